@@ -1,0 +1,102 @@
+"""Planted mistakes in the oracle (CPU only): each must make at least one pin fail.
+
+Each mutation is applied with monkeypatch to the oracle module only, so the rest of the
+suite sees the unmodified oracle.
+"""
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+import tests.test_oracle_pins as pins
+
+
+def _fails(check, *args):
+    with pytest.raises(AssertionError):
+        check(*args)
+
+
+def test_ties_to_higher_index_is_caught(monkeypatch):
+    # reverse the tie order: equal keys now prefer the higher index
+    monkeypatch.setattr(O, "_descending_stable",
+                        lambda r: (len(r) - 1 - np.argsort(-r[::-1], kind="stable")))
+    _fails(pins.check_worked_selection)
+
+
+def test_silu_sign_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "silu", lambda z: z / (1.0 + np.exp(z)))
+    _fails(pins.check_expert_vs_torch)
+    _fails(pins.check_dense_special_case)
+
+
+def test_swapped_gate_up_is_caught(monkeypatch):
+    def swapped(x_rows, w13_e, w2_e):
+        w13_e = O.f64(w13_e)
+        I = w13_e.shape[0] // 2
+        return O.__dict__["_orig_swiglu"](x_rows, np.concatenate([w13_e[I:], w13_e[:I]]), w2_e)
+    monkeypatch.setitem(O.__dict__, "_orig_swiglu", O.swiglu_expert)
+    monkeypatch.setattr(O, "swiglu_expert", swapped)
+    _fails(pins.check_expert_vs_torch)
+
+
+def test_transposed_down_projection_is_caught(monkeypatch):
+    orig = O.swiglu_expert
+
+    def transposed(x_rows, w13_e, w2_e):
+        w2 = O.f64(w2_e)
+        if w2.shape[0] != w2.shape[1]:
+            pytest.skip("needs a square case")
+        return orig(x_rows, w13_e, w2.T)
+    # use square shapes so the transposed operand still multiplies
+    monkeypatch.setattr(O, "swiglu_expert", transposed)
+    rng = np.random.default_rng(0)
+    x = rng.normal(size=(5, 6))
+    w13 = rng.normal(size=(12, 6))
+    w2 = rng.normal(size=(6, 6))
+    with pytest.raises(AssertionError):
+        np.testing.assert_allclose(O.swiglu_expert(x, w13, w2), pins._torch_swiglu(x, w13, w2),
+                                   rtol=1e-12, atol=1e-12)
+
+
+def test_wrong_source_shards_are_caught(monkeypatch):
+    # round-robin sources instead of contiguous shards
+    monkeypatch.setattr(O, "source_of_token", lambda N, P: np.arange(N, dtype=np.int64) % P)
+    _fails(pins.check_worked_layout)
+
+
+def test_missing_renormalisation_is_caught(monkeypatch):
+    orig = O.gate_weights
+    monkeypatch.setattr(O, "gate_weights", lambda z, ids, score="softmax", renormalize=True:
+                        orig(z, ids, score, False))
+    _fails(pins.check_worked_selection)
+
+
+def test_dropped_gate_in_combine_is_caught(monkeypatch):
+    orig = O.combine
+    monkeypatch.setattr(O, "combine", lambda o, lay, g, N, k, shared_out=None:
+                        orig(o, lay, np.ones_like(O.f64(g)), N, k, shared_out))
+    _fails(pins.check_worked_output)
+
+
+def test_dropped_shared_expert_is_caught(monkeypatch):
+    orig = O.moe_tokens_direct
+
+    def no_shared(cfg, *a, **kw):
+        return orig(cfg.replace(S=0), *a, **kw)
+    monkeypatch.setattr(O, "moe_tokens_direct", no_shared)
+    _fails(pins.check_shared_expert_additive)
+
+
+def test_expert_order_by_id_only_is_caught(monkeypatch):
+    # ignore the owner when ordering rows (plain argsort by expert id)
+    orig = O.dispatch_layout
+
+    def by_id(ids, E, P, expert_owner=None, S=0):
+        lay = orig(ids, E, P, expert_owner, S)
+        flat = O.i64(ids).reshape(-1)
+        row2tok = np.argsort(flat, kind="stable")
+        lay["row2tok"] = row2tok
+        lay["tok2row"] = np.empty_like(row2tok)
+        lay["tok2row"][row2tok] = np.arange(len(row2tok))
+        return lay
+    monkeypatch.setattr(O, "dispatch_layout", by_id)
+    _fails(pins.check_layout_naive_ranks, 2)
