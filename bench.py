@@ -1,0 +1,376 @@
+"""Benchmark: one MoE layer forward (router -> top-k -> dispatch layout -> permute ->
+grouped SwiGLU experts -> combine) per step, on synthetic seeded inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload fine] [--impl reference]
+
+Default workload: the fine-grained MoE layer (N=4096 tokens, d=2048, 64 routed + 2
+shared experts, top-6, I=1408, bf16).  Each step runs through the library's C ABI;
+inputs are resident in HBM when the timed region starts and L2 is flushed (a 256 MiB
+write) before every step, outside the step's CUDA-event bracket.  Under torchrun each
+rank runs its own independent batch (weak scaling, no collective on the data path);
+the time is the max over ranks.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s; grouped-GEMM TFLOP/s and permute/combine GB/s vs peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LAUNCHES_PER_STEP = 9  # router GEMM, top-k, 3 layout, permute, FC1, FC2, combine
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="fine")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def describe(cfg):
+    return (f"{cfg.name}: N={cfg.N} d={cfg.d} E={cfg.E}+{cfg.S} shared k={cfg.k} I={cfg.I} P={cfg.P} "
+            f"{cfg.score}{' renorm' if cfg.renormalize else ''}"
+            f"{f' groups {cfg.topk_groups}/{cfg.n_groups}' if cfg.n_groups > 1 else ''} {cfg.dtype}")
+
+
+def algorithmic(cfg, n_e_touched=None):
+    """Algorithmic work of one layer step: FLOPs of the two grouped GEMMs and bytes of the
+    movement kernels (each row read or written once)."""
+    A, S, N, d, I, E = cfg.N * cfg.k, cfg.S, cfg.N, cfg.d, cfg.I, cfg.E
+    b = 2 if cfg.dtype == "bf16" else 4
+    rows = A + S * N
+    touched = E if n_e_touched is None else n_e_touched
+    return dict(
+        fc1_flops=2.0 * rows * d * 2 * I,
+        fc2_flops=2.0 * rows * I * d,
+        ffn_flops=6.0 * rows * d * I,
+        fc1_weight_bytes=(touched + S) * 2 * I * d * b,
+        permute_bytes=(N + A) * d * b,
+        combine_bytes=(A + S * N + N) * d * b,
+        router_flops=2.0 * N * d * E,
+    )
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {k: float(j[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(mx), "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def source_hash(*files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload, src_hash):
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    r = rec.get(f"{kernel}/{workload}")
+    if r and r.get("source_hash") == src_hash:
+        return r["bytes_per_launch"]
+    return None
+
+
+# ------------------------------------------------------------------------------ oracle arm
+def oracle_tokens_per_s(cfg, seconds, inputs=None):
+    """Time the float64 oracle (as it stands) on consecutive 128-token slices of the
+    workload until about ``seconds`` have passed.  Returns (tokens/s, tokens, seconds, threads)."""
+    import numpy as np
+    import torch
+    from moe_inputs import make_inputs
+    from oracle import moe_oracle as O
+    threads = len(os.sched_getaffinity(0))
+    torch.set_num_threads(threads)
+    inp = inputs if inputs is not None else make_inputs(cfg, device="cpu")
+    w13 = inp["w13"].cpu()
+    w2 = inp["w2"].cpu()
+    x = inp["x"].cpu()
+    owner = inp["expert_owner"].cpu() if inp["expert_owner"] is not None else None
+    bias = inp["bias"].cpu() if inp["bias"] is not None else None
+    n_slice = 128
+    sub = cfg.replace(N=n_slice)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        s0 = done % cfg.N
+        xs = x[s0:s0 + n_slice]
+        O.moe_layer(sub.replace(N=xs.shape[0]), xs, inp["w_gate"].cpu(), bias, w13, w2, owner)
+        done += xs.shape[0]
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            return done / el, done, el, threads
+
+
+def run_reference(args, cfg, rank):
+    if rank != 0:
+        return
+    from moe_inputs import make_inputs
+    inp = make_inputs(cfg, device="cpu")
+    per_step = max(1.0, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_tokens_per_s(cfg, per_step / 4, inp)
+    tot_tok, tot_s, threads = 0, 0.0, 1
+    for _ in range(args.steps):
+        _, tok, s, threads = oracle_tokens_per_s(cfg, per_step, inp)
+        tot_tok += tok
+        tot_s += s
+    v = tot_tok / tot_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * cfg.N / v,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(cfg)},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{tot_tok} tokens of the workload in 128-token slices, whole layer in float64"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ our arm
+def main():
+    args = parse()
+    from moe_inputs import CONFIGS
+    cfg = CONFIGS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, cfg, rank)
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    import dispatch_combine_grouped_b200 as moe
+    from moe_inputs import make_inputs
+
+    dev = torch.device("cuda", local)
+    inp = make_inputs(cfg, device=dev, seed_offset=rank)
+    A, S = cfg.N * cfg.k, cfg.S
+    dt = cfg.torch_dtype
+    logits = torch.empty(cfg.N, cfg.E, dtype=torch.float32, device=dev)
+    ids = torch.empty(cfg.N, cfg.k, dtype=torch.int32, device=dev)
+    w = torch.empty(cfg.N, cfg.k, dtype=torch.float32, device=dev)
+    layout = moe.Layout(cfg, dev)
+    lay_ws = torch.empty(max(moe.layout_workspace_bytes(cfg), 1), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(A, cfg.d, dtype=dt, device=dev)
+    h = torch.empty(A + S * cfg.N, cfg.I, dtype=dt, device=dev)
+    out = torch.empty(A + S * cfg.N, cfg.d, dtype=dt, device=dev)
+    y = torch.empty(cfg.N, cfg.d, dtype=dt, device=dev)
+    ws = moe.alloc_workspace(cfg, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    x, wg, bias, owner, w13, w2 = inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], inp["w13"], inp["w2"]
+
+    def step(ev):
+        ev[0].record()
+        moe.route(cfg, x, wg, bias, out=(logits, ids, w))
+        ev[1].record()
+        moe.dispatch_layout(cfg, ids, owner, status=status, layout=layout, ws=lay_ws)
+        ev[2].record()
+        moe.permute(cfg, layout, x, out=x_perm)
+        ev[3].record()
+        moe.expert_fc1(cfg, layout, x_perm, x, w13, h=h)
+        ev[4].record()
+        moe.expert_fc2(cfg, layout, h, w2, topk_w=w, out=out)
+        ev[5].record()
+        moe.combine(cfg, layout, out, y=y)
+        ev[6].record()
+
+    def new_events():
+        return [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(new_events())
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    evs = [new_events() for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    clock_rec = clocks.stop()
+    assert status.item() == 0, f"device status {status.item()}"
+
+    names = ["route", "layout", "permute", "fc1", "fc2", "combine"]
+    stage_ms = {n: 0.0 for n in names}
+    step_ms = 0.0
+    for ev in evs:
+        for j, n in enumerate(names):
+            stage_ms[n] += ev[j].elapsed_time(ev[j + 1])
+        step_ms += ev[0].elapsed_time(ev[6])
+    t_local = torch.tensor([step_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
+    step_ms_max = float(t_local.item()) / args.steps
+    for n in names:
+        stage_ms[n] /= args.steps
+
+    # fused entry point (same kernels, one C call per step), for reference
+    fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        fev[i][0].record()
+        moe.layer_forward(cfg, x, wg, bias, owner, w13, w2, y=y, ws=ws, status=status)
+        fev[i][1].record()
+    torch.cuda.synchronize()
+    fused_ms = sum(a.elapsed_time(b) for a, b in fev) / args.steps
+
+    # end to end: pinned host input -> device, layer, result -> pinned host, per step
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(cfg.N, cfg.d, dtype=dt).pin_memory()
+    x_dev = torch.empty_like(x)
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record()
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.layer_forward(cfg, x_dev, wg, bias, owner, w13, w2, y=y, ws=ws, status=status)
+        y_host.copy_(y, non_blocking=True)
+        e2e_ev[i][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps], dtype=torch.float64,
+                          device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+
+    n_e = layout["n_e"].cpu()
+    touched = int((n_e > 0).sum())
+    alg = algorithmic(cfg, touched)
+    peaks, peak_src = load_peaks()
+    fc1_s = stage_ms["fc1"] / 1e3
+    fc1_tflops = alg["fc1_flops"] / fc1_s / 1e12
+    ffn_tflops = alg["ffn_flops"] / ((stage_ms["fc1"] + stage_ms["fc2"]) / 1e3) / 1e12
+    permute_gbs = alg["permute_bytes"] / (stage_ms["permute"] / 1e3) / 1e9
+    combine_gbs = alg["combine_bytes"] / (stage_ms["combine"] / 1e3) / 1e9
+    src = source_hash("dispatch_combine_grouped_b200/csrc/gemm_tc.cu", "dispatch_combine_grouped_b200/csrc/common.cuh")
+    traffic = recorded_traffic("fc1", cfg.name, src)
+    tokens_total = cfg.N * world
+    value = tokens_total / (step_ms_max / 1e3)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded normal inputs, random-init weights)",
+            "config": {"workload": describe(cfg), "tokens_per_gpu": cfg.N, "l2": "flushed before every step "
+                       "(256 MiB write, outside the step's event bracket)", "parallelism": f"{world} independent "
+                       "replicas (one batch per GPU)"},
+            "roofline": {"kernel": "grouped FC1 + SwiGLU (tcgen05)", "bound": "tensor", "achieved": fc1_tflops,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": fc1_tflops / peaks["bf16_tflops"],
+                         "peak_source": f"{peak_src} bf16 burst", "traffic": traffic,
+                         "flops_per_launch": alg["fc1_flops"], "ms_per_launch": stage_ms["fc1"]},
+            "stages_ms": stage_ms,
+            "ffn": {"tflops": ffn_tflops, "frac_of_peak": ffn_tflops / peaks["bf16_tflops"]},
+            "permute": {"gbs": permute_gbs, "frac_of_hbm": permute_gbs / peaks["hbm_gbs"],
+                        "frac_of_8tbs": permute_gbs / 8000.0},
+            "combine": {"gbs": combine_gbs, "frac_of_hbm": combine_gbs / peaks["hbm_gbs"],
+                        "frac_of_8tbs": combine_gbs / 8000.0},
+            "fused_ms_per_step": fused_ms,
+            "imbalance": {"max_over_mean_n_e": float(n_e.max()) / float(n_e.float().mean()),
+                          "experts_empty": int((n_e == 0).sum())},
+            "e2e": {"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": x.numel() * x.element_size(),
+                    "d2h_bytes_per_step": y.numel() * y.element_size()},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clock_rec,
+            "wall_s_timed": wall,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            v, tok, s, threads = oracle_tokens_per_s(cfg, args.cpu_seconds, {k: (t.cpu() if t is not None else None)
+                                                                             for k, t in inp.items()})
+            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                    "sample": f"{tok} tokens of the workload in 128-token slices, "
+                                              f"whole layer in float64, {s:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,272 @@
+"""Thin ctypes binding over libmoe's C ABI (include/moe.h).
+
+Argument marshalling only: tensors are passed as device pointers with the current torch
+CUDA stream, and every step of the layer runs in libmoe's CUDA kernels.  Buffers the
+ABI leaves to the caller are allocated here with torch (device memory is plumbing); the
+library itself allocates nothing.  If libmoe.so is missing or fails to load, importing
+this module raises: there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_BAD_INDEX, \
+    MOE_ERR_TIMEOUT = range(7)
+MOE_F32, MOE_BF16 = 0, 1
+MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
+
+# every symbol include/moe.h declares
+EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_config",
+            "moe_layout_workspace_bytes", "moe_workspace_bytes", "moe_route", "moe_dispatch_layout",
+            "moe_permute", "moe_permute_staged", "moe_grouped_ffn", "moe_expert_fc1", "moe_expert_fc2",
+            "moe_combine", "moe_combine_staged",
+            "moe_layer_forward"]
+
+
+class CConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ["N", "d", "E", "k", "I", "n_shared", "P", "n_groups", "topk_groups", "score",
+                 "renormalize", "dtype"]]
+
+
+LAYOUT_FIELDS = ["n_e", "expert_off", "C", "send_off", "recv_off", "tok2send", "send2row", "ret2tok",
+                 "tok2row", "row2tok", "tile_off"]
+
+
+class CLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in LAYOUT_FIELDS]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status, where, detail=""):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({_status_text(status)}) {detail}".strip())
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libmoe.so not found at {path}; build it with "
+                          f"`python -m dispatch_combine_grouped_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    cfgp, layp = ctypes.POINTER(CConfig), ctypes.POINTER(CLayout)
+    sig = {
+        "moe_version": (i32, []),
+        "moe_status_string": (ctypes.c_char_p, [i32]),
+        "moe_last_error": (ctypes.c_char_p, []),
+        "moe_check_config": (i32, [cfgp]),
+        "moe_layout_workspace_bytes": (sz, [cfgp]),
+        "moe_workspace_bytes": (sz, [cfgp]),
+        "moe_route": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_dispatch_layout": (i32, [cfgp, vp, vp, layp, vp, vp, sz, vp]),
+        "moe_permute": (i32, [cfgp, layp, vp, vp, vp]),
+        "moe_permute_staged": (i32, [cfgp, layp, vp, vp, vp, vp]),
+        "moe_grouped_ffn": (i32, [cfgp, layp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_fc1": (i32, [cfgp, layp, vp, vp, vp, vp, vp]),
+        "moe_expert_fc2": (i32, [cfgp, layp, vp, vp, vp, vp, vp]),
+        "moe_combine": (i32, [cfgp, layp, vp, vp, vp, vp]),
+        "moe_combine_staged": (i32, [cfgp, layp, vp, vp, vp, vp, vp]),
+        "moe_layer_forward": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _status_text(s):
+    try:
+        return load().moe_status_string(s).decode()
+    except Exception:  # pragma: no cover
+        return "?"
+
+
+def _check(status, where):
+    if status != MOE_OK:
+        detail = load().moe_last_error().decode()
+        raise MoEError(status, where, detail)
+
+
+def c_config(cfg) -> CConfig:
+    """moe_config from a workload description (moe_inputs.MoEConfig or any object with
+    the same attribute names)."""
+    score = cfg.score if isinstance(cfg.score, int) else \
+        {"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID}[cfg.score]
+    dtype = cfg.dtype if isinstance(cfg.dtype, int) else {"f32": MOE_F32, "bf16": MOE_BF16}[cfg.dtype]
+    return CConfig(cfg.N, cfg.d, cfg.E, cfg.k, cfg.I, cfg.S, cfg.P, cfg.n_groups, cfg.topk_groups,
+                   score, int(bool(cfg.renormalize)), dtype)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dtype(cfg):
+    return torch.float32 if c_config(cfg).dtype == MOE_F32 else torch.bfloat16
+
+
+class Layout:
+    """Caller-owned layout arrays (int32, on the device) and their C view."""
+
+    def __init__(self, cfg, device="cuda"):
+        A, E, P, S = cfg.N * cfg.k, cfg.E, cfg.P, cfg.S
+        sizes = dict(n_e=E, expert_off=E + 1, C=P * P, send_off=P * P, recv_off=P + 1, tok2send=A,
+                     send2row=A, ret2tok=A, tok2row=A, row2tok=A, tile_off=E + S + 1)
+        self.t = {k: torch.empty(max(v, 1), dtype=torch.int32, device=device) for k, v in sizes.items()}
+        self.sizes = sizes
+        self.c = CLayout(*[self.t[k].data_ptr() for k in LAYOUT_FIELDS])
+
+    def __getitem__(self, key):
+        return self.t[key][:self.sizes[key]]
+
+    def as_dict(self):
+        return {k: self[k] for k in LAYOUT_FIELDS}
+
+
+def version() -> int:
+    return load().moe_version()
+
+
+def check_config(cfg):
+    c = c_config(cfg)
+    _check(load().moe_check_config(ctypes.byref(c)), "moe_check_config")
+
+
+def workspace_bytes(cfg) -> int:
+    c = c_config(cfg)
+    return load().moe_workspace_bytes(ctypes.byref(c))
+
+
+def layout_workspace_bytes(cfg) -> int:
+    c = c_config(cfg)
+    return load().moe_layout_workspace_bytes(ctypes.byref(c))
+
+
+def route(cfg, x, w_gate, bias=None, out=None):
+    """-> (logits [N,E] fp32, topk_ids [N,k] int32, topk_w [N,k] fp32)"""
+    c = c_config(cfg)
+    if out is None:
+        dev = x.device
+        out = (torch.empty(cfg.N, cfg.E, dtype=torch.float32, device=dev),
+               torch.empty(cfg.N, cfg.k, dtype=torch.int32, device=dev),
+               torch.empty(cfg.N, cfg.k, dtype=torch.float32, device=dev))
+    logits, ids, w = out
+    _check(load().moe_route(ctypes.byref(c), _p(x), _p(w_gate), _p(bias), _p(logits), _p(ids), _p(w),
+                            _stream()), "moe_route")
+    return logits, ids, w
+
+
+def dispatch_layout(cfg, topk_ids, expert_owner=None, status=None, layout=None, ws=None):
+    c = c_config(cfg)
+    lib = load()
+    layout = layout or Layout(cfg, topk_ids.device)
+    nbytes = lib.moe_layout_workspace_bytes(ctypes.byref(c))
+    if ws is None:
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=topk_ids.device)
+    _check(lib.moe_dispatch_layout(ctypes.byref(c), _p(expert_owner), _p(topk_ids), ctypes.byref(layout.c),
+                                   _p(status), _p(ws), ws.numel(), _stream()), "moe_dispatch_layout")
+    return layout
+
+
+def permute(cfg, layout, x, out=None):
+    c = c_config(cfg)
+    if out is None:
+        out = torch.empty(cfg.N * cfg.k, cfg.d, dtype=x.dtype, device=x.device)
+    _check(load().moe_permute(ctypes.byref(c), ctypes.byref(layout.c), _p(x), _p(out), _stream()),
+           "moe_permute")
+    return out
+
+
+def permute_staged(cfg, layout, x):
+    c = c_config(cfg)
+    send = torch.empty(cfg.N * cfg.k, cfg.d, dtype=x.dtype, device=x.device)
+    out = torch.empty_like(send)
+    _check(load().moe_permute_staged(ctypes.byref(c), ctypes.byref(layout.c), _p(x), _p(send), _p(out),
+                                     _stream()), "moe_permute_staged")
+    return send, out
+
+
+def grouped_ffn(cfg, layout, x_perm, x, w13, w2, topk_w=None, h=None, out=None):
+    """-> (h [A+S*N, I], out [A+S*N, d]) in the config dtype."""
+    c = c_config(cfg)
+    rows = cfg.N * cfg.k + cfg.S * cfg.N
+    dt, dev = _dtype(cfg), x_perm.device
+    if h is None:
+        h = torch.empty(rows, cfg.I, dtype=dt, device=dev)
+    if out is None:
+        out = torch.empty(rows, cfg.d, dtype=dt, device=dev)
+    _check(load().moe_grouped_ffn(ctypes.byref(c), ctypes.byref(layout.c), _p(x_perm), _p(x), _p(w13), _p(w2),
+                                  _p(topk_w), _p(h), _p(out), _stream()), "moe_grouped_ffn")
+    return h, out
+
+
+def expert_fc1(cfg, layout, x_perm, x, w13, h=None):
+    c = c_config(cfg)
+    if h is None:
+        h = torch.empty(cfg.N * cfg.k + cfg.S * cfg.N, cfg.I, dtype=_dtype(cfg), device=x_perm.device)
+    _check(load().moe_expert_fc1(ctypes.byref(c), ctypes.byref(layout.c), _p(x_perm), _p(x), _p(w13), _p(h),
+                                 _stream()), "moe_expert_fc1")
+    return h
+
+
+def expert_fc2(cfg, layout, h, w2, topk_w=None, out=None):
+    c = c_config(cfg)
+    if out is None:
+        out = torch.empty(cfg.N * cfg.k + cfg.S * cfg.N, cfg.d, dtype=_dtype(cfg), device=h.device)
+    _check(load().moe_expert_fc2(ctypes.byref(c), ctypes.byref(layout.c), _p(h), _p(w2), _p(topk_w), _p(out),
+                                 _stream()), "moe_expert_fc2")
+    return out
+
+
+def combine(cfg, layout, out_rows, topk_w=None, y=None):
+    c = c_config(cfg)
+    if y is None:
+        y = torch.empty(cfg.N, cfg.d, dtype=out_rows.dtype, device=out_rows.device)
+    _check(load().moe_combine(ctypes.byref(c), ctypes.byref(layout.c), _p(out_rows), _p(topk_w), _p(y),
+                              _stream()), "moe_combine")
+    return y
+
+
+def combine_staged(cfg, layout, out_rows, topk_w=None):
+    c = c_config(cfg)
+    ret = torch.empty(cfg.N * cfg.k, cfg.d, dtype=out_rows.dtype, device=out_rows.device)
+    y = torch.empty(cfg.N, cfg.d, dtype=out_rows.dtype, device=out_rows.device)
+    _check(load().moe_combine_staged(ctypes.byref(c), ctypes.byref(layout.c), _p(out_rows), _p(topk_w), _p(ret),
+                                     _p(y), _stream()), "moe_combine_staged")
+    return ret, y
+
+
+def alloc_workspace(cfg, device="cuda"):
+    return torch.empty(max(workspace_bytes(cfg), 1), dtype=torch.uint8, device=device)
+
+
+def layer_forward(cfg, x, w_gate, bias, expert_owner, w13, w2, y=None, ws=None, layout=None, status=None):
+    """The whole layer through moe_layer_forward; -> y [N, d]."""
+    c = c_config(cfg)
+    if ws is None:
+        ws = alloc_workspace(cfg, x.device)
+    if y is None:
+        y = torch.empty(cfg.N, cfg.d, dtype=x.dtype, device=x.device)
+    lay = ctypes.byref(layout.c) if layout is not None else None
+    _check(load().moe_layer_forward(ctypes.byref(c), _p(x), _p(w_gate), _p(bias), _p(expert_owner), _p(w13),
+                                    _p(w2), _p(y), lay, _p(status), _p(ws), ws.numel(), _stream()),
+           "moe_layer_forward")
+    return y

@@ -1,0 +1,78 @@
+// Internal declarations shared by the translation units of libmoe.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kMaxE = 256;        // routed experts
+constexpr int kMaxK = 8;          // top-k
+constexpr int kMaxP = 32;         // virtual owners
+constexpr int kMaxGroups = 32;    // expert groups
+constexpr int kMaxTopkGroups = 8; // groups kept per token
+constexpr int kMaxShared = 8;     // shared experts
+constexpr int kLayoutChunk = 1024;  // assignments per counting chunk
+constexpr int kTileRows = 128;      // rows per block in tile_off
+
+// ---- layout.cu
+size_t layout_ws_bytes(int A, int E, int P, int nchunks);
+cudaError_t launch_layout(const moe_config& cfg, const int32_t* owner, const int32_t* ids, const moe_layout& L,
+                          int32_t* status, void* ws, cudaStream_t st);
+
+// ---- route.cu : top-k selection and gates from fp32 logits
+cudaError_t launch_topk(const moe_config& cfg, const float* logits, int32_t* ids, float* w, cudaStream_t st);
+
+// ---- movement.cu : permute / combine and their two-hop (staged) forms
+cudaError_t launch_permute(const moe_config& cfg, const moe_layout& L, const void* x, void* x_perm,
+                           cudaStream_t st);
+cudaError_t launch_permute_staged(const moe_config& cfg, const moe_layout& L, const void* x, void* send_buf,
+                                  void* x_perm, cudaStream_t st);
+cudaError_t launch_combine(const moe_config& cfg, const moe_layout& L, const void* out, const float* topk_w,
+                           void* y, cudaStream_t st);
+cudaError_t launch_combine_staged(const moe_config& cfg, const moe_layout& L, const void* out,
+                                  const float* topk_w, void* ret_buf, void* y, cudaStream_t st);
+
+// ---- GEMM family: a "group" is a block of rows multiplied by one weight matrix.
+// Groups 0..E-1 are routed experts (rows [expert_off[g], +n_e[g]) of A map 0); groups
+// E..E+S-1 are shared experts over N rows (from A map 1 when shared_from_map1, else
+// from A map 0 starting at row A_routed + s*N).  The router is one shared group.
+enum GemmMode { MODE_ROUTER = 0, MODE_FC1 = 1, MODE_FC2 = 2 };
+
+struct GemmArgs {
+  int mode;
+  int G;             // groups
+  int E;             // routed groups (first E)
+  int N;             // rows of a shared group
+  int A_routed;      // rows of all routed groups (= N*k for the FFN, 0 for the router)
+  int K;             // reduction length
+  int n_out;         // valid output columns (E, I or d)
+  int I;             // FC1: row offset of W_up inside W13
+  int shared_from_map1;
+  const int32_t* n_e;
+  const int32_t* expert_off;
+  const int32_t* row2tok;
+  const float* gate_w;  // FC2: routed row r is scaled by gate_w[row2tok[r]] (NULL: no scale)
+  const float* bias;    // router: added to every logit (NULL: none)
+  void* out;
+  long long ldo;        // output row stride in elements
+  int* status;
+  // raw operand pointers (SIMT path; the tensor-core path reads through tensor maps)
+  const void* a0;
+  const void* a1;
+  const void* b;
+  long long b_rows;     // rows of one weight matrix (2I, d or E)
+};
+
+// tensor-core (tcgen05) path, bf16 operands, fp32 accumulation
+cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStream_t st);
+// CUDA-core path, fp32 operands (the fp32 configurations)
+cudaError_t launch_simt_gemm(const GemmArgs& g, cudaStream_t st);
+
+int sm_count();
+
+}  // namespace moe

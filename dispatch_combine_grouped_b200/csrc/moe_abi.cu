@@ -1,0 +1,358 @@
+// C entry points of libmoe: argument validation, workspace carving and the launch order
+// of the layer's steps.  Every step runs in this library's CUDA kernels; nothing here
+// computes on the host.
+#include <stdio.h>
+#include <string.h>
+
+#include "kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+moe_status fail(moe_status s, const char* what) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s", what);
+  return s;
+}
+
+moe_status cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return MOE_OK;
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorString(e));
+  return MOE_ERR_CUDA;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int elem_bytes(const moe_config& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
+
+moe_status check_config(const moe_config* c) {
+  if (!c) return fail(MOE_ERR_INVALID_ARG, "config is NULL");
+  if (c->N < 0 || c->d <= 0 || c->E <= 0 || c->k <= 0 || c->I <= 0 || c->n_shared < 0 || c->P <= 0)
+    return fail(MOE_ERR_INVALID_ARG, "sizes must be positive (N >= 0)");
+  if (c->n_groups <= 0 || c->topk_groups <= 0 || c->topk_groups > c->n_groups || c->E % c->n_groups != 0)
+    return fail(MOE_ERR_INVALID_ARG, "need 1 <= topk_groups <= n_groups and E % n_groups == 0");
+  if ((long long)c->k > (long long)c->topk_groups * (c->E / c->n_groups))
+    return fail(MOE_ERR_INVALID_ARG, "k exceeds the experts of the kept groups");
+  if ((c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID) ||
+      (c->dtype != MOE_F32 && c->dtype != MOE_BF16) || (c->renormalize != 0 && c->renormalize != 1))
+    return fail(MOE_ERR_INVALID_ARG, "score, dtype or renormalize out of range");
+  if (c->k > kMaxK || c->E > kMaxE || c->P > kMaxP || c->n_groups > kMaxGroups ||
+      c->topk_groups > kMaxTopkGroups || c->n_shared > kMaxShared)
+    return fail(MOE_ERR_UNSUPPORTED, "k <= 8, E <= 256, P <= 32, n_groups <= 32, topk_groups <= 8, S <= 8");
+  const int eb = elem_bytes(*c);
+  if ((c->d * eb) % 16 != 0 || (c->I * eb) % 16 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "rows of d and I elements must be multiples of 16 bytes");
+  const long long rows = (long long)c->N * c->k + (long long)c->n_shared * c->N;
+  if (rows >= (1LL << 31) / 2) return fail(MOE_ERR_UNSUPPORTED, "N * (k + S) too large");
+  return MOE_OK;
+}
+
+moe_status check_owner(const moe_config& c, const int32_t* owner) {
+  if (!owner && c.E % c.P != 0) return fail(MOE_ERR_INVALID_ARG, "contiguous placement needs E % P == 0");
+  return MOE_OK;
+}
+
+bool layout_complete(const moe_layout* L) {
+  return L && L->n_e && L->expert_off && L->C && L->send_off && L->recv_off && L->tok2send && L->send2row &&
+         L->ret2tok && L->tok2row && L->row2tok && L->tile_off;
+}
+
+size_t layout_scratch(const moe_config& c) {
+  const int A = c.N * c.k;
+  const int nchunks = (A + kLayoutChunk - 1) / kLayoutChunk;
+  return align256(layout_ws_bytes(A, c.E, c.P, nchunks));
+}
+
+struct FwdWs {
+  float* logits;
+  int32_t* ids;
+  float* w;
+  moe_layout lay;
+  void* lay_ws;
+  void* x_perm;
+  void* h;
+  void* out;
+  size_t total;
+};
+
+FwdWs carve_forward(const moe_config& c, char* base) {
+  FwdWs w;
+  memset(&w, 0, sizeof(w));
+  const size_t A = (size_t)c.N * c.k, E = c.E, P = c.P, S = c.n_shared, eb = elem_bytes(c);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off += align256(bytes ? bytes : 1);
+    return p;
+  };
+  w.logits = reinterpret_cast<float*>(take((size_t)c.N * E * 4));
+  w.ids = reinterpret_cast<int32_t*>(take(A * 4));
+  w.w = reinterpret_cast<float*>(take(A * 4));
+  w.lay.n_e = reinterpret_cast<int32_t*>(take(E * 4));
+  w.lay.expert_off = reinterpret_cast<int32_t*>(take((E + 1) * 4));
+  w.lay.C = reinterpret_cast<int32_t*>(take(P * P * 4));
+  w.lay.send_off = reinterpret_cast<int32_t*>(take(P * P * 4));
+  w.lay.recv_off = reinterpret_cast<int32_t*>(take((P + 1) * 4));
+  w.lay.tok2send = reinterpret_cast<int32_t*>(take(A * 4));
+  w.lay.send2row = reinterpret_cast<int32_t*>(take(A * 4));
+  w.lay.ret2tok = reinterpret_cast<int32_t*>(take(A * 4));
+  w.lay.tok2row = reinterpret_cast<int32_t*>(take(A * 4));
+  w.lay.row2tok = reinterpret_cast<int32_t*>(take(A * 4));
+  w.lay.tile_off = reinterpret_cast<int32_t*>(take((E + S + 1) * 4));
+  w.lay_ws = take(layout_scratch(c));
+  w.x_perm = take(A * c.d * eb);
+  w.h = take((A + S * c.N) * c.I * eb);
+  w.out = take((A + S * c.N) * c.d * eb);
+  w.total = off;
+  return w;
+}
+
+moe_status route_impl(const moe_config& c, const void* x, const void* w_gate, const float* bias, float* logits,
+                      int32_t* ids, float* w, cudaStream_t st) {
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.mode = MODE_ROUTER;
+  g.G = 1;
+  g.E = 0;
+  g.N = c.N;
+  g.A_routed = 0;
+  g.K = c.d;
+  g.n_out = c.E;
+  g.shared_from_map1 = 1;
+  g.bias = bias;
+  g.out = logits;
+  g.ldo = c.E;
+  g.a0 = x;
+  g.a1 = x;
+  g.b = w_gate;
+  g.b_rows = c.E;
+  cudaError_t e = c.dtype == MOE_BF16 ? launch_tc_gemm(g, c.N, c.N, st) : launch_simt_gemm(g, st);
+  if (e != cudaSuccess) return cuda_status(e, "router GEMM");
+  return cuda_status(launch_topk(c, logits, ids, w, st), "top-k");
+}
+
+GemmArgs fc1_args(const moe_config& c, const moe_layout& L, const void* x_perm, const void* x, const void* w13,
+                  void* h) {
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.mode = MODE_FC1;
+  g.G = c.E + c.n_shared;
+  g.E = c.E;
+  g.N = c.N;
+  g.A_routed = c.N * c.k;
+  g.K = c.d;
+  g.n_out = c.I;
+  g.I = c.I;
+  g.shared_from_map1 = 1;
+  g.n_e = L.n_e;
+  g.expert_off = L.expert_off;
+  g.row2tok = L.row2tok;
+  g.out = h;
+  g.ldo = c.I;
+  g.a0 = x_perm;
+  g.a1 = c.n_shared > 0 ? x : nullptr;
+  g.b = w13;
+  g.b_rows = 2LL * c.I;
+  return g;
+}
+
+GemmArgs fc2_args(const moe_config& c, const moe_layout& L, const void* h, const void* w2, const float* topk_w,
+                  void* out) {
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.mode = MODE_FC2;
+  g.G = c.E + c.n_shared;
+  g.E = c.E;
+  g.N = c.N;
+  g.A_routed = c.N * c.k;
+  g.K = c.I;
+  g.n_out = c.d;
+  g.I = c.I;
+  g.shared_from_map1 = 0;
+  g.n_e = L.n_e;
+  g.expert_off = L.expert_off;
+  g.row2tok = L.row2tok;
+  g.gate_w = topk_w;
+  g.out = out;
+  g.ldo = c.d;
+  g.a0 = h;
+  g.b = w2;
+  g.b_rows = c.d;
+  return g;
+}
+
+moe_status fc1_impl(const moe_config& c, const moe_layout& L, const void* x_perm, const void* x, const void* w13,
+                    void* h, cudaStream_t st) {
+  const GemmArgs g = fc1_args(c, L, x_perm, x, w13, h);
+  cudaError_t e = c.dtype == MOE_BF16 ? launch_tc_gemm(g, c.N * c.k, c.N, st) : launch_simt_gemm(g, st);
+  return cuda_status(e, "FC1 grouped GEMM");
+}
+
+moe_status fc2_impl(const moe_config& c, const moe_layout& L, const void* h, const void* w2, const float* topk_w,
+                    void* out, cudaStream_t st) {
+  const GemmArgs g = fc2_args(c, L, h, w2, topk_w, out);
+  cudaError_t e = c.dtype == MOE_BF16 ? launch_tc_gemm(g, c.N * c.k + c.n_shared * c.N, 0, st)
+                                      : launch_simt_gemm(g, st);
+  return cuda_status(e, "FC2 grouped GEMM");
+}
+
+moe_status ffn_impl(const moe_config& c, const moe_layout& L, const void* x_perm, const void* x, const void* w13,
+                    const void* w2, const float* topk_w, void* h, void* out, cudaStream_t st) {
+  moe_status s = fc1_impl(c, L, x_perm, x, w13, h, st);
+  if (s != MOE_OK) return s;
+  return fc2_impl(c, L, h, w2, topk_w, out, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t moe_version(void) { return 100; }
+
+const char* moe_status_string(int32_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported size";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_BAD_INDEX: return "expert id or owner out of range (device)";
+    case MOE_ERR_TIMEOUT: return "bounded wait timed out (device)";
+    default: return "unknown status";
+  }
+}
+
+const char* moe_last_error(void) { return g_last_error; }
+
+moe_status moe_check_config(const moe_config* cfg) { return check_config(cfg); }
+
+size_t moe_layout_workspace_bytes(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return layout_scratch(*cfg);
+}
+
+size_t moe_workspace_bytes(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return carve_forward(*cfg, nullptr).total;
+}
+
+moe_status moe_route(const moe_config* cfg, const void* x, const void* w_gate, const float* bias, float* logits,
+                     int32_t* topk_ids, float* topk_w, moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->N == 0) return MOE_OK;
+  if (!x || !w_gate || !logits || !topk_ids || !topk_w) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return route_impl(*cfg, x, w_gate, bias, logits, topk_ids, topk_w, (cudaStream_t)stream);
+}
+
+moe_status moe_dispatch_layout(const moe_config* cfg, const int32_t* expert_owner, const int32_t* topk_ids,
+                               const moe_layout* out, int32_t* dev_status, void* ws, size_t ws_bytes,
+                               moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
+  if (!layout_complete(out) || (cfg->N > 0 && !topk_ids)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!ws || ws_bytes < layout_scratch(*cfg)) return fail(MOE_ERR_WORKSPACE, "layout workspace too small");
+  return cuda_status(launch_layout(*cfg, expert_owner, topk_ids, *out, dev_status, ws, (cudaStream_t)stream),
+                     "layout");
+}
+
+moe_status moe_permute(const moe_config* cfg, const moe_layout* layout, const void* x, void* x_perm,
+                       moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->N == 0) return MOE_OK;
+  if (!layout || !layout->tok2row || !x || !x_perm) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return cuda_status(launch_permute(*cfg, *layout, x, x_perm, (cudaStream_t)stream), "permute");
+}
+
+moe_status moe_permute_staged(const moe_config* cfg, const moe_layout* layout, const void* x, void* send_buf,
+                              void* x_perm, moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->N == 0) return MOE_OK;
+  if (!layout || !layout->tok2send || !layout->send2row || !x || !send_buf || !x_perm)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return cuda_status(launch_permute_staged(*cfg, *layout, x, send_buf, x_perm, (cudaStream_t)stream),
+                     "permute (staged)");
+}
+
+moe_status moe_grouped_ffn(const moe_config* cfg, const moe_layout* layout, const void* x_perm, const void* x,
+                           const void* w13, const void* w2, const float* topk_w, void* h_ws, void* out,
+                           moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->N == 0) return MOE_OK;
+  if (!layout || !layout->n_e || !layout->expert_off || !layout->row2tok || !x_perm || !w13 || !w2 || !h_ws ||
+      !out || (cfg->n_shared > 0 && !x))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return ffn_impl(*cfg, *layout, x_perm, x, w13, w2, topk_w, h_ws, out, (cudaStream_t)stream);
+}
+
+moe_status moe_expert_fc1(const moe_config* cfg, const moe_layout* layout, const void* x_perm, const void* x,
+                          const void* w13, void* h_ws, moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->N == 0) return MOE_OK;
+  if (!layout || !layout->n_e || !layout->expert_off || !x_perm || !w13 || !h_ws || (cfg->n_shared > 0 && !x))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return fc1_impl(*cfg, *layout, x_perm, x, w13, h_ws, (cudaStream_t)stream);
+}
+
+moe_status moe_expert_fc2(const moe_config* cfg, const moe_layout* layout, const void* h_ws, const void* w2,
+                          const float* topk_w, void* out, moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->N == 0) return MOE_OK;
+  if (!layout || !layout->n_e || !layout->expert_off || !layout->row2tok || !h_ws || !w2 || !out)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return fc2_impl(*cfg, *layout, h_ws, w2, topk_w, out, (cudaStream_t)stream);
+}
+
+moe_status moe_combine(const moe_config* cfg, const moe_layout* layout, const void* out, const float* topk_w,
+                       void* y, moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->N == 0) return MOE_OK;
+  if (!layout || !layout->tok2row || !out || !y) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return cuda_status(launch_combine(*cfg, *layout, out, topk_w, y, (cudaStream_t)stream), "combine");
+}
+
+moe_status moe_combine_staged(const moe_config* cfg, const moe_layout* layout, const void* out,
+                              const float* topk_w, void* ret_buf, void* y, moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->N == 0) return MOE_OK;
+  if (!layout || !layout->tok2send || !layout->send2row || !out || !ret_buf || !y)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return cuda_status(launch_combine_staged(*cfg, *layout, out, topk_w, ret_buf, y, (cudaStream_t)stream),
+                     "combine (staged)");
+}
+
+moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
+                             const int32_t* expert_owner, const void* w13, const void* w2, void* y,
+                             const moe_layout* layout_out, int32_t* dev_status, void* ws, size_t ws_bytes,
+                             moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
+  const moe_config& c = *cfg;
+  FwdWs w = carve_forward(c, nullptr);
+  if (!ws || ws_bytes < w.total) return fail(MOE_ERR_WORKSPACE, "forward workspace too small");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return fail(MOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if (layout_out && !layout_complete(layout_out)) return fail(MOE_ERR_INVALID_ARG, "incomplete layout_out");
+  if (c.N > 0 && (!x || !w_gate || !w13 || !w2 || !y)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  w = carve_forward(c, static_cast<char*>(ws));
+  const moe_layout& L = layout_out ? *layout_out : w.lay;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (c.N > 0 && (s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
+  if ((s = cuda_status(launch_layout(c, expert_owner, w.ids, L, dev_status, w.lay_ws, st), "layout")) != MOE_OK)
+    return s;
+  if (c.N == 0) return MOE_OK;
+  if ((s = cuda_status(launch_permute(c, L, x, w.x_perm, st), "permute")) != MOE_OK) return s;
+  if ((s = ffn_impl(c, L, w.x_perm, x, w13, w2, w.w, w.h, w.out, st)) != MOE_OK) return s;
+  return cuda_status(launch_combine(c, L, w.out, nullptr, y, st), "combine");
+}
+
+}  // extern "C"

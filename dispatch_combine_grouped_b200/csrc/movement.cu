@@ -1,0 +1,230 @@
+// Token movement: permute (dispatch) and combine, plus their two-hop "staged" forms.
+//
+// "MoE我们喜欢你（四）" §4 gives the pipeline permute_by_expert -> a2a dispatch ->
+// grouped_gemm -> a2a combine -> unpermute_and_weighted_sum; the ep_deepep explainer §3
+// says the source buckets by owner and the combine returns rows to the source, where
+// they are summed by gate.  On one GPU the all-to-all is a transpose of row blocks, so
+// the fused kernels compose it with the permute / unpermute through the layout maps;
+// the staged kernels materialise the send (or return) buffer in between.
+//
+// All kernels: one warp per row (or token), 16-byte vectors, rows are d * elem bytes
+// (a multiple of 16).  Permute is a bit copy and ignores the dtype.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+constexpr int kMoveWarps = 8;   // warps per CTA
+constexpr int kMoveUnroll = 4;  // 16-byte vectors in flight per lane per step
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// Token-centric scatter: dst[map[t*k + j]] = src[t] for j < k (each source row read once).
+__global__ void __launch_bounds__(kMoveWarps * 32) scatter_token_rows(const uint4* __restrict__ src,
+                                                                       uint4* __restrict__ dst,
+                                                                       const int32_t* __restrict__ map, int N,
+                                                                       int k, int vpr) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kMoveWarps + (threadIdx.x >> 5);
+  if (t >= N) return;
+  const int my = lane < k ? map[(size_t)t * k + lane] : 0;
+  int rows[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) rows[j] = __shfl_sync(0xffffffffu, my, j);
+  const uint4* s = src + (size_t)t * vpr;
+  for (int v0 = 0; v0 < vpr; v0 += 32 * kMoveUnroll) {
+    uint4 buf[kMoveUnroll];
+#pragma unroll
+    for (int u = 0; u < kMoveUnroll; ++u) {
+      const int v = v0 + u * 32 + lane;
+      if (v < vpr) buf[u] = ld_stream(s + v);
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j < k) {
+        uint4* d = dst + (size_t)rows[j] * vpr;
+#pragma unroll
+        for (int u = 0; u < kMoveUnroll; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (v < vpr) d[v] = buf[u];
+        }
+      }
+    }
+  }
+}
+
+// Row gather: dst[i] = src[map[i]] for i < rows  (map == NULL: dst[map_inv...] not used)
+// Row scatter: dst[map[i]] = src[i]
+template <bool kScatter>
+__global__ void __launch_bounds__(kMoveWarps * 32) move_rows(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                              const int32_t* __restrict__ map, int rows, int vpr) {
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kMoveWarps + (threadIdx.x >> 5);
+  if (i >= rows) return;
+  const int m = map[i];
+  const uint4* s = src + (size_t)(kScatter ? i : m) * vpr;
+  uint4* d = dst + (size_t)(kScatter ? m : i) * vpr;
+  for (int v0 = 0; v0 < vpr; v0 += 32 * kMoveUnroll) {
+    uint4 buf[kMoveUnroll];
+#pragma unroll
+    for (int u = 0; u < kMoveUnroll; ++u) {
+      const int v = v0 + u * 32 + lane;
+      if (v < vpr) buf[u] = ld_stream(s + v);
+    }
+#pragma unroll
+    for (int u = 0; u < kMoveUnroll; ++u) {
+      const int v = v0 + u * 32 + lane;
+      if (v < vpr) d[v] = buf[u];
+    }
+  }
+}
+
+template <typename T>
+struct Vec;
+template <>
+struct Vec<float> {
+  static constexpr int n = 4;
+  __device__ static void unpack(const uint4& q, float (&f)[8]) {
+    f[0] = __uint_as_float(q.x);
+    f[1] = __uint_as_float(q.y);
+    f[2] = __uint_as_float(q.z);
+    f[3] = __uint_as_float(q.w);
+  }
+  __device__ static uint4 pack(const float (&f)[8]) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3]));
+  }
+};
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int n = 8;
+  __device__ static void unpack(const uint4& q, float (&f)[8]) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  __device__ static uint4 pack(const float (&f)[8]) {
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                      pack_bf16x2(f[6], f[7]));
+  }
+};
+
+// y_t = sum_{j<k} g_{t,j} * routed[map[t*k+j]] + sum_{s<S} shared[s*N + t], fp32
+// accumulation in exactly this order, one rounding.
+template <typename T>
+__global__ void __launch_bounds__(kMoveWarps * 32) combine_kernel(const uint4* __restrict__ routed,
+                                                                   const uint4* __restrict__ shared,
+                                                                   const int32_t* __restrict__ map,
+                                                                   const float* __restrict__ gates,
+                                                                   uint4* __restrict__ y, int N, int k, int S,
+                                                                   int vpr) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kMoveWarps + (threadIdx.x >> 5);
+  if (t >= N) return;
+  const int my_row = lane < k ? map[(size_t)t * k + lane] : 0;
+  const float my_g = (lane < k && gates) ? gates[(size_t)t * k + lane] : 1.0f;
+  int rows[kMaxK];
+  float gs[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {  // broadcast before the (possibly divergent) vector loop
+    rows[j] = __shfl_sync(0xffffffffu, my_row, j);
+    gs[j] = __shfl_sync(0xffffffffu, my_g, j);
+  }
+  for (int v = lane; v < vpr; v += 32) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    uint4 q[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (j < k) q[j] = ld_stream(routed + (size_t)rows[j] * vpr + v);
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j < k) {
+        float f[8];
+        Vec<T>::unpack(q[j], f);
+#pragma unroll
+        for (int i = 0; i < Vec<T>::n; ++i) acc[i] = fmaf(gs[j], f[i], acc[i]);
+      }
+    }
+    for (int s = 0; s < S; ++s) {
+      float f[8];
+      Vec<T>::unpack(ld_stream(shared + ((size_t)s * N + t) * vpr + v), f);
+#pragma unroll
+      for (int i = 0; i < Vec<T>::n; ++i) acc[i] += f[i];
+    }
+    y[(size_t)t * vpr + v] = Vec<T>::pack(acc);
+  }
+}
+
+static inline int elem_bytes(const moe_config& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
+static inline int vecs_per_row(const moe_config& c) { return c.d * elem_bytes(c) / 16; }
+static inline unsigned blocks_for(long long rows) { return (unsigned)((rows + kMoveWarps - 1) / kMoveWarps); }
+
+cudaError_t launch_permute(const moe_config& c, const moe_layout& L, const void* x, void* x_perm, cudaStream_t st) {
+  if (c.N == 0) return cudaSuccess;
+  scatter_token_rows<<<blocks_for(c.N), kMoveWarps * 32, 0, st>>>(
+      static_cast<const uint4*>(x), static_cast<uint4*>(x_perm), L.tok2row, c.N, c.k, vecs_per_row(c));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_staged(const moe_config& c, const moe_layout& L, const void* x, void* send_buf,
+                                  void* x_perm, cudaStream_t st) {
+  if (c.N == 0) return cudaSuccess;
+  const int vpr = vecs_per_row(c);
+  const int A = c.N * c.k;
+  // hop 1: each source buckets its rows by destination owner (send buffer)
+  scatter_token_rows<<<blocks_for(c.N), kMoveWarps * 32, 0, st>>>(
+      static_cast<const uint4*>(x), static_cast<uint4*>(send_buf), L.tok2send, c.N, c.k, vpr);
+  // hop 2: the transpose to the owners plus the expert-local order
+  move_rows<true><<<blocks_for(A), kMoveWarps * 32, 0, st>>>(static_cast<const uint4*>(send_buf),
+                                                             static_cast<uint4*>(x_perm), L.send2row, A, vpr);
+  return cudaGetLastError();
+}
+
+template <typename T>
+static void combine_launch(const moe_config& c, const uint4* routed, const uint4* shared, const int32_t* map,
+                           const float* gates, uint4* y, cudaStream_t st) {
+  combine_kernel<T><<<blocks_for(c.N), kMoveWarps * 32, 0, st>>>(routed, shared, map, gates, y, c.N, c.k,
+                                                                  c.n_shared, vecs_per_row(c));
+}
+
+cudaError_t launch_combine(const moe_config& c, const moe_layout& L, const void* out, const float* topk_w, void* y,
+                           cudaStream_t st) {
+  if (c.N == 0) return cudaSuccess;
+  const size_t A = (size_t)c.N * c.k;
+  const uint4* o = static_cast<const uint4*>(out);
+  const uint4* sh = o + A * vecs_per_row(c);
+  if (c.dtype == MOE_BF16)
+    combine_launch<__nv_bfloat16>(c, o, sh, L.tok2row, topk_w, static_cast<uint4*>(y), st);
+  else
+    combine_launch<float>(c, o, sh, L.tok2row, topk_w, static_cast<uint4*>(y), st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_staged(const moe_config& c, const moe_layout& L, const void* out, const float* topk_w,
+                                  void* ret_buf, void* y, cudaStream_t st) {
+  if (c.N == 0) return cudaSuccess;
+  const int vpr = vecs_per_row(c);
+  const int A = c.N * c.k;
+  const uint4* o = static_cast<const uint4*>(out);
+  // hop 1: owners return rows in send-slot order (reverse transpose): ret[s] = out[send2row[s]]
+  move_rows<false><<<blocks_for(A), kMoveWarps * 32, 0, st>>>(o, static_cast<uint4*>(ret_buf), L.send2row, A, vpr);
+  // hop 2: unpermute + weighted sum at the source through tok2send
+  const uint4* sh = o + (size_t)A * vpr;
+  if (c.dtype == MOE_BF16)
+    combine_launch<__nv_bfloat16>(c, static_cast<const uint4*>(ret_buf), sh, L.tok2send, topk_w,
+                                  static_cast<uint4*>(y), st);
+  else
+    combine_launch<float>(c, static_cast<const uint4*>(ret_buf), sh, L.tok2send, topk_w, static_cast<uint4*>(y),
+                          st);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,248 @@
+/*
+ * moe.h — C ABI of libmoe: one Mixture-of-Experts layer's token movement and expert
+ * compute on one NVIDIA B200 (sm_100a).
+ *
+ * The layer (router -> top-k -> dispatch layout -> permute -> grouped SwiGLU experts ->
+ * combine) follows these web pages, cited by title and section:
+ *   [EP-DeepEP] ep_deepep explainer (papers-3lj.pages.dev): §2 y_t = sum_{e in I_t}
+ *               g_{t,e} Expert_e(x_t) and n_e; §3 dispatch/combine; §5 interface: input
+ *               = token layout + routing info, output = an owner-local computable
+ *               layout, completion and buffer lifetime explicit; §6 the three maps.
+ *   [DSMoE]     "深入浅出 DeepSeek MoE：EP 与 FSDP 经典二次开发实战指南": naive 5-step
+ *               forward; EP as a distributed transpose; DeepEP dispatch -> handle ->
+ *               combine(handle) split (Automodel excerpt).
+ *   [DeepEP]    DeepEP notes (lizn-zn.github.io) §2-3: all-to-all transpose, counts first.
+ *   [WideEP]    "Wide EP：当 MoE Expert Parallel 横跨几十张 GPU": count matrix C_ij,
+ *               receive load R_r, group-limited routing, E_local placement.
+ *   [MoE-IV]    "MoE我们喜欢你（四）：DeepEP 与 GroupedGEMM 如何拆解通信和计算瓶颈" §4:
+ *               permute -> a2a -> grouped_gemm -> a2a -> unpermute_and_weighted_sum.
+ *
+ * Conventions for every call
+ *   - All array arguments are DEVICE pointers to row-major, contiguous memory, 16-byte
+ *     aligned, allocated and owned by the caller.  The library allocates nothing, keeps
+ *     no state between calls, and never synchronises with the host.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Host-detectable errors (bad sizes, NULL pointers, small workspace) return a
+ *     non-zero moe_status immediately and launch nothing.
+ *   - Device-detected errors (an expert id outside [0, E), a wait that timed out) are
+ *     written to *dev_status (an int32 the caller zeroes and reads after synchronising);
+ *     the first error wins.  dev_status may be NULL, in which case they go unreported.
+ *   - Sizes: A = N * k assignments, a = t * k + slot indexes them.  E % P == 0 unless an
+ *     explicit expert_owner table is given.  k <= 8, E <= 256 (E >= k), P <= 32,
+ *     n_groups <= 32 with E % n_groups == 0, topk_groups <= 8.
+ *     bf16: d % 8 == 0, I % 8 == 0.   f32: d % 4 == 0, I % 4 == 0.
+ *   - dtype applies to activations, weights and expert outputs; every reduction
+ *     accumulates in fp32.  Router logits and gate weights are fp32.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* NULL pointer, negative or inconsistent size */
+  MOE_ERR_UNSUPPORTED = 2, /* valid request outside the sizes this build supports */
+  MOE_ERR_WORKSPACE = 3,   /* workspace smaller than the matching *_workspace_bytes() */
+  MOE_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed (launch, tensor map) */
+  MOE_ERR_BAD_INDEX = 5,   /* device: an expert id outside [0, E) was seen */
+  MOE_ERR_TIMEOUT = 6      /* device: a bounded wait gave up */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score;
+
+/* Shape and routing rule of one layer. */
+typedef struct {
+  int32_t N;           /* tokens */
+  int32_t d;           /* hidden size */
+  int32_t E;           /* routed experts */
+  int32_t k;           /* experts per token (top-k) */
+  int32_t I;           /* expert intermediate size (SwiGLU) */
+  int32_t n_shared;    /* S: shared experts, always active, added with weight 1 */
+  int32_t P;           /* virtual expert-owner ranks (EP size) */
+  int32_t n_groups;    /* expert groups for group-limited routing; 1 = plain top-k */
+  int32_t topk_groups; /* groups kept per token (1 when n_groups == 1) */
+  int32_t score;       /* moe_score: softmax over E, or per-expert sigmoid */
+  int32_t renormalize; /* 1: gates renormalised to sum 1 over the chosen k */
+  int32_t dtype;       /* moe_dtype */
+} moe_config;
+
+/*
+ * The dispatch layout ("handle"): caller-owned device arrays, all int32.
+ *   n_e[E]          tokens per expert                         ([EP-DeepEP] §2)
+ *   expert_off[E+1] first row of expert e in the expert-contiguous buffer; experts are
+ *                   ordered by (owner, expert id); expert_off[E] = A
+ *   C[P*P]          C[i*P+j] = assignments from source rank i to owner j ([WideEP])
+ *   send_off[P*P]   start of block (i, j) in the send buffer (ordered by source, then owner)
+ *   recv_off[P+1]   start of owner j's rows; recv_off[j+1]-recv_off[j] = R_j = sum_i C_ij
+ *   tok2send[A]     assignment a -> send slot                 ([EP-DeepEP] §6, map 1)
+ *   send2row[A]     send slot -> expert-contiguous row         ([EP-DeepEP] §6, map 2)
+ *   ret2tok[A]      return row (= send slot of the combine all-to-all) -> assignment a
+ *                                                             ([EP-DeepEP] §6, map 3)
+ *   tok2row[A]      a -> row (= send2row[tok2send[a]])
+ *   row2tok[A]      row -> a (inverse of tok2row)
+ *   tile_off[E+S+1] prefix of ceil(rows/128) over routed experts (id order) then the S
+ *                   shared groups of N rows
+ * Source rank of token t is t / ceil(N/P).  Inside an expert, rows ascend in a.
+ */
+typedef struct {
+  int32_t* n_e;
+  int32_t* expert_off;
+  int32_t* C;
+  int32_t* send_off;
+  int32_t* recv_off;
+  int32_t* tok2send;
+  int32_t* send2row;
+  int32_t* ret2tok;
+  int32_t* tok2row;
+  int32_t* row2tok;
+  int32_t* tile_off;
+} moe_layout;
+
+/* Library version (major*10000 + minor*100 + patch) and a text for a status code. */
+int32_t moe_version(void);
+const char* moe_status_string(int32_t status);
+
+/* Host-side description of the last error returned on this thread ("" if none). */
+const char* moe_last_error(void);
+
+/* Validate a configuration on the host (the same checks every call makes). */
+moe_status moe_check_config(const moe_config* cfg);
+
+/* Bytes of scratch moe_dispatch_layout needs (ws argument). */
+size_t moe_layout_workspace_bytes(const moe_config* cfg);
+
+/* Bytes of scratch moe_layer_forward needs: logits, ids, gates, layout, layout scratch,
+ * permuted rows [A, d], SwiGLU activations [A+S*N, I] and expert outputs [A+S*N, d]. */
+size_t moe_workspace_bytes(const moe_config* cfg);
+
+/*
+ * Router and top-k selection ([DSMoE] naive forward steps 1-2; [EP-DeepEP] §2;
+ * [WideEP] "Group-limited routing"; renormalisation as named in [MoE-IV] §4.2).
+ *   x        [N, d]  dtype      w_gate [E, d] dtype (one row per expert)
+ *   bias     [E] fp32 or NULL   added to the logits before selection and gating
+ *   logits   [N, E] fp32, required: written with z = x W_g^T (+ b); the selection
+ *            reads back exactly these fp32 values
+ *   topk_ids [N, k] int32: slot 0 = largest logit; ties go to the lower expert index.
+ *            With n_groups > 1 a token first keeps the topk_groups groups with the
+ *            largest group max (ties to the lower group), then takes its top-k there.
+ *   topk_w   [N, k] fp32 gate weights:
+ *            softmax: exp(z_e - m) / sum_{all E} exp(z - m), or over the chosen k when
+ *            renormalize; sigmoid: 1/(1+exp(-z_e)), divided by their sum when renormalize.
+ */
+moe_status moe_route(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
+                     float* logits, int32_t* topk_ids, float* topk_w, moe_stream_t stream);
+
+/*
+ * Dispatch layout from the top-k ids ([EP-DeepEP] §3 and §6; [WideEP] C_ij, R_r;
+ * [DeepEP] §3 "counts first"; [DSMoE] VeOmni preprocess).  Pure integer work, bit-exact
+ * and deterministic; nothing is copied to the host.
+ *   expert_owner [E] int32 or NULL (NULL = owner e / (E/P)); each owner's experts keep
+ *                id order and its rows are contiguous
+ *   topk_ids     [N, k] int32, ids outside [0, E) set *dev_status = MOE_ERR_BAD_INDEX
+ *                and are treated as expert 0 (no out-of-bounds write happens)
+ *   out          the layout arrays (all must be non-NULL)
+ *   ws, ws_bytes scratch of at least moe_layout_workspace_bytes(cfg)
+ */
+moe_status moe_dispatch_layout(const moe_config* cfg, const int32_t* expert_owner, const int32_t* topk_ids,
+                               const moe_layout* out, int32_t* dev_status, void* ws, size_t ws_bytes,
+                               moe_stream_t stream);
+
+/*
+ * Permute ([MoE-IV] §4 permute_by_expert; [DSMoE] token_pre_all2all): the dispatch
+ * all-to-all and the expert sort composed into one gather, x_perm[tok2row[a]] = x[a/k].
+ * Each token row is read once and written k times.
+ *   x [N, d] dtype  ->  x_perm [A, d] dtype (expert-contiguous, owner-major)
+ */
+moe_status moe_permute(const moe_config* cfg, const moe_layout* layout, const void* x, void* x_perm,
+                       moe_stream_t stream);
+
+/*
+ * The same movement in two explicit hops, for inspection of the virtual all-to-all
+ * ([DeepEP] §2 transpose figure; [EP-DeepEP] §3): send_buf[tok2send[a]] = x[a/k]
+ * (each source buckets by owner), then x_perm[send2row[s]] = send_buf[s] (transpose to
+ * the owners and expert-local sort).  Bit-identical to moe_permute.
+ *   send_buf [A, d] dtype scratch owned by the caller.
+ */
+moe_status moe_permute_staged(const moe_config* cfg, const moe_layout* layout, const void* x, void* send_buf,
+                              void* x_perm, moe_stream_t stream);
+
+/*
+ * Grouped SwiGLU experts ([MoE-IV] §4.1 "FC1, activation, FC2"; [EP-DeepEP] §2
+ * Expert_e):  for each expert e with n_e > 0 and its rows X_e of x_perm,
+ *   H_e = SiLU(X_e W_gate_e^T) * (X_e W_up_e^T),   O_e = H_e W_down_e^T  (x gate if topk_w)
+ * and for each shared expert s the same over all N rows of x.
+ *   x_perm [A, d], x [N, d] (read only when n_shared > 0)
+ *   w13 [E+S, 2I, d]: rows [0, I) = W_gate, rows [I, 2I) = W_up; shared experts last
+ *   w2  [E+S, d, I]
+ *   topk_w [N, k] fp32 or NULL: when given, routed output row r is scaled by
+ *          topk_w[row2tok[r]] before rounding (the combine's gate, applied here)
+ *   h_ws [A + S*N, I] dtype scratch (the SwiGLU activations)
+ *   out  [A + S*N, d] dtype: routed rows [0, A) in expert-contiguous order, then shared
+ *        expert s's N rows at A + s*N, in token order
+ * Each routed row's numbers depend only on that row and its expert: rows past an
+ * expert's end are computed in no other expert's tile result.
+ */
+moe_status moe_grouped_ffn(const moe_config* cfg, const moe_layout* layout, const void* x_perm, const void* x,
+                           const void* w13, const void* w2, const float* topk_w, void* h_ws, void* out,
+                           moe_stream_t stream);
+
+/*
+ * The two halves of moe_grouped_ffn, for callers that schedule them separately:
+ *   moe_expert_fc1: h_ws = SiLU(X W_gate^T) * (X W_up^T) for every group (routed rows of
+ *                   x_perm, then each shared expert over the N rows of x)
+ *   moe_expert_fc2: out = (h_ws W_down^T), routed rows scaled by topk_w[row2tok[r]] when
+ *                   topk_w is non-NULL
+ * Shapes, layouts and errors as for moe_grouped_ffn.
+ */
+moe_status moe_expert_fc1(const moe_config* cfg, const moe_layout* layout, const void* x_perm, const void* x,
+                          const void* w13, void* h_ws, moe_stream_t stream);
+moe_status moe_expert_fc2(const moe_config* cfg, const moe_layout* layout, const void* h_ws, const void* w2,
+                          const float* topk_w, void* out, moe_stream_t stream);
+
+/*
+ * Combine ([EP-DeepEP] §2-3; [DSMoE] combine = gate-weighted sum at the source;
+ * [MoE-IV] §4 unpermute_and_weighted_sum): the combine all-to-all composed with the
+ * unpermute and the weighted sum,
+ *   y_t = sum_{slot<k} g_{t,slot} * out[tok2row[t*k+slot]] + sum_{s<S} out[A + s*N + t]
+ * accumulated in fp32 in that fixed order and rounded once to dtype.
+ *   topk_w [N, k] fp32, or NULL when moe_grouped_ffn already applied the gates
+ *   y [N, d] dtype, token order
+ */
+moe_status moe_combine(const moe_config* cfg, const moe_layout* layout, const void* out, const float* topk_w,
+                       void* y, moe_stream_t stream);
+
+/*
+ * The combine in two explicit hops: ret_buf[s] = out[send2row[s]] (reverse transpose,
+ * the owners send rows back in send-slot order), then
+ * y_t = sum_slot g * ret_buf[tok2send[t*k+slot]] + shared rows.  Bit-identical to
+ * moe_combine.   ret_buf [A, d] dtype scratch owned by the caller.
+ */
+moe_status moe_combine_staged(const moe_config* cfg, const moe_layout* layout, const void* out,
+                              const float* topk_w, void* ret_buf, void* y, moe_stream_t stream);
+
+/*
+ * The whole layer on one stream: moe_route -> moe_dispatch_layout -> moe_permute ->
+ * moe_grouped_ffn (gates applied in the down-projection epilogue) -> moe_combine.
+ * No host synchronisation, no allocation; capturable in a CUDA graph.
+ *   layout_out  NULL, or caller arrays that receive the layout (otherwise it lives in ws)
+ *   ws          at least moe_workspace_bytes(cfg) bytes, 256-byte aligned
+ */
+moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
+                             const int32_t* expert_owner, const void* w13, const void* w2, void* y,
+                             const moe_layout* layout_out, int32_t* dev_status, void* ws, size_t ws_bytes,
+                             moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -10,4 +10,11 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
-    config.addinivalue_line("markers", "slow: long-running CPU test")
+    # the C ABI library is built in-tree from source (nvcc cross-compiles without a GPU)
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_moe_build", os.path.join(ROOT, "dispatch_combine_grouped_b200", "build.py"))
+    _build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(_build)
+    if not _build.up_to_date():
+        _build.build()
