@@ -74,50 +74,66 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    """Reads the SM clock and the clock-event (throttle) reasons through NVML every 2 ms
+    in a background thread while the timed steps run (reading only; no setting is
+    changed)."""
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+               "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
+
+    def __init__(self, device_index):
+        import threading
+        self.samples = []
+        self.stop_ev = threading.Event()
+        self.thread = None
+        self.nvml = None
+        try:
+            import pynvml as nv
+            import torch
+            nv.nvmlInit()
+            pr = torch.cuda.get_device_properties(device_index)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            self.h = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.nvml = nv
+        except Exception:
+            self.nvml = None
+
+    def _run(self):
+        nv = self.nvml
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)))
+            except Exception:
+                pass
+            self.stop_ev.wait(0.002)
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.proc = None
+        if self.nvml is None:
+            return
+        import threading
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.nvml is None or self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=10)
-        except Exception:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
+        self.stop_ev.set()
+        self.thread.join()
+        if not self.samples:
             return None
-        sm.sort()
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(mx), "reasons": sorted(reasons), "samples": len(sm)}
+        sm = sorted(x for x, _ in self.samples)
+        reasons = set()
+        for _, bits in self.samples:
+            for name, const in self.REASONS.items():
+                if hasattr(self.nvml, const) and bits & getattr(self.nvml, const):
+                    reasons.add(name)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.max_mhz, "sm_min_mhz": sm[0],
+                "reasons": sorted(reasons), "samples": len(sm), "source": "NVML, every 2 ms, warm-up + timed steps"}
 
 
 def source_hash(*files):
@@ -252,24 +268,26 @@ def main():
     def new_events():
         return [torch.cuda.Event(enable_timing=True) for _ in range(7)]
 
+    clocks = ClockSampler(local)
+    evs = [new_events() for _ in range(args.steps)]
+    clocks.start()
+    torch.cuda.nvtx.range_push("warmup")
     for _ in range(args.warmup):
         flush.zero_()
         step(new_events())
     torch.cuda.synchronize()
-
-    clocks = ClockSampler(local)
-    evs = [new_events() for _ in range(args.steps)]
+    torch.cuda.nvtx.range_pop()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
+    torch.cuda.nvtx.range_push("timed")
     wall0 = time.perf_counter()
     for i in range(args.steps):
         flush.zero_()
         step(evs[i])
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
+    torch.cuda.nvtx.range_pop()
     if world > 1:
         dist.barrier()
     clock_rec = clocks.stop()
