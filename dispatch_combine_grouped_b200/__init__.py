@@ -5,7 +5,7 @@ The compute lives in libmoe.so (C ABI in include/moe.h); this package is its Pyt
 binding.  Importing it loads the library and fails loudly when it is missing.
 """
 from .binding import (EXPORTED, Layout, MoEError, alloc_workspace, c_config, check_config, combine,  # noqa: F401
-                      combine_staged, dispatch_layout, expert_fc1, expert_fc2, grouped_ffn, layer_forward, layout_workspace_bytes,
+                      combine_staged, dispatch_layout, dispatch_layout_noalloc, expert_fc1, expert_fc2, grouped_ffn, layer_forward, layout_workspace_bytes,
                       load, permute, permute_staged, route, version, workspace_bytes)
 
 load()

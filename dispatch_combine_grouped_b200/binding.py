@@ -24,6 +24,7 @@ MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
 # every symbol include/moe.h declares
 EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_config",
             "moe_layout_workspace_bytes", "moe_workspace_bytes", "moe_route", "moe_dispatch_layout",
+            "moe_dispatch_layout_noalloc",
             "moe_permute", "moe_permute_staged", "moe_grouped_ffn", "moe_expert_fc1", "moe_expert_fc2",
             "moe_combine", "moe_combine_staged",
             "moe_layer_forward"]
@@ -71,6 +72,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_workspace_bytes": (sz, [cfgp]),
         "moe_route": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_dispatch_layout": (i32, [cfgp, vp, vp, layp, vp, vp, sz, vp]),
+        "moe_dispatch_layout_noalloc": (i32, [cfgp, vp, vp, layp, vp, vp]),
         "moe_permute": (i32, [cfgp, layp, vp, vp, vp]),
         "moe_permute_staged": (i32, [cfgp, layp, vp, vp, vp, vp]),
         "moe_grouped_ffn": (i32, [cfgp, layp, vp, vp, vp, vp, vp, vp, vp, vp]),
@@ -183,6 +185,17 @@ def dispatch_layout(cfg, topk_ids, expert_owner=None, status=None, layout=None, 
         ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=topk_ids.device)
     _check(lib.moe_dispatch_layout(ctypes.byref(c), _p(expert_owner), _p(topk_ids), ctypes.byref(layout.c),
                                    _p(status), _p(ws), ws.numel(), _stream()), "moe_dispatch_layout")
+    return layout
+
+
+def dispatch_layout_noalloc(cfg, topk_ids, expert_owner=None, status=None, layout=None):
+    """moe_dispatch_layout_noalloc: the layout with the library's built-in scratch (no
+    workspace argument; for callers that cannot allocate device memory)."""
+    c = c_config(cfg)
+    layout = layout or Layout(cfg, topk_ids.device)
+    _check(load().moe_dispatch_layout_noalloc(ctypes.byref(c), _p(expert_owner), _p(topk_ids),
+                                              ctypes.byref(layout.c), _p(status), _stream()),
+           "moe_dispatch_layout_noalloc")
     return layout
 
 

@@ -157,6 +157,29 @@ moe_status moe_dispatch_layout(const moe_config* cfg, const int32_t* expert_owne
                                moe_stream_t stream);
 
 /*
+ * moe_dispatch_layout for callers that cannot allocate GPU memory (no counterpart in
+ * the pages: it exists for deployment, not for the method).  A plugin inside a runtime
+ * that owns all device buffers, a serving loop that must not call cudaMalloc (which
+ * synchronises the device), or a service with a memory budget fixed at start-up may
+ * have no workspace to pass.  This call computes exactly what moe_dispatch_layout
+ * computes, with the same kernels, but takes no ws argument: the scratch is a 2 MiB
+ * array compiled into the library, which every GPU that loads the library holds until
+ * the process exits.  It allocates nothing and calls no allocating routine.
+ *   Limit: moe_layout_workspace_bytes(cfg) <= 2 MiB (about N*k <= 131072 assignments
+ *          with E <= 256, P <= 32); larger configurations return MOE_ERR_UNSUPPORTED.
+ *   Set-up: the first call on each device looks up the array's device address
+ *          (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *          first call before any stream capture.
+ *   Sharing: all calls on a device use the same array, so calls that overlap on the GPU
+ *          (different streams, or different host threads) race and corrupt each other's
+ *          results; serialise them.  Contents left by an earlier call are harmless:
+ *          every scratch word is written before it is read within a call.
+ * Arguments, layout and device-side errors are those of moe_dispatch_layout.
+ */
+moe_status moe_dispatch_layout_noalloc(const moe_config* cfg, const int32_t* expert_owner, const int32_t* topk_ids,
+                                       const moe_layout* out, int32_t* dev_status, moe_stream_t stream);
+
+/*
  * Permute ([MoE-IV] §4 permute_by_expert; [DSMoE] token_pre_all2all): the dispatch
  * all-to-all and the expert sort composed into one gather, x_perm[tok2row[a]] = x[a/k].
  * Each token row is read once and written k times.
