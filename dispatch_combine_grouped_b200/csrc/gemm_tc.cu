@@ -129,6 +129,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       orow = p.A_routed + s * p.N;
       arow = p.shared_from_map1 ? 0 : orow;
     }
+    if (p.tail_only) {  // the pair kernel covers the first pair_rows(rows) rows
+      const int pr = pair_rows(rows);
+      rows = rows > pr ? rows - pr : 0;
+      arow += pr;
+      orow += pr;
+    }
     s_rows[g] = rows;
     s_arow[g] = arow;
     s_orow[g] = orow;
@@ -394,7 +400,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 // 2D bf16 map over [rows, K] (K contiguous), box [128 rows, 64 cols], 128B swizzle.
-static bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K) {
+bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)(rows > 0 ? rows : 1)};
@@ -407,7 +413,7 @@ static bool make_map_a(CUtensorMap* m, const void* base, long long rows, long lo
 }
 
 // 3D bf16 map over [G, R, K], box [1, box_rows, 64], 128B swizzle.
-static bool make_map_b(CUtensorMap* m, const void* base, long long G, long long R, long long K, int box_rows) {
+bool make_map_b(CUtensorMap* m, const void* base, long long G, long long R, long long K, int box_rows) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)R, (cuuint64_t)G};
@@ -457,7 +463,7 @@ cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStre
   CUtensorMap a0, a1, b;
   if (!make_map_a(&a0, g.a0, a0_rows, g.K)) return cudaErrorInvalidValue;
   if (!make_map_a(&a1, g.a1 ? g.a1 : g.a0, g.a1 ? a1_rows : a0_rows, g.K)) return cudaErrorInvalidValue;
-  if (!make_map_b(&b, g.b, g.G - 0 * g.E, g.b_rows, g.K, BN / 2)) return cudaErrorInvalidValue;
+  if (!make_map_b(&b, g.b, g.G, g.b_rows, g.K, BN / 2)) return cudaErrorInvalidValue;
   // upper bound on tiles: every group adds at most one partial row block
   long long rows_total = (long long)g.A_routed + (long long)(g.G - g.E) * g.N;
   long long blocks = (rows_total + BM - 1) / BM + g.G;

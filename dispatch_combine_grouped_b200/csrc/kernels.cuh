@@ -53,6 +53,7 @@ struct GemmArgs {
   int n_out;         // valid output columns (E, I or d)
   int I;             // FC1: row offset of W_up inside W13
   int shared_from_map1;
+  int tail_only;        // 1-CTA kernel: only the rows left after the 256-row pair tiles
   const int32_t* n_e;
   const int32_t* expert_off;
   const int32_t* row2tok;
@@ -68,11 +69,15 @@ struct GemmArgs {
   long long b_rows;     // rows of one weight matrix (2I, d or E)
 };
 
-// tensor-core (tcgen05) path, bf16 operands, fp32 accumulation
+// tensor-core (tcgen05) path, bf16 operands, fp32 accumulation: one CTA per tile
 cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStream_t st);
+// the same over CTA pairs (cta_group::2, 256 x 256 tiles) for the rows pair_rows() covers
+cudaError_t launch_tc_gemm_pair(const GemmArgs& g, int a0_rows, int a1_rows, cudaStream_t st);
 // CUDA-core path, fp32 operands (the fp32 configurations)
 cudaError_t launch_simt_gemm(const GemmArgs& g, cudaStream_t st);
 
 int sm_count();
+bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K);
+bool make_map_b(CUtensorMap* m, const void* base, long long G, long long R, long long K, int box_rows);
 
 }  // namespace moe

@@ -24,6 +24,20 @@ def assert_close_fro(got, ref, max_abs=MAX_ABS, rel_fro=REL_FRO, what=""):
     return float(err.max()), float(fro)
 
 
+def assert_close_rel(got, ref, rel=1e-2, rel_fro=REL_FRO, what=""):
+    """For bf16 intermediates of any magnitude: |err| <= rel * max(|ref|, 1) elementwise
+    (bf16 keeps 8 significant bits: rounding alone is up to 2^-9 of the value) and the
+    relative Frobenius error bound."""
+    got = O.f64(got)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), what
+    worst = (np.abs(got - ref) / np.maximum(np.abs(ref), 1.0)).max()
+    fro = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert worst <= rel, f"{what}: scaled err {worst:.3e} > {rel}"
+    assert fro <= rel_fro, f"{what}: rel Frobenius err {fro:.3e} > {rel_fro}"
+
+
 def layout_to_numpy(layout):
     return {k: v.cpu().numpy().astype(np.int64) for k, v in layout.as_dict().items()}
 

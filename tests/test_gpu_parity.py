@@ -14,8 +14,8 @@ import torch
 import dispatch_combine_grouped_b200 as moe
 from moe_inputs import CONFIGS, MoEConfig, small_config
 from oracle import moe_oracle as O
-from tests.gpu_cases import (assert_close_fro, assert_layout_equal, check_route, gpu_inputs, layout_to_numpy,
-                             run_steps)
+from tests.gpu_cases import (assert_close_fro, assert_close_rel, assert_layout_equal, check_route, gpu_inputs,
+                             layout_to_numpy, run_steps)
 
 pytestmark = pytest.mark.gpu
 
@@ -29,6 +29,7 @@ SMALL = [
     small_config("s_bf16_grouped", cfg_id=72, N=190, d=192, E=32, S=1, k=4, I=128, P=8, n_groups=8,
                  topk_groups=3, score="sigmoid"),
     small_config("s_bf16_tiny_n", cfg_id=73, N=7, d=64, E=8, S=0, k=2, I=64, P=2),
+    small_config("s_bf16_pairs", cfg_id=79, N=700, d=4096, E=8, S=1, k=2, I=200, P=4),
     small_config("s_bf16_one_tok", cfg_id=74, N=1, d=128, E=64, S=1, k=6, I=96, P=8),
     small_config("s_f32", cfg_id=75, N=129, d=96, E=8, S=1, k=2, I=72, P=4, dtype="f32"),
     small_config("s_f32_grouped", cfg_id=76, N=64, d=64, E=16, S=0, k=4, I=40, P=4, n_groups=4, topk_groups=2,
@@ -183,3 +184,54 @@ def test_empty_batch():
     torch.cuda.synchronize()
     assert lay["n_e"].sum().item() == 0 and lay["C"].sum().item() == 0
     assert lay["expert_off"].tolist() == [0] * 9
+
+
+def _ids_with_counts(counts, N, k, seed):
+    """Distinct experts per token with exact per-expert counts (greedy by remaining count)."""
+    rem = list(counts)
+    rows = []
+    for _ in range(N):
+        order = sorted(range(len(rem)), key=lambda e: (-rem[e], e))[:k]
+        for e in order:
+            rem[e] -= 1
+        rows.append(order)
+    assert all(r == 0 for r in rem)
+    ids = np.array(rows)
+    rng = np.random.default_rng(seed)
+    ids = ids[rng.permutation(N)]
+    for t in range(N):  # random slot order inside each token
+        ids[t] = ids[t][rng.permutation(k)]
+    return ids
+
+
+def test_ffn_pair_and_tail_row_splits():
+    """Groups of 256 (one pair tile), 300 (pair + 44-row tail), 400 (two pair tiles,
+    the second 144/256 full), 128 and 95 (tails only), 1, 0 rows, plus a shared expert of
+    640 rows (512 in pairs + a 128-row tail).  d = 4096 selects the CTA-pair kernel."""
+    counts = [256, 300, 400, 128, 1, 0, 95, 100]
+    cfg = small_config("splits", cfg_id=78, N=640, d=4096, E=8, S=1, k=2, I=192, P=4)
+    inp = gpu_inputs(cfg)
+    ids = _ids_with_counts(counts, cfg.N, cfg.k, 3)
+    ids_t = torch.tensor(ids, dtype=torch.int32, device="cuda")
+    gates = torch.rand(cfg.N, cfg.k, generator=torch.Generator().manual_seed(5)).float().cuda()
+    lay = moe.dispatch_layout(cfg, ids_t)
+    xp = moe.permute(cfg, lay, inp["x"])
+    h, out = moe.grouped_ffn(cfg, lay, xp, inp["x"], inp["w13"], inp["w2"], topk_w=gates)
+    torch.cuda.synchronize()
+    ref = O.dispatch_layout(ids, cfg.E, cfg.P, None, cfg.S)
+    assert layout_to_numpy(lay)["n_e"].tolist() == counts
+    o_ref = O.experts_on_rows(O.permute(inp["x"], ref, cfg.k), ref, inp["w13"], inp["w2"], cfg.E)
+    g_row = O.f64(gates).reshape(-1)[ref["row2tok"]]
+    A = cfg.N * cfg.k
+    assert_close_fro(out[:A], o_ref * g_row[:, None], what="routed rows")
+    shared = O.swiglu_expert(inp["x"], inp["w13"][cfg.E], inp["w2"][cfg.E])
+    assert_close_fro(out[A:], shared, what="shared rows")
+    # h (FC1 output) against the float64 SwiGLU activations, for every routed row
+    xp64 = O.permute(inp["x"], ref, cfg.k)
+    for e in range(cfg.E):
+        n, r0 = ref["n_e"][e], ref["expert_off"][e]
+        if n == 0:
+            continue
+        w13 = O.f64(inp["w13"][e])
+        hh = O.silu(xp64[r0:r0 + n] @ w13[:cfg.I].T) * (xp64[r0:r0 + n] @ w13[cfg.I:].T)
+        assert_close_rel(h[r0:r0 + n], hh, what=f"h expert {e}")
