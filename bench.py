@@ -25,7 +25,6 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s; grouped-GEMM TFLOP/s and permute/combine GB/s vs peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 9  # router GEMM, top-k, 3 layout, permute, FC1, FC2, combine
 
 
 def parse():
@@ -250,7 +249,38 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     x, wg, bias, owner, w13, w2 = inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], inp["w13"], inp["w2"]
 
+    side = torch.cuda.Stream(device=dev)
+    main = torch.cuda.current_stream(dev)
+
     def step(ev):
+        """One layer pass as the product runs it (moe_layer_forward_overlapped's order):
+        router; then the shared experts on a side stream while layout, permute and the
+        routed experts run on the main stream; join; combine."""
+        ev[0].record()
+        moe.route(cfg, x, wg, bias, out=(logits, ids, w))
+        ev[1].record()
+        if S:
+            fork, join = torch.cuda.Event(), torch.cuda.Event()
+            fork.record(main)
+            side.wait_event(fork)
+            moe.expert_fc1(cfg, None, None, x, w13, h=h, groups="shared", stream=side)
+            moe.expert_fc2(cfg, None, h, w2, out=out, groups="shared", stream=side)
+            join.record(side)
+        moe.dispatch_layout(cfg, ids, owner, status=status, layout=layout, ws=lay_ws)
+        ev[2].record()
+        moe.permute(cfg, layout, x, out=x_perm)
+        ev[3].record()
+        moe.expert_fc1(cfg, layout, x_perm, x, w13, h=h, groups="routed")
+        ev[4].record()
+        moe.expert_fc2(cfg, layout, h, w2, topk_w=w, out=out, groups="routed")
+        ev[5].record()
+        if S:
+            main.wait_event(join)
+        moe.combine(cfg, layout, out, y=y)
+        ev[6].record()
+
+    def step_sequential(ev):
+        """The same kernels one after another on one stream (diagnostic breakdown)."""
         ev[0].record()
         moe.route(cfg, x, wg, bias, out=(logits, ids, w))
         ev[1].record()
@@ -307,12 +337,21 @@ def main():
     for n in names:
         stage_ms[n] /= args.steps
 
-    # fused entry point (same kernels, one C call per step), for reference
+    # diagnostic: the same kernels one after another on one stream (per-stage breakdown)
+    seq_evs = [new_events() for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        step_sequential(seq_evs[i])
+    torch.cuda.synchronize()
+    seq_ms = {n: sum(ev[j].elapsed_time(ev[j + 1]) for ev in seq_evs) / args.steps for j, n in enumerate(names)}
+    seq_step_ms = sum(ev[0].elapsed_time(ev[6]) for ev in seq_evs) / args.steps
+
+    # the fused entry point (one C call per step, same kernels and order as the timed step)
     fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for i in range(args.steps):
         flush.zero_()
         fev[i][0].record()
-        moe.layer_forward(cfg, x, wg, bias, owner, w13, w2, y=y, ws=ws, status=status)
+        moe.layer_forward_overlapped(cfg, x, wg, bias, owner, w13, w2, side, y=y, ws=ws, status=status)
         fev[i][1].record()
     torch.cuda.synchronize()
     fused_ms = sum(a.elapsed_time(b) for a, b in fev) / args.steps
@@ -326,7 +365,7 @@ def main():
         flush.zero_()
         e2e_ev[i][0].record()
         x_dev.copy_(x_host, non_blocking=True)
-        moe.layer_forward(cfg, x_dev, wg, bias, owner, w13, w2, y=y, ws=ws, status=status)
+        moe.layer_forward_overlapped(cfg, x_dev, wg, bias, owner, w13, w2, side, y=y, ws=ws, status=status)
         y_host.copy_(y, non_blocking=True)
         e2e_ev[i][1].record()
     torch.cuda.synchronize()
@@ -340,15 +379,20 @@ def main():
     touched = int((n_e > 0).sum())
     alg = algorithmic(cfg, touched)
     peaks, peak_src = load_peaks()
-    fc1_s = stage_ms["fc1"] / 1e3
-    fc1_tflops = alg["fc1_flops"] / fc1_s / 1e12
-    ffn_tflops = alg["ffn_flops"] / ((stage_ms["fc1"] + stage_ms["fc2"]) / 1e3) / 1e12
+    A_rows = cfg.N * cfg.k
+    routed_fc1_flops = 4.0 * A_rows * cfg.d * cfg.I
+    routed_ffn_flops = 6.0 * A_rows * cfg.d * cfg.I
+    fc1_tflops = routed_fc1_flops / (stage_ms["fc1"] / 1e3) / 1e12
+    ffn_seq_tflops = alg["ffn_flops"] / ((seq_ms["fc1"] + seq_ms["fc2"]) / 1e3) / 1e12
     permute_gbs = alg["permute_bytes"] / (stage_ms["permute"] / 1e3) / 1e9
-    combine_gbs = alg["combine_bytes"] / (stage_ms["combine"] / 1e3) / 1e9
-    src = source_hash("dispatch_combine_grouped_b200/csrc/gemm_tc.cu", "dispatch_combine_grouped_b200/csrc/common.cuh")
-    traffic = recorded_traffic("fc1", cfg.name, src)
+    combine_gbs = alg["combine_bytes"] / (seq_ms["combine"] / 1e3) / 1e9
+    src = source_hash("dispatch_combine_grouped_b200/csrc/gemm_tc.cu", "dispatch_combine_grouped_b200/csrc/gemm_tc2.cu",
+                      "dispatch_combine_grouped_b200/csrc/common.cuh")
+    traffic = recorded_traffic("fc1_routed", cfg.name, src)
     tokens_total = cfg.N * world
     value = tokens_total / (step_ms_max / 1e3)
+    gl = 2 if (cfg.dtype == "bf16" and cfg.N > 128 and cfg.d >= 4096) else 1   # pair + tail launches
+    launches_per_step = 2 + 3 + 1 + 2 * gl + (2 * gl if S else 0) + 1
 
     if rank == 0:
         line = {
@@ -358,12 +402,16 @@ def main():
             "config": {"workload": describe(cfg), "tokens_per_gpu": cfg.N, "l2": "flushed before every step "
                        "(256 MiB write, outside the step's event bracket)", "parallelism": f"{world} independent "
                        "replicas (one batch per GPU)"},
-            "roofline": {"kernel": "grouped FC1 + SwiGLU (tcgen05)", "bound": "tensor", "achieved": fc1_tflops,
-                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": fc1_tflops / peaks["bf16_tflops"],
-                         "peak_source": f"{peak_src} bf16 burst", "traffic": traffic,
-                         "flops_per_launch": alg["fc1_flops"], "ms_per_launch": stage_ms["fc1"]},
+            "roofline": {"kernel": "routed grouped FC1 + SwiGLU (tcgen05)", "bound": "tensor",
+                         "achieved": fc1_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": fc1_tflops / peaks["bf16_tflops"], "peak_source": f"{peak_src} bf16 burst",
+                         "traffic": traffic, "flops_per_launch": routed_fc1_flops, "ms_per_launch": stage_ms["fc1"],
+                         "note": "timed inside the step, with the shared experts running on a side stream"},
             "stages_ms": stage_ms,
-            "ffn": {"tflops": ffn_tflops, "frac_of_peak": ffn_tflops / peaks["bf16_tflops"]},
+            "sequential": {"ms_per_step": seq_step_ms, "stages_ms": seq_ms,
+                           "ffn_tflops": ffn_seq_tflops, "ffn_frac_of_peak": ffn_seq_tflops / peaks["bf16_tflops"]},
+            "ffn": {"tflops": ffn_seq_tflops, "frac_of_peak": ffn_seq_tflops / peaks["bf16_tflops"],
+                    "routed_tflops_overlapped": routed_ffn_flops / ((stage_ms["fc1"] + stage_ms["fc2"]) / 1e3) / 1e12},
             "permute": {"gbs": permute_gbs, "frac_of_hbm": permute_gbs / peaks["hbm_gbs"],
                         "frac_of_8tbs": permute_gbs / 8000.0},
             "combine": {"gbs": combine_gbs, "frac_of_hbm": combine_gbs / peaks["hbm_gbs"],
@@ -374,7 +422,7 @@ def main():
             "e2e": {"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": x.numel() * x.element_size(),
                     "d2h_bytes_per_step": y.numel() * y.element_size()},
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "gpu_launches": launches_per_step * args.steps,
             "clocks": clock_rec,
             "wall_s_timed": wall,
         }

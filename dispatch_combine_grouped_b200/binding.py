@@ -20,12 +20,14 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUD
     MOE_ERR_TIMEOUT = range(7)
 MOE_F32, MOE_BF16 = 0, 1
 MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
+GROUPS = {"all": 0, "routed": 1, "shared": 2}
 
 # every symbol include/moe.h declares
 EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_config",
             "moe_layout_workspace_bytes", "moe_workspace_bytes", "moe_route", "moe_dispatch_layout",
             "moe_dispatch_layout_noalloc",
             "moe_permute", "moe_permute_staged", "moe_grouped_ffn", "moe_expert_fc1", "moe_expert_fc2",
+            "moe_routed_ffn", "moe_shared_ffn", "moe_layer_forward_overlapped",
             "moe_combine", "moe_combine_staged",
             "moe_layer_forward"]
 
@@ -76,8 +78,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_permute": (i32, [cfgp, layp, vp, vp, vp]),
         "moe_permute_staged": (i32, [cfgp, layp, vp, vp, vp, vp]),
         "moe_grouped_ffn": (i32, [cfgp, layp, vp, vp, vp, vp, vp, vp, vp, vp]),
-        "moe_expert_fc1": (i32, [cfgp, layp, vp, vp, vp, vp, vp]),
-        "moe_expert_fc2": (i32, [cfgp, layp, vp, vp, vp, vp, vp]),
+        "moe_expert_fc1": (i32, [cfgp, layp, vp, vp, vp, vp, i32, vp]),
+        "moe_expert_fc2": (i32, [cfgp, layp, vp, vp, vp, vp, i32, vp]),
+        "moe_routed_ffn": (i32, [cfgp, layp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_shared_ffn": (i32, [cfgp, vp, vp, vp, vp, vp, vp]),
+        "moe_layer_forward_overlapped": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp, vp]),
         "moe_combine": (i32, [cfgp, layp, vp, vp, vp, vp]),
         "moe_combine_staged": (i32, [cfgp, layp, vp, vp, vp, vp, vp]),
         "moe_layer_forward": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp]),
@@ -231,22 +236,47 @@ def grouped_ffn(cfg, layout, x_perm, x, w13, w2, topk_w=None, h=None, out=None):
     return h, out
 
 
-def expert_fc1(cfg, layout, x_perm, x, w13, h=None):
+def expert_fc1(cfg, layout, x_perm, x, w13, h=None, groups="all", stream=None):
     c = c_config(cfg)
     if h is None:
-        h = torch.empty(cfg.N * cfg.k + cfg.S * cfg.N, cfg.I, dtype=_dtype(cfg), device=x_perm.device)
-    _check(load().moe_expert_fc1(ctypes.byref(c), ctypes.byref(layout.c), _p(x_perm), _p(x), _p(w13), _p(h),
-                                 _stream()), "moe_expert_fc1")
+        dev = (x_perm if x_perm is not None else x).device
+        h = torch.empty(cfg.N * cfg.k + cfg.S * cfg.N, cfg.I, dtype=_dtype(cfg), device=dev)
+    st = ctypes.c_void_p(stream.cuda_stream) if stream is not None else _stream()
+    lay = ctypes.byref(layout.c) if layout is not None else None
+    _check(load().moe_expert_fc1(ctypes.byref(c), lay, _p(x_perm), _p(x), _p(w13), _p(h), GROUPS[groups], st),
+           "moe_expert_fc1")
     return h
 
 
-def expert_fc2(cfg, layout, h, w2, topk_w=None, out=None):
+def expert_fc2(cfg, layout, h, w2, topk_w=None, out=None, groups="all", stream=None):
     c = c_config(cfg)
     if out is None:
         out = torch.empty(cfg.N * cfg.k + cfg.S * cfg.N, cfg.d, dtype=_dtype(cfg), device=h.device)
-    _check(load().moe_expert_fc2(ctypes.byref(c), ctypes.byref(layout.c), _p(h), _p(w2), _p(topk_w), _p(out),
-                                 _stream()), "moe_expert_fc2")
+    st = ctypes.c_void_p(stream.cuda_stream) if stream is not None else _stream()
+    lay = ctypes.byref(layout.c) if layout is not None else None
+    _check(load().moe_expert_fc2(ctypes.byref(c), lay, _p(h), _p(w2), _p(topk_w), _p(out), GROUPS[groups], st),
+           "moe_expert_fc2")
     return out
+
+
+def routed_ffn(cfg, layout, x_perm, w13, w2, topk_w=None, h=None, out=None):
+    c = c_config(cfg)
+    rows = cfg.N * cfg.k + cfg.S * cfg.N
+    if h is None:
+        h = torch.empty(rows, cfg.I, dtype=_dtype(cfg), device=x_perm.device)
+    if out is None:
+        out = torch.empty(rows, cfg.d, dtype=_dtype(cfg), device=x_perm.device)
+    _check(load().moe_routed_ffn(ctypes.byref(c), ctypes.byref(layout.c), _p(x_perm), _p(w13), _p(w2), _p(topk_w),
+                                 _p(h), _p(out), _stream()), "moe_routed_ffn")
+    return h, out
+
+
+def shared_ffn(cfg, x, w13, w2, h, out, stream=None):
+    """Shared experts into rows [A, A+S*N) of h and out, on ``stream`` (default: current)."""
+    c = c_config(cfg)
+    st = ctypes.c_void_p(stream.cuda_stream) if stream is not None else _stream()
+    _check(load().moe_shared_ffn(ctypes.byref(c), _p(x), _p(w13), _p(w2), _p(h), _p(out), st), "moe_shared_ffn")
+    return h, out
 
 
 def combine(cfg, layout, out_rows, topk_w=None, y=None):
@@ -269,6 +299,22 @@ def combine_staged(cfg, layout, out_rows, topk_w=None):
 
 def alloc_workspace(cfg, device="cuda"):
     return torch.empty(max(workspace_bytes(cfg), 1), dtype=torch.uint8, device=device)
+
+
+def layer_forward_overlapped(cfg, x, w_gate, bias, expert_owner, w13, w2, side_stream, y=None, ws=None, layout=None,
+                             status=None):
+    """moe_layer_forward_overlapped: shared experts on ``side_stream`` (a torch.cuda.Stream)."""
+    c = c_config(cfg)
+    if ws is None:
+        ws = alloc_workspace(cfg, x.device)
+    if y is None:
+        y = torch.empty(cfg.N, cfg.d, dtype=x.dtype, device=x.device)
+    lay = ctypes.byref(layout.c) if layout is not None else None
+    _check(load().moe_layer_forward_overlapped(ctypes.byref(c), _p(x), _p(w_gate), _p(bias), _p(expert_owner),
+                                               _p(w13), _p(w2), _p(y), lay, _p(status), _p(ws), ws.numel(), _stream(),
+                                               ctypes.c_void_p(side_stream.cuda_stream)),
+           "moe_layer_forward_overlapped")
+    return y
 
 
 def layer_forward(cfg, x, w_gate, bias, expert_owner, w13, w2, y=None, ws=None, layout=None, status=None):

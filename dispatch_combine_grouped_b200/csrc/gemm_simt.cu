@@ -22,11 +22,12 @@ __global__ void __launch_bounds__(kSimtThreads) simt_gemm_kernel(const GemmArgs 
   const int G = p.G;
   for (int g = tid; g < G; g += kSimtThreads) {
     int rows, arow, orow;
-    if (g < p.E) {
-      rows = p.n_e[g];
-      arow = orow = p.expert_off[g];
+    const int gg = p.g0 + g;  // global group
+    if (gg < p.E) {
+      rows = p.n_e[gg];
+      arow = orow = p.expert_off[gg];
     } else {
-      const int s = g - p.E;
+      const int s = gg - p.E;
       rows = p.N;
       orow = p.A_routed + s * p.N;
       arow = p.shared_from_map1 ? 0 : orow;
@@ -72,9 +73,10 @@ __global__ void __launch_bounds__(kSimtThreads) simt_gemm_kernel(const GemmArgs 
     const int local = t - s_prefix[g] * n_tiles;
     const int n_blk = local / mt, m_blk = local - n_blk * mt;
     const int rows = s_rows[g];
-    const float* Abase = (g >= p.E && p.shared_from_map1) ? A1 : Aall;
+    const int gz = p.g0 + g;  // global group = weight index
+    const float* Abase = (gz >= p.E && p.shared_from_map1) ? A1 : Aall;
     const long long arow0 = (long long)s_arow[g] + (long long)m_blk * SBM;
-    const float* W = Ball + (long long)g * p.b_rows * p.K;
+    const float* W = Ball + (long long)gz * p.b_rows * p.K;
     const int n0 = n_blk * SBN;
 
     float accg[4][4] = {}, accu[4][4] = {};
@@ -136,7 +138,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_gemm_kernel(const GemmArgs 
       if (r >= rows) continue;
       const long long orow = (long long)s_orow[g] + r;
       float scale = 1.0f;
-      if (MODE == MODE_FC2 && p.gate_w && g < p.E) scale = p.gate_w[p.row2tok[orow]];
+      if (MODE == MODE_FC2 && p.gate_w && gz < p.E) scale = p.gate_w[p.row2tok[orow]];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int col = n0 + tx * 4 + j;
@@ -152,7 +154,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_gemm_kernel(const GemmArgs 
 }
 
 cudaError_t launch_simt_gemm(const GemmArgs& g, cudaStream_t st) {
-  const long long rows_total = (long long)g.A_routed + (long long)(g.G - g.E) * g.N;
+  const long long rows_total = launch_rows(g);
   const long long blocks = (rows_total + SBM - 1) / SBM + g.G;
   const long long tiles = blocks * ((g.n_out + SBN - 1) / SBN);
   long long grid = 4LL * sm_count();

@@ -120,11 +120,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // group table: rows, first A row, first output row
   for (int g = threadIdx.x; g < G; g += kThreads) {
     int rows, arow, orow;
-    if (g < p.E) {
-      rows = p.n_e[g];
-      arow = orow = p.expert_off[g];
+    const int gg = p.g0 + g;  // global group
+    if (gg < p.E) {
+      rows = p.n_e[gg];
+      arow = orow = p.expert_off[gg];
     } else {
-      const int s = g - p.E;
+      const int s = gg - p.E;
       rows = p.N;
       orow = p.A_routed + s * p.N;
       arow = p.shared_from_map1 ? 0 : orow;
@@ -175,7 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const TileDesc td = decode_tile(t, s_prefix, G, n_tiles);
-        const CUtensorMap* mapA = (td.g >= p.E && p.shared_from_map1) ? &tmA1 : &tmA0;
+        const int gz = p.g0 + td.g;  // global group = weight index
+        const CUtensorMap* mapA = (gz >= p.E && p.shared_from_map1) ? &tmA1 : &tmA0;
         const int a_row = s_arow[td.g] + td.m_blk * BM;
         int b_row0, b_row1;
         if (MODE == MODE_FC1) {
@@ -192,8 +194,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&full[stage], TX_BYTES);
           tma_load_2d(sA + stage * A_BYTES, mapA, &full[stage], kb * BK, a_row);
-          tma_load_3d(sB + stage * B_BYTES, &tmB, &full[stage], kb * BK, b_row0, td.g);
-          tma_load_3d(sB + stage * B_BYTES + HALF_B, &tmB, &full[stage], kb * BK, b_row1, td.g);
+          tma_load_3d(sB + stage * B_BYTES, &tmB, &full[stage], kb * BK, b_row0, gz);
+          tma_load_3d(sB + stage * B_BYTES + HALF_B, &tmB, &full[stage], kb * BK, b_row1, gz);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -346,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {  // MODE_FC2
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + orow * p.ldo;
         float scale = 1.0f;
-        if (row_ok && p.gate_w && td.g < p.E) scale = p.gate_w[p.row2tok[orow]];
+        if (row_ok && p.gate_w && p.g0 + td.g < p.E) scale = p.gate_w[p.row2tok[orow]];
         const int col_base = td.n_blk * BN;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -463,9 +465,9 @@ cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStre
   CUtensorMap a0, a1, b;
   if (!make_map_a(&a0, g.a0, a0_rows, g.K)) return cudaErrorInvalidValue;
   if (!make_map_a(&a1, g.a1 ? g.a1 : g.a0, g.a1 ? a1_rows : a0_rows, g.K)) return cudaErrorInvalidValue;
-  if (!make_map_b(&b, g.b, g.G, g.b_rows, g.K, BN / 2)) return cudaErrorInvalidValue;
+  if (!make_map_b(&b, g.b, g.g0 + g.G, g.b_rows, g.K, BN / 2)) return cudaErrorInvalidValue;
   // upper bound on tiles: every group adds at most one partial row block
-  long long rows_total = (long long)g.A_routed + (long long)(g.G - g.E) * g.N;
+  long long rows_total = launch_rows(g);
   long long blocks = (rows_total + BM - 1) / BM + g.G;
   long long n_tiles = g.mode == MODE_FC1 ? (g.n_out + BN / 2 - 1) / (BN / 2) : (g.n_out + BN - 1) / BN;
   long long max_tiles = blocks * n_tiles;

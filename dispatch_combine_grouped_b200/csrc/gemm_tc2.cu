@@ -92,11 +92,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   // group table over the rows that pair tiles cover
   for (int g = threadIdx.x; g < G; g += kPairThreads) {
     int rows, arow, orow;
-    if (g < p.E) {
-      rows = p.n_e[g];
-      arow = orow = p.expert_off[g];
+    const int gg = p.g0 + g;  // global group
+    if (gg < p.E) {
+      rows = p.n_e[gg];
+      arow = orow = p.expert_off[gg];
     } else {
-      const int s = g - p.E;
+      const int s = gg - p.E;
       rows = p.N;
       orow = p.A_routed + s * p.N;
       arow = p.shared_from_map1 ? 0 : orow;
@@ -151,7 +152,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const int g = lo, mt = s_prefix[g + 1] - s_prefix[g];
         const int local = t - s_prefix[g] * n_tiles;
         const int n_blk = local / mt, m_blk = local - n_blk * mt;
-        const CUtensorMap* mapA = (g >= p.E && p.shared_from_map1) ? &tmA1 : &tmA0;
+        const int gz = p.g0 + g;  // global group = weight index
+        const CUtensorMap* mapA = (gz >= p.E && p.shared_from_map1) ? &tmA1 : &tmA0;
         const int a_row = s_arow[g] + m_blk * PM + (int)rank * 128;
         // FC1: the even CTA stages the W_gate rows, the odd CTA the W_up rows of the same
         // 128 outputs, so accumulator columns [0,128) are gate and [128,256) are up
@@ -165,7 +167,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
           const uint32_t bar = lead_full0 + (uint32_t)(stage * sizeof(uint64_t));
           tma_load_2d_pair(sA + stage * A_BYTES, mapA, bar, kb * PK, a_row);
-          tma_load_3d_pair(sB + stage * B_BYTES, &tmB, bar, kb * PK, b_row, g);
+          tma_load_3d_pair(sB + stage * B_BYTES, &tmB, bar, kb * PK, b_row, gz);
           if (++stage == kPairStages) {
             stage = 0;
             ph ^= 1u;
@@ -288,7 +290,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
       } else {
         float scale = 1.0f;
-        if (row_ok && p.gate_w && g < p.E) scale = p.gate_w[p.row2tok[orow]];
+        if (row_ok && p.gate_w && p.g0 + g < p.E) scale = p.gate_w[p.row2tok[orow]];
         const int col_base = n_blk * PN;
 #pragma unroll 1
         for (int c0 = 0; c0 < PN; c0 += 32) {
@@ -334,8 +336,8 @@ cudaError_t launch_tc_gemm_pair(const GemmArgs& g, int a0_rows, int a1_rows, cud
   CUtensorMap a0, a1, b;
   if (!make_map_a(&a0, g.a0, a0_rows, g.K)) return cudaErrorInvalidValue;
   if (!make_map_a(&a1, g.a1 ? g.a1 : g.a0, g.a1 ? a1_rows : a0_rows, g.K)) return cudaErrorInvalidValue;
-  if (!make_map_b(&b, g.b, g.G, g.b_rows, g.K, PN / 2)) return cudaErrorInvalidValue;
-  const long long rows_total = (long long)g.A_routed + (long long)(g.G - g.E) * g.N;
+  if (!make_map_b(&b, g.b, g.g0 + g.G, g.b_rows, g.K, PN / 2)) return cudaErrorInvalidValue;
+  const long long rows_total = launch_rows(g);
   const long long pairs = (rows_total + PM - 1) / PM + g.G;
   const long long n_tiles = g.mode == MODE_FC1 ? (g.n_out + PN / 2 - 1) / (PN / 2) : (g.n_out + PN - 1) / PN;
   long long grid = (sm_count() / 2) * 2;

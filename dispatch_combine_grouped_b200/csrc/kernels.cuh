@@ -45,8 +45,9 @@ enum GemmMode { MODE_ROUTER = 0, MODE_FC1 = 1, MODE_FC2 = 2 };
 
 struct GemmArgs {
   int mode;
-  int G;             // groups
-  int E;             // routed groups (first E)
+  int G;             // groups in this launch: global groups g0 .. g0+G-1
+  int g0;            // first global group (routed experts are 0..E-1, shared E..E+S-1)
+  int E;             // routed groups
   int N;             // rows of a shared group
   int A_routed;      // rows of all routed groups (= N*k for the FFN, 0 for the router)
   int K;             // reduction length
@@ -68,6 +69,13 @@ struct GemmArgs {
   const void* b;
   long long b_rows;     // rows of one weight matrix (2I, d or E)
 };
+
+// Rows a launch covers, for grid sizing: routed rows if any routed group is in range,
+// plus N rows per shared group in range.
+inline long long launch_rows(const GemmArgs& g) {
+  const int routed = (g.g0 < g.E) ? ((g.g0 + g.G < g.E ? g.g0 + g.G : g.E) - g.g0) : 0;
+  return (routed > 0 ? (long long)g.A_routed : 0LL) + (long long)(g.G - routed) * g.N;
+}
 
 // tensor-core (tcgen05) path, bf16 operands, fp32 accumulation: one CTA per tile
 cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStream_t st);

@@ -197,25 +197,32 @@ cudaError_t tc_grouped(GemmArgs g, const moe_config& c, int a0_rows, int a1_rows
 }
 
 moe_status fc1_impl(const moe_config& c, const moe_layout& L, const void* x_perm, const void* x, const void* w13,
-                    void* h, cudaStream_t st) {
-  const GemmArgs g = fc1_args(c, L, x_perm, x, w13, h);
+                    void* h, cudaStream_t st, int g0 = 0, int G = -1) {
+  GemmArgs g = fc1_args(c, L, x_perm, x, w13, h);
+  g.g0 = g0;
+  if (G >= 0) g.G = G;
+  if (g.G == 0) return MOE_OK;
   cudaError_t e = c.dtype == MOE_BF16 ? tc_grouped(g, c, c.N * c.k, c.N, st) : launch_simt_gemm(g, st);
   return cuda_status(e, "FC1 grouped GEMM");
 }
 
 moe_status fc2_impl(const moe_config& c, const moe_layout& L, const void* h, const void* w2, const float* topk_w,
-                    void* out, cudaStream_t st) {
-  const GemmArgs g = fc2_args(c, L, h, w2, topk_w, out);
+                    void* out, cudaStream_t st, int g0 = 0, int G = -1) {
+  GemmArgs g = fc2_args(c, L, h, w2, topk_w, out);
+  g.g0 = g0;
+  if (G >= 0) g.G = G;
+  if (g.G == 0) return MOE_OK;
   cudaError_t e = c.dtype == MOE_BF16 ? tc_grouped(g, c, c.N * c.k + c.n_shared * c.N, 0, st)
                                       : launch_simt_gemm(g, st);
   return cuda_status(e, "FC2 grouped GEMM");
 }
 
 moe_status ffn_impl(const moe_config& c, const moe_layout& L, const void* x_perm, const void* x, const void* w13,
-                    const void* w2, const float* topk_w, void* h, void* out, cudaStream_t st) {
-  moe_status s = fc1_impl(c, L, x_perm, x, w13, h, st);
+                    const void* w2, const float* topk_w, void* h, void* out, cudaStream_t st, int g0 = 0,
+                    int G = -1) {
+  moe_status s = fc1_impl(c, L, x_perm, x, w13, h, st, g0, G);
   if (s != MOE_OK) return s;
-  return fc2_impl(c, L, h, w2, topk_w, out, st);
+  return fc2_impl(c, L, h, w2, topk_w, out, st, g0, G);
 }
 
 }  // namespace
@@ -304,24 +311,66 @@ moe_status moe_grouped_ffn(const moe_config* cfg, const moe_layout* layout, cons
   return ffn_impl(*cfg, *layout, x_perm, x, w13, w2, topk_w, h_ws, out, (cudaStream_t)stream);
 }
 
+static bool group_range(const moe_config& c, int32_t groups, int* g0, int* G) {
+  switch (groups) {
+    case MOE_GROUPS_ALL: *g0 = 0; *G = c.E + c.n_shared; return true;
+    case MOE_GROUPS_ROUTED: *g0 = 0; *G = c.E; return true;
+    case MOE_GROUPS_SHARED: *g0 = c.E; *G = c.n_shared; return true;
+    default: return false;
+  }
+}
+
 moe_status moe_expert_fc1(const moe_config* cfg, const moe_layout* layout, const void* x_perm, const void* x,
-                          const void* w13, void* h_ws, moe_stream_t stream) {
+                          const void* w13, void* h_ws, int32_t groups, moe_stream_t stream) {
   moe_status s = check_config(cfg);
   if (s != MOE_OK) return s;
+  int g0, G;
+  if (!group_range(*cfg, groups, &g0, &G)) return fail(MOE_ERR_INVALID_ARG, "groups out of range");
   if (cfg->N == 0) return MOE_OK;
-  if (!layout || !layout->n_e || !layout->expert_off || !x_perm || !w13 || !h_ws || (cfg->n_shared > 0 && !x))
+  const bool routed = groups != MOE_GROUPS_SHARED, shared = groups != MOE_GROUPS_ROUTED && cfg->n_shared > 0;
+  if (!w13 || !h_ws || (routed && (!layout || !layout->n_e || !layout->expert_off || !x_perm)) || (shared && !x))
     return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
-  return fc1_impl(*cfg, *layout, x_perm, x, w13, h_ws, (cudaStream_t)stream);
+  moe_layout none;
+  memset(&none, 0, sizeof(none));
+  return fc1_impl(*cfg, routed ? *layout : none, x_perm, x, w13, h_ws, (cudaStream_t)stream, g0, G);
 }
 
 moe_status moe_expert_fc2(const moe_config* cfg, const moe_layout* layout, const void* h_ws, const void* w2,
-                          const float* topk_w, void* out, moe_stream_t stream) {
+                          const float* topk_w, void* out, int32_t groups, moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  int g0, G;
+  if (!group_range(*cfg, groups, &g0, &G)) return fail(MOE_ERR_INVALID_ARG, "groups out of range");
+  if (cfg->N == 0) return MOE_OK;
+  const bool routed = groups != MOE_GROUPS_SHARED;
+  if (!h_ws || !w2 || !out || (routed && (!layout || !layout->n_e || !layout->expert_off || !layout->row2tok)))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  moe_layout none;
+  memset(&none, 0, sizeof(none));
+  return fc2_impl(*cfg, routed ? *layout : none, h_ws, w2, topk_w, out, (cudaStream_t)stream, g0, G);
+}
+
+moe_status moe_routed_ffn(const moe_config* cfg, const moe_layout* layout, const void* x_perm, const void* w13,
+                          const void* w2, const float* topk_w, void* h_ws, void* out, moe_stream_t stream) {
   moe_status s = check_config(cfg);
   if (s != MOE_OK) return s;
   if (cfg->N == 0) return MOE_OK;
-  if (!layout || !layout->n_e || !layout->expert_off || !layout->row2tok || !h_ws || !w2 || !out)
+  if (!layout || !layout->n_e || !layout->expert_off || !layout->row2tok || !x_perm || !w13 || !w2 || !h_ws ||
+      !out)
     return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
-  return fc2_impl(*cfg, *layout, h_ws, w2, topk_w, out, (cudaStream_t)stream);
+  return ffn_impl(*cfg, *layout, x_perm, nullptr, w13, w2, topk_w, h_ws, out, (cudaStream_t)stream, 0, cfg->E);
+}
+
+moe_status moe_shared_ffn(const moe_config* cfg, const void* x, const void* w13, const void* w2, void* h_ws,
+                          void* out, moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->N == 0 || cfg->n_shared == 0) return MOE_OK;
+  if (!x || !w13 || !w2 || !h_ws || !out) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  moe_layout none;
+  memset(&none, 0, sizeof(none));
+  return ffn_impl(*cfg, none, nullptr, x, w13, w2, nullptr, h_ws, out, (cudaStream_t)stream, cfg->E,
+                  cfg->n_shared);
 }
 
 moe_status moe_combine(const moe_config* cfg, const moe_layout* layout, const void* out, const float* topk_w,
@@ -366,6 +415,54 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* w
   if (c.N == 0) return MOE_OK;
   if ((s = cuda_status(launch_permute(c, L, x, w.x_perm, st), "permute")) != MOE_OK) return s;
   if ((s = ffn_impl(c, L, w.x_perm, x, w13, w2, w.w, w.h, w.out, st)) != MOE_OK) return s;
+  return cuda_status(launch_combine(c, L, w.out, nullptr, y, st), "combine");
+}
+
+moe_status moe_layer_forward_overlapped(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
+                                        const int32_t* expert_owner, const void* w13, const void* w2, void* y,
+                                        const moe_layout* layout_out, int32_t* dev_status, void* ws, size_t ws_bytes,
+                                        moe_stream_t stream, moe_stream_t side_stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
+  const moe_config& c = *cfg;
+  if (c.n_shared == 0 || c.N == 0 || side_stream == stream)
+    return moe_layer_forward(cfg, x, w_gate, bias, expert_owner, w13, w2, y, layout_out, dev_status, ws, ws_bytes,
+                             stream);
+  FwdWs w = carve_forward(c, nullptr);
+  if (!ws || ws_bytes < w.total) return fail(MOE_ERR_WORKSPACE, "forward workspace too small");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return fail(MOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if (layout_out && !layout_complete(layout_out)) return fail(MOE_ERR_INVALID_ARG, "incomplete layout_out");
+  if (!x || !w_gate || !w13 || !w2 || !y) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  w = carve_forward(c, static_cast<char*>(ws));
+  const moe_layout& L = layout_out ? *layout_out : w.lay;
+  cudaStream_t st = (cudaStream_t)stream, side = (cudaStream_t)side_stream;
+  if ((s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaError_t e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventRecord(fork, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
+  if (e != cudaSuccess) {
+    if (fork) cudaEventDestroy(fork);
+    if (join) cudaEventDestroy(join);
+    return cuda_status(e, "fork");
+  }
+  // side stream: shared experts (they read only x)
+  moe_layout none;
+  memset(&none, 0, sizeof(none));
+  s = ffn_impl(c, none, nullptr, x, w13, w2, nullptr, w.h, w.out, side, c.E, c.n_shared);
+  e = cudaEventRecord(join, side);
+  // main stream: layout, permute, routed experts
+  if (s == MOE_OK)
+    s = cuda_status(launch_layout(c, expert_owner, w.ids, L, dev_status, w.lay_ws, st), "layout");
+  if (s == MOE_OK) s = cuda_status(launch_permute(c, L, x, w.x_perm, st), "permute");
+  if (s == MOE_OK) s = ffn_impl(c, L, w.x_perm, x, w13, w2, w.w, w.h, w.out, st, 0, c.E);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, join, 0);  // join even after an error
+  cudaEventDestroy(fork);
+  cudaEventDestroy(join);
+  if (s != MOE_OK) return s;
+  if (e != cudaSuccess) return cuda_status(e, "join");
   return cuda_status(launch_combine(c, L, w.out, nullptr, y, st), "combine");
 }
 

@@ -218,18 +218,36 @@ moe_status moe_grouped_ffn(const moe_config* cfg, const moe_layout* layout, cons
                            const void* w13, const void* w2, const float* topk_w, void* h_ws, void* out,
                            moe_stream_t stream);
 
+/* Which expert groups an FFN call covers. */
+typedef enum { MOE_GROUPS_ALL = 0, MOE_GROUPS_ROUTED = 1, MOE_GROUPS_SHARED = 2 } moe_group_set;
+
 /*
  * The two halves of moe_grouped_ffn, for callers that schedule them separately:
- *   moe_expert_fc1: h_ws = SiLU(X W_gate^T) * (X W_up^T) for every group (routed rows of
- *                   x_perm, then each shared expert over the N rows of x)
+ *   moe_expert_fc1: h_ws = SiLU(X W_gate^T) * (X W_up^T) for every group in `groups`
+ *                   (routed rows of x_perm; each shared expert over the N rows of x)
  *   moe_expert_fc2: out = (h_ws W_down^T), routed rows scaled by topk_w[row2tok[r]] when
  *                   topk_w is non-NULL
- * Shapes, layouts and errors as for moe_grouped_ffn.
+ * `groups` is a moe_group_set.  Shapes, layouts and errors as for moe_grouped_ffn; with
+ * MOE_GROUPS_SHARED the layout may be NULL.
  */
 moe_status moe_expert_fc1(const moe_config* cfg, const moe_layout* layout, const void* x_perm, const void* x,
-                          const void* w13, void* h_ws, moe_stream_t stream);
+                          const void* w13, void* h_ws, int32_t groups, moe_stream_t stream);
 moe_status moe_expert_fc2(const moe_config* cfg, const moe_layout* layout, const void* h_ws, const void* w2,
-                          const float* topk_w, void* out, moe_stream_t stream);
+                          const float* topk_w, void* out, int32_t groups, moe_stream_t stream);
+
+/*
+ * moe_grouped_ffn split by expert kind, so that the shared experts (which need only x)
+ * can run concurrently with the routing and dispatch of the routed ones:
+ *   moe_routed_ffn: FC1 + SwiGLU and FC2 (x topk_w when non-NULL) for the routed experts,
+ *                   rows [0, A) of h_ws and out
+ *   moe_shared_ffn: the same for the S shared experts over all N rows of x, rows
+ *                   [A, A + S*N) of h_ws and out (no layout is needed)
+ * Together they write exactly what moe_grouped_ffn writes.
+ */
+moe_status moe_routed_ffn(const moe_config* cfg, const moe_layout* layout, const void* x_perm, const void* w13,
+                          const void* w2, const float* topk_w, void* h_ws, void* out, moe_stream_t stream);
+moe_status moe_shared_ffn(const moe_config* cfg, const void* x, const void* w13, const void* w2, void* h_ws,
+                          void* out, moe_stream_t stream);
 
 /*
  * Combine ([EP-DeepEP] §2-3; [DSMoE] combine = gate-weighted sum at the source;
@@ -263,6 +281,21 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* w
                              const int32_t* expert_owner, const void* w13, const void* w2, void* y,
                              const moe_layout* layout_out, int32_t* dev_status, void* ws, size_t ws_bytes,
                              moe_stream_t stream);
+
+/*
+ * moe_layer_forward with the shared experts overlapped (the pages' overlap lever:
+ * [EP-DeepEP] §7 pipelining; [WideEP] dual-batch overlap; [MoE-IV] §4.2 overlap): the
+ * router runs on `stream`; then the shared experts run on `side_stream` while the
+ * layout, permute and routed experts run on `stream`; `stream` waits for `side_stream`
+ * before the combine.  Same result as moe_layer_forward, bit for bit.  Two events are
+ * created and destroyed per call (no device memory is allocated).  With n_shared == 0 or
+ * side_stream == stream this is moe_layer_forward.  When the call returns, `stream`
+ * orders after all the work; `side_stream` may be reused immediately.
+ */
+moe_status moe_layer_forward_overlapped(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
+                                        const int32_t* expert_owner, const void* w13, const void* w2, void* y,
+                                        const moe_layout* layout_out, int32_t* dev_status, void* ws, size_t ws_bytes,
+                                        moe_stream_t stream, moe_stream_t side_stream);
 
 #ifdef __cplusplus
 }

@@ -235,3 +235,22 @@ def test_ffn_pair_and_tail_row_splits():
         w13 = O.f64(inp["w13"][e])
         hh = O.silu(xp64[r0:r0 + n] @ w13[:cfg.I].T) * (xp64[r0:r0 + n] @ w13[cfg.I:].T)
         assert_close_rel(h[r0:r0 + n], hh, what=f"h expert {e}")
+
+
+@pytest.mark.parametrize("cfg", [SMALL[1], SMALL[4], SMALL[5]], ids=_ids([SMALL[1], SMALL[4], SMALL[5]]))
+def test_overlapped_forward_and_split_ffn_match_bitwise(cfg):
+    """Shared experts on a side stream give the same bits as the one-stream forward, and
+    moe_routed_ffn + moe_shared_ffn write exactly what moe_grouped_ffn writes."""
+    inp = gpu_inputs(cfg)
+    res = run_steps(cfg, inp)
+    side = torch.cuda.Stream()
+    lay = moe.Layout(cfg)
+    y = moe.layer_forward_overlapped(cfg, inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], inp["w13"],
+                                     inp["w2"], side, layout=lay)
+    torch.cuda.synchronize()
+    assert torch.equal(y, res["y"])
+    assert torch.equal(lay["tok2row"], res["layout"]["tok2row"])
+    h, out = moe.routed_ffn(cfg, res["layout"], res["x_perm"], inp["w13"], inp["w2"], topk_w=res["w"])
+    moe.shared_ffn(cfg, inp["x"], inp["w13"], inp["w2"], h, out)
+    torch.cuda.synchronize()
+    assert torch.equal(h, res["h"]) and torch.equal(out, res["out"])
