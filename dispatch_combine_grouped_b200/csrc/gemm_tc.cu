@@ -294,6 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (MODE == MODE_ROUTER) {
         float* dst = static_cast<float*>(p.out) + orow * p.ldo;
+        const int col_base = td.n_blk * BN;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 32) {
           uint32_t v[32];
@@ -302,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (row_ok) {
 #pragma unroll
             for (int q = 0; q < 32; q += 4) {
-              const int col = c0 + q;
+              const int col = col_base + c0 + q;
               float f[4];
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
@@ -441,12 +442,15 @@ int sm_count() {
 template <int BN, int MODE>
 static cudaError_t launch_bn(const GemmArgs& g, const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                              long long max_tiles, cudaStream_t st) {
-  constexpr int STAGES = 4;
+  // as many stages as fit in ~192 KB, at most 8 (narrow router tiles get deeper rings)
+  constexpr int STAGE_KB = (BM * BK * 2 + BN * BK * 2) / 1024;
+  constexpr int STAGES = (192 / STAGE_KB) > 8 ? 8 : (192 / STAGE_KB);
   constexpr int smem = smem_bytes_for<BN, STAGES>();
   auto kern = tc_gemm_kernel<BN, MODE, STAGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   long long grid = sm_count();
+  if (g.max_ctas > 0 && g.max_ctas < grid) grid = g.max_ctas;
   if (max_tiles < grid) grid = max_tiles;
   if (grid < 1) grid = 1;
   kern<<<(unsigned)grid, kThreads, smem, st>>>(a0, a1, b, g);
@@ -457,8 +461,13 @@ cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStre
   // B box rows: half the tile (two boxes per stage)
   int BN;
   if (g.mode == MODE_ROUTER) {
+    // one tile column holds every expert when that already gives ~a wave of tiles;
+    // with few 128-token row blocks the experts are split over narrower tile columns
+    // so that more SMs stream x
     BN = 32;
     while (BN < g.n_out) BN <<= 1;
+    const long long row_blocks = ((long long)g.N + BM - 1) / BM;
+    while (BN > 32 && row_blocks * ((g.n_out + BN - 1) / BN) < 120) BN >>= 1;
   } else {
     BN = 256;
   }

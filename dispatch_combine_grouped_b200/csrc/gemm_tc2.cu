@@ -341,6 +341,7 @@ cudaError_t launch_tc_gemm_pair(const GemmArgs& g, int a0_rows, int a1_rows, cud
   const long long pairs = (rows_total + PM - 1) / PM + g.G;
   const long long n_tiles = g.mode == MODE_FC1 ? (g.n_out + PN / 2 - 1) / (PN / 2) : (g.n_out + PN - 1) / PN;
   long long grid = (sm_count() / 2) * 2;
+  if (g.max_ctas > 0 && g.max_ctas < grid) grid = (g.max_ctas / 2) * 2;
   if (2 * pairs * n_tiles < grid) grid = 2 * pairs * n_tiles;
   if (grid < 2) grid = 2;
   cudaError_t e;

@@ -68,6 +68,7 @@ struct GemmArgs {
   const void* a1;
   const void* b;
   long long b_rows;     // rows of one weight matrix (2I, d or E)
+  int max_ctas;         // cap on the persistent grid (0 = one CTA per SM)
 };
 
 // Rows a launch covers, for grid sizing: routed rows if any routed group is in range,

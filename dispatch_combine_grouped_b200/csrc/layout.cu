@@ -188,27 +188,45 @@ __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutArgs p,
   const int PP = p.P * p.P;
 
   // per-expert and per-owner chunk bases (in place), totals
+  // column scans over chunks; loads are batched so that 8 are in flight at a time
+  constexpr int B = 8;
   if (tid < p.E) {
     int s = 0;
-    for (int c = 0; c < nchunks; ++c) {
-      int v = w.hist_e[(size_t)c * p.E + tid];
-      w.hist_e[(size_t)c * p.E + tid] = s;
-      s += v;
+    for (int c0 = 0; c0 < nchunks; c0 += B) {
+      int v[B];
+#pragma unroll
+      for (int u = 0; u < B; ++u) v[u] = c0 + u < nchunks ? w.hist_e[(size_t)(c0 + u) * p.E + tid] : 0;
+#pragma unroll
+      for (int u = 0; u < B; ++u) {
+        if (c0 + u < nchunks) w.hist_e[(size_t)(c0 + u) * p.E + tid] = s;
+        s += v[u];
+      }
     }
     s_ne[tid] = s;
     L.n_e[tid] = s;
   } else if (tid >= 512 && tid < 512 + p.P) {
     const int j = tid - 512;
     int s = 0;
-    for (int c = 0; c < nchunks; ++c) {
-      int v = w.hist_j[(size_t)c * p.P + j];
-      w.hist_j[(size_t)c * p.P + j] = s;
-      s += v;
+    for (int c0 = 0; c0 < nchunks; c0 += B) {
+      int v[B];
+#pragma unroll
+      for (int u = 0; u < B; ++u) v[u] = c0 + u < nchunks ? w.hist_j[(size_t)(c0 + u) * p.P + j] : 0;
+#pragma unroll
+      for (int u = 0; u < B; ++u) {
+        if (c0 + u < nchunks) w.hist_j[(size_t)(c0 + u) * p.P + j] = s;
+        s += v[u];
+      }
     }
   }
   for (int x = tid; x < PP; x += kScanThreads) {
     int s = 0;
-    for (int c = 0; c < nchunks; ++c) s += w.hist_ij[(size_t)c * PP + x];
+    for (int c0 = 0; c0 < nchunks; c0 += B) {
+      int v[B];
+#pragma unroll
+      for (int u = 0; u < B; ++u) v[u] = c0 + u < nchunks ? w.hist_ij[(size_t)(c0 + u) * PP + x] : 0;
+#pragma unroll
+      for (int u = 0; u < B; ++u) s += v[u];
+    }
     s_C[x] = s;
     L.C[x] = s;
   }
@@ -247,12 +265,17 @@ __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutArgs p,
     int v = tid < p.E ? s_ne[tid] : 0;
     int ex = block_exclusive_scan(v, nullptr);
     if (tid < p.E) L.expert_off[tid] = ex;
-  } else if (tid < p.E) {
-    const int j = owner_of(p, tid);
-    int s = s_recv[j];
-    for (int e2 = 0; e2 < tid; ++e2)
-      if (owner_of(p, e2) == j) s += s_ne[e2];
-    L.expert_off[tid] = s;
+  } else {
+    __shared__ int s_own[kMaxE];
+    if (tid < p.E) s_own[tid] = owner_of(p, tid);
+    __syncthreads();
+    if (tid < p.E) {
+      const int j = s_own[tid];
+      int s = s_recv[j];
+      for (int e2 = 0; e2 < tid; ++e2)
+        if (s_own[e2] == j) s += s_ne[e2];
+      L.expert_off[tid] = s;
+    }
   }
   if (tid == 0) L.expert_off[p.E] = p.A;
 

@@ -196,10 +196,19 @@ cudaError_t tc_grouped(GemmArgs g, const moe_config& c, int a0_rows, int a1_rows
   return launch_tc_gemm(g, a0_rows, a1_rows, st);
 }
 
+// A launch over the shared experts alone runs beside the routing kernels of the same
+// layer (moe_layer_forward_overlapped): it leaves this many SMs to them.
+constexpr int kSharedReserveSMs = 16;
+
+int shared_cap(const moe_config& c, int g0) {
+  return (g0 >= c.E && sm_count() > 2 * kSharedReserveSMs) ? sm_count() - kSharedReserveSMs : 0;
+}
+
 moe_status fc1_impl(const moe_config& c, const moe_layout& L, const void* x_perm, const void* x, const void* w13,
                     void* h, cudaStream_t st, int g0 = 0, int G = -1) {
   GemmArgs g = fc1_args(c, L, x_perm, x, w13, h);
   g.g0 = g0;
+  g.max_ctas = shared_cap(c, g0);
   if (G >= 0) g.G = G;
   if (g.G == 0) return MOE_OK;
   cudaError_t e = c.dtype == MOE_BF16 ? tc_grouped(g, c, c.N * c.k, c.N, st) : launch_simt_gemm(g, st);
@@ -210,6 +219,7 @@ moe_status fc2_impl(const moe_config& c, const moe_layout& L, const void* h, con
                     void* out, cudaStream_t st, int g0 = 0, int G = -1) {
   GemmArgs g = fc2_args(c, L, h, w2, topk_w, out);
   g.g0 = g0;
+  g.max_ctas = shared_cap(c, g0);
   if (G >= 0) g.G = G;
   if (g.G == 0) return MOE_OK;
   cudaError_t e = c.dtype == MOE_BF16 ? tc_grouped(g, c, c.N * c.k + c.n_shared * c.N, 0, st)

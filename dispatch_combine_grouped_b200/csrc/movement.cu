@@ -118,7 +118,11 @@ struct Vec<__nv_bfloat16> {
 };
 
 // y_t = sum_{j<k} g_{t,j} * routed[map[t*k+j]] + sum_{s<S} shared[s*N + t], fp32
-// accumulation in exactly this order, one rounding.
+// accumulation in exactly this order, one rounding.  A warp handles one (token, chunk of
+// 64 vectors) item: each lane issues the loads of its 2 vectors for all k (+S) rows
+// before using any, so up to 2*(k+S) 16-byte loads per lane are in flight.
+constexpr int kCombVec = 2;
+
 template <typename T>
 __global__ void __launch_bounds__(kMoveWarps * 32) combine_kernel(const uint4* __restrict__ routed,
                                                                    const uint4* __restrict__ shared,
@@ -127,28 +131,38 @@ __global__ void __launch_bounds__(kMoveWarps * 32) combine_kernel(const uint4* _
                                                                    uint4* __restrict__ y, int N, int k, int S,
                                                                    int vpr) {
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kMoveWarps + (threadIdx.x >> 5);
-  if (t >= N) return;
+  const int chunks = (vpr + 32 * kCombVec - 1) / (32 * kCombVec);
+  const long long item = (long long)blockIdx.x * kMoveWarps + (threadIdx.x >> 5);
+  if (item >= (long long)N * chunks) return;
+  const int t = (int)(item / chunks);
+  const int v0 = (int)(item - (long long)t * chunks) * 32 * kCombVec + lane;
   const int my_row = lane < k ? map[(size_t)t * k + lane] : 0;
   const float my_g = (lane < k && gates) ? gates[(size_t)t * k + lane] : 1.0f;
   int rows[kMaxK];
   float gs[kMaxK];
 #pragma unroll
-  for (int j = 0; j < kMaxK; ++j) {  // broadcast before the (possibly divergent) vector loop
+  for (int j = 0; j < kMaxK; ++j) {
     rows[j] = __shfl_sync(0xffffffffu, my_row, j);
     gs[j] = __shfl_sync(0xffffffffu, my_g, j);
   }
-  for (int v = lane; v < vpr; v += 32) {
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    uint4 q[kMaxK];
+  uint4 q[kCombVec][kMaxK];
+#pragma unroll
+  for (int u = 0; u < kCombVec; ++u) {
+    const int v = v0 + u * 32;
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j)
-      if (j < k) q[j] = ld_stream(routed + (size_t)rows[j] * vpr + v);
+      if (j < k && v < vpr) q[u][j] = ld_stream(routed + (size_t)rows[j] * vpr + v);
+  }
+#pragma unroll
+  for (int u = 0; u < kCombVec; ++u) {
+    const int v = v0 + u * 32;
+    if (v >= vpr) continue;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
       if (j < k) {
         float f[8];
-        Vec<T>::unpack(q[j], f);
+        Vec<T>::unpack(q[u][j], f);
 #pragma unroll
         for (int i = 0; i < Vec<T>::n; ++i) acc[i] = fmaf(gs[j], f[i], acc[i]);
       }
@@ -191,8 +205,10 @@ cudaError_t launch_permute_staged(const moe_config& c, const moe_layout& L, cons
 template <typename T>
 static void combine_launch(const moe_config& c, const uint4* routed, const uint4* shared, const int32_t* map,
                            const float* gates, uint4* y, cudaStream_t st) {
-  combine_kernel<T><<<blocks_for(c.N), kMoveWarps * 32, 0, st>>>(routed, shared, map, gates, y, c.N, c.k,
-                                                                  c.n_shared, vecs_per_row(c));
+  const int vpr = vecs_per_row(c);
+  const long long items = (long long)c.N * ((vpr + 32 * kCombVec - 1) / (32 * kCombVec));
+  combine_kernel<T><<<blocks_for(items), kMoveWarps * 32, 0, st>>>(routed, shared, map, gates, y, c.N, c.k,
+                                                                    c.n_shared, vpr);
 }
 
 cudaError_t launch_combine(const moe_config& c, const moe_layout& L, const void* out, const float* topk_w, void* y,

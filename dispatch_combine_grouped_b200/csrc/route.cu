@@ -41,6 +41,9 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs p) {
     v[q] = col < p.E ? row[col] : -INFINITY;
   }
   const int gsize = p.E / p.n_groups;
+  int grp[kLanesE];  // group of each logit this lane holds (no division in the loops below)
+#pragma unroll
+  for (int q = 0; q < kLanesE; ++q) grp[q] = (lane + 32 * q) / gsize;
 
   // group-limited routing: keep topk_groups groups by their max logit
   uint32_t allowed = 0xffffffffu;
@@ -57,7 +60,7 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs p) {
 #pragma unroll
       for (int q = 0; q < kLanesE; ++q) {
         const int col = lane + 32 * q;
-        if (col < p.E && col / gsize == g) m = fmaxf(m, v[q]);
+        if (col < p.E && grp[q] == g) m = fmaxf(m, v[q]);
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -96,7 +99,7 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs p) {
 #pragma unroll
       for (int q = 0; q < kLanesE; ++q) {
         const int col = lane + 32 * q;
-        const bool ok = col < p.E && !((taken >> q) & 1u) && ((allowed >> (col / gsize)) & 1u);
+        const bool ok = col < p.E && !((taken >> q) & 1u) && ((allowed >> grp[q]) & 1u);
         if (ok && ranks_before(v[q], col, bv, bi)) {
           bv = v[q];
           bi = col;

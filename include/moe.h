@@ -228,7 +228,7 @@ typedef enum { MOE_GROUPS_ALL = 0, MOE_GROUPS_ROUTED = 1, MOE_GROUPS_SHARED = 2 
  *   moe_expert_fc2: out = (h_ws W_down^T), routed rows scaled by topk_w[row2tok[r]] when
  *                   topk_w is non-NULL
  * `groups` is a moe_group_set.  Shapes, layouts and errors as for moe_grouped_ffn; with
- * MOE_GROUPS_SHARED the layout may be NULL.
+ * MOE_GROUPS_SHARED the layout may be NULL and, as in moe_shared_ffn, 16 SMs are left free.
  */
 moe_status moe_expert_fc1(const moe_config* cfg, const moe_layout* layout, const void* x_perm, const void* x,
                           const void* w13, void* h_ws, int32_t groups, moe_stream_t stream);
@@ -241,7 +241,8 @@ moe_status moe_expert_fc2(const moe_config* cfg, const moe_layout* layout, const
  *   moe_routed_ffn: FC1 + SwiGLU and FC2 (x topk_w when non-NULL) for the routed experts,
  *                   rows [0, A) of h_ws and out
  *   moe_shared_ffn: the same for the S shared experts over all N rows of x, rows
- *                   [A, A + S*N) of h_ws and out (no layout is needed)
+ *                   [A, A + S*N) of h_ws and out (no layout is needed); it leaves 16 SMs
+ *                   free for the routing kernels meant to run beside it
  * Together they write exactly what moe_grouped_ffn writes.
  */
 moe_status moe_routed_ffn(const moe_config* cfg, const moe_layout* layout, const void* x_perm, const void* w13,
