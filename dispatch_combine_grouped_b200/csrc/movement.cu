@@ -59,6 +59,60 @@ __global__ void __launch_bounds__(kMoveWarps * 32) scatter_token_rows(const uint
   }
 }
 
+// The same scatter with 32-byte vectors (rows whose size is a multiple of 32 bytes):
+// half the load / store instructions of the 16-byte version.
+struct alignas(32) V32 {
+  uint32_t w[8];
+};
+
+__device__ __forceinline__ V32 ld_stream32(const V32* p) {
+  V32 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]), "=r"(r.w[4]), "=r"(r.w[5]), "=r"(r.w[6]),
+                 "=r"(r.w[7])
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void st32(V32* p, const V32& v) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v.w[0]), "r"(v.w[1]),
+               "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]), "r"(v.w[7])
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kMoveWarps * 32) scatter_token_rows32(const V32* __restrict__ src,
+                                                                         V32* __restrict__ dst,
+                                                                         const int32_t* __restrict__ map, int N,
+                                                                         int k, int vpr) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kMoveWarps + (threadIdx.x >> 5);
+  if (t >= N) return;
+  const int my = lane < k ? map[(size_t)t * k + lane] : 0;
+  int rows[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) rows[j] = __shfl_sync(0xffffffffu, my, j);
+  const V32* s = src + (size_t)t * vpr;
+  for (int v0 = 0; v0 < vpr; v0 += 32 * kMoveUnroll) {
+    V32 buf[kMoveUnroll];
+#pragma unroll
+    for (int u = 0; u < kMoveUnroll; ++u) {
+      const int v = v0 + u * 32 + lane;
+      if (v < vpr) buf[u] = ld_stream32(s + v);
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j < k) {
+        V32* d = dst + (size_t)rows[j] * vpr;
+#pragma unroll
+        for (int u = 0; u < kMoveUnroll; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (v < vpr) st32(d + v, buf[u]);
+        }
+      }
+    }
+  }
+}
+
 // Row gather: dst[i] = src[map[i]] for i < rows  (map == NULL: dst[map_inv...] not used)
 // Row scatter: dst[map[i]] = src[i]
 template <bool kScatter>
@@ -177,12 +231,86 @@ __global__ void __launch_bounds__(kMoveWarps * 32) combine_kernel(const uint4* _
   }
 }
 
+// The combine with 32-byte vectors (rows whose size is a multiple of 32 bytes): one
+// vector per lane per item, k (+S) loads in flight per lane.
+template <typename T>
+__global__ void __launch_bounds__(kMoveWarps * 32) combine_kernel32(const V32* __restrict__ routed,
+                                                                     const V32* __restrict__ shared,
+                                                                     const int32_t* __restrict__ map,
+                                                                     const float* __restrict__ gates,
+                                                                     V32* __restrict__ y, int N, int k, int S,
+                                                                     int vpr) {
+  const int lane = threadIdx.x & 31;
+  const int chunks = (vpr + 31) / 32;
+  const long long item = (long long)blockIdx.x * kMoveWarps + (threadIdx.x >> 5);
+  if (item >= (long long)N * chunks) return;
+  const int t = (int)(item / chunks);
+  const int v = (int)(item - (long long)t * chunks) * 32 + lane;
+  const int my_row = lane < k ? map[(size_t)t * k + lane] : 0;
+  const float my_g = (lane < k && gates) ? gates[(size_t)t * k + lane] : 1.0f;
+  int rows[kMaxK];
+  float gs[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    rows[j] = __shfl_sync(0xffffffffu, my_row, j);
+    gs[j] = __shfl_sync(0xffffffffu, my_g, j);
+  }
+  if (v >= vpr) return;
+  V32 q[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j)
+    if (j < k) q[j] = ld_stream32(routed + (size_t)rows[j] * vpr + v);
+  constexpr int n = Vec<T>::n;  // elements per 16 bytes
+  float acc[2 * 8];
+#pragma unroll
+  for (int i = 0; i < 2 * n; ++i) acc[i] = 0.f;
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    if (j < k) {
+      float f[8];
+      Vec<T>::unpack(make_uint4(q[j].w[0], q[j].w[1], q[j].w[2], q[j].w[3]), f);
+#pragma unroll
+      for (int i = 0; i < n; ++i) acc[i] = fmaf(gs[j], f[i], acc[i]);
+      Vec<T>::unpack(make_uint4(q[j].w[4], q[j].w[5], q[j].w[6], q[j].w[7]), f);
+#pragma unroll
+      for (int i = 0; i < n; ++i) acc[n + i] = fmaf(gs[j], f[i], acc[n + i]);
+    }
+  }
+  for (int s = 0; s < S; ++s) {
+    const V32 sv = ld_stream32(shared + ((size_t)s * N + t) * vpr + v);
+    float f[8];
+    Vec<T>::unpack(make_uint4(sv.w[0], sv.w[1], sv.w[2], sv.w[3]), f);
+#pragma unroll
+    for (int i = 0; i < n; ++i) acc[i] += f[i];
+    Vec<T>::unpack(make_uint4(sv.w[4], sv.w[5], sv.w[6], sv.w[7]), f);
+#pragma unroll
+    for (int i = 0; i < n; ++i) acc[n + i] += f[i];
+  }
+  float lo[8], hi[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    lo[i] = i < n ? acc[i] : 0.f;
+    hi[i] = i < n ? acc[n + i] : 0.f;
+  }
+  const uint4 a = Vec<T>::pack(lo), b = Vec<T>::pack(hi);
+  V32 o;
+  o.w[0] = a.x; o.w[1] = a.y; o.w[2] = a.z; o.w[3] = a.w;
+  o.w[4] = b.x; o.w[5] = b.y; o.w[6] = b.z; o.w[7] = b.w;
+  st32(y + (size_t)t * vpr + v, o);
+}
+
 static inline int elem_bytes(const moe_config& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
 static inline int vecs_per_row(const moe_config& c) { return c.d * elem_bytes(c) / 16; }
 static inline unsigned blocks_for(long long rows) { return (unsigned)((rows + kMoveWarps - 1) / kMoveWarps); }
 
 cudaError_t launch_permute(const moe_config& c, const moe_layout& L, const void* x, void* x_perm, cudaStream_t st) {
   if (c.N == 0) return cudaSuccess;
+  const int row_bytes = c.d * elem_bytes(c);
+  if (row_bytes % 32 == 0) {
+    scatter_token_rows32<<<blocks_for(c.N), kMoveWarps * 32, 0, st>>>(
+        static_cast<const V32*>(x), static_cast<V32*>(x_perm), L.tok2row, c.N, c.k, row_bytes / 32);
+    return cudaGetLastError();
+  }
   scatter_token_rows<<<blocks_for(c.N), kMoveWarps * 32, 0, st>>>(
       static_cast<const uint4*>(x), static_cast<uint4*>(x_perm), L.tok2row, c.N, c.k, vecs_per_row(c));
   return cudaGetLastError();
@@ -205,6 +333,17 @@ cudaError_t launch_permute_staged(const moe_config& c, const moe_layout& L, cons
 template <typename T>
 static void combine_launch(const moe_config& c, const uint4* routed, const uint4* shared, const int32_t* map,
                            const float* gates, uint4* y, cudaStream_t st) {
+#ifndef MOE_COMBINE16
+  const int row_bytes = c.d * elem_bytes(c);
+  if (row_bytes % 32 == 0) {
+    const int vpr32 = row_bytes / 32;
+    const long long items = (long long)c.N * ((vpr32 + 31) / 32);
+    combine_kernel32<T><<<blocks_for(items), kMoveWarps * 32, 0, st>>>(
+        reinterpret_cast<const V32*>(routed), reinterpret_cast<const V32*>(shared), map, gates,
+        reinterpret_cast<V32*>(y), c.N, c.k, c.n_shared, vpr32);
+    return;
+  }
+#endif
   const int vpr = vecs_per_row(c);
   const long long items = (long long)c.N * ((vpr + 32 * kCombVec - 1) / (32 * kCombVec));
   combine_kernel<T><<<blocks_for(items), kMoveWarps * 32, 0, st>>>(routed, shared, map, gates, y, c.N, c.k,
