@@ -155,6 +155,24 @@ def recorded_traffic(kernel, workload, src_hash):
     return None
 
 
+# ------------------------------------------------------------------------------ multi-rank aggregation
+def max_over_ranks(value: float, world: int, device="cpu") -> float:
+    """The largest of the ranks' values (each rank passes its own); world == 1: value."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(tokens_per_rank: int, world: int, slowest_ms_per_step: float) -> float:
+    """Every rank processes its own batch of tokens_per_rank tokens per step (weak scaling);
+    the job's rate is all ranks' tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / (slowest_ms_per_step / 1e3)
+
+
 # ------------------------------------------------------------------------------ oracle arm
 def oracle_tokens_per_s(cfg, seconds, inputs=None):
     """Time the float64 oracle (as it stands) on consecutive 128-token slices of the
@@ -330,10 +348,7 @@ def main():
         for j, n in enumerate(names):
             stage_ms[n] += ev[j].elapsed_time(ev[j + 1])
         step_ms += ev[0].elapsed_time(ev[6])
-    t_local = torch.tensor([step_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
-    step_ms_max = float(t_local.item()) / args.steps
+    step_ms_max = max_over_ranks(step_ms, world, dev) / args.steps
     for n in names:
         stage_ms[n] /= args.steps
 
@@ -369,11 +384,7 @@ def main():
         y_host.copy_(y, non_blocking=True)
         e2e_ev[i][1].record()
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps], dtype=torch.float64,
-                          device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps, world, dev)
 
     n_e = layout["n_e"].cpu()
     touched = int((n_e > 0).sum())
@@ -390,7 +401,7 @@ def main():
                       "dispatch_combine_grouped_b200/csrc/common.cuh")
     traffic = recorded_traffic("fc1_routed", cfg.name, src)
     tokens_total = cfg.N * world
-    value = tokens_total / (step_ms_max / 1e3)
+    value = whole_job_tokens_per_s(cfg.N, world, step_ms_max)
     gl = 2 if (cfg.dtype == "bf16" and cfg.N > 128 and cfg.d >= 4096) else 1   # pair + tail launches
     launches_per_step = 2 + 3 + 1 + 2 * gl + (2 * gl if S else 0) + 1
 
@@ -419,7 +430,7 @@ def main():
             "fused_ms_per_step": fused_ms,
             "imbalance": {"max_over_mean_n_e": float(n_e.max()) / float(n_e.float().mean()),
                           "experts_empty": int((n_e == 0).sum())},
-            "e2e": {"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s",
+            "e2e": {"value": whole_job_tokens_per_s(cfg.N, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": x.numel() * x.element_size(),
                     "d2h_bytes_per_step": y.numel() * y.element_size()},
             "gpu_launches": launches_per_step * args.steps,

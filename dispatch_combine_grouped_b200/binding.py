@@ -27,7 +27,7 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_con
             "moe_layout_workspace_bytes", "moe_workspace_bytes", "moe_route", "moe_dispatch_layout",
             "moe_dispatch_layout_noalloc",
             "moe_permute", "moe_permute_staged", "moe_grouped_ffn", "moe_expert_fc1", "moe_expert_fc2",
-            "moe_routed_ffn", "moe_shared_ffn", "moe_layer_forward_overlapped",
+            "moe_routed_ffn", "moe_shared_ffn", "moe_layer_forward_overlapped", "moe_selftest_bounded_wait",
             "moe_combine", "moe_combine_staged",
             "moe_layer_forward"]
 
@@ -83,6 +83,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_routed_ffn": (i32, [cfgp, layp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_shared_ffn": (i32, [cfgp, vp, vp, vp, vp, vp, vp]),
         "moe_layer_forward_overlapped": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp, vp]),
+        "moe_selftest_bounded_wait": (i32, [vp, ctypes.c_uint64, vp]),
         "moe_combine": (i32, [cfgp, layp, vp, vp, vp, vp]),
         "moe_combine_staged": (i32, [cfgp, layp, vp, vp, vp, vp, vp]),
         "moe_layer_forward": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp]),
@@ -146,6 +147,11 @@ class Layout:
 
     def as_dict(self):
         return {k: self[k] for k in LAYOUT_FIELDS}
+
+
+def selftest_bounded_wait(status, limit_ns=20_000_000):
+    """Run the bounded-wait self-test kernel; it writes MOE_ERR_TIMEOUT into ``status``."""
+    _check(load().moe_selftest_bounded_wait(_p(status), limit_ns, _stream()), "moe_selftest_bounded_wait")
 
 
 def version() -> int:

@@ -65,17 +65,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait until the phase with the given parity has completed.  Bounded: gives up (returns
 // false) when *abort becomes non-zero or after MOE_WAIT_LIMIT_NS, so that no wait in this
 // library can spin forever.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1; it != 0; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0u) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > MOE_WAIT_LIMIT_NS) return false;
+      if (global_timer_ns() - t0 > limit_ns) return false;
     }
   }
   return false;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_for(bar, parity, abort, MOE_WAIT_LIMIT_NS);
 }
 
 // ------------------------------------------------------------------ TMA

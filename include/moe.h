@@ -284,6 +284,15 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* w
                              moe_stream_t stream);
 
 /*
+ * Self-test of the failure path (no counterpart in the pages).  Launches one thread that
+ * waits, with the library's bounded-wait routine and a limit of `limit_ns` nanoseconds
+ * (1 .. 1e10), on an mbarrier that nothing will ever arrive on.  The wait gives up, the
+ * kernel writes MOE_ERR_TIMEOUT to *dev_status and returns; the context stays usable.
+ * Every wait in the library's kernels behaves this way (limit 2 s).
+ */
+moe_status moe_selftest_bounded_wait(int32_t* dev_status, uint64_t limit_ns, moe_stream_t stream);
+
+/*
  * moe_layer_forward with the shared experts overlapped (the pages' overlap lever:
  * [EP-DeepEP] §7 pipelining; [WideEP] dual-batch overlap; [MoE-IV] §4.2 overlap): the
  * router runs on `stream`; then the shared experts run on `side_stream` while the

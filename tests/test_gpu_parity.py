@@ -254,3 +254,29 @@ def test_overlapped_forward_and_split_ffn_match_bitwise(cfg):
     moe.shared_ffn(cfg, inp["x"], inp["w13"], inp["w2"], h, out)
     torch.cuda.synchronize()
     assert torch.equal(h, res["h"]) and torch.equal(out, res["out"])
+
+
+def test_bounded_wait_gives_up_and_context_stays_usable():
+    """A wait on a barrier that nothing arrives on ends after its limit with
+    MOE_ERR_TIMEOUT in the status word; the GPU keeps working afterwards."""
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    moe.selftest_bounded_wait(status, limit_ns=50_000_000)  # 50 ms
+    torch.cuda.synchronize()
+    assert status.item() == 6  # MOE_ERR_TIMEOUT
+    cfg = small_config("after", N=64, d=64, E=8, S=0, k=2, I=64, P=2)
+    ids = torch.zeros(64, 2, dtype=torch.int32, device="cuda")
+    ids[:, 1] = 1
+    lay = moe.dispatch_layout(cfg, ids)
+    torch.cuda.synchronize()
+    assert lay["n_e"].tolist()[:2] == [64, 64]
+
+
+def test_bad_owner_table_sets_status():
+    cfg = small_config("badown", N=32, d=64, E=8, S=0, k=2, I=64, P=2)
+    ids = torch.stack([torch.arange(32) % 8, (torch.arange(32) + 1) % 8], 1).to(torch.int32).cuda()
+    owner = torch.tensor([0, 1, 0, 1, 0, 1, 5, 1], dtype=torch.int32, device="cuda")  # 5 >= P
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lay = moe.dispatch_layout(cfg, ids, owner, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 5
+    assert sorted(lay["tok2row"].cpu().tolist()) == list(range(64))
