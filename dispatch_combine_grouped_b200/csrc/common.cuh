@@ -136,6 +136,21 @@ __device__ __forceinline__ uint64_t smem_desc_k128(uint32_t saddr) {
   return d;
 }
 
+// The same for rows of SWB bytes (128, 64 or 32) with the matching swizzle: what TMA
+// writes for a box whose inner extent is SWB bytes; 8-row groups 8*SWB bytes apart.
+template <int SWB>
+__device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr) {
+  static_assert(SWB == 128 || SWB == 64 || SWB == 32, "swizzle width");
+  constexpr uint64_t layout = SWB == 128 ? 2u : (SWB == 64 ? 4u : 6u);
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)((8u * SWB) >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= layout << 61;
+  return d;
+}
+
 // Instruction descriptor: D fp32, A and B bf16, both K-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)                         // D format: f32

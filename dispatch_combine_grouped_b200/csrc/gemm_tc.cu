@@ -32,7 +32,10 @@
 namespace moe {
 
 constexpr int BM = 128;
-constexpr int BK = 64;
+constexpr int BK = 64;  // k per stage of the pair kernel and the router; FC tiles use MOE_GEMM_BK
+#ifndef MOE_GEMM_BK
+#define MOE_GEMM_BK 64
+#endif
 constexpr int kThreads = 192;
 constexpr int kMaxGroupsGemm = kMaxE + kMaxShared;
 
@@ -40,10 +43,16 @@ struct SmemPlan {
   int a_bytes, b_bytes, stages, total;
 };
 
-template <int BN, int STAGES>
+// barriers: full/empty per stage, 2 tfull, 2 tempty, drain, then TMEM holder + abort flag
+template <int STAGES>
+__host__ __device__ constexpr int barrier_bytes() {
+  return ((2 * STAGES + 5) * 8 + 8 + 15) & ~15;
+}
+
+template <int BN, int STAGES, int BKT>
 __host__ __device__ constexpr int smem_bytes_for() {
   // 1 KB alignment slack + stages + barriers/flags + group tables
-  return 1024 + STAGES * (BM * BK * 2 + BN * BK * 2) + 256 + 4 * (4 * kMaxGroupsGemm + 8);
+  return 1024 + STAGES * (BM * BKT * 2 + BN * BKT * 2) + barrier_bytes<STAGES>() + 4 * (4 * kMaxGroupsGemm + 8);
 }
 
 struct TileDesc {
@@ -67,12 +76,12 @@ __device__ __forceinline__ TileDesc decode_tile(int t, const int* prefix, int G,
   return d;
 }
 
-template <int BN, int MODE, int STAGES>
+template <int BN, int MODE, int STAGES, int BKT>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
-  constexpr int A_BYTES = BM * BK * 2;
-  constexpr int B_BYTES = BN * BK * 2;
+  constexpr int A_BYTES = BM * BKT * 2;
+  constexpr int B_BYTES = BN * BKT * 2;
   constexpr int HALF_B = B_BYTES / 2;
   constexpr uint32_t TMEM_COLS = 2 * BN;  // BN is a power of two >= 32
   constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
@@ -89,7 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
-  int* s_prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + 256);
+  int* s_prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + barrier_bytes<STAGES>());
   int* s_arow = s_prefix + (kMaxGroupsGemm + 1);
   int* s_orow = s_arow + kMaxGroupsGemm;
   int* s_rows = s_orow + kMaxGroupsGemm;
@@ -164,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_holder;
   const int n_tiles = (MODE == MODE_FC1) ? (p.n_out + BN / 2 - 1) / (BN / 2) : (p.n_out + BN - 1) / BN;
   const int total = s_prefix[G] * n_tiles;
-  const int num_kb = (p.K + BK - 1) / BK;
+  const int num_kb = (p.K + BKT - 1) / BKT;
   volatile int* abort_v = abort_flag;
 
   if (warp == 0) {
@@ -193,9 +202,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[stage], TX_BYTES);
-          tma_load_2d(sA + stage * A_BYTES, mapA, &full[stage], kb * BK, a_row);
-          tma_load_3d(sB + stage * B_BYTES, &tmB, &full[stage], kb * BK, b_row0, gz);
-          tma_load_3d(sB + stage * B_BYTES + HALF_B, &tmB, &full[stage], kb * BK, b_row1, gz);
+          tma_load_2d(sA + stage * A_BYTES, mapA, &full[stage], kb * BKT, a_row);
+          tma_load_3d(sB + stage * B_BYTES, &tmB, &full[stage], kb * BKT, b_row0, gz);
+          tma_load_3d(sB + stage * B_BYTES + HALF_B, &tmB, &full[stage], kb * BKT, b_row1, gz);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -242,8 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            umma_bf16(d_tmem, smem_desc_k128(a_addr + kk * 32), smem_desc_k128(b_addr + kk * 32), IDESC,
+          for (int kk = 0; kk < BKT / 16; ++kk) {
+            umma_bf16(d_tmem, smem_desc_kmajor<BKT * 2>(a_addr + kk * 32), smem_desc_kmajor<BKT * 2>(b_addr + kk * 32),
+                      IDESC,
                       (kb | kk) != 0 ? 1u : 0u);
           }
           any = true;
@@ -402,29 +412,33 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// 2D bf16 map over [rows, K] (K contiguous), box [128 rows, 64 cols], 128B swizzle.
-bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K) {
+static CUtensorMapSwizzle swizzle_for(int box_k) {
+  return box_k == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : (box_k == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
+// 2D bf16 map over [rows, K] (K contiguous), box [128 rows, box_k cols], swizzle = 2*box_k bytes.
+bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K, int box_k) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)(rows > 0 ? rows : 1)};
   cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  cuuint32_t box[2] = {BK, BM};
+  cuuint32_t box[2] = {(cuuint32_t)box_k, BM};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(box_k), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3D bf16 map over [G, R, K], box [1, box_rows, 64], 128B swizzle.
-bool make_map_b(CUtensorMap* m, const void* base, long long G, long long R, long long K, int box_rows) {
+// 3D bf16 map over [G, R, K], box [1, box_rows, box_k], swizzle = 2*box_k bytes.
+bool make_map_b(CUtensorMap* m, const void* base, long long G, long long R, long long K, int box_rows, int box_k) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)R, (cuuint64_t)G};
   cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)(R * K * 2)};
-  cuuint32_t box[3] = {BK, (cuuint32_t)box_rows, 1};
+  cuuint32_t box[3] = {(cuuint32_t)box_k, (cuuint32_t)box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(box_k), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -439,14 +453,14 @@ int sm_count() {
   return n;
 }
 
-template <int BN, int MODE>
+template <int BN, int MODE, int BKT>
 static cudaError_t launch_bn(const GemmArgs& g, const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                              long long max_tiles, cudaStream_t st) {
-  // as many stages as fit in ~192 KB, at most 8 (narrow router tiles get deeper rings)
-  constexpr int STAGE_KB = (BM * BK * 2 + BN * BK * 2) / 1024;
-  constexpr int STAGES = (192 / STAGE_KB) > 8 ? 8 : (192 / STAGE_KB);
-  constexpr int smem = smem_bytes_for<BN, STAGES>();
-  auto kern = tc_gemm_kernel<BN, MODE, STAGES>;
+  // as many stages as fit in ~192 KB, at most 16
+  constexpr int STAGE_B = BM * BKT * 2 + BN * BKT * 2;
+  constexpr int STAGES = (192 * 1024 / STAGE_B) > 16 ? 16 : (192 * 1024 / STAGE_B);
+  constexpr int smem = smem_bytes_for<BN, STAGES, BKT>();
+  auto kern = tc_gemm_kernel<BN, MODE, STAGES, BKT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   long long grid = sm_count();
@@ -471,10 +485,11 @@ cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStre
   } else {
     BN = 256;
   }
+  const int bk = g.mode == MODE_ROUTER ? BK : MOE_GEMM_BK;
   CUtensorMap a0, a1, b;
-  if (!make_map_a(&a0, g.a0, a0_rows, g.K)) return cudaErrorInvalidValue;
-  if (!make_map_a(&a1, g.a1 ? g.a1 : g.a0, g.a1 ? a1_rows : a0_rows, g.K)) return cudaErrorInvalidValue;
-  if (!make_map_b(&b, g.b, g.g0 + g.G, g.b_rows, g.K, BN / 2)) return cudaErrorInvalidValue;
+  if (!make_map_a(&a0, g.a0, a0_rows, g.K, bk)) return cudaErrorInvalidValue;
+  if (!make_map_a(&a1, g.a1 ? g.a1 : g.a0, g.a1 ? a1_rows : a0_rows, g.K, bk)) return cudaErrorInvalidValue;
+  if (!make_map_b(&b, g.b, g.g0 + g.G, g.b_rows, g.K, BN / 2, bk)) return cudaErrorInvalidValue;
   // upper bound on tiles: every group adds at most one partial row block
   long long rows_total = launch_rows(g);
   long long blocks = (rows_total + BM - 1) / BM + g.G;
@@ -482,15 +497,15 @@ cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStre
   long long max_tiles = blocks * n_tiles;
   switch (g.mode) {
     case MODE_FC1:
-      return launch_bn<256, MODE_FC1>(g, a0, a1, b, max_tiles, st);
+      return launch_bn<256, MODE_FC1, MOE_GEMM_BK>(g, a0, a1, b, max_tiles, st);
     case MODE_FC2:
-      return launch_bn<256, MODE_FC2>(g, a0, a1, b, max_tiles, st);
+      return launch_bn<256, MODE_FC2, MOE_GEMM_BK>(g, a0, a1, b, max_tiles, st);
     default:
       switch (BN) {
-        case 32: return launch_bn<32, MODE_ROUTER>(g, a0, a1, b, max_tiles, st);
-        case 64: return launch_bn<64, MODE_ROUTER>(g, a0, a1, b, max_tiles, st);
-        case 128: return launch_bn<128, MODE_ROUTER>(g, a0, a1, b, max_tiles, st);
-        case 256: return launch_bn<256, MODE_ROUTER>(g, a0, a1, b, max_tiles, st);
+        case 32: return launch_bn<32, MODE_ROUTER, BK>(g, a0, a1, b, max_tiles, st);
+        case 64: return launch_bn<64, MODE_ROUTER, BK>(g, a0, a1, b, max_tiles, st);
+        case 128: return launch_bn<128, MODE_ROUTER, BK>(g, a0, a1, b, max_tiles, st);
+        case 256: return launch_bn<256, MODE_ROUTER, BK>(g, a0, a1, b, max_tiles, st);
         default: return cudaErrorInvalidValue;
       }
   }

@@ -86,7 +86,9 @@ cudaError_t launch_tc_gemm_pair(const GemmArgs& g, int a0_rows, int a1_rows, cud
 cudaError_t launch_simt_gemm(const GemmArgs& g, cudaStream_t st);
 
 int sm_count();
-bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K);
-bool make_map_b(CUtensorMap* m, const void* base, long long G, long long R, long long K, int box_rows);
+// TMA maps for bf16 K-major operands; box_k (64, 32 or 16) selects the 128/64/32-byte swizzle
+bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K, int box_k = 64);
+bool make_map_b(CUtensorMap* m, const void* base, long long G, long long R, long long K, int box_rows,
+                int box_k = 64);
 
 }  // namespace moe

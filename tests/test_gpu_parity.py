@@ -280,3 +280,30 @@ def test_bad_owner_table_sets_status():
     torch.cuda.synchronize()
     assert status.item() == 5
     assert sorted(lay["tok2row"].cpu().tolist()) == list(range(64))
+
+
+@pytest.mark.parametrize("cfg", [SMALL[1], SMALL[5]], ids=_ids([SMALL[1], SMALL[5]]))
+def test_forward_captures_into_cuda_graph(cfg):
+    """moe_layer_forward launches only device work on its stream (no host sync, no
+    allocation), so it captures into a CUDA graph; replays give the eager result."""
+    inp = gpu_inputs(cfg)
+    ws = moe.alloc_workspace(cfg)
+    y_eager = moe.layer_forward(cfg, inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], inp["w13"],
+                                inp["w2"], ws=ws)
+    torch.cuda.synchronize()
+    y = torch.empty_like(y_eager)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        moe.layer_forward(cfg, inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], inp["w13"], inp["w2"],
+                          y=y, ws=ws)  # warm-up on the capture stream
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            moe.layer_forward(cfg, inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], inp["w13"],
+                              inp["w2"], y=y, ws=ws)
+    for _ in range(2):
+        y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_eager)
