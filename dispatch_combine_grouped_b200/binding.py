@@ -35,7 +35,7 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_con
 class CConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ["N", "d", "E", "k", "I", "n_shared", "P", "n_groups", "topk_groups", "score",
-                 "renormalize", "dtype"]]
+                 "renormalize", "dtype", "bias_mode"]]
 
 
 LAYOUT_FIELDS = ["n_e", "expert_off", "C", "send_off", "recv_off", "tok2send", "send2row", "ret2tok",
@@ -115,8 +115,10 @@ def c_config(cfg) -> CConfig:
     score = cfg.score if isinstance(cfg.score, int) else \
         {"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID}[cfg.score]
     dtype = cfg.dtype if isinstance(cfg.dtype, int) else {"f32": MOE_F32, "bf16": MOE_BF16}[cfg.dtype]
+    bias_mode = getattr(cfg, "bias_mode", "logits")
+    bias_mode = bias_mode if isinstance(bias_mode, int) else {"logits": 0, "selection": 1}[bias_mode]
     return CConfig(cfg.N, cfg.d, cfg.E, cfg.k, cfg.I, cfg.S, cfg.P, cfg.n_groups, cfg.topk_groups,
-                   score, int(bool(cfg.renormalize)), dtype)
+                   score, int(bool(cfg.renormalize)), dtype, bias_mode)
 
 
 def _p(t):

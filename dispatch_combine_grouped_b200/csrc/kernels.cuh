@@ -25,7 +25,9 @@ cudaError_t launch_layout(const moe_config& cfg, const int32_t* owner, const int
                           int32_t* status, void* ws, cudaStream_t st);
 
 // ---- route.cu : top-k selection and gates from fp32 logits
-cudaError_t launch_topk(const moe_config& cfg, const float* logits, int32_t* ids, float* w, cudaStream_t st);
+// gate_bias: NULL, or the router bias to subtract from the selection keys before gating
+cudaError_t launch_topk(const moe_config& cfg, const float* logits, const float* gate_bias, int32_t* ids, float* w,
+                        cudaStream_t st);
 
 // ---- movement.cu : permute / combine and their two-hop (staged) forms
 cudaError_t launch_permute(const moe_config& cfg, const moe_layout& L, const void* x, void* x_perm,

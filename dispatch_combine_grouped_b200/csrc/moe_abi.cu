@@ -35,8 +35,9 @@ moe_status check_config(const moe_config* c) {
   if ((long long)c->k > (long long)c->topk_groups * (c->E / c->n_groups))
     return fail(MOE_ERR_INVALID_ARG, "k exceeds the experts of the kept groups");
   if ((c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID) ||
-      (c->dtype != MOE_F32 && c->dtype != MOE_BF16) || (c->renormalize != 0 && c->renormalize != 1))
-    return fail(MOE_ERR_INVALID_ARG, "score, dtype or renormalize out of range");
+      (c->dtype != MOE_F32 && c->dtype != MOE_BF16) || (c->renormalize != 0 && c->renormalize != 1) ||
+      (c->bias_mode != MOE_BIAS_LOGITS && c->bias_mode != MOE_BIAS_SELECTION))
+    return fail(MOE_ERR_INVALID_ARG, "score, dtype, renormalize or bias_mode out of range");
   if (c->k > kMaxK || c->E > kMaxE || c->P > kMaxP || c->n_groups > kMaxGroups ||
       c->topk_groups > kMaxTopkGroups || c->n_shared > kMaxShared)
     return fail(MOE_ERR_UNSUPPORTED, "k <= 8, E <= 256, P <= 32, n_groups <= 32, topk_groups <= 8, S <= 8");
@@ -129,7 +130,8 @@ moe_status route_impl(const moe_config& c, const void* x, const void* w_gate, co
   g.b_rows = c.E;
   cudaError_t e = c.dtype == MOE_BF16 ? launch_tc_gemm(g, c.N, c.N, st) : launch_simt_gemm(g, st);
   if (e != cudaSuccess) return cuda_status(e, "router GEMM");
-  return cuda_status(launch_topk(c, logits, ids, w, st), "top-k");
+  return cuda_status(launch_topk(c, logits, c.bias_mode == MOE_BIAS_SELECTION ? bias : nullptr, ids, w, st),
+                     "top-k");
 }
 
 GemmArgs fc1_args(const moe_config& c, const moe_layout& L, const void* x_perm, const void* x, const void* w13,

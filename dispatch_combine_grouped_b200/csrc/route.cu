@@ -17,6 +17,7 @@ namespace moe {
 
 struct TopkArgs {
   const float* logits;
+  const float* gate_bias;  // correction bias: selection on logits, gates on logits - bias
   int32_t* ids;
   float* w;
   int N, E, k, n_groups, topk_groups, score, renorm;
@@ -121,6 +122,18 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs p) {
     }
   }
 
+  // gate inputs: the selection keys, or with a correction bias the unbiased logits
+  if (p.gate_bias) {
+#pragma unroll
+    for (int q = 0; q < kLanesE; ++q) {
+      const int col = lane + 32 * q;
+      if (col < p.E) v[q] -= p.gate_bias[col];
+    }
+#pragma unroll
+    for (int s = 0; s < kMaxK; ++s)
+      if (s < p.k) sel_v[s] -= p.gate_bias[sel_i[s]];
+  }
+
   // softmax denominator over all E (only needed without renormalisation)
   float gmax = -INFINITY, den_all = 0.f;
   if (p.score == MOE_SCORE_SOFTMAX && !p.renorm) {
@@ -134,6 +147,10 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs p) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) den_all += __shfl_xor_sync(0xffffffffu, den_all, o);
   }
+  float smax = -INFINITY;  // max of the chosen gate inputs (softmax renormalised)
+#pragma unroll
+  for (int s = 0; s < kMaxK; ++s)
+    if (s < p.k) smax = fmaxf(smax, sel_v[s]);
 
   if (lane == 0) {
     float g[kMaxK];
@@ -143,7 +160,7 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs p) {
       g[s] = 0.f;
       if (s < p.k) {
         if (p.score == MOE_SCORE_SOFTMAX) {
-          g[s] = p.renorm ? expf(sel_v[s] - sel_v[0]) : expf(sel_v[s] - gmax) / den_all;
+          g[s] = p.renorm ? expf(sel_v[s] - smax) : expf(sel_v[s] - gmax) / den_all;
         } else {
           g[s] = 1.0f / (1.0f + expf(-sel_v[s]));
         }
@@ -160,10 +177,12 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs p) {
   }
 }
 
-cudaError_t launch_topk(const moe_config& cfg, const float* logits, int32_t* ids, float* w, cudaStream_t st) {
+cudaError_t launch_topk(const moe_config& cfg, const float* logits, const float* gate_bias, int32_t* ids, float* w,
+                        cudaStream_t st) {
   if (cfg.N == 0) return cudaSuccess;
   TopkArgs p;
   p.logits = logits;
+  p.gate_bias = gate_bias;
   p.ids = ids;
   p.w = w;
   p.N = cfg.N;

@@ -58,6 +58,10 @@ typedef enum {
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score;
+/* MOE_BIAS_LOGITS: z = x W_g^T + b feeds both the selection and the gates.
+ * MOE_BIAS_SELECTION: a correction bias ([MoE-IV] §4.2 "correction_bias"): the selection
+ * uses z + b, the gate weights use the unbiased z of the chosen experts. */
+typedef enum { MOE_BIAS_LOGITS = 0, MOE_BIAS_SELECTION = 1 } moe_bias_mode;
 
 /* Shape and routing rule of one layer. */
 typedef struct {
@@ -73,6 +77,7 @@ typedef struct {
   int32_t score;       /* moe_score: softmax over E, or per-expert sigmoid */
   int32_t renormalize; /* 1: gates renormalised to sum 1 over the chosen k */
   int32_t dtype;       /* moe_dtype */
+  int32_t bias_mode;   /* moe_bias_mode: how the router bias (when given) is used */
 } moe_config;
 
 /*
@@ -128,7 +133,7 @@ size_t moe_workspace_bytes(const moe_config* cfg);
  * Router and top-k selection ([DSMoE] naive forward steps 1-2; [EP-DeepEP] §2;
  * [WideEP] "Group-limited routing"; renormalisation as named in [MoE-IV] §4.2).
  *   x        [N, d]  dtype      w_gate [E, d] dtype (one row per expert)
- *   bias     [E] fp32 or NULL   added to the logits before selection and gating
+ *   bias     [E] fp32 or NULL   added to the logits (see moe_bias_mode)
  *   logits   [N, E] fp32, required: written with z = x W_g^T (+ b); the selection
  *            reads back exactly these fp32 values
  *   topk_ids [N, k] int32: slot 0 = largest logit; ties go to the lower expert index.
@@ -137,6 +142,7 @@ size_t moe_workspace_bytes(const moe_config* cfg);
  *   topk_w   [N, k] fp32 gate weights:
  *            softmax: exp(z_e - m) / sum_{all E} exp(z - m), or over the chosen k when
  *            renormalize; sigmoid: 1/(1+exp(-z_e)), divided by their sum when renormalize.
+ *            With MOE_BIAS_SELECTION, z here is the unbiased x W_g^T (logits holds z + b).
  */
 moe_status moe_route(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
                      float* logits, int32_t* topk_ids, float* topk_w, moe_stream_t stream);

@@ -42,6 +42,7 @@ class MoEConfig:
     dtype: str = "bf16"      # "f32" | "bf16"
     bias: str = "none"       # "none" | "zipf"
     bias_alpha: float = 0.0  # b_e = alpha * ln(1 / rank_e), rank_e = e + 1
+    bias_mode: str = "logits"  # "logits": bias in selection and gates | "selection": selection only
     owner: str = "contiguous"  # "contiguous" | "hot4"
 
     @property

@@ -39,6 +39,7 @@ Readings where the pages are silent (each is listed in the design notes):
     gives the expert-local order; owners' buffers follow each other in owner order.
   * Return row = send slot (the combine all-to-all is the inverse transpose).
   * Shared experts are added with weight 1.
+  * A correction bias (bias_mode "selection") shifts the selection keys only.
 """
 from __future__ import annotations
 
@@ -168,6 +169,15 @@ def gate_weights(logits, ids, score: str = "softmax", renormalize: bool = True) 
             return s / s.sum(axis=1, keepdims=True)
         return s
     raise ValueError(score)
+
+
+def gate_logits(cfg, x, w_gate, bias):
+    """Logits the gate weights are computed from: x W_g^T + b, or with a correction bias
+    (bias_mode "selection", named as router correction_bias in [MoE-IV] §4.2) the
+    unbiased x W_g^T — the bias then only steers which experts are selected."""
+    if getattr(cfg, "bias_mode", "logits") == "selection":
+        return router_logits(x, w_gate, None)
+    return router_logits(x, w_gate, bias)
 
 
 # ---------------------------------------------------------------------------------------
@@ -324,7 +334,7 @@ def moe_layer(cfg, x, w_gate, bias, w13, w2, expert_owner=None, select_keys=None
     z = router_logits(x, w_gate, bias)
     keys = z if select_keys is None else np.asarray(select_keys)
     ids = select_experts(keys, cfg.k, cfg.n_groups, cfg.topk_groups)
-    g = gate_weights(z, ids, cfg.score, cfg.renormalize)
+    g = gate_weights(gate_logits(cfg, x, w_gate, bias), ids, cfg.score, cfg.renormalize)
     lay = dispatch_layout(ids, cfg.E, cfg.P, expert_owner, cfg.S)
     xp = permute(x, lay, cfg.k)
     o = experts_on_rows(xp, lay, w13, w2, cfg.E)

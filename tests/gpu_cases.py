@@ -68,12 +68,13 @@ def run_steps(cfg, inp, status=None):
 def check_route(cfg, inp, res, logit_tol):
     """Stages (i)-(iii) of the near-tie protocol."""
     z64 = O.router_logits(inp["x"], inp["w_gate"], inp["bias"])
+    zgate = O.gate_logits(cfg, inp["x"], inp["w_gate"], inp["bias"])
     zg = res["logits"].cpu().numpy()
     assert np.abs(zg.astype(np.float64) - z64).max() <= logit_tol, "router logits"
     ids_ref = O.select_experts(zg, cfg.k, cfg.n_groups, cfg.topk_groups)   # on the GPU's fp32 logits
     ids = res["ids"].cpu().numpy().astype(np.int64)
     assert np.array_equal(ids, ids_ref), "top-k ids (selection on the same fp32 logits)"
-    g_ref = O.gate_weights(z64, ids, cfg.score, cfg.renormalize)
+    g_ref = O.gate_weights(zgate, ids, cfg.score, cfg.renormalize)
     np.testing.assert_allclose(res["w"].cpu().numpy(), g_ref, rtol=0, atol=1e-5)
     # report how many tokens the oracle's own fp64 selection would route differently
     ids64 = O.select_experts(z64, cfg.k, cfg.n_groups, cfg.topk_groups)

@@ -40,7 +40,7 @@ def test_full_config(name):
     assert torch.equal(xp, inp["x"][torch.tensor(a_s // cfg.k, device="cuda")]), "permute rows"
 
     tokens = np.sort(rng.choice(cfg.N, size=SAMPLE_TOKENS[name], replace=False))
-    z64 = O.router_logits(inp["x"][torch.tensor(tokens, device="cuda")], inp["w_gate"], inp["bias"])
+    z64 = O.gate_logits(cfg, inp["x"][torch.tensor(tokens, device="cuda")], inp["w_gate"], inp["bias"])
     g64 = O.gate_weights(z64, ids[tokens], cfg.score, cfg.renormalize)
     gates = np.zeros((cfg.N, cfg.k))
     gates[tokens] = g64

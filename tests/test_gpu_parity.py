@@ -30,6 +30,8 @@ SMALL = [
                  topk_groups=3, score="sigmoid"),
     small_config("s_bf16_tiny_n", cfg_id=73, N=7, d=64, E=8, S=0, k=2, I=64, P=2),
     small_config("s_bf16_pairs", cfg_id=79, N=700, d=4096, E=8, S=1, k=2, I=200, P=4),
+    small_config("s_bf16_corrbias", cfg_id=81, N=333, d=256, E=32, S=1, k=4, I=128, P=8, n_groups=8,
+                 topk_groups=3, score="sigmoid", bias="zipf", bias_alpha=0.7, bias_mode="selection"),
     small_config("s_bf16_one_tok", cfg_id=74, N=1, d=128, E=64, S=1, k=6, I=96, P=8),
     small_config("s_f32", cfg_id=75, N=129, d=96, E=8, S=1, k=2, I=72, P=4, dtype="f32"),
     small_config("s_f32_grouped", cfg_id=76, N=64, d=64, E=16, S=0, k=4, I=40, P=4, n_groups=4, topk_groups=2,
@@ -55,8 +57,7 @@ def test_small_end_to_end(cfg):
     xp_ref = O.permute(inp["x"], ref, cfg.k)
     assert np.array_equal(O.f64(res["x_perm"]), xp_ref)
     # full oracle on the GPU's routing (gates from the fp64 logits)
-    z64 = O.router_logits(inp["x"], inp["w_gate"], inp["bias"])
-    g64 = O.gate_weights(z64, ids, cfg.score, cfg.renormalize)
+    g64 = O.gate_weights(O.gate_logits(cfg, inp["x"], inp["w_gate"], inp["bias"]), ids, cfg.score, cfg.renormalize)
     o_ref = O.experts_on_rows(xp_ref, ref, inp["w13"], inp["w2"], cfg.E)
     A = cfg.N * cfg.k
     o_gpu = O.f64(res["out"][:A])

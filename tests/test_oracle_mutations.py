@@ -100,3 +100,9 @@ def test_expert_order_by_id_only_is_caught(monkeypatch):
         return lay
     monkeypatch.setattr(O, "dispatch_layout", by_id)
     _fails(pins.check_layout_naive_ranks, 2)
+
+
+def test_bias_leaking_into_gates_is_caught(monkeypatch):
+    # a correction bias that also shifts the gates
+    monkeypatch.setattr(O, "gate_logits", lambda cfg, x, w_gate, bias: O.router_logits(x, w_gate, bias))
+    _fails(pins.check_correction_bias)

@@ -337,3 +337,26 @@ def test_imbalance_and_page_arithmetic():
     # tiny config: mean n_e = N k / E
     lay = O.dispatch_layout(np.arange(512).reshape(256, 2) % 8, E=8, P=2)
     assert lay["n_e"].mean() == 256 * 2 / 8
+
+
+def check_correction_bias():
+    """The bias steers the selection only: keys z + b pick (1, 0) over z's own (0, 2);
+    the renormalised softmax gates then come from z: (e^0, e^1) / (e^0 + e^1)."""
+    cfg = MoEConfig("cb", 0, N=1, d=3, E=3, S=0, k=2, I=8, P=1, score="softmax", renormalize=True,
+                    dtype="f32", bias="zipf", bias_mode="selection")
+    x = np.array([[1.0, 0.0, 0.5]])
+    w_gate = np.eye(3)                                     # z = x
+    bias = np.array([0.0, 2.0, 0.0])
+    keys = O.router_logits(x, w_gate, bias)
+    ids = O.select_experts(keys, 2)
+    assert ids.tolist() == [[1, 0]]
+    g = O.gate_weights(O.gate_logits(cfg, x, w_gate, bias), ids, cfg.score, cfg.renormalize)
+    e = math.e
+    np.testing.assert_allclose(g, [[1 / (1 + e), e / (1 + e)]], atol=1e-15)
+    # the default mode feeds the bias to the gates too
+    g2 = O.gate_weights(O.gate_logits(cfg.replace(bias_mode="logits"), x, w_gate, bias), ids, "softmax", True)
+    np.testing.assert_allclose(g2, [[e ** 2 / (e ** 2 + e), e / (e ** 2 + e)]], atol=1e-15)
+
+
+def test_correction_bias_closed_form():
+    check_correction_bias()
