@@ -106,3 +106,34 @@ def test_bias_leaking_into_gates_is_caught(monkeypatch):
     # a correction bias that also shifts the gates
     monkeypatch.setattr(O, "gate_logits", lambda cfg, x, w_gate, bias: O.router_logits(x, w_gate, bias))
     _fails(pins.check_correction_bias)
+
+
+# ---- EPLB oracle (redundant expert slots)
+import tests.test_eplb_oracle as eplb_pins
+from oracle import eplb as EP
+
+
+def test_copies_to_the_coldest_expert_are_caught(monkeypatch):
+    def coldest(load, R):
+        load = np.asarray(load, dtype=np.int64)
+        r = np.ones(len(load), dtype=np.int64)
+        for _ in range(R):
+            r[int(np.argmin(load / r))] += 1
+        return r
+    monkeypatch.setattr(EP, "replica_counts", coldest)
+    _fails(eplb_pins.check_copy_counts_optimal, 3, 2, np.array([30, 5, 1]))
+    _fails(eplb_pins.check_worked_example)
+
+
+def test_replica_rank_off_by_one_is_caught(monkeypatch):
+    def shifted(ids, replica_off, replica_slots):
+        ids = np.asarray(ids, dtype=np.int64)
+        flat = ids.reshape(-1)
+        out = np.empty_like(flat)
+        for e in range(len(replica_off) - 1):
+            rows = np.flatnonzero(flat == e)
+            r = replica_off[e + 1] - replica_off[e]
+            out[rows] = np.asarray(replica_slots)[replica_off[e] + (np.arange(len(rows)) + 1) % r]
+        return out.reshape(ids.shape)
+    monkeypatch.setattr(EP, "assign", shifted)
+    _fails(eplb_pins.check_worked_example)
