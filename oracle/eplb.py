@@ -22,18 +22,17 @@ in the design notes), in the plainest form that meets the stated goal:
      turn goes to the expert with the largest load per copy, load_e / r_e (ties to the
      lower expert id).  Giving the next copy to the current maximum is what lowers the
      maximum, so this minimises max_e load_e / r_e.
-  2. Placement: the E + R copies, each carrying load_e / r_e, are taken in descending
-     load order (ties: lower expert id, then lower copy number) and each goes to the
-     owner with free room (E_local slots per owner) that holds no copy of the same
-     expert yet if there is one, then the smallest load so far, then the lower owner.
+  2. Placement: copy c of expert e carries the rows reading 4 gives it,
+     floor(load_e / r_e) + (1 if c < load_e mod r_e else 0).  The E + R copies are taken
+     in descending load order (ties: lower expert id, then lower copy number) and each
+     goes to the owner with free room (E_local slots per owner) that holds no copy of the
+     same expert yet if there is one, then the smallest load so far, then the lower owner.
   3. Slot ids: owner j holds slots [j E_local, (j+1) E_local), in ascending (expert id,
-     copy number) order; a logical expert's replicas are listed in ascending slot id.
+     copy number) order; a logical expert's replicas are listed by copy number.
   4. Assignment: the q-th assignment of logical expert e in ascending a = t k + slot order
      goes to replica q mod r_e, so the copies of e share its n_e to within one row.
 """
 from __future__ import annotations
-
-import math
 
 import numpy as np
 
@@ -52,9 +51,14 @@ def replica_counts(load, R: int) -> np.ndarray:
     return r
 
 
+def copy_load(load_e: int, r_e: int, c: int) -> int:
+    """Rows copy c of an expert with load_e rows and r_e copies receives (reading 4)."""
+    return load_e // r_e + (1 if c < load_e % r_e else 0)
+
+
 def plan(load, R: int, P: int) -> dict:
-    """Readings 1-3.  Returns replica_off [E+1], replica_slots [E+R], slot_expert [E+R],
-    slot_owner [E+R] (all int64)."""
+    """Readings 1-3.  Returns copies [E], replica_off [E+1], replica_slots [E+R] (slot of
+    copy c of expert e at replica_off[e] + c), slot_expert [E+R], slot_owner [E+R]."""
     load = np.asarray(load, dtype=np.int64)
     E = len(load)
     S = E + R
@@ -62,27 +66,15 @@ def plan(load, R: int, P: int) -> dict:
         raise ValueError("E + R must be a multiple of P")
     per = S // P
     r = replica_counts(load, R)
-    # copies as (load numerator, denominator, expert, copy number); order by load desc
-    copies = [(int(load[e]), int(r[e]), e, c) for e in range(E) for c in range(r[e])]
+    copies = [(copy_load(int(load[e]), int(r[e]), c), e, c) for e in range(E) for c in range(r[e])]
+    # descending load, then ascending expert id, then ascending copy number
+    order = sorted(copies, key=lambda u: (-u[0], u[1], u[2]))
 
-    def before(u, v):  # u is placed before v
-        lu, lv = u[0] * v[1], v[0] * u[1]
-        if lu != lv:
-            return lu > lv
-        return (u[2], u[3]) < (v[2], v[3])
-
-    order = []
-    for item in copies:  # insertion sort by `before` (n <= 288: plain and exact)
-        pos = len(order)
-        while pos > 0 and before(item, order[pos - 1]):
-            pos -= 1
-        order.insert(pos, item)
-
-    owner_load = [(0, 1)] * P  # fractions as (numerator, denominator)
+    owner_load = [0] * P
     owner_room = [per] * P
     holds = [set() for _ in range(P)]
     owner_of = {}
-    for (num, den, e, c) in order:
+    for (cl, e, c) in order:
         best = -1
         for j in range(P):
             if owner_room[j] == 0:
@@ -95,33 +87,28 @@ def plan(load, R: int, P: int) -> dict:
                 if fresh_j:
                     best = j
                 continue
-            a_num, a_den = owner_load[j]
-            b_num, b_den = owner_load[best]
-            if a_num * b_den < b_num * a_den:
+            if owner_load[j] < owner_load[best]:
                 best = j
         owner_of[(e, c)] = best
-        n0, d0 = owner_load[best]
-        owner_load[best] = (n0 * den + num * d0, d0 * den)
-        g = math.gcd(owner_load[best][0], owner_load[best][1])
-        if g > 1:
-            owner_load[best] = (owner_load[best][0] // g, owner_load[best][1] // g)
+        owner_load[best] += cl
         owner_room[best] -= 1
         holds[best].add(e)
 
     slot_expert = np.empty(S, dtype=np.int64)
     slot_owner = np.empty(S, dtype=np.int64)
-    for j in range(P):
-        mine = sorted((e, c) for (e, c), o in owner_of.items() if o == j)
-        for i, (e, c) in enumerate(mine):
-            slot_expert[j * per + i] = e
-            slot_owner[j * per + i] = j
     replica_off = np.zeros(E + 1, dtype=np.int64)
     replica_off[1:] = np.cumsum(r)
     replica_slots = np.empty(S, dtype=np.int64)
-    for e in range(E):
-        replica_slots[replica_off[e]:replica_off[e + 1]] = np.flatnonzero(slot_expert == e)
+    for j in range(P):
+        mine = sorted((e, c) for (e, c), o in owner_of.items() if o == j)
+        for i, (e, c) in enumerate(mine):
+            slot = j * per + i
+            slot_expert[slot] = e
+            slot_owner[slot] = j
+            replica_slots[replica_off[e] + c] = slot
     return {"replica_off": replica_off, "replica_slots": replica_slots,
-            "slot_expert": slot_expert, "slot_owner": slot_owner, "copies": r}
+            "slot_expert": slot_expert, "slot_owner": slot_owner, "copies": r,
+            "owner_load": np.asarray(owner_load, dtype=np.int64)}
 
 
 def assign(ids, replica_off, replica_slots) -> np.ndarray:

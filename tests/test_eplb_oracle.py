@@ -24,8 +24,8 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "eplb_example.json")
 def check_worked_example():
     g = json.load(open(GOLDEN))
     pl = EP.plan(g["load"], g["R"], g["P"])
-    for key in ("copies", "slot_expert", "slot_owner", "replica_off", "replica_slots"):
-        assert pl[key].tolist() == g[key], key
+    for key in ("copies", "owner_loads", "slot_expert", "slot_owner", "replica_off", "replica_slots"):
+        assert pl[key if key != "owner_loads" else "owner_load"].tolist() == g[key], key
     assert EP.assign(g["ids"], pl["replica_off"], pl["replica_slots"]).tolist() == g["phys_ids"]
 
 
@@ -64,10 +64,11 @@ def test_plan_is_a_valid_placement():
         assert (pl["slot_owner"] == np.arange(S) // per).all()
         for e in range(E):
             slots = pl["replica_slots"][pl["replica_off"][e]:pl["replica_off"][e + 1]]
-            assert (np.diff(slots) > 0).all() and (pl["slot_expert"][slots] == e).all()
+            assert len(set(slots.tolist())) == len(slots) and (pl["slot_expert"][slots] == e).all()
             if pl["copies"][e] <= P:  # copies of one expert land on distinct owners here
                 assert len(set(pl["slot_owner"][slots].tolist())) == len(slots)
         assert sorted(pl["replica_slots"].tolist()) == list(range(S))
+        assert pl["owner_load"].sum() == load.sum()
 
 
 def test_identity_replicas_are_the_plain_routing():
@@ -89,6 +90,10 @@ def test_assignment_keeps_the_expert_and_splits_its_load():
     for e in range(E):
         per = n_slot[pl["replica_slots"][pl["replica_off"][e]:pl["replica_off"][e + 1]]]
         assert per.sum() == load[e] and per.max() - per.min() <= 1
+        # the plan's copy loads are exactly the rows the assignment delivers
+        assert per.tolist() == [EP.copy_load(load[e], len(per), c) for c in range(len(per))]
+    n_owner = np.bincount(pl["slot_owner"][phys.reshape(-1)], minlength=P)
+    assert n_owner.tolist() == pl["owner_load"].tolist()
 
 
 def check_layer_unchanged_by_replicas(R):
