@@ -29,7 +29,8 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_con
             "moe_permute", "moe_permute_staged", "moe_grouped_ffn", "moe_expert_fc1", "moe_expert_fc2",
             "moe_routed_ffn", "moe_shared_ffn", "moe_layer_forward_overlapped", "moe_selftest_bounded_wait",
             "moe_combine", "moe_combine_staged",
-            "moe_layer_forward"]
+            "moe_layer_forward", "moe_eplb_plan", "moe_eplb_workspace_bytes", "moe_eplb_assign",
+            "moe_eplb_place_weights"]
 
 
 class CConfig(ctypes.Structure):
@@ -87,6 +88,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_combine": (i32, [cfgp, layp, vp, vp, vp, vp]),
         "moe_combine_staged": (i32, [cfgp, layp, vp, vp, vp, vp, vp]),
         "moe_layer_forward": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp]),
+        "moe_eplb_plan": (i32, [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_eplb_workspace_bytes": (sz, [cfgp]),
+        "moe_eplb_assign": (i32, [cfgp, vp, vp, vp, i32, vp, vp, vp, sz, vp]),
+        "moe_eplb_place_weights": (i32, [vp, i32, i32, i32, sz, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -337,3 +342,59 @@ def layer_forward(cfg, x, w_gate, bias, expert_owner, w13, w2, y=None, ws=None, 
                                     _p(w2), _p(y), lay, _p(status), _p(ws), ws.numel(), _stream()),
            "moe_layer_forward")
     return y
+
+
+# ---------------------------------------------------------------- redundant expert slots (EPLB)
+def _np_ptr(a):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def eplb_plan(load_per_expert, R: int, P: int) -> dict:
+    """moe_eplb_plan (host): copies per expert, slot tables and planned owner loads.
+    Returns int32/int64 NumPy arrays: copies [E], replica_off [E+1], replica_slots [E+R],
+    slot_expert [E+R], slot_owner [E+R], owner_load [P]."""
+    import numpy as np
+    load_np = np.ascontiguousarray(np.asarray(load_per_expert, dtype=np.int64))
+    E = len(load_np)
+    out = {"copies": np.zeros(E, np.int32), "replica_off": np.zeros(E + 1, np.int32),
+           "replica_slots": np.zeros(E + R, np.int32), "slot_expert": np.zeros(E + R, np.int32),
+           "slot_owner": np.zeros(E + R, np.int32), "owner_load": np.zeros(P, np.int64)}
+    _check(load().moe_eplb_plan(E, R, P, _np_ptr(load_np), _np_ptr(out["copies"]), _np_ptr(out["replica_off"]),
+                                _np_ptr(out["replica_slots"]), _np_ptr(out["slot_expert"]),
+                                _np_ptr(out["slot_owner"]), _np_ptr(out["owner_load"])), "moe_eplb_plan")
+    return out
+
+
+def physical_config(cfg, R: int):
+    """The configuration of the E + R physical slots (same sizes, plain top-k grouping:
+    the slots are never routed to directly)."""
+    import dataclasses
+    return dataclasses.replace(cfg, E=cfg.E + R, n_groups=1, topk_groups=1)
+
+
+def eplb_assign(cfg, topk_ids, replica_off, replica_slots, n_slots: int, status=None, out=None, ws=None):
+    """moe_eplb_assign: physical slot ids [N, k] int32 for the logical ids (device)."""
+    c = c_config(cfg)
+    lib = load()
+    dev = topk_ids.device
+    if out is None:
+        out = torch.empty_like(topk_ids)
+    if ws is None:
+        ws = torch.empty(max(lib.moe_eplb_workspace_bytes(ctypes.byref(c)), 1), dtype=torch.uint8, device=dev)
+    _check(lib.moe_eplb_assign(ctypes.byref(c), _p(topk_ids), _p(replica_off), _p(replica_slots), n_slots,
+                               _p(out), _p(status), _p(ws), ws.numel(), _stream()), "moe_eplb_assign")
+    return out
+
+
+def eplb_place_weights(slot_expert, E: int, n_shared: int, w):
+    """moe_eplb_place_weights: [n_slots + n_shared, ...] copy of w [E + n_shared, ...] whose
+    slot s holds expert slot_expert[s] (host int array)."""
+    import numpy as np
+    se = np.ascontiguousarray(np.asarray(slot_expert, dtype=np.int32))
+    n_slots = len(se)
+    out = torch.empty((n_slots + n_shared,) + tuple(w.shape[1:]), dtype=w.dtype, device=w.device)
+    expert_bytes = w[0].numel() * w.element_size()
+    _check(load().moe_eplb_place_weights(_np_ptr(se), n_slots, E, n_shared, expert_bytes, _p(w), _p(out),
+                                         _stream()), "moe_eplb_place_weights")
+    return out
+

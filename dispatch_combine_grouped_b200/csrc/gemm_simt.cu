@@ -10,7 +10,7 @@ namespace moe {
 
 constexpr int SBM = 64, SBN = 64, SBK = 16;
 constexpr int kSimtThreads = 256;
-constexpr int kSimtGroups = kMaxE + kMaxShared;
+constexpr int kSimtGroups = kMaxSlots + kMaxShared;
 
 template <int MODE>
 __global__ void __launch_bounds__(kSimtThreads) simt_gemm_kernel(const GemmArgs p) {

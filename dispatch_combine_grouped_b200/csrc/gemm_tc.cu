@@ -37,7 +37,7 @@ constexpr int BK = 64;  // k per stage of the pair kernel and the router; FC til
 #define MOE_GEMM_BK 64
 #endif
 constexpr int kThreads = 192;
-constexpr int kMaxGroupsGemm = kMaxE + kMaxShared;
+constexpr int kMaxGroupsGemm = kMaxSlots + kMaxShared;
 
 struct SmemPlan {
   int a_bytes, b_bytes, stages, total;

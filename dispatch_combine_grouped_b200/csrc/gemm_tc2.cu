@@ -33,7 +33,7 @@ constexpr int PN = 256;             // MMA N (each CTA stages PN/2 rows of B)
 constexpr int PK = 64;              // k per stage
 constexpr int kPairThreads = 192;
 constexpr int kPairStages = 6;
-constexpr int kPairGroups = kMaxE + kMaxShared;
+constexpr int kPairGroups = kMaxSlots + kMaxShared;
 constexpr int A_BYTES = 128 * PK * 2;          // 16 KB
 constexpr int B_BYTES = (PN / 2) * PK * 2;     // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;

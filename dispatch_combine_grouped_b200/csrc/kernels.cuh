@@ -10,7 +10,8 @@
 
 namespace moe {
 
-constexpr int kMaxE = 256;        // routed experts
+constexpr int kMaxE = 256;        // routed experts a router scores
+constexpr int kMaxSlots = 512;    // experts (or physical expert slots) the layout and expert GEMMs take
 constexpr int kMaxK = 8;          // top-k
 constexpr int kMaxP = 32;         // virtual owners
 constexpr int kMaxGroups = 32;    // expert groups
@@ -86,6 +87,14 @@ cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStre
 cudaError_t launch_tc_gemm_pair(const GemmArgs& g, int a0_rows, int a1_rows, cudaStream_t st);
 // CUDA-core path, fp32 operands (the fp32 configurations)
 cudaError_t launch_simt_gemm(const GemmArgs& g, cudaStream_t st);
+
+// redundant expert slots (eplb.cu)
+size_t eplb_ws_bytes(const moe_config& c);
+cudaError_t launch_eplb_assign(const moe_config& c, const int32_t* ids, const int32_t* replica_off,
+                               const int32_t* replica_slots, int n_slots, int32_t* phys, int32_t* status, void* ws,
+                               cudaStream_t st);
+moe_status eplb_plan(int E, int R, int P, const int64_t* load, int32_t* copies, int32_t* replica_off,
+                     int32_t* replica_slots, int32_t* slot_expert, int32_t* slot_owner, int64_t* owner_load);
 
 int sm_count();
 // TMA maps for bf16 K-major operands; box_k (64, 32 or 16) selects the 128/64/32-byte swizzle

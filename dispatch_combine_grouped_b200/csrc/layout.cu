@@ -78,9 +78,9 @@ __device__ __forceinline__ int owner_of(const LayoutArgs& p, int e) {
 }
 
 __global__ void __launch_bounds__(kLayoutThreads) layout_count_kernel(LayoutArgs p, LayoutWs w) {
-  __shared__ int run_e[kMaxE];
+  __shared__ int run_e[kMaxSlots];
   __shared__ int run_j[kMaxP];
-  __shared__ int wcnt_e[kLayoutWarps][kMaxE];
+  __shared__ int wcnt_e[kLayoutWarps][kMaxSlots];
   __shared__ int wcnt_j[kLayoutWarps][kMaxP];
   __shared__ int hist_ij[kMaxP * kMaxP];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -181,7 +181,7 @@ constexpr int kScanThreads = 1024;
 
 __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutArgs p, LayoutWs w, moe_layout L,
                                                                    int nchunks) {
-  __shared__ int s_ne[kMaxE];
+  __shared__ int s_ne[kMaxSlots];
   __shared__ int s_C[kMaxP * kMaxP];
   __shared__ int s_recv[kMaxP + 1];
   const int tid = threadIdx.x;
@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutArgs p,
     int ex = block_exclusive_scan(v, nullptr);
     if (tid < p.E) L.expert_off[tid] = ex;
   } else {
-    __shared__ int s_own[kMaxE];
+    __shared__ int s_own[kMaxSlots];
     if (tid < p.E) s_own[tid] = owner_of(p, tid);
     __syncthreads();
     if (tid < p.E) {

@@ -38,14 +38,21 @@ moe_status check_config(const moe_config* c) {
       (c->dtype != MOE_F32 && c->dtype != MOE_BF16) || (c->renormalize != 0 && c->renormalize != 1) ||
       (c->bias_mode != MOE_BIAS_LOGITS && c->bias_mode != MOE_BIAS_SELECTION))
     return fail(MOE_ERR_INVALID_ARG, "score, dtype, renormalize or bias_mode out of range");
-  if (c->k > kMaxK || c->E > kMaxE || c->P > kMaxP || c->n_groups > kMaxGroups ||
+  if (c->k > kMaxK || c->E > kMaxSlots || c->P > kMaxP || c->n_groups > kMaxGroups ||
       c->topk_groups > kMaxTopkGroups || c->n_shared > kMaxShared)
-    return fail(MOE_ERR_UNSUPPORTED, "k <= 8, E <= 256, P <= 32, n_groups <= 32, topk_groups <= 8, S <= 8");
+    return fail(MOE_ERR_UNSUPPORTED, "k <= 8, E <= 512, P <= 32, n_groups <= 32, topk_groups <= 8, S <= 8");
   const int eb = elem_bytes(*c);
   if ((c->d * eb) % 16 != 0 || (c->I * eb) % 16 != 0)
     return fail(MOE_ERR_UNSUPPORTED, "rows of d and I elements must be multiples of 16 bytes");
   const long long rows = (long long)c->N * c->k + (long long)c->n_shared * c->N;
   if (rows >= (1LL << 31) / 2) return fail(MOE_ERR_UNSUPPORTED, "N * (k + S) too large");
+  return MOE_OK;
+}
+
+// The router (and so every call that routes) scores at most kMaxE experts; the layout,
+// movement and expert calls take up to kMaxSlots (e.g. E + R physical expert slots).
+moe_status check_router(const moe_config& c) {
+  if (c.E > kMaxE) return fail(MOE_ERR_UNSUPPORTED, "the router scores at most 256 experts");
   return MOE_OK;
 }
 
@@ -274,6 +281,7 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_gate, c
                      int32_t* topk_ids, float* topk_w, moe_stream_t stream) {
   moe_status s = check_config(cfg);
   if (s != MOE_OK) return s;
+  if ((s = check_router(*cfg)) != MOE_OK) return s;
   if (cfg->N == 0) return MOE_OK;
   if (!x || !w_gate || !logits || !topk_ids || !topk_w) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
   return route_impl(*cfg, x, w_gate, bias, logits, topk_ids, topk_w, (cudaStream_t)stream);
@@ -411,6 +419,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* w
                              moe_stream_t stream) {
   moe_status s = check_config(cfg);
   if (s != MOE_OK) return s;
+  if ((s = check_router(*cfg)) != MOE_OK) return s;
   if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
   const moe_config& c = *cfg;
   FwdWs w = carve_forward(c, nullptr);
@@ -436,6 +445,7 @@ moe_status moe_layer_forward_overlapped(const moe_config* cfg, const void* x, co
                                         moe_stream_t stream, moe_stream_t side_stream) {
   moe_status s = check_config(cfg);
   if (s != MOE_OK) return s;
+  if ((s = check_router(*cfg)) != MOE_OK) return s;
   if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
   const moe_config& c = *cfg;
   if (c.n_shared == 0 || c.N == 0 || side_stream == stream)
@@ -476,6 +486,62 @@ moe_status moe_layer_forward_overlapped(const moe_config* cfg, const void* x, co
   if (s != MOE_OK) return s;
   if (e != cudaSuccess) return cuda_status(e, "join");
   return cuda_status(launch_combine(c, L, w.out, nullptr, y, st), "combine");
+}
+
+size_t moe_eplb_workspace_bytes(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return eplb_ws_bytes(*cfg);
+}
+
+moe_status moe_eplb_plan(int32_t E, int32_t R, int32_t P, const int64_t* load, int32_t* copies,
+                         int32_t* replica_off, int32_t* replica_slots, int32_t* slot_expert, int32_t* slot_owner,
+                         int64_t* owner_load) {
+  if (E < 1 || R < 0 || P < 1) return fail(MOE_ERR_INVALID_ARG, "need E >= 1, R >= 0, P >= 1");
+  if ((E + R) % P != 0) return fail(MOE_ERR_INVALID_ARG, "E + R must be a multiple of P");
+  if (E + R > kMaxSlots) return fail(MOE_ERR_UNSUPPORTED, "E + R <= 512");
+  if (!load || !copies || !replica_off || !replica_slots || !slot_expert || !slot_owner || !owner_load)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  for (int e = 0; e < E; ++e)
+    if (load[e] < 0 || load[e] > (1LL << 40)) return fail(MOE_ERR_INVALID_ARG, "load out of range [0, 2^40]");
+  return eplb_plan(E, R, P, load, copies, replica_off, replica_slots, slot_expert, slot_owner, owner_load);
+}
+
+moe_status moe_eplb_assign(const moe_config* cfg, const int32_t* topk_ids, const int32_t* replica_off,
+                           const int32_t* replica_slots, int32_t n_slots, int32_t* phys_ids, int32_t* dev_status,
+                           void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (n_slots < cfg->E || n_slots > kMaxSlots) return fail(MOE_ERR_INVALID_ARG, "need E <= n_slots <= 512");
+  if (!replica_off || !replica_slots || (cfg->N > 0 && (!topk_ids || !phys_ids)))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!ws || ws_bytes < eplb_ws_bytes(*cfg)) return fail(MOE_ERR_WORKSPACE, "EPLB workspace too small");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return fail(MOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  return cuda_status(launch_eplb_assign(*cfg, topk_ids, replica_off, replica_slots, n_slots, phys_ids, dev_status,
+                                        ws, (cudaStream_t)stream),
+                     "eplb assign");
+}
+
+moe_status moe_eplb_place_weights(const int32_t* slot_expert, int32_t n_slots, int32_t E, int32_t n_shared,
+                                  size_t expert_bytes, const void* w_logical, void* w_physical, moe_stream_t stream) {
+  if (n_slots < 1 || n_slots > kMaxSlots || E < 1 || n_shared < 0 || n_shared > kMaxShared)
+    return fail(MOE_ERR_INVALID_ARG, "need 1 <= n_slots <= 512, E >= 1, 0 <= n_shared <= 8");
+  if (!slot_expert || !w_logical || !w_physical) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  for (int i = 0; i < n_slots; ++i)
+    if (slot_expert[i] < 0 || slot_expert[i] >= E) return fail(MOE_ERR_INVALID_ARG, "slot_expert out of [0, E)");
+  const char* src = static_cast<const char*>(w_logical);
+  char* dst = static_cast<char*>(w_physical);
+  cudaStream_t st = (cudaStream_t)stream;
+  for (int i = 0; i < n_slots; ++i) {
+    cudaError_t e = cudaMemcpyAsync(dst + (size_t)i * expert_bytes, src + (size_t)slot_expert[i] * expert_bytes,
+                                    expert_bytes, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_status(e, "eplb place weights");
+  }
+  if (n_shared > 0) {
+    cudaError_t e = cudaMemcpyAsync(dst + (size_t)n_slots * expert_bytes, src + (size_t)E * expert_bytes,
+                                    (size_t)n_shared * expert_bytes, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_status(e, "eplb place weights");
+  }
+  return MOE_OK;
 }
 
 }  // extern "C"

@@ -28,8 +28,10 @@
  *     written to *dev_status (an int32 the caller zeroes and reads after synchronising);
  *     the first error wins.  dev_status may be NULL, in which case they go unreported.
  *   - Sizes: A = N * k assignments, a = t * k + slot indexes them.  E % P == 0 unless an
- *     explicit expert_owner table is given.  k <= 8, E <= 256 (E >= k), P <= 32,
- *     n_groups <= 32 with E % n_groups == 0, topk_groups <= 8.
+ *     explicit expert_owner table is given.  k <= 8, E >= k, P <= 32,
+ *     n_groups <= 32 with E % n_groups == 0, topk_groups <= 8.  The router (moe_route
+ *     and the fused forwards) takes E <= 256; the layout, movement and expert calls take
+ *     E <= 512 (e.g. E + R physical expert slots, see moe_eplb_*).
  *     bf16: d % 8 == 0, I % 8 == 0.   f32: d % 4 == 0, I % 4 == 0.
  *   - dtype applies to activations, weights and expert outputs; every reduction
  *     accumulates in fp32.  Router logits and gate weights are fp32.
@@ -312,6 +314,81 @@ moe_status moe_layer_forward_overlapped(const moe_config* cfg, const void* x, co
                                         const int32_t* expert_owner, const void* w13, const void* w2, void* y,
                                         const moe_layout* layout_out, int32_t* dev_status, void* ws, size_t ws_bytes,
                                         moe_stream_t stream, moe_stream_t side_stream);
+
+/*
+ * Redundant expert slots, EPLB ([WideEP] "为什么要把 EP 做宽": E logical experts plus R
+ * copies make E + R physical experts, (E + R) / P per owner; "DeepSeek-V3/R1 的两个具体
+ * 布局": 256 + 32 = 288 slots; "Expert 副本在 Wide EP 中还有整除作用": hot experts are
+ * copied and a logical expert's assignments are spread over its copies; "三种负载必须同时
+ * 平衡": the balancer minimises the largest expert / receive load).  The router's choice
+ * is kept; only which copy serves an assignment changes.  Use:
+ *   1. moe_eplb_plan on the host, from per-expert loads (e.g. n_e of earlier batches);
+ *   2. moe_eplb_place_weights once per plan: W13 / W2 of the E + R slots (+ shared);
+ *   3. per batch: moe_route (E logical experts) -> moe_eplb_assign -> the layout, permute,
+ *      expert and combine calls with a config whose E is E + R (slot s is owned by
+ *      s / ((E + R) / P), so expert_owner may be NULL), the physical weights and the same
+ *      topk_w.  The output equals the layer without copies.
+ */
+
+/*
+ * Plan (host only; all pointers are HOST memory; no GPU work).  Steps, since the pages
+ * give the goal but no algorithm:
+ *   copies: every expert keeps one copy; each of the R extra copies in turn goes to the
+ *           expert with the largest load per copy, load_e / copies_e (ties: lower id),
+ *           which minimises max_e load_e / copies_e;
+ *   placement: copy c of expert e carries load_e / copies_e rounded down, plus one when
+ *           c < load_e mod copies_e (the rows moe_eplb_assign gives it); copies are
+ *           placed in descending load order (ties: lower expert, lower copy) on the
+ *           owner with free room that holds no copy of the same expert if there is one,
+ *           then the least loaded owner, then the lower owner;
+ *   slots:  owner j holds slots [j (E+R)/P, (j+1) (E+R)/P) in (expert, copy) order.
+ *   load          [E] int64, 0 .. 2^40
+ *   copies        [E] out: copies per expert (sum E + R)
+ *   replica_off   [E+1] out: copies of expert e are replica_slots[replica_off[e] ..)
+ *   replica_slots [E+R] out: slot of copy c of expert e at replica_off[e] + c
+ *   slot_expert   [E+R] out: logical expert of each slot
+ *   slot_owner    [E+R] out: owner of each slot
+ *   owner_load    [P] out: planned rows per owner
+ * Errors: (E + R) % P != 0 or a NULL pointer -> MOE_ERR_INVALID_ARG; E + R > 512 ->
+ * MOE_ERR_UNSUPPORTED.
+ */
+moe_status moe_eplb_plan(int32_t E, int32_t R, int32_t P, const int64_t* load, int32_t* copies,
+                         int32_t* replica_off, int32_t* replica_slots, int32_t* slot_expert, int32_t* slot_owner,
+                         int64_t* owner_load);
+
+/* Bytes of scratch moe_eplb_assign needs (a one-owner dispatch layout of the logical ids). */
+size_t moe_eplb_workspace_bytes(const moe_config* cfg);
+
+/*
+ * Replica assignment (device): the q-th assignment of logical expert e, in ascending
+ * a = t*k + slot, goes to copy q mod copies_e: phys_ids[a] = replica_slots[replica_off[e]
+ * + q mod (replica_off[e+1] - replica_off[e])].  Copies of e thus get n_e / copies_e rows
+ * to within one.  q comes from a dispatch layout of the logical ids with one owner,
+ * computed in the workspace.
+ *   cfg            the LOGICAL configuration (E experts)
+ *   topk_ids       [N, k] int32 logical ids
+ *   replica_off    [E+1], replica_slots [n_slots] int32 device copies of the plan
+ *   n_slots        E + R (E <= n_slots <= 512)
+ *   phys_ids       [N, k] int32 out: slot ids in [0, n_slots)
+ *   ws, ws_bytes   scratch of at least moe_eplb_workspace_bytes(cfg), 256-byte aligned
+ * Device errors (MOE_ERR_BAD_INDEX in *dev_status): an id outside [0, E) (counted as
+ * expert 0), an expert without copies or a slot outside [0, n_slots) (slot 0 written).
+ */
+moe_status moe_eplb_assign(const moe_config* cfg, const int32_t* topk_ids, const int32_t* replica_off,
+                           const int32_t* replica_slots, int32_t n_slots, int32_t* phys_ids, int32_t* dev_status,
+                           void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Weights of the physical slots: w_physical[s] = w_logical[slot_expert[s]] for the
+ * n_slots slots, then the n_shared shared experts w_logical[E ..] after them.  One
+ * device-to-device copy per slot (plus one for the shared experts) on `stream`; a
+ * placement step, run once per plan.
+ *   slot_expert  [n_slots] HOST int32 in [0, E)
+ *   expert_bytes bytes of one expert's matrix (2*I*d*b for W13, d*I*b for W2)
+ *   w_logical    [E + n_shared] matrices, w_physical [n_slots + n_shared] matrices (device)
+ */
+moe_status moe_eplb_place_weights(const int32_t* slot_expert, int32_t n_slots, int32_t E, int32_t n_shared,
+                                  size_t expert_bytes, const void* w_logical, void* w_physical, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

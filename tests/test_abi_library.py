@@ -44,7 +44,7 @@ def test_host_validation_without_gpu():
     for cfg in CONFIGS.values():
         moe.check_config(cfg)
         assert moe.workspace_bytes(cfg) > 0
-    bad = [dict(k=9), dict(E=512), dict(P=64), dict(d=100), dict(N=-1), dict(n_groups=3),
+    bad = [dict(k=9), dict(E=513), dict(P=64), dict(d=100), dict(N=-1), dict(n_groups=3),
            dict(n_groups=4, topk_groups=5), dict(S=9)]
     for kw in bad:
         with pytest.raises(moe.MoEError):
@@ -68,3 +68,51 @@ def test_calls_reject_null_without_launching():
         == binding.MOE_ERR_INVALID_ARG
     assert lib.moe_layer_forward(ctypes.byref(cfg), None, None, None, None, None, None, None, None, None, None, 0,
                                  None) == binding.MOE_ERR_WORKSPACE
+
+
+def test_router_takes_at_most_256_experts():
+    """Layout and expert calls accept up to 512 experts (physical slots); the router 256.
+    The check happens on the host before anything launches."""
+    cfg = small_config(N=8, d=64, E=288, S=0, k=2, I=64, P=2)
+    moe.check_config(cfg)
+    c = binding.c_config(cfg)
+    lib = binding.load()
+    assert lib.moe_route(ctypes.byref(c), None, None, None, None, None, None, None) == binding.MOE_ERR_UNSUPPORTED
+    assert lib.moe_layer_forward(ctypes.byref(c), None, None, None, None, None, None, None, None, None, None, 0,
+                                 None) == binding.MOE_ERR_UNSUPPORTED
+
+
+def test_eplb_plan_matches_the_oracle_on_the_host():
+    """moe_eplb_plan is host code: its tables equal the oracle's plan (same steps, written
+    independently), for random and skewed loads."""
+    import numpy as np
+    from oracle import eplb as EP
+    rng = np.random.default_rng(11)
+    cases = [(4, 2, 3, np.array([10, 4, 3, 1]))]
+    for E, R, P in [(8, 4, 4), (16, 16, 8), (32, 0, 8), (128, 16, 16), (256, 32, 32), (6, 3, 9), (64, 0, 8)]:
+        cases.append((E, R, P, rng.zipf(1.3, size=E).astype(np.int64) % 100000))
+        cases.append((E, R, P, rng.integers(0, 5, size=E)))
+    for E, R, P, load in cases:
+        got = moe.eplb_plan(load, R, P)
+        ref = EP.plan(load, R, P)
+        for key in ("copies", "replica_off", "replica_slots", "slot_expert", "slot_owner", "owner_load"):
+            assert got[key].tolist() == ref[key].tolist(), (E, R, P, key)
+
+
+def test_eplb_calls_reject_bad_arguments_without_launching():
+    import numpy as np
+    lib = binding.load()
+    with pytest.raises(moe.MoEError):
+        moe.eplb_plan(np.ones(8), 3, 4)  # 11 slots over 4 owners
+    with pytest.raises(moe.MoEError):
+        moe.eplb_plan(np.ones(500), 20, 4)  # 520 slots
+    c = binding.c_config(small_config(N=8, d=64, E=8, S=0, k=2, I=64, P=2))
+    assert lib.moe_eplb_workspace_bytes(ctypes.byref(c)) > 0
+    assert lib.moe_eplb_assign(ctypes.byref(c), None, None, None, 12, None, None, None, 0, None) \
+        == binding.MOE_ERR_INVALID_ARG
+    assert lib.moe_eplb_assign(ctypes.byref(c), None, None, None, 4, None, None, None, 0, None) \
+        == binding.MOE_ERR_INVALID_ARG  # fewer slots than experts
+    se = np.array([0, 1, 9], dtype=np.int32)  # expert 9 does not exist
+    assert lib.moe_eplb_place_weights(ctypes.c_void_p(se.ctypes.data), 3, 8, 0, 16, ctypes.c_void_p(16),
+                                      ctypes.c_void_p(16), None) == binding.MOE_ERR_INVALID_ARG
+
