@@ -20,6 +20,8 @@ import subprocess
 import sys
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -36,6 +38,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--eplb", type=int, default=0, metavar="R",
+                    help="run the routed experts over E + R physical slots (redundant copies of the "
+                         "hot experts, planned from the batch's own counts)")
     return ap.parse_args()
 
 
@@ -270,6 +275,33 @@ def main():
     side = torch.cuda.Stream(device=dev)
     main = torch.cuda.current_stream(dev)
 
+    # redundant expert slots: plan from this batch's counts, copy the slot weights once
+    R = args.eplb
+    pcfg, ids_l, w13_l, w2_l, owner_l = cfg, ids, w13, w2, owner
+    eplb_info = None
+    if R:
+        moe.route(cfg, x, wg, bias, out=(logits, ids, w))
+        n_e0 = torch.bincount(ids.reshape(-1).long(), minlength=cfg.E).cpu().numpy()
+        plan = moe.eplb_plan(n_e0, R, cfg.P)
+        rep_off = torch.tensor(plan["replica_off"], dtype=torch.int32, device=dev)
+        rep_slots = torch.tensor(plan["replica_slots"], dtype=torch.int32, device=dev)
+        eplb_ws = torch.empty(max(moe.eplb_workspace_bytes(cfg), 1), dtype=torch.uint8, device=dev)
+        pcfg = moe.physical_config(cfg, R)
+        ids_l = torch.empty_like(ids)
+        w13_l = moe.eplb_place_weights(plan["slot_expert"], cfg.E, S, w13)
+        w2_l = moe.eplb_place_weights(plan["slot_expert"], cfg.E, S, w2)
+        owner_l = None
+        layout = moe.Layout(pcfg, dev)
+        lay_ws = torch.empty(max(moe.layout_workspace_bytes(pcfg), 1), dtype=torch.uint8, device=dev)
+        own = owner.long().cpu().numpy() if owner is not None else np.arange(cfg.E) // (cfg.E // cfg.P)
+        before = np.bincount(own, weights=n_e0, minlength=cfg.P)
+        eplb_info = {"copies": R, "slots": cfg.E + R, "planned_owner_load": plan["owner_load"].tolist(),
+                     "owner_max_over_mean_before": float(before.max() / before.mean())}
+
+    def assign():
+        if R:
+            moe.eplb_assign(cfg, ids, rep_off, rep_slots, cfg.E + R, status=status, out=ids_l, ws=eplb_ws)
+
     def step(ev):
         """One layer pass as the product runs it (moe_layer_forward_overlapped's order):
         router; then the shared experts on a side stream while layout, permute and the
@@ -281,20 +313,21 @@ def main():
             fork, join = torch.cuda.Event(), torch.cuda.Event()
             fork.record(main)
             side.wait_event(fork)
-            moe.expert_fc1(cfg, None, None, x, w13, h=h, groups="shared", stream=side)
-            moe.expert_fc2(cfg, None, h, w2, out=out, groups="shared", stream=side)
+            moe.expert_fc1(pcfg, None, None, x, w13_l, h=h, groups="shared", stream=side)
+            moe.expert_fc2(pcfg, None, h, w2_l, out=out, groups="shared", stream=side)
             join.record(side)
-        moe.dispatch_layout(cfg, ids, owner, status=status, layout=layout, ws=lay_ws)
+        assign()
+        moe.dispatch_layout(pcfg, ids_l, owner_l, status=status, layout=layout, ws=lay_ws)
         ev[2].record()
-        moe.permute(cfg, layout, x, out=x_perm)
+        moe.permute(pcfg, layout, x, out=x_perm)
         ev[3].record()
-        moe.expert_fc1(cfg, layout, x_perm, x, w13, h=h, groups="routed")
+        moe.expert_fc1(pcfg, layout, x_perm, x, w13_l, h=h, groups="routed")
         ev[4].record()
-        moe.expert_fc2(cfg, layout, h, w2, topk_w=w, out=out, groups="routed")
+        moe.expert_fc2(pcfg, layout, h, w2_l, topk_w=w, out=out, groups="routed")
         ev[5].record()
         if S:
             main.wait_event(join)
-        moe.combine(cfg, layout, out, y=y)
+        moe.combine(pcfg, layout, out, y=y)
         ev[6].record()
 
     def step_sequential(ev):
@@ -302,15 +335,16 @@ def main():
         ev[0].record()
         moe.route(cfg, x, wg, bias, out=(logits, ids, w))
         ev[1].record()
-        moe.dispatch_layout(cfg, ids, owner, status=status, layout=layout, ws=lay_ws)
+        assign()
+        moe.dispatch_layout(pcfg, ids_l, owner_l, status=status, layout=layout, ws=lay_ws)
         ev[2].record()
-        moe.permute(cfg, layout, x, out=x_perm)
+        moe.permute(pcfg, layout, x, out=x_perm)
         ev[3].record()
-        moe.expert_fc1(cfg, layout, x_perm, x, w13, h=h)
+        moe.expert_fc1(pcfg, layout, x_perm, x, w13_l, h=h)
         ev[4].record()
-        moe.expert_fc2(cfg, layout, h, w2, topk_w=w, out=out)
+        moe.expert_fc2(pcfg, layout, h, w2_l, topk_w=w, out=out)
         ev[5].record()
-        moe.combine(cfg, layout, out, y=y)
+        moe.combine(pcfg, layout, out, y=y)
         ev[6].record()
 
     def new_events():
@@ -405,7 +439,12 @@ def main():
     tokens_total = cfg.N * world
     value = whole_job_tokens_per_s(cfg.N, world, step_ms_max)
     gl = 2 if (cfg.dtype == "bf16" and cfg.N > 128 and cfg.d >= 4096) else 1   # pair + tail launches
-    launches_per_step = 2 + 3 + 1 + 2 * gl + (2 * gl if S else 0) + 1
+    launches_per_step = 2 + 3 + 1 + 2 * gl + (2 * gl if S else 0) + 1 + (4 if R else 0)
+    if R:
+        R_after = np.diff(layout["recv_off"].cpu().numpy())
+        eplb_info["owner_max_over_mean_after"] = float(R_after.max() / R_after.mean())
+        eplb_info["note"] = ("stages_ms.layout includes the replica assignment; the fused and e2e "
+                             "numbers run the layer without copies")
 
     if rank == 0:
         line = {
@@ -436,6 +475,7 @@ def main():
                     "h2d_bytes_per_step": x.numel() * x.element_size(),
                     "d2h_bytes_per_step": y.numel() * y.element_size()},
             "gpu_launches": launches_per_step * args.steps,
+            **({"eplb": eplb_info} if R else {}),
             "clocks": clock_rec,
             "wall_s_timed": wall,
         }

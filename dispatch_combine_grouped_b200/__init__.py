@@ -6,7 +6,7 @@ binding.  Importing it loads the library and fails loudly when it is missing.
 """
 from .binding import (EXPORTED, Layout, MoEError, alloc_workspace, c_config, check_config,  # noqa: F401
                       combine, combine_staged, dispatch_layout, dispatch_layout_noalloc, eplb_assign,
-                      eplb_place_weights, eplb_plan, expert_fc1, physical_config,
+                      eplb_place_weights, eplb_plan, eplb_workspace_bytes, expert_fc1, physical_config,
                       expert_fc2, grouped_ffn, layer_forward, layer_forward_overlapped, layout_workspace_bytes,
                       load, permute, permute_staged, route, routed_ffn, selftest_bounded_wait, shared_ffn, version,
                       workspace_bytes)

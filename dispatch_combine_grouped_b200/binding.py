@@ -372,6 +372,11 @@ def physical_config(cfg, R: int):
     return dataclasses.replace(cfg, E=cfg.E + R, n_groups=1, topk_groups=1)
 
 
+def eplb_workspace_bytes(cfg) -> int:
+    c = c_config(cfg)
+    return load().moe_eplb_workspace_bytes(ctypes.byref(c))
+
+
 def eplb_assign(cfg, topk_ids, replica_off, replica_slots, n_slots: int, status=None, out=None, ws=None):
     """moe_eplb_assign: physical slot ids [N, k] int32 for the logical ids (device)."""
     c = c_config(cfg)
