@@ -137,3 +137,23 @@ def test_replica_rank_off_by_one_is_caught(monkeypatch):
         return out.reshape(ids.shape)
     monkeypatch.setattr(EP, "assign", shifted)
     _fails(eplb_pins.check_worked_example)
+
+
+# ---- FP8 oracle
+import tests.test_fp8_oracle as fp8_pins
+from oracle import fp8 as F8
+
+
+def test_fp8_ties_away_from_even_are_caught(monkeypatch):
+    orig = F8.e4m3_encode
+
+    def up(v):
+        v = np.asarray(v, dtype=np.float64)
+        return orig(np.nextafter(np.abs(v), np.inf) * np.where(np.signbit(v), -1, 1))
+    monkeypatch.setattr(F8, "e4m3_encode", up)
+    _fails(fp8_pins.test_ties_go_to_the_even_code_and_large_values_saturate)
+
+
+def test_fp8_wrong_scale_is_caught(monkeypatch):
+    monkeypatch.setattr(F8, "E4M3_MAX", 240.0)
+    _fails(fp8_pins.test_row_quantisation)
