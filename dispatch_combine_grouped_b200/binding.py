@@ -30,7 +30,8 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_con
             "moe_routed_ffn", "moe_shared_ffn", "moe_layer_forward_overlapped", "moe_selftest_bounded_wait",
             "moe_combine", "moe_combine_staged",
             "moe_layer_forward", "moe_eplb_plan", "moe_eplb_workspace_bytes", "moe_eplb_assign",
-            "moe_eplb_place_weights"]
+            "moe_eplb_place_weights", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8",
+            "moe_workspace_bytes_fp8", "moe_layer_forward_fp8"]
 
 
 class CConfig(ctypes.Structure):
@@ -92,6 +93,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_eplb_workspace_bytes": (sz, [cfgp]),
         "moe_eplb_assign": (i32, [cfgp, vp, vp, vp, i32, vp, vp, vp, sz, vp]),
         "moe_eplb_place_weights": (i32, [vp, i32, i32, i32, sz, vp, vp, vp]),
+        "moe_quantize_fp8": (i32, [vp, ctypes.c_int64, i32, vp, vp, vp]),
+        "moe_permute_fp8": (i32, [cfgp, layp, vp, vp, vp]),
+        "moe_grouped_ffn_fp8": (i32, [cfgp, layp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_workspace_bytes_fp8": (sz, [cfgp]),
+        "moe_layer_forward_fp8": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -402,4 +408,62 @@ def eplb_place_weights(slot_expert, E: int, n_shared: int, w):
     _check(load().moe_eplb_place_weights(_np_ptr(se), n_slots, E, n_shared, expert_bytes, _p(w), _p(out),
                                          _stream()), "moe_eplb_place_weights")
     return out
+
+
+# ---------------------------------------------------------------- FP8 (e4m3) expert path
+def quantize_fp8(src, out=None, scale=None):
+    """moe_quantize_fp8: per-row e4m3 codes (uint8, same shape) and fp32 scales of a bf16
+    tensor whose last dimension is the row."""
+    rows = src.numel() // src.shape[-1]
+    cols = src.shape[-1]
+    if out is None:
+        out = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+    if scale is None:
+        scale = torch.empty(src.shape[:-1], dtype=torch.float32, device=src.device)
+    _check(load().moe_quantize_fp8(_p(src), rows, cols, _p(out), _p(scale), _stream()), "moe_quantize_fp8")
+    return out, scale
+
+
+def permute_fp8(cfg, layout, x_q, out=None):
+    c = c_config(cfg)
+    if out is None:
+        out = torch.empty(cfg.N * cfg.k, cfg.d, dtype=torch.uint8, device=x_q.device)
+    _check(load().moe_permute_fp8(ctypes.byref(c), ctypes.byref(layout.c), _p(x_q), _p(out), _stream()),
+           "moe_permute_fp8")
+    return out
+
+
+def grouped_ffn_fp8(cfg, layout, x_q_perm, x_q, x_scale, w13_q, w13_scale, w2_q, w2_scale, topk_w=None,
+                    h=None, h_q=None, h_scale=None, out=None):
+    """-> (h bf16, h_q e4m3, h_scale, out bf16) over [A + S*N] rows."""
+    c = c_config(cfg)
+    dev = x_q_perm.device
+    rows = cfg.N * cfg.k + cfg.S * cfg.N
+    h = h if h is not None else torch.empty(rows, cfg.I, dtype=torch.bfloat16, device=dev)
+    h_q = h_q if h_q is not None else torch.empty(rows, cfg.I, dtype=torch.uint8, device=dev)
+    h_scale = h_scale if h_scale is not None else torch.empty(rows, dtype=torch.float32, device=dev)
+    out = out if out is not None else torch.empty(rows, cfg.d, dtype=torch.bfloat16, device=dev)
+    _check(load().moe_grouped_ffn_fp8(ctypes.byref(c), ctypes.byref(layout.c), _p(x_q_perm), _p(x_q), _p(x_scale),
+                                      _p(w13_q), _p(w13_scale), _p(w2_q), _p(w2_scale), _p(topk_w), _p(h), _p(h_q),
+                                      _p(h_scale), _p(out), _stream()), "moe_grouped_ffn_fp8")
+    return h, h_q, h_scale, out
+
+
+def workspace_bytes_fp8(cfg) -> int:
+    c = c_config(cfg)
+    return load().moe_workspace_bytes_fp8(ctypes.byref(c))
+
+
+def layer_forward_fp8(cfg, x, w_gate, bias, expert_owner, w13_q, w13_scale, w2_q, w2_scale, y=None, ws=None,
+                      layout=None, status=None):
+    c = c_config(cfg)
+    if y is None:
+        y = torch.empty(cfg.N, cfg.d, dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = torch.empty(max(workspace_bytes_fp8(cfg), 1), dtype=torch.uint8, device=x.device)
+    _check(load().moe_layer_forward_fp8(ctypes.byref(c), _p(x), _p(w_gate), _p(bias), _p(expert_owner), _p(w13_q),
+                                        _p(w13_scale), _p(w2_q), _p(w2_scale), _p(y),
+                                        ctypes.byref(layout.c) if layout is not None else None, _p(status), _p(ws),
+                                        ws.numel(), _stream()), "moe_layer_forward_fp8")
+    return y
 

@@ -49,10 +49,10 @@ __host__ __device__ constexpr int barrier_bytes() {
   return ((2 * STAGES + 5) * 8 + 8 + 15) & ~15;
 }
 
-template <int BN, int STAGES, int BKT>
+template <int BN, int STAGES, int BKT, int ES>
 __host__ __device__ constexpr int smem_bytes_for() {
   // 1 KB alignment slack + stages + barriers/flags + group tables
-  return 1024 + STAGES * (BM * BKT * 2 + BN * BKT * 2) + barrier_bytes<STAGES>() + 4 * (4 * kMaxGroupsGemm + 8);
+  return 1024 + STAGES * (BM * BKT * ES + BN * BKT * ES) + barrier_bytes<STAGES>() + 4 * (4 * kMaxGroupsGemm + 8);
 }
 
 struct TileDesc {
@@ -76,15 +76,19 @@ __device__ __forceinline__ TileDesc decode_tile(int t, const int* prefix, int G,
   return d;
 }
 
-template <int BN, int MODE, int STAGES, int BKT>
+// F8: e4m3 operands (BKT = 128 k per stage, the same 128-byte rows), kind::f8f6f4 MMAs and
+// the row x column scales applied to the accumulator in the epilogue.
+template <int BN, int MODE, int STAGES, int BKT, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
-  constexpr int A_BYTES = BM * BKT * 2;
-  constexpr int B_BYTES = BN * BKT * 2;
+  constexpr int ES = F8 ? 1 : 2;        // bytes per element
+  constexpr int ROWB = BKT * ES;        // bytes of one row of a stage
+  constexpr int A_BYTES = BM * ROWB;
+  constexpr int B_BYTES = BN * ROWB;
   constexpr int HALF_B = B_BYTES / 2;
   constexpr uint32_t TMEM_COLS = 2 * BN;  // BN is a power of two >= 32
-  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+  constexpr uint32_t IDESC = F8 ? idesc_e4m3_f32(BM, BN) : idesc_bf16_f32(BM, BN);
   constexpr uint32_t TX_BYTES = A_BYTES + B_BYTES;
 
   extern __shared__ uint8_t smem_raw[];
@@ -251,10 +255,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BKT / 16; ++kk) {
-            umma_bf16(d_tmem, smem_desc_kmajor<BKT * 2>(a_addr + kk * 32), smem_desc_kmajor<BKT * 2>(b_addr + kk * 32),
-                      IDESC,
-                      (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < ROWB / 32; ++kk) {  // 32 bytes of k per MMA
+            if (F8)
+              umma_e4m3(d_tmem, smem_desc_kmajor<ROWB>(a_addr + kk * 32), smem_desc_kmajor<ROWB>(b_addr + kk * 32),
+                        IDESC, (kb | kk) != 0 ? 1u : 0u);
+            else
+              umma_bf16(d_tmem, smem_desc_kmajor<ROWB>(a_addr + kk * 32), smem_desc_kmajor<ROWB>(b_addr + kk * 32),
+                        IDESC, (kb | kk) != 0 ? 1u : 0u);
           }
           any = true;
           umma_commit(&empty[stage]);  // frees the smem stage when these MMAs complete
@@ -332,12 +339,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (MODE == MODE_FC1) {
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + orow * p.ldo;
         const int col_base = td.n_blk * (BN / 2);
+        float ra = 1.0f;  // FP8: scale of this row's token
+        const float* sb = nullptr;
+        if (F8) {
+          const int gz = p.g0 + td.g;
+          if (row_ok) ra = p.a_scale[gz < p.E ? p.row2tok[orow] / p.k : r];
+          sb = p.b_scale + (size_t)gz * p.b_rows;
+        }
 #pragma unroll 1
         for (int c0 = 0; c0 < BN / 2; c0 += 32) {
           uint32_t gv[32], uv[32];
           tmem_ld32(taddr + c0, gv);
           tmem_ld32(taddr + BN / 2 + c0, uv);
           tmem_wait_ld();
+          if (F8 && row_ok) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              const int col = min(col_base + c0 + q, p.n_out - 1);
+              gv[q] = __float_as_uint(__uint_as_float(gv[q]) * ra * __ldg(sb + col));
+              uv[q] = __float_as_uint(__uint_as_float(uv[q]) * ra * __ldg(sb + p.I + col));
+            }
+          }
           if (row_ok) {
 #pragma unroll
             for (int q = 0; q < 32; q += 8) {
@@ -360,12 +382,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + orow * p.ldo;
         float scale = 1.0f;
         if (row_ok && p.gate_w && p.g0 + td.g < p.E) scale = p.gate_w[p.row2tok[orow]];
+        const float* sb = nullptr;
+        if (F8) {
+          if (row_ok) scale *= p.a_scale[orow];  // FP8: scale of this h row
+          sb = p.b_scale + (size_t)(p.g0 + td.g) * p.b_rows;
+        }
         const int col_base = td.n_blk * BN;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 32) {
           uint32_t v[32];
           tmem_ld32(taddr + c0, v);
           tmem_wait_ld();
+          if (F8 && row_ok) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              v[q] = __float_as_uint(__uint_as_float(v[q]) * __ldg(sb + min(col_base + c0 + q, p.n_out - 1)));
+          }
           if (row_ok) {
 #pragma unroll
             for (int q = 0; q < 32; q += 8) {
@@ -412,34 +444,39 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-static CUtensorMapSwizzle swizzle_for(int box_k) {
-  return box_k == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : (box_k == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+static CUtensorMapSwizzle swizzle_for(int row_bytes) {
+  return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
-// 2D bf16 map over [rows, K] (K contiguous), box [128 rows, box_k cols], swizzle = 2*box_k bytes.
-bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K, int box_k) {
+// 2D map over [rows, K] (K contiguous; bf16, or bytes when u8), box [128 rows, box_k
+// elements], swizzle = the box's row bytes.
+bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K, int box_k, bool u8) {
   auto enc = get_encode();
   if (!enc) return false;
+  const int es = u8 ? 1 : 2;
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)(rows > 0 ? rows : 1)};
-  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint64_t strides[1] = {(cuuint64_t)K * es};
   cuuint32_t box[2] = {(cuuint32_t)box_k, BM};
-  cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(box_k), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(box_k * es),
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3D bf16 map over [G, R, K], box [1, box_rows, box_k], swizzle = 2*box_k bytes.
-bool make_map_b(CUtensorMap* m, const void* base, long long G, long long R, long long K, int box_rows, int box_k) {
+// 3D map over [G, R, K] (bf16, or bytes when u8), box [1, box_rows, box_k elements].
+bool make_map_b(CUtensorMap* m, const void* base, long long G, long long R, long long K, int box_rows, int box_k,
+                bool u8) {
   auto enc = get_encode();
   if (!enc) return false;
+  const int es = u8 ? 1 : 2;
   cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)R, (cuuint64_t)G};
-  cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)(R * K * 2)};
+  cuuint64_t strides[2] = {(cuuint64_t)K * es, (cuuint64_t)(R * K * es)};
   cuuint32_t box[3] = {(cuuint32_t)box_k, (cuuint32_t)box_rows, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(box_k), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(box_k * es),
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int sm_count() {
@@ -453,14 +490,15 @@ int sm_count() {
   return n;
 }
 
-template <int BN, int MODE, int BKT>
+template <int BN, int MODE, int BKT, bool F8 = false>
 static cudaError_t launch_bn(const GemmArgs& g, const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                              long long max_tiles, cudaStream_t st) {
   // as many stages as fit in ~192 KB, at most 16
-  constexpr int STAGE_B = BM * BKT * 2 + BN * BKT * 2;
+  constexpr int ES = F8 ? 1 : 2;
+  constexpr int STAGE_B = BM * BKT * ES + BN * BKT * ES;
   constexpr int STAGES = (192 * 1024 / STAGE_B) > 16 ? 16 : (192 * 1024 / STAGE_B);
-  constexpr int smem = smem_bytes_for<BN, STAGES, BKT>();
-  auto kern = tc_gemm_kernel<BN, MODE, STAGES, BKT>;
+  constexpr int smem = smem_bytes_for<BN, STAGES, BKT, ES>();
+  auto kern = tc_gemm_kernel<BN, MODE, STAGES, BKT, F8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   long long grid = sm_count();
@@ -485,11 +523,12 @@ cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStre
   } else {
     BN = 256;
   }
-  const int bk = g.mode == MODE_ROUTER ? BK : MOE_GEMM_BK;
+  const bool f8 = g.fp8 != 0 && g.mode != MODE_ROUTER;
+  const int bk = f8 ? 128 : (g.mode == MODE_ROUTER ? BK : MOE_GEMM_BK);  // k per stage
   CUtensorMap a0, a1, b;
-  if (!make_map_a(&a0, g.a0, a0_rows, g.K, bk)) return cudaErrorInvalidValue;
-  if (!make_map_a(&a1, g.a1 ? g.a1 : g.a0, g.a1 ? a1_rows : a0_rows, g.K, bk)) return cudaErrorInvalidValue;
-  if (!make_map_b(&b, g.b, g.g0 + g.G, g.b_rows, g.K, BN / 2, bk)) return cudaErrorInvalidValue;
+  if (!make_map_a(&a0, g.a0, a0_rows, g.K, bk, f8)) return cudaErrorInvalidValue;
+  if (!make_map_a(&a1, g.a1 ? g.a1 : g.a0, g.a1 ? a1_rows : a0_rows, g.K, bk, f8)) return cudaErrorInvalidValue;
+  if (!make_map_b(&b, g.b, g.g0 + g.G, g.b_rows, g.K, BN / 2, bk, f8)) return cudaErrorInvalidValue;
   // upper bound on tiles: every group adds at most one partial row block
   long long rows_total = launch_rows(g);
   long long blocks = (rows_total + BM - 1) / BM + g.G;
@@ -497,8 +536,10 @@ cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStre
   long long max_tiles = blocks * n_tiles;
   switch (g.mode) {
     case MODE_FC1:
+      if (f8) return launch_bn<256, MODE_FC1, 128, true>(g, a0, a1, b, max_tiles, st);
       return launch_bn<256, MODE_FC1, MOE_GEMM_BK>(g, a0, a1, b, max_tiles, st);
     case MODE_FC2:
+      if (f8) return launch_bn<256, MODE_FC2, 128, true>(g, a0, a1, b, max_tiles, st);
       return launch_bn<256, MODE_FC2, MOE_GEMM_BK>(g, a0, a1, b, max_tiles, st);
     default:
       switch (BN) {

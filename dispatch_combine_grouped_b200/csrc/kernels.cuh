@@ -72,6 +72,11 @@ struct GemmArgs {
   const void* b;
   long long b_rows;     // rows of one weight matrix (2I, d or E)
   int max_ctas;         // cap on the persistent grid (0 = one CTA per SM)
+  // FP8 (e4m3) operands: accumulator x a_scale(row) x b_scale(weight row)
+  int fp8;
+  int k;                // top-k (FC1: routed row -> token = row2tok / k)
+  const float* a_scale; // FC1: per token [N]; FC2: per h row [A + S*N]
+  const float* b_scale; // per weight row [groups, b_rows]
 };
 
 // Rows a launch covers, for grid sizing: routed rows if any routed group is in range,
@@ -88,6 +93,13 @@ cudaError_t launch_tc_gemm_pair(const GemmArgs& g, int a0_rows, int a1_rows, cud
 // CUDA-core path, fp32 operands (the fp32 configurations)
 cudaError_t launch_simt_gemm(const GemmArgs& g, cudaStream_t st);
 
+// rows of row_bytes bytes (the FP8 dispatch payload moves d bytes per row)
+cudaError_t launch_permute_bytes(const moe_config& c, const moe_layout& L, const void* x, void* x_perm,
+                                 int row_bytes, cudaStream_t st);
+// FP8 (fp8.cu): per-row e4m3 quantisation of bf16 rows, scale = amax / 448
+cudaError_t launch_quantize_rows(const void* src, long long rows, int cols, void* dst, float* scale,
+                                 cudaStream_t st);
+
 // redundant expert slots (eplb.cu)
 size_t eplb_ws_bytes(const moe_config& c);
 cudaError_t launch_eplb_assign(const moe_config& c, const int32_t* ids, const int32_t* replica_off,
@@ -98,8 +110,8 @@ moe_status eplb_plan(int E, int R, int P, const int64_t* load, int32_t* copies, 
 
 int sm_count();
 // TMA maps for bf16 K-major operands; box_k (64, 32 or 16) selects the 128/64/32-byte swizzle
-bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K, int box_k = 64);
+bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K, int box_k = 64, bool u8 = false);
 bool make_map_b(CUtensorMap* m, const void* base, long long G, long long R, long long K, int box_rows,
-                int box_k = 64);
+                int box_k = 64, bool u8 = false);
 
 }  // namespace moe

@@ -81,10 +81,16 @@ struct FwdWs {
   void* x_perm;
   void* h;
   void* out;
+  // FP8 forward only
+  void* x_q;
+  float* x_scale;
+  void* h_q;
+  float* h_scale;
   size_t total;
 };
 
-FwdWs carve_forward(const moe_config& c, char* base) {
+// fp8: the FP8 forward's buffers (x_perm holds e4m3 rows, plus x_q, h_q and the scales)
+FwdWs carve_forward(const moe_config& c, char* base, bool fp8 = false) {
   FwdWs w;
   memset(&w, 0, sizeof(w));
   const size_t A = (size_t)c.N * c.k, E = c.E, P = c.P, S = c.n_shared, eb = elem_bytes(c);
@@ -109,9 +115,15 @@ FwdWs carve_forward(const moe_config& c, char* base) {
   w.lay.row2tok = reinterpret_cast<int32_t*>(take(A * 4));
   w.lay.tile_off = reinterpret_cast<int32_t*>(take((E + S + 1) * 4));
   w.lay_ws = take(layout_scratch(c));
-  w.x_perm = take(A * c.d * eb);
+  w.x_perm = take(A * c.d * (fp8 ? 1 : eb));
   w.h = take((A + S * c.N) * c.I * eb);
   w.out = take((A + S * c.N) * c.d * eb);
+  if (fp8) {
+    w.x_q = take((size_t)c.N * c.d);
+    w.x_scale = reinterpret_cast<float*>(take((size_t)c.N * 4));
+    w.h_q = take((A + S * c.N) * c.I);
+    w.h_scale = reinterpret_cast<float*>(take((A + S * c.N) * 4));
+  }
   w.total = off;
   return w;
 }
@@ -234,6 +246,55 @@ moe_status fc2_impl(const moe_config& c, const moe_layout& L, const void* h, con
   cudaError_t e = c.dtype == MOE_BF16 ? tc_grouped(g, c, c.N * c.k + c.n_shared * c.N, 0, st)
                                       : launch_simt_gemm(g, st);
   return cuda_status(e, "FC2 grouped GEMM");
+}
+
+// FP8 expert FFN over groups [g0, g0+G): FC1 on e4m3 rows -> h (bf16) -> per-row e4m3
+// quantisation of h -> FC2 on e4m3 rows.  Always the one-CTA tensor-core kernel.
+struct Fp8Ffn {
+  const void *x_q_perm, *x_q;
+  const float* x_scale;
+  const void* w13_q;
+  const float* w13_scale;
+  const void* w2_q;
+  const float* w2_scale;
+  const float* topk_w;
+  void* h;
+  void* h_q;
+  float* h_scale;
+  void* out;
+};
+
+moe_status ffn_fp8_impl(const moe_config& c, const moe_layout& L, const Fp8Ffn& f, cudaStream_t st, int g0 = 0,
+                        int G = -1) {
+  if (G < 0) G = c.E + c.n_shared - g0;
+  if (G == 0) return MOE_OK;
+  const long long A = (long long)c.N * c.k;
+  GemmArgs g = fc1_args(c, L, f.x_q_perm, f.x_q, f.w13_q, f.h);
+  g.g0 = g0;
+  g.G = G;
+  g.max_ctas = shared_cap(c, g0);
+  g.fp8 = 1;
+  g.k = c.k;
+  g.a_scale = f.x_scale;
+  g.b_scale = f.w13_scale;
+  cudaError_t e = launch_tc_gemm(g, (int)A, c.N, st);
+  if (e != cudaSuccess) return cuda_status(e, "FC1 grouped GEMM (fp8)");
+  // rows of h this group range wrote: all routed rows [0, A) if a routed group is in
+  // range, then the N-row blocks of the shared experts in range
+  const long long r0 = g0 < c.E ? 0 : A + (long long)(g0 - c.E) * c.N;
+  const long long r1 = (g0 + G <= c.E) ? A : A + (long long)(g0 + G - c.E) * c.N;
+  e = launch_quantize_rows(static_cast<const uint16_t*>(f.h) + r0 * c.I, r1 - r0, c.I,
+                           static_cast<uint8_t*>(f.h_q) + r0 * c.I, f.h_scale + r0, st);
+  if (e != cudaSuccess) return cuda_status(e, "h quantisation");
+  GemmArgs g2 = fc2_args(c, L, f.h_q, f.w2_q, f.topk_w, f.out);
+  g2.g0 = g0;
+  g2.G = G;
+  g2.max_ctas = shared_cap(c, g0);
+  g2.fp8 = 1;
+  g2.k = c.k;
+  g2.a_scale = f.h_scale;
+  g2.b_scale = f.w2_scale;
+  return cuda_status(launch_tc_gemm(g2, (int)(A + (long long)c.n_shared * c.N), 0, st), "FC2 grouped GEMM (fp8)");
 }
 
 moe_status ffn_impl(const moe_config& c, const moe_layout& L, const void* x_perm, const void* x, const void* w13,
@@ -542,6 +603,81 @@ moe_status moe_eplb_place_weights(const int32_t* slot_expert, int32_t n_slots, i
     if (e != cudaSuccess) return cuda_status(e, "eplb place weights");
   }
   return MOE_OK;
+}
+
+moe_status moe_quantize_fp8(const void* src, int64_t rows, int32_t cols, void* dst, float* scale,
+                            moe_stream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 8 != 0) return fail(MOE_ERR_INVALID_ARG, "need rows >= 0, cols % 8 == 0");
+  if (rows > 0 && (!src || !dst || !scale)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return cuda_status(launch_quantize_rows(src, rows, cols, dst, scale, (cudaStream_t)stream), "fp8 quantisation");
+}
+
+moe_status moe_permute_fp8(const moe_config* cfg, const moe_layout* layout, const void* x_q, void* x_q_perm,
+                           moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->N == 0) return MOE_OK;
+  if (cfg->d % 16 != 0) return fail(MOE_ERR_UNSUPPORTED, "fp8 rows need d % 16 == 0");
+  if (!layout || !layout->tok2row || !x_q || !x_q_perm) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return cuda_status(launch_permute_bytes(*cfg, *layout, x_q, x_q_perm, cfg->d, (cudaStream_t)stream),
+                     "permute (fp8)");
+}
+
+static moe_status check_fp8(const moe_config* cfg) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "the FP8 path takes a bf16 configuration");
+  if (cfg->d % 16 != 0 || cfg->I % 16 != 0) return fail(MOE_ERR_UNSUPPORTED, "fp8 rows need d, I % 16 == 0");
+  return MOE_OK;
+}
+
+moe_status moe_grouped_ffn_fp8(const moe_config* cfg, const moe_layout* layout, const void* x_q_perm,
+                               const void* x_q, const float* x_scale, const void* w13_q, const float* w13_scale,
+                               const void* w2_q, const float* w2_scale, const float* topk_w, void* h, void* h_q,
+                               float* h_scale, void* out, moe_stream_t stream) {
+  moe_status s = check_fp8(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->N == 0) return MOE_OK;
+  if (!layout || !layout_complete(layout) || !x_q_perm || !x_scale || !w13_q || !w13_scale || !w2_q || !w2_scale ||
+      !h || !h_q || !h_scale || !out || (cfg->n_shared > 0 && !x_q))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  Fp8Ffn f{x_q_perm, x_q, x_scale, w13_q, w13_scale, w2_q, w2_scale, topk_w, h, h_q, h_scale, out};
+  return ffn_fp8_impl(*cfg, *layout, f, (cudaStream_t)stream);
+}
+
+size_t moe_workspace_bytes_fp8(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return carve_forward(*cfg, nullptr, true).total;
+}
+
+moe_status moe_layer_forward_fp8(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
+                                 const int32_t* expert_owner, const void* w13_q, const float* w13_scale,
+                                 const void* w2_q, const float* w2_scale, void* y, const moe_layout* layout_out,
+                                 int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status s = check_fp8(cfg);
+  if (s != MOE_OK) return s;
+  if ((s = check_router(*cfg)) != MOE_OK) return s;
+  if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
+  const moe_config& c = *cfg;
+  FwdWs w = carve_forward(c, nullptr, true);
+  if (!ws || ws_bytes < w.total) return fail(MOE_ERR_WORKSPACE, "forward workspace too small");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return fail(MOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if (layout_out && !layout_complete(layout_out)) return fail(MOE_ERR_INVALID_ARG, "incomplete layout_out");
+  if (c.N > 0 && (!x || !w_gate || !w13_q || !w13_scale || !w2_q || !w2_scale || !y))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  w = carve_forward(c, static_cast<char*>(ws), true);
+  const moe_layout& L = layout_out ? *layout_out : w.lay;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (c.N > 0 && (s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
+  if ((s = cuda_status(launch_layout(c, expert_owner, w.ids, L, dev_status, w.lay_ws, st), "layout")) != MOE_OK)
+    return s;
+  if (c.N == 0) return MOE_OK;
+  if ((s = cuda_status(launch_quantize_rows(x, c.N, c.d, w.x_q, w.x_scale, st), "x quantisation")) != MOE_OK)
+    return s;
+  if ((s = cuda_status(launch_permute_bytes(c, L, w.x_q, w.x_perm, c.d, st), "permute (fp8)")) != MOE_OK) return s;
+  Fp8Ffn f{w.x_perm, w.x_q, w.x_scale, w13_q, w13_scale, w2_q, w2_scale, w.w, w.h, w.h_q, w.h_scale, w.out};
+  if ((s = ffn_fp8_impl(c, L, f, st)) != MOE_OK) return s;
+  return cuda_status(launch_combine(c, L, w.out, nullptr, y, st), "combine");
 }
 
 }  // extern "C"

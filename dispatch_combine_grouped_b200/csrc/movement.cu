@@ -303,17 +303,22 @@ static inline int elem_bytes(const moe_config& c) { return c.dtype == MOE_BF16 ?
 static inline int vecs_per_row(const moe_config& c) { return c.d * elem_bytes(c) / 16; }
 static inline unsigned blocks_for(long long rows) { return (unsigned)((rows + kMoveWarps - 1) / kMoveWarps); }
 
-cudaError_t launch_permute(const moe_config& c, const moe_layout& L, const void* x, void* x_perm, cudaStream_t st) {
+// x_perm[tok2row[a]] = x[a / k] for rows of row_bytes bytes (a multiple of 16)
+cudaError_t launch_permute_bytes(const moe_config& c, const moe_layout& L, const void* x, void* x_perm,
+                                 int row_bytes, cudaStream_t st) {
   if (c.N == 0) return cudaSuccess;
-  const int row_bytes = c.d * elem_bytes(c);
   if (row_bytes % 32 == 0) {
     scatter_token_rows32<<<blocks_for(c.N), kMoveWarps * 32, 0, st>>>(
         static_cast<const V32*>(x), static_cast<V32*>(x_perm), L.tok2row, c.N, c.k, row_bytes / 32);
     return cudaGetLastError();
   }
   scatter_token_rows<<<blocks_for(c.N), kMoveWarps * 32, 0, st>>>(
-      static_cast<const uint4*>(x), static_cast<uint4*>(x_perm), L.tok2row, c.N, c.k, vecs_per_row(c));
+      static_cast<const uint4*>(x), static_cast<uint4*>(x_perm), L.tok2row, c.N, c.k, row_bytes / 16);
   return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const moe_config& c, const moe_layout& L, const void* x, void* x_perm, cudaStream_t st) {
+  return launch_permute_bytes(c, L, x, x_perm, c.d * elem_bytes(c), st);
 }
 
 cudaError_t launch_permute_staged(const moe_config& c, const moe_layout& L, const void* x, void* send_buf,

@@ -390,6 +390,53 @@ moe_status moe_eplb_assign(const moe_config* cfg, const int32_t* topk_ids, const
 moe_status moe_eplb_place_weights(const int32_t* slot_expert, int32_t n_slots, int32_t E, int32_t n_shared,
                                   size_t expert_bytes, const void* w_logical, void* w_physical, moe_stream_t stream);
 
+/*
+ * FP8 (e4m3) expert path ([MoE-IV] FP8 dispatch payloads and FP8 grouped GEMMs;
+ * [WideEP] FP8 weights and dispatch; [EP-DeepEP] §7 low-precision dispatch with the
+ * combine in higher precision).  The pages fix neither format nor scaling; this library
+ * uses e4m3 without infinities (largest finite 448) and one fp32 scale per row of every
+ * operand: s = amax(|row|) / 448 (fp32 division; 1 for an all-zero row), code = round to
+ * nearest even of x / s (fp32 division), saturating at +-448.  A GEMM on e4m3 rows
+ * computes (sum_k qa qb) * s_a(row) * s_b(weight row) with fp32 accumulation.  The
+ * configuration stays bf16 (dtype = MOE_BF16): x, y, h, expert outputs and the combine are
+ * bf16 / fp32 as in the bf16 path; d % 16 == 0 and I % 16 == 0.
+ */
+
+/* Per-row quantisation: src [rows, cols] bf16 -> dst [rows, cols] e4m3 codes (one byte
+ * each), scale [rows] fp32.  cols % 8 == 0.  Used for weights (once), x and h (per step). */
+moe_status moe_quantize_fp8(const void* src, int64_t rows, int32_t cols, void* dst, float* scale,
+                            moe_stream_t stream);
+
+/* FP8 dispatch payload: x_q_perm[tok2row[a]] = x_q[a / k], rows of d bytes (the permute
+ * of moe_permute on e4m3 rows; the token scales stay in token order). */
+moe_status moe_permute_fp8(const moe_config* cfg, const moe_layout* layout, const void* x_q, void* x_q_perm,
+                           moe_stream_t stream);
+
+/*
+ * FP8 grouped SwiGLU FFN, routed and shared experts:
+ *   h   = SiLU(Xq Wq_gate^T * s) * (Xq Wq_up^T * s)     (bf16 [A + S*N, I])
+ *   h_q, h_scale = moe_quantize_fp8(h)                  (e4m3 [A + S*N, I], fp32 [A + S*N])
+ *   out = (h_q W2q^T) * h_scale(row) * w2_scale(col) * gate(row)  (bf16 [A + S*N, d])
+ *   x_q_perm [A, d] e4m3 (moe_permute_fp8), x_q [N, d] e4m3 (shared experts' rows),
+ *   x_scale [N] per token; w13_q [E+S, 2I, d] e4m3, w13_scale [E+S, 2I]; w2_q [E+S, d, I]
+ *   e4m3, w2_scale [E+S, d]; topk_w as in moe_grouped_ffn (NULL: no gate scale).
+ */
+moe_status moe_grouped_ffn_fp8(const moe_config* cfg, const moe_layout* layout, const void* x_q_perm,
+                               const void* x_q, const float* x_scale, const void* w13_q, const float* w13_scale,
+                               const void* w2_q, const float* w2_scale, const float* topk_w, void* h, void* h_q,
+                               float* h_scale, void* out, moe_stream_t stream);
+
+/* Bytes of scratch moe_layer_forward_fp8 needs. */
+size_t moe_workspace_bytes_fp8(const moe_config* cfg);
+
+/* The whole layer with the FP8 expert path, one stream: moe_route -> moe_dispatch_layout
+ * -> moe_quantize_fp8(x) -> moe_permute_fp8 -> moe_grouped_ffn_fp8 -> moe_combine.  The
+ * weights come quantised (moe_quantize_fp8 of W13 and W2 rows, once). */
+moe_status moe_layer_forward_fp8(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
+                                 const int32_t* expert_owner, const void* w13_q, const float* w13_scale,
+                                 const void* w2_q, const float* w2_scale, void* y, const moe_layout* layout_out,
+                                 int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
