@@ -38,6 +38,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--fp8", action="store_true",
+                    help="the FP8 (e4m3) expert path: quantised dispatch payload and expert GEMMs")
     ap.add_argument("--eplb", type=int, default=0, metavar="R",
                     help="run the routed experts over E + R physical slots (redundant copies of the "
                          "hot experts, planned from the batch's own counts)")
@@ -234,6 +236,133 @@ def run_reference(args, cfg, rank):
 
 
 # ------------------------------------------------------------------------------ our arm
+def run_fp8(args, cfg, world, rank, local):
+    """The layer with the FP8 expert path on one stream: route -> layout -> quantise x +
+    FP8 permute -> FP8 grouped FFN (FC1, h quantisation, FC2) -> combine.  Weights are
+    quantised once, before timing (a load-time step)."""
+    import torch
+    import torch.distributed  # noqa: F401
+    import dispatch_combine_grouped_b200 as moe
+    from moe_inputs import make_inputs
+
+    dev = torch.device("cuda", local)
+    inp = make_inputs(cfg, device=dev, seed_offset=rank)
+    A, S = cfg.N * cfg.k, cfg.S
+    rows = A + S * cfg.N
+    x, wg, bias, owner = inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"]
+    w13_q, w13_s = moe.quantize_fp8(inp["w13"])
+    w2_q, w2_s = moe.quantize_fp8(inp["w2"])
+    del inp
+    logits = torch.empty(cfg.N, cfg.E, dtype=torch.float32, device=dev)
+    ids = torch.empty(cfg.N, cfg.k, dtype=torch.int32, device=dev)
+    w = torch.empty(cfg.N, cfg.k, dtype=torch.float32, device=dev)
+    layout = moe.Layout(cfg, dev)
+    lay_ws = torch.empty(max(moe.layout_workspace_bytes(cfg), 1), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    x_q = torch.empty(cfg.N, cfg.d, dtype=torch.uint8, device=dev)
+    x_s = torch.empty(cfg.N, dtype=torch.float32, device=dev)
+    x_perm = torch.empty(A, cfg.d, dtype=torch.uint8, device=dev)
+    h = torch.empty(rows, cfg.I, dtype=torch.bfloat16, device=dev)
+    h_q = torch.empty(rows, cfg.I, dtype=torch.uint8, device=dev)
+    h_s = torch.empty(rows, dtype=torch.float32, device=dev)
+    out = torch.empty(rows, cfg.d, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(cfg.N, cfg.d, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(moe.workspace_bytes_fp8(cfg), 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step(ev):
+        ev[0].record()
+        moe.route(cfg, x, wg, bias, out=(logits, ids, w))
+        ev[1].record()
+        moe.dispatch_layout(cfg, ids, owner, status=status, layout=layout, ws=lay_ws)
+        ev[2].record()
+        moe.quantize_fp8(x, out=x_q, scale=x_s)
+        moe.permute_fp8(cfg, layout, x_q, out=x_perm)
+        ev[3].record()
+        moe.grouped_ffn_fp8(cfg, layout, x_perm, x_q, x_s, w13_q, w13_s, w2_q, w2_s, topk_w=w, h=h, h_q=h_q,
+                            h_scale=h_s, out=out)
+        ev[4].record()
+        moe.combine(cfg, layout, out, y=y)
+        ev[5].record()
+
+    def events(n):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    clocks = ClockSampler(local)
+    evs = [events(6) for _ in range(args.steps)]
+    clocks.start()
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(events(6))
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clock_rec = clocks.stop()
+    assert status.item() == 0, f"device status {status.item()}"
+    names = ["route", "layout", "quantize_permute", "ffn", "combine"]
+    stage_ms = {n: sum(ev[j].elapsed_time(ev[j + 1]) for ev in evs) / args.steps for j, n in enumerate(names)}
+    step_ms = max_over_ranks(sum(ev[0].elapsed_time(ev[5]) for ev in evs) / args.steps, world, dev)
+    fev = [events(2) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        fev[i][0].record()
+        moe.layer_forward_fp8(cfg, x, wg, bias, owner, w13_q, w13_s, w2_q, w2_s, y=y, ws=ws, status=status)
+        fev[i][1].record()
+    torch.cuda.synchronize()
+    fused_ms = sum(a.elapsed_time(b) for a, b in fev) / args.steps
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(cfg.N, cfg.d, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    eev = [events(2) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        eev[i][0].record()
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.layer_forward_fp8(cfg, x_dev, wg, bias, owner, w13_q, w13_s, w2_q, w2_s, y=y, ws=ws, status=status)
+        y_host.copy_(y, non_blocking=True)
+        eev[i][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eev) / args.steps, world, dev)
+
+    alg = algorithmic(cfg)
+    peaks, peak_src = load_peaks()
+    fp8_peak = 2.0 * peaks["bf16_tflops"]  # e4m3 dense rate = 2 x bf16 (4.5 vs 2.25 PFLOP/s nominal)
+    ffn_tflops = alg["ffn_flops"] / (stage_ms["ffn"] / 1e3) / 1e12
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": whole_job_tokens_per_s(cfg.N, world, step_ms), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 expert GEMM operands and dispatch payload (fp32 accumulate), bf16 activations",
+            "data": "synthetic (seeded normal inputs, random-init weights)",
+            "config": {"workload": describe(cfg) + " with the FP8 expert path", "tokens_per_gpu": cfg.N,
+                       "l2": "flushed before every step (256 MiB write, outside the step's event bracket)",
+                       "parallelism": f"{world} independent replicas (one batch per GPU)"},
+            "roofline": {"kernel": "FP8 grouped FFN (FC1 + h quantisation + FC2, tcgen05 kind::f8f6f4)",
+                         "bound": "tensor", "achieved": ffn_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": ffn_tflops / fp8_peak,
+                         "peak_source": f"{peak_src} bf16 burst x 2 (nominal e4m3 / bf16 ratio)",
+                         "traffic": None, "flops_per_launch": alg["ffn_flops"], "ms_per_launch": stage_ms["ffn"]},
+            "stages_ms": stage_ms,
+            "ffn": {"tflops": ffn_tflops, "frac_of_fp8_peak": ffn_tflops / fp8_peak,
+                    "frac_of_bf16_peak": ffn_tflops / peaks["bf16_tflops"]},
+            "fused_ms_per_step": fused_ms,
+            "e2e": {"value": whole_job_tokens_per_s(cfg.N, world, e2e_ms), "unit": "tokens/s",
+                    "h2d_bytes_per_step": x.numel() * x.element_size(),
+                    "d2h_bytes_per_step": y.numel() * y.element_size()},
+            "gpu_launches": 11 * args.steps,
+            "clocks": clock_rec,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     from moe_inputs import CONFIGS
@@ -250,6 +379,12 @@ def main():
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.fp8:
+        run_fp8(args, cfg, world, rank, local)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
     import dispatch_combine_grouped_b200 as moe
     from moe_inputs import make_inputs
