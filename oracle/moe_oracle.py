@@ -40,6 +40,10 @@ Readings where the pages are silent (each is listed in the design notes):
   * Return row = send slot (the combine all-to-all is the inverse transpose).
   * Shared experts are added with weight 1.
   * A correction bias (bias_mode "selection") shifts the selection keys only.
+  * Capacity ([EP-DeepEP] §4, capacity factor): an expert receives at most
+    ceil(factor * N * k / E) assignments, the first ones in ascending a; the others are
+    dropped (id -1): they take no row and add nothing to y, and the gates of the kept
+    assignments are left as they are.
 """
 from __future__ import annotations
 
@@ -203,15 +207,20 @@ def dispatch_layout(ids, E: int, P: int, expert_owner=None, S: int = 0) -> dict:
     Returns int64 arrays:
       n_e[E], expert_off[E+1], C[P,P], send_off[P,P], recv_off[P+1],
       tok2send[A], send2row[A], ret2tok[A], tok2row[A], row2tok[A], tile_off[E+S+1].
+    Dropped assignments (id -1) take no row and no send slot: their tok2send / tok2row
+    are -1, and the slots / rows past the A_kept used ones are -1 in send2row, ret2tok
+    and row2tok; expert_off[E] = A_kept.
     """
     ids = i64(ids)
     N, k = ids.shape
     A = N * k
     owner = default_owner(E, P) if expert_owner is None else i64(expert_owner)
-    flat = ids.reshape(-1)                       # expert of assignment a = t*k + slot
-    a_idx = np.arange(A, dtype=np.int64)
-    src = source_of_token(N, P)[a_idx // k]      # source rank of each assignment
-    dst = owner[flat]                            # destination owner of each assignment
+    flat_all = ids.reshape(-1)                   # expert of assignment a = t*k + slot
+    kept = np.flatnonzero(flat_all >= 0)         # assignments that are dispatched
+    A_kept = len(kept)
+    flat = flat_all[kept]
+    src = source_of_token(N, P)[kept // k]       # source rank of each kept assignment
+    dst = owner[flat]                            # destination owner of each kept assignment
 
     n_e = np.bincount(flat, minlength=E).astype(np.int64)
 
@@ -220,9 +229,10 @@ def dispatch_layout(ids, E: int, P: int, expert_owner=None, S: int = 0) -> dict:
         C[i, j] += 1
 
     # Send buffer: each source buckets its assignments by owner, keeping token order.
-    send_list = np.lexsort((a_idx, dst, src))    # primary src, then owner, then a
-    tok2send = np.empty(A, dtype=np.int64)
-    tok2send[send_list] = np.arange(A)
+    order_send = np.lexsort((kept, dst, src))    # primary src, then owner, then a
+    send_list = kept[order_send]                 # assignment in each send slot
+    tok2send = np.full(A, -1, dtype=np.int64)
+    tok2send[send_list] = np.arange(A_kept)
     send_off = np.zeros((P, P), dtype=np.int64)
     flatC = C.reshape(-1)
     send_off.reshape(-1)[1:] = np.cumsum(flatC)[:-1]
@@ -230,20 +240,23 @@ def dispatch_layout(ids, E: int, P: int, expert_owner=None, S: int = 0) -> dict:
     # Receive buffers (the transpose): owner j gets blocks i->j for i = 0..P-1 in order.
     rows = []
     R = np.zeros(P, dtype=np.int64)
+    dst_of = np.full(A, -1, dtype=np.int64)
+    dst_of[kept] = dst
     for j in range(P):
-        recv_j = send_list[dst[send_list] == j]  # source-major, token order inside
+        recv_j = send_list[dst_of[send_list] == j]  # source-major, token order inside
         R[j] = len(recv_j)
-        order = np.argsort(flat[recv_j], kind="stable")   # expert-local order
+        order = np.argsort(flat_all[recv_j], kind="stable")   # expert-local order
         rows.append(recv_j[order])
     row_list = np.concatenate(rows) if rows else np.zeros(0, dtype=np.int64)
     recv_off = np.zeros(P + 1, dtype=np.int64)
     recv_off[1:] = np.cumsum(R)
 
-    row2tok = row_list
-    tok2row = np.empty(A, dtype=np.int64)
-    tok2row[row2tok] = np.arange(A)
-    send2row = tok2row[send_list]
-    ret2tok = send_list.copy()
+    tail = np.full(A - A_kept, -1, dtype=np.int64)
+    row2tok = np.concatenate([row_list, tail])
+    tok2row = np.full(A, -1, dtype=np.int64)
+    tok2row[row_list] = np.arange(A_kept)
+    send2row = np.concatenate([tok2row[send_list], tail])
+    ret2tok = np.concatenate([send_list, tail])
 
     # expert_off[e]: first row of expert e; experts follow owner order, then id order.
     expert_off = np.zeros(E + 1, dtype=np.int64)
@@ -253,7 +266,7 @@ def dispatch_layout(ids, E: int, P: int, expert_owner=None, S: int = 0) -> dict:
             if owner[e] == j:
                 expert_off[e] = run
                 run += n_e[e]
-    expert_off[E] = A
+    expert_off[E] = A_kept
 
     # Row-block prefix over groups in id order (routed experts, then S shared groups of N rows).
     blocks = [-(-int(n) // TILE_M) for n in n_e] + [-(-N // TILE_M)] * S
@@ -290,12 +303,13 @@ def swiglu_expert(x_rows, w13_e, w2_e) -> np.ndarray:
 
 
 def permute(x, layout, k: int) -> np.ndarray:
-    """x_perm[tok2row[a]] = x[a // k]  (token rows in expert-contiguous order)."""
+    """x_perm[tok2row[a]] = x[a // k]  (token rows in expert-contiguous order); rows past
+    the kept ones stay zero."""
     x = f64(x)
     tok2row = layout["tok2row"]
-    out = np.empty((len(tok2row), x.shape[1]))
-    a = np.arange(len(tok2row))
-    out[tok2row] = x[a // k]
+    out = np.zeros((len(tok2row), x.shape[1]))
+    a = np.flatnonzero(tok2row >= 0)
+    out[tok2row[a]] = x[a // k]
     return out
 
 
@@ -306,7 +320,8 @@ def combine(o_rows, layout, gates, N: int, k: int, shared_out=None) -> np.ndarra
     y = np.zeros((N, o_rows.shape[1]))
     for slot in range(k):
         rows = layout["tok2row"][np.arange(N) * k + slot]
-        y += g[:, slot:slot + 1] * o_rows[rows]
+        live = rows >= 0  # a dropped assignment adds nothing
+        y[live] += g[live, slot:slot + 1] * o_rows[rows[live]]
     if shared_out is not None:
         for so in shared_out:
             y += so
@@ -354,7 +369,8 @@ def moe_tokens_direct(cfg, x, ids, gates, w13, w2, tokens) -> np.ndarray:
     by_expert = {}
     for n, t in enumerate(tokens):
         for slot in range(ids.shape[1]):
-            by_expert.setdefault(int(ids[t, slot]), []).append((n, t, slot))
+            if ids[t, slot] >= 0:  # a dropped assignment adds nothing
+                by_expert.setdefault(int(ids[t, slot]), []).append((n, t, slot))
     for e, lst in sorted(by_expert.items()):
         rows = np.array([t for _, t, _ in lst])
         oe = swiglu_expert(x[rows], w13[e], w2[e])
@@ -363,3 +379,20 @@ def moe_tokens_direct(cfg, x, ids, gates, w13, w2, tokens) -> np.ndarray:
     for s in range(cfg.S):
         out += swiglu_expert(x[tokens], w13[cfg.E + s], w2[cfg.E + s])
     return out
+
+
+def capacity(factor: float, N: int, k: int, E: int) -> int:
+    """Assignments one expert may receive: ceil(factor * N * k / E) ([EP-DeepEP] §4: the
+    uniform share N k / E times the capacity factor)."""
+    return int(np.ceil(factor * N * k / E))
+
+
+def capacity_keep(ids, E: int, cap: int) -> np.ndarray:
+    """Ids with every assignment past the first `cap` of its expert (ascending a) set to -1."""
+    ids = i64(ids)
+    flat = ids.reshape(-1).copy()
+    for e in range(E):
+        rows = np.flatnonzero(flat == e)
+        flat[rows[cap:]] = -1
+    return flat.reshape(ids.shape)
+

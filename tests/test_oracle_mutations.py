@@ -157,3 +157,30 @@ def test_fp8_ties_away_from_even_are_caught(monkeypatch):
 def test_fp8_wrong_scale_is_caught(monkeypatch):
     monkeypatch.setattr(F8, "E4M3_MAX", 240.0)
     _fails(fp8_pins.test_row_quantisation)
+
+
+# ---- capacity (dropped assignments)
+import tests.test_capacity_oracle as cap_pins
+
+
+def test_dropping_the_first_instead_of_the_last_is_caught(monkeypatch):
+    def last(ids, E, cap):
+        ids = O.i64(ids)
+        flat = ids.reshape(-1).copy()
+        for e in range(E):
+            rows = np.flatnonzero(flat == e)
+            flat[rows[:max(len(rows) - cap, 0)]] = -1
+        return flat.reshape(ids.shape)
+    monkeypatch.setattr(O, "capacity_keep", last)
+    _fails(cap_pins.check_worked_example)
+
+
+def test_dropped_rows_leaking_into_combine_are_caught(monkeypatch):
+    orig = O.combine
+
+    def leaky(o_rows, layout, gates, N, k, shared_out=None):
+        lay = dict(layout)
+        lay["tok2row"] = np.where(layout["tok2row"] < 0, 0, layout["tok2row"])
+        return orig(o_rows, lay, gates, N, k, shared_out)
+    monkeypatch.setattr(O, "combine", leaky)
+    _fails(cap_pins.check_layout_path_with_drops, 0.8)
