@@ -31,7 +31,7 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_con
             "moe_combine", "moe_combine_staged",
             "moe_layer_forward", "moe_eplb_plan", "moe_eplb_workspace_bytes", "moe_eplb_assign",
             "moe_eplb_place_weights", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8",
-            "moe_workspace_bytes_fp8", "moe_layer_forward_fp8"]
+            "moe_workspace_bytes_fp8", "moe_layer_forward_fp8", "moe_capacity_drop"]
 
 
 class CConfig(ctypes.Structure):
@@ -98,6 +98,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_grouped_ffn_fp8": (i32, [cfgp, layp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_workspace_bytes_fp8": (sz, [cfgp]),
         "moe_layer_forward_fp8": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp]),
+        "moe_capacity_drop": (i32, [cfgp, vp, i32, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -466,4 +467,26 @@ def layer_forward_fp8(cfg, x, w_gate, bias, expert_owner, w13_q, w13_scale, w2_q
                                         ctypes.byref(layout.c) if layout is not None else None, _p(status), _p(ws),
                                         ws.numel(), _stream()), "moe_layer_forward_fp8")
     return y
+
+
+# ---------------------------------------------------------------- capacity factor
+def capacity_of(factor: float, cfg) -> int:
+    """ceil(factor * N * k / E): the uniform share of one expert times the factor."""
+    import math
+    return int(math.ceil(factor * cfg.N * cfg.k / cfg.E))
+
+
+def capacity_drop(cfg, topk_ids, capacity: int, status=None, out=None, ws=None):
+    """moe_capacity_drop: topk_ids with the assignments past each expert's first
+    `capacity` (ascending a) set to -1."""
+    c = c_config(cfg)
+    lib = load()
+    if out is None:
+        out = torch.empty_like(topk_ids)
+    if ws is None:
+        ws = torch.empty(max(lib.moe_eplb_workspace_bytes(ctypes.byref(c)), 1), dtype=torch.uint8,
+                         device=topk_ids.device)
+    _check(lib.moe_capacity_drop(ctypes.byref(c), _p(topk_ids), int(capacity), _p(out), _p(status), _p(ws),
+                                 ws.numel(), _stream()), "moe_capacity_drop")
+    return out
 

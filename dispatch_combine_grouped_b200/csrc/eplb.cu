@@ -1,4 +1,5 @@
-// Redundant expert slots (EPLB): plan, replica assignment, weight placement.
+// Redundant expert slots (EPLB): plan, replica assignment, weight placement; and the
+// capacity cut, which needs the same per-expert rank of each assignment.
 //
 // "Wide EP：当 MoE Expert Parallel 横跨几十张 GPU", sections "为什么要把 EP 做宽"
 // (E logical experts + R copies = E + R physical experts, E_local = (E + R) / P_e per
@@ -34,6 +35,10 @@ __global__ void eplb_assign_kernel(const int32_t* __restrict__ ids, const int32_
   const int a = blockIdx.x * blockDim.x + threadIdx.x;
   if (a >= A) return;
   int e = ids[a];
+  if (e == -1) {  // a dropped assignment stays dropped
+    phys[a] = -1;
+    return;
+  }
   if (e < 0 || e >= E) {  // the layout pass counted it as expert 0 as well
     report(status, MOE_ERR_BAD_INDEX);
     e = 0;
@@ -99,6 +104,22 @@ static moe_config one_owner(const moe_config& c) {
 
 size_t eplb_ws_bytes(const moe_config& c) { return carve_eplb(one_owner(c), nullptr).total; }
 
+// Capacity ("ep_deepep" explainer §4): the q-th assignment of expert e (ascending a) is
+// kept when q < capacity, else dropped (-1).  q comes from the same one-owner layout.
+__global__ void capacity_keep_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ tok2row,
+                                     const int32_t* __restrict__ expert_off, int A, int E, int capacity,
+                                     int32_t* __restrict__ kept) {
+  const int a = blockIdx.x * blockDim.x + threadIdx.x;
+  if (a >= A) return;
+  int e = ids[a];
+  if (e == -1) {
+    kept[a] = -1;
+    return;
+  }
+  if (e < 0 || e >= E) e = 0;  // reported by the layout pass, counted as expert 0 there
+  kept[a] = (tok2row[a] - expert_off[e] < capacity) ? e : -1;
+}
+
 cudaError_t launch_eplb_assign(const moe_config& c, const int32_t* ids, const int32_t* replica_off,
                                const int32_t* replica_slots, int n_slots, int32_t* phys, int32_t* status, void* ws,
                                cudaStream_t st) {
@@ -110,6 +131,19 @@ cudaError_t launch_eplb_assign(const moe_config& c, const int32_t* ids, const in
   if (A == 0) return cudaSuccess;
   eplb_assign_kernel<<<(A + 255) / 256, 256, 0, st>>>(ids, w.lay.tok2row, w.lay.expert_off, replica_off,
                                                       replica_slots, A, c.E, n_slots, phys, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_capacity_keep(const moe_config& c, const int32_t* ids, int capacity, int32_t* kept,
+                                 int32_t* status, void* ws, cudaStream_t st) {
+  const moe_config o = one_owner(c);
+  EplbWs w = carve_eplb(o, ws);
+  cudaError_t e = launch_layout(o, nullptr, ids, w.lay, status, w.scratch, st);
+  if (e != cudaSuccess) return e;
+  const int A = c.N * c.k;
+  if (A == 0) return cudaSuccess;
+  capacity_keep_kernel<<<(A + 255) / 256, 256, 0, st>>>(ids, w.lay.tok2row, w.lay.expert_off, A, c.E, capacity,
+                                                        kept);
   return cudaGetLastError();
 }
 

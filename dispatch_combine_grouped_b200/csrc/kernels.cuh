@@ -105,6 +105,8 @@ size_t eplb_ws_bytes(const moe_config& c);
 cudaError_t launch_eplb_assign(const moe_config& c, const int32_t* ids, const int32_t* replica_off,
                                const int32_t* replica_slots, int n_slots, int32_t* phys, int32_t* status, void* ws,
                                cudaStream_t st);
+cudaError_t launch_capacity_keep(const moe_config& c, const int32_t* ids, int capacity, int32_t* kept,
+                                 int32_t* status, void* ws, cudaStream_t st);
 moe_status eplb_plan(int E, int R, int P, const int64_t* load, int32_t* copies, int32_t* replica_off,
                      int32_t* replica_slots, int32_t* slot_expert, int32_t* slot_owner, int64_t* owner_load);
 

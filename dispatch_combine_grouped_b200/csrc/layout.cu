@@ -58,8 +58,10 @@ struct LayoutArgs {
   int* status;
 };
 
+// Expert of assignment a; -1 marks a dropped assignment (capacity), which takes no row.
 __device__ __forceinline__ int expert_of(const LayoutArgs& p, int a) {
   int e = p.ids[a];
+  if (e == -1) return -1;
   if (e < 0 || e >= p.E) {
     report(p.status, MOE_ERR_BAD_INDEX);
     e = 0;
@@ -101,12 +103,12 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_count_kernel(LayoutArgs
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int r = 0; r < kLayoutChunk / kLayoutThreads; ++r) {
     const int a = a_begin + r * kLayoutThreads + tid;
-    const bool valid = a < p.A;
     int e = -1, j = -1;
-    if (valid) {
+    if (a < p.A) {
       e = expert_of(p, a);
-      j = owner_of(p, e);
+      if (e >= 0) j = owner_of(p, e);
     }
+    const bool valid = e >= 0;  // in range and not dropped
     const unsigned me = __match_any_sync(0xffffffffu, e);
     const unsigned mj = __match_any_sync(0xffffffffu, j);
     const int lre = __popc(me & lt_mask), lrj = __popc(mj & lt_mask);
@@ -277,7 +279,7 @@ __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutArgs p,
       L.expert_off[tid] = s;
     }
   }
-  if (tid == 0) L.expert_off[p.E] = p.A;
+  if (tid == 0) L.expert_off[p.E] = s_recv[p.P];  // rows in use (A minus dropped)
 
   // tile_off: prefix of ceil(rows / 128) over routed experts then shared groups
   {
@@ -295,7 +297,18 @@ __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutArgs p,
 __global__ void layout_maps_kernel(LayoutArgs p, LayoutWs w, moe_layout L) {
   const int a = blockIdx.x * blockDim.x + threadIdx.x;
   if (a >= p.A) return;
+  // rows and send slots past the ones in use (dropped assignments) are marked -1
+  if (a >= L.recv_off[p.P]) {
+    L.row2tok[a] = -1;
+    L.ret2tok[a] = -1;
+    L.send2row[a] = -1;
+  }
   const int e = expert_of(p, a);
+  if (e < 0) {
+    L.tok2send[a] = -1;
+    L.tok2row[a] = -1;
+    return;
+  }
   const int j = owner_of(p, e);
   const int c = a / kLayoutChunk;
   const int i = (a / p.k) / p.shard;

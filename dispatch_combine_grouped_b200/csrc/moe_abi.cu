@@ -680,4 +680,16 @@ moe_status moe_layer_forward_fp8(const moe_config* cfg, const void* x, const voi
   return cuda_status(launch_combine(c, L, w.out, nullptr, y, st), "combine");
 }
 
+moe_status moe_capacity_drop(const moe_config* cfg, const int32_t* topk_ids, int32_t capacity, int32_t* kept_ids,
+                             int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (capacity < 0) return fail(MOE_ERR_INVALID_ARG, "capacity must be >= 0");
+  if (cfg->N > 0 && (!topk_ids || !kept_ids)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!ws || ws_bytes < eplb_ws_bytes(*cfg)) return fail(MOE_ERR_WORKSPACE, "capacity workspace too small");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return fail(MOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  return cuda_status(launch_capacity_keep(*cfg, topk_ids, capacity, kept_ids, dev_status, ws, (cudaStream_t)stream),
+                     "capacity");
+}
+
 }  // extern "C"

@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(kMoveWarps * 32) scatter_token_rows(const uint
     }
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
-      if (j < k) {
+      if (j < k && rows[j] >= 0) {  // a dropped assignment (-1) has no row
         uint4* d = dst + (size_t)rows[j] * vpr;
 #pragma unroll
         for (int u = 0; u < kMoveUnroll; ++u) {
@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kMoveWarps * 32) scatter_token_rows32(const V3
     }
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
-      if (j < k) {
+      if (j < k && rows[j] >= 0) {  // a dropped assignment (-1) has no row
         V32* d = dst + (size_t)rows[j] * vpr;
 #pragma unroll
         for (int u = 0; u < kMoveUnroll; ++u) {
@@ -122,6 +122,7 @@ __global__ void __launch_bounds__(kMoveWarps * 32) move_rows(const uint4* __rest
   const int i = blockIdx.x * kMoveWarps + (threadIdx.x >> 5);
   if (i >= rows) return;
   const int m = map[i];
+  if (m < 0) return;  // an unused slot / a dropped assignment
   const uint4* s = src + (size_t)(kScatter ? i : m) * vpr;
   uint4* d = dst + (size_t)(kScatter ? m : i) * vpr;
   for (int v0 = 0; v0 < vpr; v0 += 32 * kMoveUnroll) {
@@ -205,7 +206,7 @@ __global__ void __launch_bounds__(kMoveWarps * 32) combine_kernel(const uint4* _
     const int v = v0 + u * 32;
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j)
-      if (j < k && v < vpr) q[u][j] = ld_stream(routed + (size_t)rows[j] * vpr + v);
+      if (j < k && rows[j] >= 0 && v < vpr) q[u][j] = ld_stream(routed + (size_t)rows[j] * vpr + v);
   }
 #pragma unroll
   for (int u = 0; u < kCombVec; ++u) {
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(kMoveWarps * 32) combine_kernel(const uint4* _
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
-      if (j < k) {
+      if (j < k && rows[j] >= 0) {  // a dropped assignment adds nothing
         float f[8];
         Vec<T>::unpack(q[u][j], f);
 #pragma unroll
@@ -259,14 +260,14 @@ __global__ void __launch_bounds__(kMoveWarps * 32) combine_kernel32(const V32* _
   V32 q[kMaxK];
 #pragma unroll
   for (int j = 0; j < kMaxK; ++j)
-    if (j < k) q[j] = ld_stream32(routed + (size_t)rows[j] * vpr + v);
+    if (j < k && rows[j] >= 0) q[j] = ld_stream32(routed + (size_t)rows[j] * vpr + v);
   constexpr int n = Vec<T>::n;  // elements per 16 bytes
   float acc[2 * 8];
 #pragma unroll
   for (int i = 0; i < 2 * n; ++i) acc[i] = 0.f;
 #pragma unroll
   for (int j = 0; j < kMaxK; ++j) {
-    if (j < k) {
+    if (j < k && rows[j] >= 0) {  // a dropped assignment adds nothing
       float f[8];
       Vec<T>::unpack(make_uint4(q[j].w[0], q[j].w[1], q[j].w[2], q[j].w[3]), f);
 #pragma unroll

@@ -356,7 +356,25 @@ moe_status moe_eplb_plan(int32_t E, int32_t R, int32_t P, const int64_t* load, i
                          int32_t* replica_off, int32_t* replica_slots, int32_t* slot_expert, int32_t* slot_owner,
                          int64_t* owner_load);
 
-/* Bytes of scratch moe_eplb_assign needs (a one-owner dispatch layout of the logical ids). */
+/*
+ * Capacity factor with dropping ([EP-DeepEP] §4: a capacity factor caps the assignments an
+ * expert receives per round and the excess may be dropped): the q-th assignment of expert
+ * e in ascending a = t*k + slot is kept when q < capacity, else dropped.  kept_ids [N, k]
+ * = topk_ids with the dropped ones set to -1 (a -1 in topk_ids stays -1).  The usual
+ * capacity is ceil(factor * N * k / E).  A dropped assignment takes no row and no send
+ * slot: moe_dispatch_layout gives it tok2row = tok2send = -1, counts only the kept ones
+ * (expert_off[E] = recv_off[P] = the rows in use, A_kept), and marks the unused tails
+ * [A_kept, A) of row2tok, send2row and ret2tok with -1; the permute skips it and the
+ * combine adds nothing for it (the other gates are not renormalised).  Routed rows of the
+ * FFN buffers are [0, A_kept); shared experts' rows still start at A = N*k.
+ *   ws, ws_bytes: at least moe_eplb_workspace_bytes(cfg), 256-byte aligned.
+ * Device errors: ids outside [0, E) other than -1 -> MOE_ERR_BAD_INDEX (counted as 0).
+ */
+moe_status moe_capacity_drop(const moe_config* cfg, const int32_t* topk_ids, int32_t capacity, int32_t* kept_ids,
+                             int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Bytes of scratch moe_eplb_assign and moe_capacity_drop need (a one-owner dispatch
+ * layout of the logical ids). */
 size_t moe_eplb_workspace_bytes(const moe_config* cfg);
 
 /*
