@@ -17,6 +17,8 @@
 //              accumulator barriers of both CTAs; both CTAs: TMEM alloc / dealloc
 //   warps 2-5  epilogue of this CTA's 128 rows, from its own TMEM; each warp releases
 //              the accumulator to both CTAs' barriers
+// F8: e4m3 operands, a 128-element k-step (the same 128-byte rows), kind::f8f6f4 MMAs and
+// the row x column scales applied to the accumulator in the epilogue.
 // No TMA multicast is used.  Every wait is bounded (2 s); on timeout the kernel writes
 // MOE_ERR_TIMEOUT and every role leaves its loop.
 #include <cudaTypedefs.h>
@@ -41,12 +43,13 @@ constexpr int kPairSmem = 1024 + kPairStages * STAGE_BYTES + 256 + 4 * (4 * kPai
 
 }  // namespace
 
-template <int MODE>
+template <int MODE, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                         const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
   constexpr uint32_t TMEM_COLS = 2 * PN;  // double-buffered 128 x 256 fp32 accumulator
-  constexpr uint32_t IDESC = idesc_bf16_f32(PM, PN);
+  constexpr uint32_t IDESC = F8 ? idesc_e4m3_f32(PM, PN) : idesc_bf16_f32(PM, PN);
+  constexpr int KSTEP = F8 ? 2 * PK : PK;  // elements of k per stage (128-byte rows either way)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -131,7 +134,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const uint32_t tmem_base = *tmem_holder;
   const int n_tiles = (MODE == MODE_FC1) ? (p.n_out + PN / 2 - 1) / (PN / 2) : (p.n_out + PN - 1) / PN;
   const int total = s_prefix[G] * n_tiles;
-  const int num_kb = (p.K + PK - 1) / PK;
+  const int num_kb = (p.K + KSTEP - 1) / KSTEP;
   const int pair_id = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
   volatile int* abort_v = abort_flag;
 
@@ -166,8 +169,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           }
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
           const uint32_t bar = lead_full0 + (uint32_t)(stage * sizeof(uint64_t));
-          tma_load_2d_pair(sA + stage * A_BYTES, mapA, bar, kb * PK, a_row);
-          tma_load_3d_pair(sB + stage * B_BYTES, &tmB, bar, kb * PK, b_row, gz);
+          tma_load_2d_pair(sA + stage * A_BYTES, mapA, bar, kb * KSTEP, a_row);
+          tma_load_3d_pair(sB + stage * B_BYTES, &tmB, bar, kb * KSTEP, b_row, gz);
           if (++stage == kPairStages) {
             stage = 0;
             ph ^= 1u;
@@ -203,9 +206,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < PK / 16; ++kk) {
-            umma_bf16_pair(d_tmem, smem_desc_k128(a_addr + kk * 32), smem_desc_k128(b_addr + kk * 32), IDESC,
-                           (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {  // 32 bytes of k per MMA
+            if (F8)
+              umma_e4m3_pair(d_tmem, smem_desc_k128(a_addr + kk * 32), smem_desc_k128(b_addr + kk * 32), IDESC,
+                             (kb | kk) != 0 ? 1u : 0u);
+            else
+              umma_bf16_pair(d_tmem, smem_desc_k128(a_addr + kk * 32), smem_desc_k128(b_addr + kk * 32), IDESC,
+                             (kb | kk) != 0 ? 1u : 0u);
           }
           any = true;
           umma_commit_pair(&empty[stage], 0x3);  // frees this stage in both CTAs
@@ -264,12 +271,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + orow * p.ldo;
       if (MODE == MODE_FC1) {
         const int col_base = n_blk * (PN / 2);
+        float ra = 1.0f;  // FP8: scale of this row's token
+        const float* sb = nullptr;
+        if (F8) {
+          const int gz = p.g0 + g;
+          // token of the row: routed rows through row2tok; a shared expert's rows are the
+          // tokens in order, after A_routed and the earlier shared experts' blocks
+          if (row_ok)
+            ra = p.a_scale[gz < p.E ? p.row2tok[orow] / p.k : (int)(orow - p.A_routed - (long long)(gz - p.E) * p.N)];
+          sb = p.b_scale + (size_t)gz * p.b_rows;
+        }
 #pragma unroll 1
         for (int c0 = 0; c0 < PN / 2; c0 += 32) {
           uint32_t gv[32], uv[32];
           tmem_ld32(taddr + c0, gv);
           tmem_ld32(taddr + PN / 2 + c0, uv);
           tmem_wait_ld();
+          if (F8 && row_ok) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              const int col = min(col_base + c0 + q, p.n_out - 1);
+              gv[q] = __float_as_uint(__uint_as_float(gv[q]) * ra * __ldg(sb + col));
+              uv[q] = __float_as_uint(__uint_as_float(uv[q]) * ra * __ldg(sb + p.I + col));
+            }
+          }
           if (row_ok) {
 #pragma unroll
             for (int q = 0; q < 32; q += 8) {
@@ -291,12 +316,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       } else {
         float scale = 1.0f;
         if (row_ok && p.gate_w && p.g0 + g < p.E) scale = p.gate_w[p.row2tok[orow]];
+        const float* sb = nullptr;
+        if (F8) {
+          if (row_ok) scale *= p.a_scale[orow];  // FP8: scale of this h row
+          sb = p.b_scale + (size_t)(p.g0 + g) * p.b_rows;
+        }
         const int col_base = n_blk * PN;
 #pragma unroll 1
         for (int c0 = 0; c0 < PN; c0 += 32) {
           uint32_t v[32];
           tmem_ld32(taddr + c0, v);
           tmem_wait_ld();
+          if (F8 && row_ok) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              v[q] = __float_as_uint(__uint_as_float(v[q]) * __ldg(sb + min(col_base + c0 + q, p.n_out - 1)));
+          }
           if (row_ok) {
 #pragma unroll
             for (int q = 0; q < 32; q += 8) {
@@ -334,9 +369,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
 cudaError_t launch_tc_gemm_pair(const GemmArgs& g, int a0_rows, int a1_rows, cudaStream_t st) {
   CUtensorMap a0, a1, b;
-  if (!make_map_a(&a0, g.a0, a0_rows, g.K)) return cudaErrorInvalidValue;
-  if (!make_map_a(&a1, g.a1 ? g.a1 : g.a0, g.a1 ? a1_rows : a0_rows, g.K)) return cudaErrorInvalidValue;
-  if (!make_map_b(&b, g.b, g.g0 + g.G, g.b_rows, g.K, PN / 2)) return cudaErrorInvalidValue;
+  const bool f8 = g.fp8 != 0;
+  const int bk = f8 ? 2 * PK : PK;
+  if (!make_map_a(&a0, g.a0, a0_rows, g.K, bk, f8)) return cudaErrorInvalidValue;
+  if (!make_map_a(&a1, g.a1 ? g.a1 : g.a0, g.a1 ? a1_rows : a0_rows, g.K, bk, f8)) return cudaErrorInvalidValue;
+  if (!make_map_b(&b, g.b, g.g0 + g.G, g.b_rows, g.K, PN / 2, bk, f8)) return cudaErrorInvalidValue;
   const long long rows_total = launch_rows(g);
   const long long pairs = (rows_total + PM - 1) / PM + g.G;
   const long long n_tiles = g.mode == MODE_FC1 ? (g.n_out + PN / 2 - 1) / (PN / 2) : (g.n_out + PN - 1) / PN;
@@ -344,17 +381,14 @@ cudaError_t launch_tc_gemm_pair(const GemmArgs& g, int a0_rows, int a1_rows, cud
   if (g.max_ctas > 0 && g.max_ctas < grid) grid = (g.max_ctas / 2) * 2;
   if (2 * pairs * n_tiles < grid) grid = 2 * pairs * n_tiles;
   if (grid < 2) grid = 2;
-  cudaError_t e;
-  if (g.mode == MODE_FC1) {
-    e = cudaFuncSetAttribute(tc_gemm_pair_kernel<MODE_FC1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
+  auto run = [&](auto kern) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
     if (e != cudaSuccess) return e;
-    tc_gemm_pair_kernel<MODE_FC1><<<(unsigned)grid, kPairThreads, kPairSmem, st>>>(a0, a1, b, g);
-  } else {
-    e = cudaFuncSetAttribute(tc_gemm_pair_kernel<MODE_FC2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
-    if (e != cudaSuccess) return e;
-    tc_gemm_pair_kernel<MODE_FC2><<<(unsigned)grid, kPairThreads, kPairSmem, st>>>(a0, a1, b, g);
-  }
-  return cudaGetLastError();
+    kern<<<(unsigned)grid, kPairThreads, kPairSmem, st>>>(a0, a1, b, g);
+    return cudaGetLastError();
+  };
+  if (g.mode == MODE_FC1) return f8 ? run(tc_gemm_pair_kernel<MODE_FC1, true>) : run(tc_gemm_pair_kernel<MODE_FC1, false>);
+  return f8 ? run(tc_gemm_pair_kernel<MODE_FC2, true>) : run(tc_gemm_pair_kernel<MODE_FC2, false>);
 }
 
 }  // namespace moe

@@ -249,7 +249,7 @@ moe_status fc2_impl(const moe_config& c, const moe_layout& L, const void* h, con
 }
 
 // FP8 expert FFN over groups [g0, g0+G): FC1 on e4m3 rows -> h (bf16) -> per-row e4m3
-// quantisation of h -> FC2 on e4m3 rows.  Always the one-CTA tensor-core kernel.
+// quantisation of h -> FC2 on e4m3 rows, on the same tile kernels as bf16.
 struct Fp8Ffn {
   const void *x_q_perm, *x_q;
   const float* x_scale;
@@ -277,7 +277,7 @@ moe_status ffn_fp8_impl(const moe_config& c, const moe_layout& L, const Fp8Ffn& 
   g.k = c.k;
   g.a_scale = f.x_scale;
   g.b_scale = f.w13_scale;
-  cudaError_t e = launch_tc_gemm(g, (int)A, c.N, st);
+  cudaError_t e = tc_grouped(g, c, (int)A, c.N, st);
   if (e != cudaSuccess) return cuda_status(e, "FC1 grouped GEMM (fp8)");
   // rows of h this group range wrote: all routed rows [0, A) if a routed group is in
   // range, then the N-row blocks of the shared experts in range
@@ -294,7 +294,7 @@ moe_status ffn_fp8_impl(const moe_config& c, const moe_layout& L, const Fp8Ffn& 
   g2.k = c.k;
   g2.a_scale = f.h_scale;
   g2.b_scale = f.w2_scale;
-  return cuda_status(launch_tc_gemm(g2, (int)(A + (long long)c.n_shared * c.N), 0, st), "FC2 grouped GEMM (fp8)");
+  return cuda_status(tc_grouped(g2, c, (int)(A + (long long)c.n_shared * c.N), 0, st), "FC2 grouped GEMM (fp8)");
 }
 
 moe_status ffn_impl(const moe_config& c, const moe_layout& L, const void* x_perm, const void* x, const void* w13,

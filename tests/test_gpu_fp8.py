@@ -59,6 +59,8 @@ SMALL = [
     small_config("f8_small", cfg_id=85, N=700, d=256, E=16, S=1, k=4, I=128, P=8),
     small_config("f8_ragged", cfg_id=86, N=333, d=512, E=8, S=2, k=2, I=208, P=4, score="sigmoid"),
     small_config("f8_wide_d", cfg_id=87, N=300, d=4096, E=8, S=1, k=2, I=192, P=4),
+    # d = 4096 with groups over 128 rows: 256-row CTA-pair tiles plus one-CTA tails
+    small_config("f8_pairs", cfg_id=99, N=640, d=4096, E=8, S=1, k=2, I=192, P=4),
 ]
 
 
@@ -132,10 +134,12 @@ def test_fp8_layer_staged(cfg):
     assert torch.equal(y, r["y"])
 
 
-def test_fp8_full_size_fine_sampled():
-    """The bench's fine-grained workload at full size: quantisation bit-exact, sampled
-    rows of h and out against the oracle on the same codes, fused == staged."""
-    cfg = CONFIGS["fine"]
+@pytest.mark.parametrize("name", ["fine", "hot_cal"])
+def test_fp8_full_size_sampled(name):
+    """Full-size workloads (fine: one-CTA tiles; hot_cal: CTA-pair tiles): x quantisation
+    bit-exact, the weight codes of the sampled experts bit-exact, sampled rows of h and out
+    against the oracle on the same codes, fused == staged."""
+    cfg = CONFIGS[name]
     inp = gpu_inputs(cfg)
     r = _staged(cfg, inp)
     k, I, E = cfg.k, cfg.I, cfg.E
@@ -150,7 +154,9 @@ def test_fp8_full_size_fine_sampled():
     w2s = _np(r["w2_s"]).reshape(E + cfg.S, cfg.d)
     hq = _np(r["h_q"])
     hs = _np(r["h_s"])
-    for e in rng.choice(E, 6, replace=False):
+    for e in rng.choice(np.flatnonzero(n_e > 0), 6, replace=False):
+        wq_ref, ws_ref = F.quantize_rows(inp["w13"][e].float().cpu().numpy())
+        assert np.array_equal(w13q[e], wq_ref) and np.array_equal(w13s[e], ws_ref)
         rows = off[e] + rng.choice(n_e[e], min(8, n_e[e]), replace=False)
         tok = row2tok[rows] // k
         assert_close_rel(r["h"][torch.tensor(rows)], F.fc1(xq_ref[tok], xs_ref[tok], w13q[e], w13s[e], I),
