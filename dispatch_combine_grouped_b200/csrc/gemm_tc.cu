@@ -1,5 +1,5 @@
-// Grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM, fed by TMA), bf16
-// operands with fp32 accumulation, one kernel family for three jobs:
+// Grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM, fed by TMA), bf16 or
+// e4m3 (F8) operands with fp32 accumulation, one kernel family for three jobs:
 //   MODE_ROUTER  logits = x W_g^T (+ b), fp32 out                ("深入浅出 DeepSeek MoE", step 1)
 //   MODE_FC1     h = SiLU(X W_gate^T) * (X W_up^T), bf16 out     ("MoE我们喜欢你（四）" §4.1 FC1 + activation)
 //   MODE_FC2     o = (h W_down^T) * gate(row), bf16 out          (§4.1 FC2; the combine's gate applied here)
@@ -7,8 +7,9 @@
 // (ep_deepep explainer §2: work per expert is n_e, critical work max_e n_e).
 //
 // Structure (one CTA per SM, persistent, 6 warps):
-//   warp 0      TMA producer: A tile [128 x 64] + B tile [BN x 64] per stage, 128B swizzle
-//   warp 1      MMA issuer: 4 x tcgen05.mma (M=128, N=BN, K=16) per stage into TMEM;
+//   warp 0      TMA producer: A tile [128 x 128 B] + B tile [BN x 128 B] per stage (64
+//               bf16 or 128 e4m3 k values per row), 128B swizzle
+//   warp 1      MMA issuer: 4 x tcgen05.mma (M=128, N=BN, K=16 bf16 / 32 e4m3) per stage;
 //               owns the TMEM allocation (2 x BN fp32 columns: double-buffered accumulator)
 //   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes, SwiGLU / gate scale / bias,
 //               vectorised stores; overlaps the next tile's mainloop

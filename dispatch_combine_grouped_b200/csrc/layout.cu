@@ -16,7 +16,9 @@
 //   3. maps  : every assignment's row and send slot from bases + ranks; scatter of the
 //              five maps
 // Ranks come from counts, never from atomic arrival order, so the result is identical
-// on every run.
+// on every run.  An id of -1 marks a dropped assignment (capacity factor): it is not
+// counted, gets no row and no send slot (its tok2row / tok2send are -1), and the unused
+// tails [A_kept, A) of row2tok, send2row and ret2tok are -1.
 #include "common.cuh"
 #include "kernels.cuh"
 

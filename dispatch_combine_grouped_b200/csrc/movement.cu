@@ -8,7 +8,8 @@
 // the staged kernels materialise the send (or return) buffer in between.
 //
 // All kernels: one warp per row (or token), 16-byte vectors, rows are d * elem bytes
-// (a multiple of 16).  Permute is a bit copy and ignores the dtype.
+// (a multiple of 16).  Permute is a bit copy and ignores the dtype.  A map entry of -1
+// (a dropped assignment, an unused slot) is skipped: nothing is moved or added for it.
 #include "common.cuh"
 #include "kernels.cuh"
 

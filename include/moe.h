@@ -24,7 +24,8 @@
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
  *   - Host-detectable errors (bad sizes, NULL pointers, small workspace) return a
  *     non-zero moe_status immediately and launch nothing.
- *   - Device-detected errors (an expert id outside [0, E), a wait that timed out) are
+ *   - Device-detected errors (an expert id outside [0, E) other than -1, which marks a
+ *     dropped assignment (moe_capacity_drop), or a wait that timed out) are
  *     written to *dev_status (an int32 the caller zeroes and reads after synchronising);
  *     the first error wins.  dev_status may be NULL, in which case they go unreported.
  *   - Sizes: A = N * k assignments, a = t * k + slot indexes them.  E % P == 0 unless an
@@ -54,7 +55,7 @@ typedef enum {
   MOE_ERR_UNSUPPORTED = 2, /* valid request outside the sizes this build supports */
   MOE_ERR_WORKSPACE = 3,   /* workspace smaller than the matching *_workspace_bytes() */
   MOE_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed (launch, tensor map) */
-  MOE_ERR_BAD_INDEX = 5,   /* device: an expert id outside [0, E) was seen */
+  MOE_ERR_BAD_INDEX = 5,   /* device: an expert id outside [0, E) (other than -1) was seen */
   MOE_ERR_TIMEOUT = 6      /* device: a bounded wait gave up */
 } moe_status;
 
@@ -155,7 +156,8 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_gate, c
  * and deterministic; nothing is copied to the host.
  *   expert_owner [E] int32 or NULL (NULL = owner e / (E/P)); each owner's experts keep
  *                id order and its rows are contiguous
- *   topk_ids     [N, k] int32, ids outside [0, E) set *dev_status = MOE_ERR_BAD_INDEX
+ *   topk_ids     [N, k] int32; -1 marks a dropped assignment (no row, see
+ *                moe_capacity_drop); other ids outside [0, E) set *dev_status = MOE_ERR_BAD_INDEX
  *                and are treated as expert 0 (no out-of-bounds write happens)
  *   out          the layout arrays (all must be non-NULL)
  *   ws, ws_bytes scratch of at least moe_layout_workspace_bytes(cfg)
