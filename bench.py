@@ -252,6 +252,49 @@ def run_reference(args, cfg, rank):
 
 
 # ------------------------------------------------------------------------------ our arm
+def e2e_pipelined(forward, x, y, flush, steps):
+    """End to end through the public call, the way a serving loop runs it: every step
+    copies its input from pinned host memory to the device (copy-in stream), runs the
+    layer (current stream) and copies its result back to pinned host memory (copy-out
+    stream); with two device buffers each way, step i's layer overlaps step i+1's input
+    copy and step i-1's result copy.  Returns ms per step, device-timed from the first
+    copy-in to the last copy-out (L2 flushed before every layer call, inside the window)."""
+    import torch
+    dev = x.device
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    comp = torch.cuda.current_stream(dev)
+    x_host = x.cpu().pin_memory()
+    y_hosts = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(2)]
+    x_devs = [torch.empty_like(x) for _ in range(2)]
+    y_devs = [torch.empty_like(y) for _ in range(2)]
+    in_done = [torch.cuda.Event() for _ in range(steps)]
+    comp_done = [torch.cuda.Event() for _ in range(steps)]
+    out_done = [torch.cuda.Event() for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(s_in)
+    for i in range(steps):
+        b = i % 2
+        if i >= 2:
+            s_in.wait_event(comp_done[i - 2])  # the layer of step i-2 has read x_devs[b]
+        with torch.cuda.stream(s_in):
+            x_devs[b].copy_(x_host, non_blocking=True)
+        in_done[i].record(s_in)
+        comp.wait_event(in_done[i])
+        if i >= 2:
+            comp.wait_event(out_done[i - 2])   # y_devs[b] has been copied out
+        flush.zero_()
+        forward(x_devs[b], y_devs[b])
+        comp_done[i].record(comp)
+        s_out.wait_event(comp_done[i])
+        with torch.cuda.stream(s_out):
+            y_hosts[b].copy_(y_devs[b], non_blocking=True)
+        out_done[i].record(s_out)
+    t1.record(s_out)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / steps
+
+
 def run_fp8(args, cfg, world, rank, local):
     """The layer with the FP8 expert path on one stream: route -> layout -> quantise x +
     FP8 permute -> FP8 grouped FFN (FC1, h quantisation, FC2) -> combine.  Weights are
@@ -334,19 +377,9 @@ def run_fp8(args, cfg, world, rank, local):
         fev[i][1].record()
     torch.cuda.synchronize()
     fused_ms = sum(a.elapsed_time(b) for a, b in fev) / args.steps
-    x_host = x.cpu().pin_memory()
-    y_host = torch.empty(cfg.N, cfg.d, dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(x)
-    eev = [events(2) for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.zero_()
-        eev[i][0].record()
-        x_dev.copy_(x_host, non_blocking=True)
-        moe.layer_forward_fp8(cfg, x_dev, wg, bias, owner, w13_q, w13_s, w2_q, w2_s, y=y, ws=ws, status=status)
-        y_host.copy_(y, non_blocking=True)
-        eev[i][1].record()
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eev) / args.steps, world, dev)
+    e2e_ms = max_over_ranks(e2e_pipelined(
+        lambda xd, yd: moe.layer_forward_fp8(cfg, xd, wg, bias, owner, w13_q, w13_s, w2_q, w2_s, y=yd, ws=ws,
+                                             status=status), x, y, flush, max(args.steps, 8)), world, dev)
 
     alg = algorithmic(cfg)
     peaks, peak_src = load_peaks()
@@ -375,7 +408,11 @@ def run_fp8(args, cfg, world, rank, local):
             "fused_ms_per_step": fused_ms,
             "e2e": {"value": whole_job_tokens_per_s(cfg.N, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": x.numel() * x.element_size(),
-                    "d2h_bytes_per_step": y.numel() * y.element_size()},
+                    "d2h_bytes_per_step": y.numel() * y.element_size(), "ms_per_step": e2e_ms,
+                    "how": "moe_layer_forward* per step, input copied in from pinned host memory and result "
+                           "copied out, on their own streams so that step i overlaps the copies of steps "
+                           "i+1 and i-1 (two device buffers each way); device-timed from the first copy-in "
+                           "to the last copy-out"},
             "gpu_launches": 11 * args.steps,
             "clocks": clock_rec,
         }
@@ -580,20 +617,10 @@ def main():
     torch.cuda.synchronize()
     fused_ms = sum(a.elapsed_time(b) for a, b in fev) / args.steps
 
-    # end to end: pinned host input -> device, layer, result -> pinned host, per step
-    x_host = x.cpu().pin_memory()
-    y_host = torch.empty(cfg.N, cfg.d, dtype=dt).pin_memory()
-    x_dev = torch.empty_like(x)
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.zero_()
-        e2e_ev[i][0].record()
-        x_dev.copy_(x_host, non_blocking=True)
-        moe.layer_forward_overlapped(cfg, x_dev, wg, bias, owner, w13, w2, side, y=y, ws=ws, status=status)
-        y_host.copy_(y, non_blocking=True)
-        e2e_ev[i][1].record()
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps, world, dev)
+    # end to end: pinned host input -> device, layer, result -> pinned host, every step
+    e2e_ms = max_over_ranks(e2e_pipelined(
+        lambda xd, yd: moe.layer_forward_overlapped(cfg, xd, wg, bias, owner, w13, w2, side, y=yd, ws=ws,
+                                                    status=status), x, y, flush, max(args.steps, 8)), world, dev)
 
     n_e = layout["n_e"].cpu()
     touched = int((n_e > 0).sum())
@@ -656,7 +683,11 @@ def main():
                           "experts_empty": int((n_e == 0).sum())},
             "e2e": {"value": whole_job_tokens_per_s(cfg.N, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": x.numel() * x.element_size(),
-                    "d2h_bytes_per_step": y.numel() * y.element_size()},
+                    "d2h_bytes_per_step": y.numel() * y.element_size(), "ms_per_step": e2e_ms,
+                    "how": "moe_layer_forward* per step, input copied in from pinned host memory and result "
+                           "copied out, on their own streams so that step i overlaps the copies of steps "
+                           "i+1 and i-1 (two device buffers each way); device-timed from the first copy-in "
+                           "to the last copy-out"},
             "gpu_launches": launches_per_step * args.steps,
             **({"eplb": eplb_info} if R else {}),
             "clocks": clock_rec,
