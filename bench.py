@@ -421,8 +421,8 @@ def run_fp8(args, cfg, world, rank, local):
 
 def main():
     args = parse()
-    from moe_inputs import CONFIGS
-    cfg = CONFIGS[args.workload]
+    from moe_inputs import CONFIGS, PROFILE_CASES
+    cfg = CONFIGS[args.workload] if args.workload in CONFIGS else PROFILE_CASES[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -76,6 +76,16 @@ CONFIGS = {
                          owner="hot4"),
 }
 
+# Reduced cases for profiler captures that must stay a few GB on the device: the wide
+# layer's shapes and its n_e ~ 256 per expert with 32 experts (2.9 GB of weights), and the
+# same with 4096 tokens so that the permute / combine traffic (0.5 GB) exceeds the L2.
+PROFILE_CASES = {
+    "wide_e32": MoEConfig("wide_e32", 6, N=1024, d=7168, E=32, S=1, k=8, I=2048, P=8,
+                          n_groups=8, topk_groups=4, score="sigmoid", renormalize=True),
+    "wide_e32_n4k": MoEConfig("wide_e32_n4k", 7, N=4096, d=7168, E=32, S=1, k=8, I=2048, P=8,
+                              n_groups=8, topk_groups=4, score="sigmoid", renormalize=True),
+}
+
 
 def zipf_bias(E: int, alpha: float) -> torch.Tensor:
     """Router logit bias b_e = alpha * ln(1/rank_e) with rank_e = e + 1 (expert 0 hottest)."""
