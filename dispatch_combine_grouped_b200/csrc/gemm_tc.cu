@@ -33,10 +33,9 @@
 namespace moe {
 
 constexpr int BM = 128;
-constexpr int BK = 64;  // k per stage of the pair kernel and the router; FC tiles use MOE_GEMM_BK
-#ifndef MOE_GEMM_BK
-#define MOE_GEMM_BK 64
-#endif
+// k per stage: 64 bf16 (128-byte rows with the 128B swizzle); narrower k-steps (64- and
+// 32-byte swizzles) measured 20% and 50% slower on B200
+constexpr int BK = 64;
 constexpr int kThreads = 192;
 constexpr int kMaxGroupsGemm = kMaxSlots + kMaxShared;
 
@@ -528,7 +527,7 @@ cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStre
     BN = 256;
   }
   const bool f8 = g.fp8 != 0 && g.mode != MODE_ROUTER;
-  const int bk = f8 ? 128 : (g.mode == MODE_ROUTER ? BK : MOE_GEMM_BK);  // k per stage
+  const int bk = f8 ? 128 : (g.mode == MODE_ROUTER ? BK : BK);  // k per stage
   CUtensorMap a0, a1, b;
   if (!make_map_a(&a0, g.a0, a0_rows, g.K, bk, f8)) return cudaErrorInvalidValue;
   if (!make_map_a(&a1, g.a1 ? g.a1 : g.a0, g.a1 ? a1_rows : a0_rows, g.K, bk, f8)) return cudaErrorInvalidValue;
@@ -541,10 +540,10 @@ cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStre
   switch (g.mode) {
     case MODE_FC1:
       if (f8) return launch_bn<256, MODE_FC1, 128, true>(g, a0, a1, b, max_tiles, st);
-      return launch_bn<256, MODE_FC1, MOE_GEMM_BK>(g, a0, a1, b, max_tiles, st);
+      return launch_bn<256, MODE_FC1, BK>(g, a0, a1, b, max_tiles, st);
     case MODE_FC2:
       if (f8) return launch_bn<256, MODE_FC2, 128, true>(g, a0, a1, b, max_tiles, st);
-      return launch_bn<256, MODE_FC2, MOE_GEMM_BK>(g, a0, a1, b, max_tiles, st);
+      return launch_bn<256, MODE_FC2, BK>(g, a0, a1, b, max_tiles, st);
     default:
       switch (BN) {
         case 32: return launch_bn<32, MODE_ROUTER, BK>(g, a0, a1, b, max_tiles, st);

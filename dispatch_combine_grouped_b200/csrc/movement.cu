@@ -340,7 +340,6 @@ cudaError_t launch_permute_staged(const moe_config& c, const moe_layout& L, cons
 template <typename T>
 static void combine_launch(const moe_config& c, const uint4* routed, const uint4* shared, const int32_t* map,
                            const float* gates, uint4* y, cudaStream_t st) {
-#ifndef MOE_COMBINE16
   const int row_bytes = c.d * elem_bytes(c);
   if (row_bytes % 32 == 0) {
     const int vpr32 = row_bytes / 32;
@@ -350,7 +349,6 @@ static void combine_launch(const moe_config& c, const uint4* routed, const uint4
         reinterpret_cast<V32*>(y), c.N, c.k, c.n_shared, vpr32);
     return;
   }
-#endif
   const int vpr = vecs_per_row(c);
   const long long items = (long long)c.N * ((vpr + 32 * kCombVec - 1) / (32 * kCombVec));
   combine_kernel<T><<<blocks_for(items), kMoveWarps * 32, 0, st>>>(routed, shared, map, gates, y, c.N, c.k,
