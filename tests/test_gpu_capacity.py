@@ -96,3 +96,32 @@ def test_full_size_hot_with_capacity():
     g[tokens] = O.gate_weights(z, ids_np[tokens], cfg.score, cfg.renormalize)
     y_ref = O.moe_tokens_direct(cfg, inp["x"], kept_ref, g, inp["w13"], inp["w2"], tokens)
     assert_close_fro(y[torch.tensor(tokens, device="cuda")], y_ref, what="hot_cal sampled y")
+
+
+def test_capacity_then_replicas():
+    """Dropped assignments stay dropped through the replica assignment; the layer over the
+    slots with the dropped ones gives the layer without copies, bit for bit."""
+    cfg = SMALL[0]
+    R = 8
+    inp = gpu_inputs(cfg)
+    logits, ids, w = moe.route(cfg, inp["x"], inp["w_gate"], inp["bias"])
+    kept = moe.capacity_drop(cfg, ids, moe.capacity_of(0.8, cfg))
+    n_e = torch.bincount(kept.reshape(-1)[kept.reshape(-1) >= 0].long(), minlength=cfg.E).cpu().numpy()
+    plan = moe.eplb_plan(n_e, R, cfg.P)
+    phys = moe.eplb_assign(cfg, kept, torch.tensor(plan["replica_off"], device="cuda"),
+                           torch.tensor(plan["replica_slots"], device="cuda"), cfg.E + R)
+    torch.cuda.synchronize()
+    assert torch.equal(phys < 0, kept < 0)
+    pcfg = moe.physical_config(cfg, R)
+    w13p = moe.eplb_place_weights(plan["slot_expert"], cfg.E, cfg.S, inp["w13"])
+    w2p = moe.eplb_place_weights(plan["slot_expert"], cfg.E, cfg.S, inp["w2"])
+    lay = moe.dispatch_layout(pcfg, phys)
+    xp = moe.permute(pcfg, lay, inp["x"])
+    _, out = moe.grouped_ffn(pcfg, lay, xp, inp["x"], w13p, w2p, topk_w=w)
+    y = moe.combine(pcfg, lay, out)
+    lay0 = moe.dispatch_layout(cfg, kept)
+    xp0 = moe.permute(cfg, lay0, inp["x"])
+    _, out0 = moe.grouped_ffn(cfg, lay0, xp0, inp["x"], inp["w13"], inp["w2"], topk_w=w)
+    y0 = moe.combine(cfg, lay0, out0)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y0)

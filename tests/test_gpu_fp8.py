@@ -168,3 +168,32 @@ def test_fp8_full_size_sampled(name):
                               r["w13_s"], r["w2_q"], r["w2_s"])
     torch.cuda.synchronize()
     assert torch.equal(y, r["y"])
+
+
+def test_fp8_forward_is_deterministic_and_graph_capturable():
+    """Two runs give the same bits; the fused FP8 forward captured in a CUDA graph and
+    replayed gives them too (the workspace and the weights are set up before capture)."""
+    cfg = SMALL[3]
+    inp = gpu_inputs(cfg)
+    w13_q, w13_s = moe.quantize_fp8(inp["w13"])
+    w2_q, w2_s = moe.quantize_fp8(inp["w2"])
+    ws = torch.empty(moe.workspace_bytes_fp8(cfg), dtype=torch.uint8, device="cuda")
+    args = (cfg, inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], w13_q, w13_s, w2_q, w2_s)
+    y1 = moe.layer_forward_fp8(*args, ws=ws)
+    y2 = moe.layer_forward_fp8(*args, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    y3 = torch.empty_like(y1)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        moe.layer_forward_fp8(*args, y=y3, ws=ws)  # warm-up on the capture stream
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    y3.zero_()
+    with torch.cuda.graph(graph):
+        moe.layer_forward_fp8(*args, y=y3, ws=ws)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y3, y1)
