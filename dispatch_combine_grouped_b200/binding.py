@@ -31,7 +31,8 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_con
             "moe_combine", "moe_combine_staged",
             "moe_layer_forward", "moe_eplb_plan", "moe_eplb_workspace_bytes", "moe_eplb_assign",
             "moe_eplb_place_weights", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8",
-            "moe_workspace_bytes_fp8", "moe_layer_forward_fp8", "moe_capacity_drop"]
+            "moe_workspace_bytes_fp8", "moe_layer_forward_fp8", "moe_capacity_drop",
+            "moe_layer_forward_fp8_overlapped"]
 
 
 class CConfig(ctypes.Structure):
@@ -99,6 +100,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_workspace_bytes_fp8": (sz, [cfgp]),
         "moe_layer_forward_fp8": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp]),
         "moe_capacity_drop": (i32, [cfgp, vp, i32, vp, vp, vp, sz, vp]),
+        "moe_layer_forward_fp8_overlapped": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp,
+                                                   vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -456,16 +459,21 @@ def workspace_bytes_fp8(cfg) -> int:
 
 
 def layer_forward_fp8(cfg, x, w_gate, bias, expert_owner, w13_q, w13_scale, w2_q, w2_scale, y=None, ws=None,
-                      layout=None, status=None):
+                      layout=None, status=None, side_stream=None):
+    """moe_layer_forward_fp8, or moe_layer_forward_fp8_overlapped when side_stream is given."""
     c = c_config(cfg)
     if y is None:
         y = torch.empty(cfg.N, cfg.d, dtype=torch.bfloat16, device=x.device)
     if ws is None:
         ws = torch.empty(max(workspace_bytes_fp8(cfg), 1), dtype=torch.uint8, device=x.device)
-    _check(load().moe_layer_forward_fp8(ctypes.byref(c), _p(x), _p(w_gate), _p(bias), _p(expert_owner), _p(w13_q),
-                                        _p(w13_scale), _p(w2_q), _p(w2_scale), _p(y),
-                                        ctypes.byref(layout.c) if layout is not None else None, _p(status), _p(ws),
-                                        ws.numel(), _stream()), "moe_layer_forward_fp8")
+    args = [ctypes.byref(c), _p(x), _p(w_gate), _p(bias), _p(expert_owner), _p(w13_q), _p(w13_scale), _p(w2_q),
+            _p(w2_scale), _p(y), ctypes.byref(layout.c) if layout is not None else None, _p(status), _p(ws),
+            ws.numel(), _stream()]
+    if side_stream is None:
+        _check(load().moe_layer_forward_fp8(*args), "moe_layer_forward_fp8")
+    else:
+        _check(load().moe_layer_forward_fp8_overlapped(*args, ctypes.c_void_p(side_stream.cuda_stream)),
+               "moe_layer_forward_fp8_overlapped")
     return y
 
 

@@ -650,10 +650,10 @@ size_t moe_workspace_bytes_fp8(const moe_config* cfg) {
   return carve_forward(*cfg, nullptr, true).total;
 }
 
-moe_status moe_layer_forward_fp8(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
-                                 const int32_t* expert_owner, const void* w13_q, const float* w13_scale,
-                                 const void* w2_q, const float* w2_scale, void* y, const moe_layout* layout_out,
-                                 int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream) {
+static moe_status forward_fp8(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
+                              const int32_t* expert_owner, const void* w13_q, const float* w13_scale,
+                              const void* w2_q, const float* w2_scale, void* y, const moe_layout* layout_out,
+                              int32_t* dev_status, void* ws, size_t ws_bytes, cudaStream_t st, cudaStream_t side) {
   moe_status s = check_fp8(cfg);
   if (s != MOE_OK) return s;
   if ((s = check_router(*cfg)) != MOE_OK) return s;
@@ -667,17 +667,58 @@ moe_status moe_layer_forward_fp8(const moe_config* cfg, const void* x, const voi
     return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
   w = carve_forward(c, static_cast<char*>(ws), true);
   const moe_layout& L = layout_out ? *layout_out : w.lay;
-  cudaStream_t st = (cudaStream_t)stream;
   if (c.N > 0 && (s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
-  if ((s = cuda_status(launch_layout(c, expert_owner, w.ids, L, dev_status, w.lay_ws, st), "layout")) != MOE_OK)
+  if (c.N > 0 && (s = cuda_status(launch_quantize_rows(x, c.N, c.d, w.x_q, w.x_scale, st), "x quantisation")) !=
+                     MOE_OK)
     return s;
-  if (c.N == 0) return MOE_OK;
-  if ((s = cuda_status(launch_quantize_rows(x, c.N, c.d, w.x_q, w.x_scale, st), "x quantisation")) != MOE_OK)
-    return s;
-  if ((s = cuda_status(launch_permute_bytes(c, L, w.x_q, w.x_perm, c.d, st), "permute (fp8)")) != MOE_OK) return s;
   Fp8Ffn f{w.x_perm, w.x_q, w.x_scale, w13_q, w13_scale, w2_q, w2_scale, w.w, w.h, w.h_q, w.h_scale, w.out};
-  if ((s = ffn_fp8_impl(c, L, f, st)) != MOE_OK) return s;
+  const bool overlap = side != nullptr && side != st && c.n_shared > 0 && c.N > 0;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaError_t e = cudaSuccess;
+  if (overlap) {  // the shared experts read only x_q: they run on the side stream
+    e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
+    if (e != cudaSuccess) {
+      if (fork) cudaEventDestroy(fork);
+      if (join) cudaEventDestroy(join);
+      return cuda_status(e, "fork");
+    }
+    s = ffn_fp8_impl(c, L, f, side, c.E, c.n_shared);
+    e = cudaEventRecord(join, side);
+  }
+  if (s == MOE_OK)
+    s = cuda_status(launch_layout(c, expert_owner, w.ids, L, dev_status, w.lay_ws, st), "layout");
+  if (s == MOE_OK && c.N > 0)
+    s = cuda_status(launch_permute_bytes(c, L, w.x_q, w.x_perm, c.d, st), "permute (fp8)");
+  if (s == MOE_OK && c.N > 0) s = overlap ? ffn_fp8_impl(c, L, f, st, 0, c.E) : ffn_fp8_impl(c, L, f, st);
+  if (overlap) {
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, join, 0);  // join even after an error
+    cudaEventDestroy(fork);
+    cudaEventDestroy(join);
+  }
+  if (s != MOE_OK) return s;
+  if (e != cudaSuccess) return cuda_status(e, "join");
+  if (c.N == 0) return MOE_OK;
   return cuda_status(launch_combine(c, L, w.out, nullptr, y, st), "combine");
+}
+
+moe_status moe_layer_forward_fp8(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
+                                 const int32_t* expert_owner, const void* w13_q, const float* w13_scale,
+                                 const void* w2_q, const float* w2_scale, void* y, const moe_layout* layout_out,
+                                 int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return forward_fp8(cfg, x, w_gate, bias, expert_owner, w13_q, w13_scale, w2_q, w2_scale, y, layout_out,
+                     dev_status, ws, ws_bytes, (cudaStream_t)stream, nullptr);
+}
+
+moe_status moe_layer_forward_fp8_overlapped(const moe_config* cfg, const void* x, const void* w_gate,
+                                            const float* bias, const int32_t* expert_owner, const void* w13_q,
+                                            const float* w13_scale, const void* w2_q, const float* w2_scale, void* y,
+                                            const moe_layout* layout_out, int32_t* dev_status, void* ws,
+                                            size_t ws_bytes, moe_stream_t stream, moe_stream_t side_stream) {
+  return forward_fp8(cfg, x, w_gate, bias, expert_owner, w13_q, w13_scale, w2_q, w2_scale, y, layout_out,
+                     dev_status, ws, ws_bytes, (cudaStream_t)stream, (cudaStream_t)side_stream);
 }
 
 moe_status moe_capacity_drop(const moe_config* cfg, const int32_t* topk_ids, int32_t capacity, int32_t* kept_ids,

@@ -457,6 +457,18 @@ moe_status moe_layer_forward_fp8(const moe_config* cfg, const void* x, const voi
                                  const void* w2_q, const float* w2_scale, void* y, const moe_layout* layout_out,
                                  int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_layer_forward_fp8 with the shared experts overlapped: after the router and the
+ * quantisation of x on `stream`, the shared experts' FP8 FFN runs on `side_stream` while
+ * the layout, the FP8 permute and the routed FP8 FFN run on `stream`; `stream` waits for
+ * `side_stream` before the combine.  Same result as moe_layer_forward_fp8, bit for bit;
+ * two events are created and destroyed per call.  With n_shared == 0 or side_stream ==
+ * stream this is moe_layer_forward_fp8. */
+moe_status moe_layer_forward_fp8_overlapped(const moe_config* cfg, const void* x, const void* w_gate,
+                                            const float* bias, const int32_t* expert_owner, const void* w13_q,
+                                            const float* w13_scale, const void* w2_q, const float* w2_scale, void* y,
+                                            const moe_layout* layout_out, int32_t* dev_status, void* ws,
+                                            size_t ws_bytes, moe_stream_t stream, moe_stream_t side_stream);
+
 #ifdef __cplusplus
 }
 #endif
