@@ -38,6 +38,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--movement-sweep", action="store_true",
+                    help="permute / combine bandwidth at the workload's row shape for N = 128 .. 16384 "
+                         "(one JSON line with the curve)")
     ap.add_argument("--fp8", action="store_true",
                     help="the FP8 (e4m3) expert path: quantised dispatch payload and expert GEMMs")
     ap.add_argument("--eplb", type=int, default=0, metavar="R",
@@ -295,6 +298,52 @@ def e2e_pipelined(forward, x, y, flush, steps):
     return t0.elapsed_time(t1) / steps
 
 
+def run_movement_sweep(args, cfg, local):
+    """Permute and combine at the workload's shapes (d, k, E, S) for N = 128 .. 16384:
+    each kernel timed alone, L2 flushed before every launch, median of 10, at full clock
+    (an idle pause before each size)."""
+    import torch
+    import dispatch_combine_grouped_b200 as moe
+    from moe_inputs import make_inputs
+
+    dev = torch.device("cuda", local)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    curve = []
+    n = 128
+    while n <= 16384:
+        c = cfg.replace(N=n)
+        inp = make_inputs(c, device=dev, with_experts=False)
+        _, ids, w = moe.route(c, inp["x"], inp["w_gate"], inp["bias"])
+        lay = moe.dispatch_layout(c, ids, inp["expert_owner"])
+        rows = n * c.k + c.S * n
+        xp = torch.empty(n * c.k, c.d, dtype=inp["x"].dtype, device=dev)
+        out = torch.randn(rows, c.d, device=dev).to(inp["x"].dtype)
+        y = torch.empty_like(inp["x"])
+        alg = algorithmic(c)
+        time.sleep(0.5)
+        res = {"N": n}
+        for name, fn, byt in [("permute", lambda: moe.permute(c, lay, inp["x"], out=xp), alg["permute_bytes"]),
+                              ("combine", lambda: moe.combine(c, lay, out, y=y), alg["combine_bytes"])]:
+            ts = []
+            for _ in range(10):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b.record()
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b))
+            ms = sorted(ts)[5]
+            res[f"{name}_us"] = ms * 1e3
+            res[f"{name}_gbs"] = byt / (ms / 1e3) / 1e9
+        curve.append(res)
+        del inp, xp, out, y, lay
+        n *= 2
+    peaks, src = load_peaks()
+    print(json.dumps({"movement_sweep": describe(cfg), "hbm_gbs_measured": peaks["hbm_gbs"], "curve": curve}),
+          flush=True)
+
+
 def run_fp8(args, cfg, world, rank, local):
     """The layer with the FP8 expert path on one stream: route -> layout -> quantise x +
     FP8 permute -> FP8 grouped FFN (FC1, h quantisation, FC2) -> combine.  Weights are
@@ -449,6 +498,13 @@ def main():
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.movement_sweep:
+        if rank == 0:
+            run_movement_sweep(args, cfg, local)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     if args.fp8:
         run_fp8(args, cfg, world, rank, local)
         if world > 1:
