@@ -694,6 +694,8 @@ def main():
 
     n_e = layout["n_e"].cpu()
     touched = int((n_e > 0).sum())
+    R_own = layout["recv_off"].cpu().diff().float()  # rows each virtual owner receives
+    owner_imb = float(R_own.max() / R_own.mean()) if float(R_own.mean()) > 0 else None
     alg = algorithmic(cfg, touched)
     peaks, peak_src = load_peaks()
     tpeak, tkind = tensor_peak(peaks, clock_rec)
@@ -750,7 +752,8 @@ def main():
                         "gbs_in_step": alg["combine_bytes"] / (seq_ms["combine"] / 1e3) / 1e9},
             "fused_ms_per_step": fused_ms,
             "imbalance": {"max_over_mean_n_e": float(n_e.max()) / float(n_e.float().mean()),
-                          "experts_empty": int((n_e == 0).sum())},
+                          "experts_empty": int((n_e == 0).sum()),
+                          "max_over_mean_owner_rows": owner_imb},
             "e2e": {"value": whole_job_tokens_per_s(cfg.N, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": x.numel() * x.element_size(),
                     "d2h_bytes_per_step": y.numel() * y.element_size(), "ms_per_step": e2e_ms,
