@@ -12,4 +12,6 @@ from .binding import (EXPORTED, Layout, MoEError, alloc_workspace, c_config, che
                       workspace_bytes, quantize_fp8, permute_fp8, grouped_ffn_fp8, workspace_bytes_fp8,
                       layer_forward_fp8, capacity_drop, capacity_of)
 
+from . import ep  # noqa: F401,E402  (expert parallelism across GPUs: moe_ep_*)
+
 load()

@@ -32,7 +32,9 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_con
             "moe_layer_forward", "moe_eplb_plan", "moe_eplb_workspace_bytes", "moe_eplb_assign",
             "moe_eplb_place_weights", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8",
             "moe_workspace_bytes_fp8", "moe_layer_forward_fp8", "moe_capacity_drop",
-            "moe_layer_forward_fp8_overlapped"]
+            "moe_layer_forward_fp8_overlapped", "moe_ep_window_bytes", "moe_ep_window_layout",
+            "moe_ep_workspace_bytes", "moe_ep_ipc_handle", "moe_ep_ipc_open", "moe_ep_ipc_close", "moe_ep_notify",
+            "moe_ep_layout", "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ep_layer_forward"]
 
 
 class CConfig(ctypes.Structure):
@@ -47,6 +49,15 @@ LAYOUT_FIELDS = ["n_e", "expert_off", "C", "send_off", "recv_off", "tok2send", "
 
 class CLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in LAYOUT_FIELDS]
+
+
+class CEpGroup(ctypes.Structure):
+    _fields_ = [("rank", ctypes.c_int32), ("capacity", ctypes.c_int32), ("local_experts", ctypes.c_int32),
+                ("windows", ctypes.POINTER(ctypes.c_void_p))]
+
+
+class CEpHandle(ctypes.Structure):
+    _fields_ = [("dest", ctypes.c_void_p), ("owner_n_e", ctypes.c_void_p), ("owner_off", ctypes.c_void_p)]
 
 
 class MoEError(RuntimeError):
@@ -103,6 +114,21 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_layer_forward_fp8_overlapped": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp,
                                                    vp]),
     }
+    grpp, hdp, u64 = ctypes.POINTER(CEpGroup), ctypes.POINTER(CEpHandle), ctypes.c_uint64
+    sig.update({
+        "moe_ep_window_bytes": (sz, [cfgp, i32]),
+        "moe_ep_window_layout": (i32, [cfgp, i32, vp]),
+        "moe_ep_workspace_bytes": (sz, [cfgp, i32]),
+        "moe_ep_ipc_handle": (i32, [vp, vp, ctypes.POINTER(sz)]),
+        "moe_ep_ipc_open": (i32, [vp, sz, ctypes.POINTER(vp)]),
+        "moe_ep_ipc_close": (i32, [vp, sz]),
+        "moe_ep_notify": (i32, [cfgp, grpp, u64, vp, vp, vp, sz, vp]),
+        "moe_ep_layout": (i32, [cfgp, grpp, u64, vp, vp, hdp, vp, vp, sz, vp]),
+        "moe_ep_dispatch": (i32, [cfgp, grpp, u64, vp, vp, hdp, vp]),
+        "moe_ep_expert_ffn": (i32, [cfgp, grpp, u64, vp, vp, vp, hdp, vp, vp, sz, vp]),
+        "moe_ep_combine": (i32, [cfgp, grpp, u64, hdp, vp, vp, vp]),
+        "moe_ep_layer_forward": (i32, [cfgp, grpp, u64, vp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz, vp]),
+    })
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
         f.restype = res

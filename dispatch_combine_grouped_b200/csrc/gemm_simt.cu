@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_gemm_kernel(const GemmArgs 
       if (r >= rows) continue;
       const long long orow = (long long)s_orow[g] + r;
       float scale = 1.0f;
-      if (MODE == MODE_FC2 && p.gate_w && gz < p.E) scale = p.gate_w[p.row2tok[orow]];
+      if (MODE == MODE_FC2 && p.gate_w && gz < p.E) scale = p.gate_w[p.row2tok ? p.row2tok[orow] : orow];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int col = n0 + tx * 4 + j;

@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {  // MODE_FC2
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + orow * p.ldo;
         float scale = 1.0f;
-        if (row_ok && p.gate_w && p.g0 + td.g < p.E) scale = p.gate_w[p.row2tok[orow]];
+        if (row_ok && p.gate_w && p.g0 + td.g < p.E) scale = p.gate_w[p.row2tok ? p.row2tok[orow] : orow];
         const float* sb = nullptr;
         if (F8) {
           if (row_ok) scale *= p.a_scale[orow];  // FP8: scale of this h row

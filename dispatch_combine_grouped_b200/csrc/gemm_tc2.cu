@@ -315,7 +315,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
       } else {
         float scale = 1.0f;
-        if (row_ok && p.gate_w && p.g0 + g < p.E) scale = p.gate_w[p.row2tok[orow]];
+        if (row_ok && p.gate_w && p.g0 + g < p.E) scale = p.gate_w[p.row2tok ? p.row2tok[orow] : orow];
         const float* sb = nullptr;
         if (F8) {
           if (row_ok) scale *= p.a_scale[orow];  // FP8: scale of this h row

@@ -61,7 +61,8 @@ struct GemmArgs {
   const int32_t* n_e;
   const int32_t* expert_off;
   const int32_t* row2tok;
-  const float* gate_w;  // FC2: routed row r is scaled by gate_w[row2tok[r]] (NULL: no scale)
+  const float* gate_w;  // FC2: routed row r is scaled by gate_w[row2tok[r]], or gate_w[r] when
+                        // row2tok is NULL (NULL gate_w: no scale)
   const float* bias;    // router: added to every logit (NULL: none)
   void* out;
   long long ldo;        // output row stride in elements
@@ -109,6 +110,36 @@ cudaError_t launch_capacity_keep(const moe_config& c, const int32_t* ids, int ca
                                  int32_t* status, void* ws, cudaStream_t st);
 moe_status eplb_plan(int E, int R, int P, const int64_t* load, int32_t* copies, int32_t* replica_off,
                      int32_t* replica_slots, int32_t* slot_expert, int32_t* slot_owner, int64_t* owner_load);
+
+// expert parallelism over peer memory (ep.cu).  A window is the buffer every rank
+// allocates with the same size; its parts sit at the same offsets on every rank.
+struct EpOffsets {
+  size_t cnt_flag, disp_flag, done_flag;  // [kMaxP] u64 epochs, indexed by the signalling rank
+  size_t disp_ctr;                        // u32: this rank's dispatch CTAs finished in the running launch
+  size_t cnt_tab;                         // [P, E] int32: row i = source i's expert counts
+  size_t gate;                            // [capacity] fp32: gate of each received row
+  size_t x_recv;                          // [capacity, d]: received rows, expert-major
+  size_t out_recv;                        // [capacity + S*N, d]: FC2 rows (routed, then shared)
+  size_t total;
+};
+struct EpPeers {
+  char* base[kMaxP];  // every rank's window as mapped in this process
+};
+EpOffsets ep_offsets(const moe_config& c, int capacity);
+cudaError_t launch_ep_push_counts(const EpPeers& peers, const EpOffsets& off, const int32_t* n_loc, int E, int P,
+                                  int me, uint64_t epoch, cudaStream_t st);
+cudaError_t launch_ep_layout(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me, int capacity,
+                             int local_experts, uint64_t epoch, const int32_t* owner, const int32_t* ids,
+                             const moe_layout& loc, int32_t* dest, int32_t* own_n_e, int32_t* own_off, int* status,
+                             cudaStream_t st);
+cudaError_t launch_ep_dispatch(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me,
+                               int capacity, uint64_t epoch, const void* x, const int32_t* dest,
+                               const float* topk_w, cudaStream_t st);
+cudaError_t launch_ep_wait(const uint64_t* flags, int n, uint64_t epoch, int* status, cudaStream_t st);
+cudaError_t launch_ep_signal(const EpPeers& peers, size_t flag_off, int P, int me, uint64_t epoch,
+                             cudaStream_t st);
+cudaError_t launch_ep_combine(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me, int capacity,
+                              uint64_t epoch, const int32_t* dest, void* y, int* status, cudaStream_t st);
 
 int sm_count();
 // TMA maps for bf16 K-major operands; box_k (64, 32 or 16) selects the 128/64/32-byte swizzle

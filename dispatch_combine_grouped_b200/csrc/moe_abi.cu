@@ -305,6 +305,140 @@ moe_status ffn_impl(const moe_config& c, const moe_layout& L, const void* x_perm
   return fc2_impl(c, L, h, w2, topk_w, out, st, g0, G);
 }
 
+// ---- expert parallelism across GPUs
+struct EpWs {
+  moe_layout loc;  // this rank's assignments laid out with a single owner
+  void* lay_ws;
+  void* h;         // [capacity + S*N, I]
+  // moe_ep_layer_forward only
+  float* logits;
+  int32_t* ids;
+  float* w;
+  moe_ep_handle hd;
+  size_t total;
+};
+
+moe_config one_owner(const moe_config& c) {
+  moe_config c1 = c;
+  c1.P = 1;
+  return c1;
+}
+
+EpWs carve_ep(const moe_config& c, int capacity, char* base) {
+  EpWs w;
+  memset(&w, 0, sizeof(w));
+  const size_t A = (size_t)c.N * c.k, E = c.E, S = c.n_shared, eb = elem_bytes(c);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off += align256(bytes ? bytes : 1);
+    return p;
+  };
+  auto i32 = [&](size_t n) { return reinterpret_cast<int32_t*>(take(n * 4)); };
+  w.loc.n_e = i32(E);
+  w.loc.expert_off = i32(E + 1);
+  w.loc.C = i32(1);
+  w.loc.send_off = i32(1);
+  w.loc.recv_off = i32(2);
+  w.loc.tok2send = i32(A);
+  w.loc.send2row = i32(A);
+  w.loc.ret2tok = i32(A);
+  w.loc.tok2row = i32(A);
+  w.loc.row2tok = i32(A);
+  w.loc.tile_off = i32(E + S + 1);
+  w.lay_ws = take(layout_scratch(one_owner(c)));
+  w.h = take(((size_t)capacity + S * c.N) * c.I * eb);
+  w.logits = reinterpret_cast<float*>(take((size_t)c.N * E * 4));
+  w.ids = i32(A);
+  w.w = reinterpret_cast<float*>(take(A * 4));
+  w.hd.dest = i32(A);
+  w.hd.owner_n_e = i32(E);
+  w.hd.owner_off = i32(E + 1);
+  w.total = off;
+  return w;
+}
+
+moe_status check_ep(const moe_config* cfg, const moe_ep_group* g, uint64_t epoch, EpPeers* peers) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (!g || !g->windows) return fail(MOE_ERR_INVALID_ARG, "EP group or its window table is NULL");
+  const moe_config& c = *cfg;
+  if (g->rank < 0 || g->rank >= c.P) return fail(MOE_ERR_INVALID_ARG, "rank outside [0, P)");
+  if (g->capacity < 1 || (long long)g->capacity * c.P >= (1LL << 31) ||
+      (long long)g->capacity + (long long)c.n_shared * c.N >= (1LL << 30))
+    return fail(MOE_ERR_UNSUPPORTED, "need 1 <= capacity, capacity * P < 2^31 and capacity + S*N < 2^30");
+  if (g->local_experts < 0 || g->local_experts > c.E) return fail(MOE_ERR_INVALID_ARG, "local_experts outside [0, E]");
+  if (epoch == 0) return fail(MOE_ERR_INVALID_ARG, "epochs start at 1");
+  memset(peers, 0, sizeof(*peers));
+  for (int p = 0; p < c.P; ++p) {
+    if (!g->windows[p] || (reinterpret_cast<uintptr_t>(g->windows[p]) & 255) != 0)
+      return fail(MOE_ERR_INVALID_ARG, "every window must be non-NULL and 256-byte aligned");
+    peers->base[p] = static_cast<char*>(g->windows[p]);
+  }
+  return MOE_OK;
+}
+
+moe_status check_ep_ws(const moe_config& c, const moe_ep_group* g, void* ws, size_t ws_bytes) {
+  if (!ws || ws_bytes < carve_ep(c, g->capacity, nullptr).total) return fail(MOE_ERR_WORKSPACE, "EP workspace too small");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return fail(MOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  return MOE_OK;
+}
+
+bool handle_complete(const moe_ep_handle* h) { return h && h->dest && h->owner_n_e && h->owner_off; }
+
+moe_status ep_notify_impl(const moe_config& c, const moe_ep_group& g, const EpPeers& peers, uint64_t epoch,
+                          const int32_t* ids, int32_t* status, const EpWs& w, cudaStream_t st) {
+  moe_status s = cuda_status(launch_layout(one_owner(c), nullptr, ids, w.loc, status, w.lay_ws, st), "local layout");
+  if (s != MOE_OK) return s;
+  return cuda_status(
+      launch_ep_push_counts(peers, ep_offsets(c, g.capacity), w.loc.n_e, c.E, c.P, g.rank, epoch, st),
+      "count exchange");
+}
+
+moe_status ep_layout_impl(const moe_config& c, const moe_ep_group& g, const EpPeers& peers, uint64_t epoch,
+                          const int32_t* owner, const int32_t* ids, const moe_ep_handle& hd, int32_t* status,
+                          const EpWs& w, cudaStream_t st) {
+  return cuda_status(launch_ep_layout(c, peers, ep_offsets(c, g.capacity), g.rank, g.capacity, g.local_experts,
+                                      epoch, owner, ids, w.loc, hd.dest, hd.owner_n_e, hd.owner_off, status, st),
+                     "EP layout");
+}
+
+// The owner's grouped FFN: routed groups = the owned experts over the received rows
+// (A_routed = capacity, no row map: row r's gate is gate[r]), shared groups over the
+// rank's own N tokens; outputs into the window's output rows.
+moe_status ep_ffn_impl(const moe_config& c, const moe_ep_group& g, const EpPeers& peers, uint64_t epoch,
+                       const void* x, const void* w13, const void* w2, const moe_ep_handle& hd, int32_t* status,
+                       const EpWs& w, cudaStream_t st) {
+  const EpOffsets off = ep_offsets(c, g.capacity);
+  char* win = peers.base[g.rank];
+  cudaError_t e = launch_ep_wait(reinterpret_cast<const uint64_t*>(win + off.disp_flag), c.P, epoch, status, st);
+  if (e != cudaSuccess) return cuda_status(e, "dispatch wait");
+  moe_config co = c;
+  co.E = g.local_experts;
+  moe_layout L;
+  memset(&L, 0, sizeof(L));
+  L.n_e = hd.owner_n_e;
+  L.expert_off = hd.owner_off;
+  const int S = c.N > 0 ? c.n_shared : 0;  // the shared experts have no rows without tokens
+  const int G = g.local_experts + S;
+  // pair tiles pay for wide rows when a group can exceed 128 rows
+  moe_config dec = c;
+  dec.N = g.capacity > c.N ? g.capacity : c.N;
+  if (G > 0) {
+    GemmArgs g1 = fc1_args(co, L, win + off.x_recv, S > 0 ? x : nullptr, w13, w.h);
+    g1.G = G;
+    g1.A_routed = g.capacity;
+    e = c.dtype == MOE_BF16 ? tc_grouped(g1, dec, g.capacity, c.N, st) : launch_simt_gemm(g1, st);
+    if (e != cudaSuccess) return cuda_status(e, "EP FC1 grouped GEMM");
+    GemmArgs g2 = fc2_args(co, L, w.h, w2, reinterpret_cast<const float*>(win + off.gate), win + off.out_recv);
+    g2.G = G;
+    g2.A_routed = g.capacity;
+    e = c.dtype == MOE_BF16 ? tc_grouped(g2, dec, g.capacity + S * c.N, 0, st) : launch_simt_gemm(g2, st);
+    if (e != cudaSuccess) return cuda_status(e, "EP FC2 grouped GEMM");
+  }
+  return cuda_status(launch_ep_signal(peers, off.done_flag, c.P, g.rank, epoch, st), "FFN done signal");
+}
+
 }  // namespace
 
 extern "C" {
@@ -719,6 +853,154 @@ moe_status moe_layer_forward_fp8_overlapped(const moe_config* cfg, const void* x
                                             size_t ws_bytes, moe_stream_t stream, moe_stream_t side_stream) {
   return forward_fp8(cfg, x, w_gate, bias, expert_owner, w13_q, w13_scale, w2_q, w2_scale, y, layout_out,
                      dev_status, ws, ws_bytes, (cudaStream_t)stream, (cudaStream_t)side_stream);
+}
+
+size_t moe_ep_window_bytes(const moe_config* cfg, int32_t capacity) {
+  if (check_config(cfg) != MOE_OK || capacity < 1) return 0;
+  return ep_offsets(*cfg, capacity).total;
+}
+
+size_t moe_ep_workspace_bytes(const moe_config* cfg, int32_t capacity) {
+  if (check_config(cfg) != MOE_OK || capacity < 1) return 0;
+  return carve_ep(*cfg, capacity, nullptr).total;
+}
+
+moe_status moe_ep_window_layout(const moe_config* cfg, int32_t capacity, size_t* offsets) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (capacity < 1 || !offsets) return fail(MOE_ERR_INVALID_ARG, "capacity < 1 or NULL offsets");
+  const EpOffsets o = ep_offsets(*cfg, capacity);
+  const size_t v[8] = {o.cnt_flag, o.disp_flag, o.done_flag, o.disp_ctr, o.cnt_tab, o.gate, o.x_recv, o.out_recv};
+  memcpy(offsets, v, sizeof(v));
+  return MOE_OK;
+}
+
+typedef CUresult (*GetAddressRange)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+moe_status moe_ep_ipc_handle(const void* window, void* handle, size_t* offset) {
+  if (!window || !handle || !offset) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn)
+    return fail(MOE_ERR_CUDA, "cuMemGetAddressRange unavailable");
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (reinterpret_cast<GetAddressRange>(fn)(&base, &size, reinterpret_cast<CUdeviceptr>(window)) != CUDA_SUCCESS)
+    return fail(MOE_ERR_INVALID_ARG, "window is not device memory");
+  cudaIpcMemHandle_t h;
+  cudaError_t e = cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base));
+  if (e != cudaSuccess) return cuda_status(e, "cudaIpcGetMemHandle");
+  static_assert(sizeof(h) == 64, "CUDA IPC handles are 64 bytes");
+  memcpy(handle, &h, sizeof(h));
+  *offset = reinterpret_cast<CUdeviceptr>(window) - base;
+  return MOE_OK;
+}
+
+moe_status moe_ep_ipc_open(const void* handle, size_t offset, void** window) {
+  if (!handle || !window) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  cudaIpcMemHandle_t h;
+  memcpy(&h, handle, sizeof(h));
+  void* base = nullptr;
+  cudaError_t e = cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess);
+  if (e != cudaSuccess) return cuda_status(e, "cudaIpcOpenMemHandle");
+  *window = static_cast<char*>(base) + offset;
+  return MOE_OK;
+}
+
+moe_status moe_ep_ipc_close(void* window, size_t offset) {
+  if (!window) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return cuda_status(cudaIpcCloseMemHandle(static_cast<char*>(window) - offset), "cudaIpcCloseMemHandle");
+}
+
+moe_status moe_ep_notify(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const int32_t* topk_ids,
+                         int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  EpPeers peers;
+  moe_status s = check_ep(cfg, grp, epoch, &peers);
+  if (s != MOE_OK) return s;
+  if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes)) != MOE_OK) return s;
+  if (cfg->N > 0 && !topk_ids) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return ep_notify_impl(*cfg, *grp, peers, epoch, topk_ids, dev_status, carve_ep(*cfg, grp->capacity, (char*)ws),
+                        (cudaStream_t)stream);
+}
+
+moe_status moe_ep_layout(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const int32_t* expert_owner,
+                         const int32_t* topk_ids, const moe_ep_handle* handle, int32_t* dev_status, void* ws,
+                         size_t ws_bytes, moe_stream_t stream) {
+  EpPeers peers;
+  moe_status s = check_ep(cfg, grp, epoch, &peers);
+  if (s != MOE_OK) return s;
+  if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
+  if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes)) != MOE_OK) return s;
+  if (!handle_complete(handle) || (cfg->N > 0 && !topk_ids)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return ep_layout_impl(*cfg, *grp, peers, epoch, expert_owner, topk_ids, *handle, dev_status,
+                        carve_ep(*cfg, grp->capacity, (char*)ws), (cudaStream_t)stream);
+}
+
+moe_status moe_ep_dispatch(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const void* x,
+                           const float* topk_w, const moe_ep_handle* handle, moe_stream_t stream) {
+  EpPeers peers;
+  moe_status s = check_ep(cfg, grp, epoch, &peers);
+  if (s != MOE_OK) return s;
+  if (!handle_complete(handle) || (cfg->N > 0 && (!x || !topk_w))) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return cuda_status(launch_ep_dispatch(*cfg, peers, ep_offsets(*cfg, grp->capacity), grp->rank, grp->capacity,
+                                        epoch, x, handle->dest, topk_w, (cudaStream_t)stream),
+                     "EP dispatch");
+}
+
+moe_status moe_ep_expert_ffn(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const void* x,
+                             const void* w13, const void* w2, const moe_ep_handle* handle, int32_t* dev_status,
+                             void* ws, size_t ws_bytes, moe_stream_t stream) {
+  EpPeers peers;
+  moe_status s = check_ep(cfg, grp, epoch, &peers);
+  if (s != MOE_OK) return s;
+  if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes)) != MOE_OK) return s;
+  const bool any = grp->local_experts > 0 || (cfg->N > 0 && cfg->n_shared > 0);
+  if (!handle_complete(handle) || (any && (!w13 || !w2)) || (cfg->N > 0 && cfg->n_shared > 0 && !x))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return ep_ffn_impl(*cfg, *grp, peers, epoch, x, w13, w2, *handle, dev_status,
+                     carve_ep(*cfg, grp->capacity, (char*)ws), (cudaStream_t)stream);
+}
+
+moe_status moe_ep_combine(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const moe_ep_handle* handle,
+                          void* y, int32_t* dev_status, moe_stream_t stream) {
+  EpPeers peers;
+  moe_status s = check_ep(cfg, grp, epoch, &peers);
+  if (s != MOE_OK) return s;
+  if (!handle_complete(handle) || (cfg->N > 0 && !y)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return cuda_status(launch_ep_combine(*cfg, peers, ep_offsets(*cfg, grp->capacity), grp->rank, grp->capacity, epoch,
+                                       handle->dest, y, dev_status, (cudaStream_t)stream),
+                     "EP combine");
+}
+
+moe_status moe_ep_layer_forward(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const void* x,
+                                const void* w_gate, const float* bias, const int32_t* expert_owner, const void* w13,
+                                const void* w2, void* y, const moe_ep_handle* handle_out, int32_t* dev_status,
+                                void* ws, size_t ws_bytes, moe_stream_t stream) {
+  EpPeers peers;
+  moe_status s = check_ep(cfg, grp, epoch, &peers);
+  if (s != MOE_OK) return s;
+  if ((s = check_router(*cfg)) != MOE_OK) return s;
+  if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
+  if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes)) != MOE_OK) return s;
+  if (handle_out && !handle_complete(handle_out)) return fail(MOE_ERR_INVALID_ARG, "incomplete handle_out");
+  const moe_config& c = *cfg;
+  const bool any = grp->local_experts > 0 || (c.N > 0 && c.n_shared > 0);
+  if ((c.N > 0 && (!x || !w_gate || !y)) || (any && (!w13 || !w2))) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  const EpWs w = carve_ep(c, grp->capacity, static_cast<char*>(ws));
+  const moe_ep_handle& hd = handle_out ? *handle_out : w.hd;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (c.N > 0 && (s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
+  if ((s = ep_notify_impl(c, *grp, peers, epoch, w.ids, dev_status, w, st)) != MOE_OK) return s;
+  if ((s = ep_layout_impl(c, *grp, peers, epoch, expert_owner, w.ids, hd, dev_status, w, st)) != MOE_OK) return s;
+  if ((s = cuda_status(launch_ep_dispatch(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, epoch,
+                                          x, hd.dest, w.w, st),
+                       "EP dispatch")) != MOE_OK)
+    return s;
+  if ((s = ep_ffn_impl(c, *grp, peers, epoch, x, w13, w2, hd, dev_status, w, st)) != MOE_OK) return s;
+  return cuda_status(launch_ep_combine(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, epoch, hd.dest,
+                                       y, dev_status, st),
+                     "EP combine");
 }
 
 moe_status moe_capacity_drop(const moe_config* cfg, const int32_t* topk_ids, int32_t capacity, int32_t* kept_ids,

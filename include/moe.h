@@ -469,6 +469,123 @@ moe_status moe_layer_forward_fp8_overlapped(const moe_config* cfg, const void* x
                                             const moe_layout* layout_out, int32_t* dev_status, void* ws,
                                             size_t ws_bytes, moe_stream_t stream, moe_stream_t side_stream);
 
+/* ============================================================================
+ * Expert parallelism across GPUs ([EP-DeepEP] §2-3: every rank is a source of tokens
+ * and the owner of some experts; dispatch sends each assignment to the owner of its
+ * expert, combine returns the outputs to the source; [DeepEP] §2-3: counts are exchanged
+ * first, then the all-to-all runs as a transpose; [WideEP]: the count matrix C_ij and
+ * the receive load R_j).  One rank per GPU, P = cfg->P ranks, rank r owns the experts
+ * with expert_owner[e] == r (or e / (E/P) when expert_owner is NULL), in ascending id.
+ *
+ * cfg describes THIS rank's batch: cfg->N is the rank's own tokens (its source shard);
+ * E, k, d, I, S and the routing rule are the layer's.  Rank r's receive rows are exactly
+ * rows [recv_off[r], recv_off[r+1]) of the one-GPU moe_dispatch_layout whose virtual
+ * sources are the ranks (the ranks' batches concatenated in rank order): expert-major in
+ * ascending id, inside an expert by source rank, then by assignment a.
+ *
+ * The window.  Every rank allocates one device buffer of moe_ep_window_bytes(cfg,
+ * capacity) bytes, zeroes it, and maps every other rank's window into its address space
+ * (moe_ep_ipc_handle on the owner's side, moe_ep_ipc_open on the others'), all before
+ * any rank's first step.  It holds the epoch flags, the count table [P, E], the gate and
+ * the row of each received assignment (capacity rows) and the expert output rows
+ * (capacity routed rows, then S*N shared rows).  capacity = receive rows per owner, the
+ * same on every rank; at most the layer's total assignments are ever needed.  When the
+ * routing sends more than capacity rows to an owner, the rows beyond it are dropped and
+ * MOE_ERR_WORKSPACE is written to *dev_status on every rank.
+ *
+ * epoch: 1, 2, 3, ... one per layer step, the same on every rank.  Each wait compares a
+ * flag with it; flags only grow, so nothing is reset between steps.  Every wait is
+ * bounded (2 s); on timeout MOE_ERR_TIMEOUT is written to *dev_status and the waiting
+ * kernel skips its work, so outputs of that step are undefined but no access leaves its
+ * buffer.
+ *
+ * One step on rank r, in this order on one stream:
+ *   moe_ep_notify      the local layout of r's assignments (moe_dispatch_layout with one
+ *                      owner); r's per-expert counts stored into row r of every rank's
+ *                      count table (peer stores); flag
+ *   moe_ep_layout      waits for all P count rows; the destination (owner, row) of each of
+ *                      r's assignments and the rows r receives per owned expert
+ *   moe_ep_dispatch    each token row read once and stored straight into its owners'
+ *                      receive rows (peer stores over NVLink) with its gate; flag
+ *   moe_ep_expert_ffn  waits for all P sources; grouped SwiGLU over the received rows
+ *                      (FC2 scales each row by its gate) and the shared experts over r's
+ *                      own tokens; flag to every source
+ *   moe_ep_combine     waits for all P owners; y_t = sum over slots of the owners' output
+ *                      rows (peer loads) + the shared rows, fp32, one rounding
+ * A step never waits on a later step of another rank, and a rank's next step writes
+ * another rank's window only after that rank's previous step has finished with the
+ * buffer it writes, so one window serves every step.  moe_ep_layer_forward runs the
+ * router and the five calls in this order.  The calls of one step take the same ws.
+ * ========================================================================== */
+
+typedef struct {
+  int32_t rank;          /* this rank, 0 <= rank < cfg->P */
+  int32_t capacity;      /* receive rows per owner (the same on every rank), >= 0 */
+  int32_t local_experts; /* experts this rank owns (the routed rows of its w13 / w2) */
+  void* const* windows;  /* HOST array [P] of device pointers: each rank's window as mapped in
+                            this process; windows[rank] is this rank's own */
+} moe_ep_group;
+
+/* This rank's part of the EP layout: caller-owned device arrays, all int32.
+ *   dest[N*k]                  owner * capacity + row of each local assignment a in its
+ *                              owner's receive rows; -1 = no row (dropped, or beyond capacity)
+ *   owner_n_e[local_experts]   rows received per owned expert (ascending expert id)
+ *   owner_off[local_experts+1] first receive row of each owned expert; the last entry =
+ *                              rows received (at most capacity) */
+typedef struct {
+  int32_t* dest;
+  int32_t* owner_n_e;
+  int32_t* owner_off;
+} moe_ep_handle;
+
+/* Bytes of one rank's window (0 on an invalid configuration). */
+size_t moe_ep_window_bytes(const moe_config* cfg, int32_t capacity);
+/* Byte offsets of the window's parts (the same on every rank; a rank's own N only sizes
+ * the shared rows at the end): offsets[0..7] = count flags [32] u64, dispatch flags [32]
+ * u64, done flags [32] u64 (each indexed by the signalling rank), dispatch counter u32,
+ * count table [P, E] int32, gates [capacity] fp32, received rows [capacity, d], output
+ * rows [capacity + S*N, d]. */
+moe_status moe_ep_window_layout(const moe_config* cfg, int32_t capacity, size_t* offsets);
+/* Bytes of scratch the EP calls of one step need (ws; the same ws for all calls of a step
+ * and for moe_ep_layer_forward, which also keeps the router outputs and the handle there). */
+size_t moe_ep_workspace_bytes(const moe_config* cfg, int32_t capacity);
+
+/* Window mapping (setup, off the hot path).  moe_ep_ipc_handle writes the 64-byte CUDA IPC
+ * handle of the allocation that holds `window` to handle[64] and the window's byte offset
+ * inside it to *offset; another process passes both to moe_ep_ipc_open, which maps the
+ * allocation (peer access enabled lazily) and returns the window's address there;
+ * moe_ep_ipc_close(window, offset) unmaps it. */
+moe_status moe_ep_ipc_handle(const void* window, void* handle, size_t* offset);
+moe_status moe_ep_ipc_open(const void* handle, size_t offset, void** window);
+moe_status moe_ep_ipc_close(void* window, size_t offset);
+
+/* Step 1: local layout + count exchange.  topk_ids [N, k] (-1 = dropped). */
+moe_status moe_ep_notify(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch,
+                         const int32_t* topk_ids, int32_t* dev_status, void* ws, size_t ws_bytes,
+                         moe_stream_t stream);
+/* Step 2: destinations.  expert_owner [E] or NULL; fills *handle. */
+moe_status moe_ep_layout(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch,
+                         const int32_t* expert_owner, const int32_t* topk_ids, const moe_ep_handle* handle,
+                         int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream);
+/* Step 3: dispatch.  x [N, d] dtype, topk_w [N, k] fp32 (the gates FC2 applies). */
+moe_status moe_ep_dispatch(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const void* x,
+                           const float* topk_w, const moe_ep_handle* handle, moe_stream_t stream);
+/* Step 4: this owner's experts.  x [N, d] (the shared experts' rows); w13 [local_experts + S,
+ * 2I, d] and w2 [local_experts + S, d, I]: the owned experts in ascending id, then the
+ * shared experts (the layout of moe_grouped_ffn's weights restricted to this owner). */
+moe_status moe_ep_expert_ffn(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const void* x,
+                             const void* w13, const void* w2, const moe_ep_handle* handle, int32_t* dev_status,
+                             void* ws, size_t ws_bytes, moe_stream_t stream);
+/* Step 5: combine into y [N, d] dtype, in token order. */
+moe_status moe_ep_combine(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch,
+                          const moe_ep_handle* handle, void* y, int32_t* dev_status, moe_stream_t stream);
+/* The layer on this rank: moe_route on its N tokens, then steps 1-5.  handle_out (NULL ok)
+ * receives the EP layout instead of the workspace. */
+moe_status moe_ep_layer_forward(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const void* x,
+                                const void* w_gate, const float* bias, const int32_t* expert_owner,
+                                const void* w13, const void* w2, void* y, const moe_ep_handle* handle_out,
+                                int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -278,6 +278,61 @@ def dispatch_layout(ids, E: int, P: int, expert_owner=None, S: int = 0) -> dict:
                 row2tok=row2tok, tile_off=tile_off)
 
 
+def ep_layout(ids_per_rank, E: int, P: int, expert_owner=None, capacity=None) -> dict:
+    """The dispatch across P ranks, each rank one source of tokens and the owner of some
+    experts ([EP-DeepEP] §3: tokens go to the owner of their expert and come back to
+    their source; [DeepEP] §2: owner j receives the blocks from sources 0, 1, ... in
+    order; [WideEP] the count matrix).  ids_per_rank[i] is rank i's [n_i, k] top-k ids
+    (n_i may differ, -1 = dropped).
+
+    Owner j's receive rows, from the definition: for each expert e that j owns, in
+    ascending id, the assignments to e of source 0, then of source 1, ..., each source's
+    in ascending local index a = t*k + slot.  With `capacity`, rows at or past it are not
+    received.  Returns
+      cnt[P, E]          counts of each source (the rows exchanged first)
+      recv[j]            [R_j, 2] array of (source i, local a) per receive row of owner j
+      R[P]               rows each owner is sent (before the capacity)
+      dest[i]            [n_i*k]: owner * capacity + row, -1 for dropped / not received
+      owned[j]           experts owner j holds, ascending
+      owner_n_e[j], owner_off[j]  rows received per owned expert and their first row
+                         (capped at capacity; owner_off[j][-1] = rows received)
+    """
+    owner = default_owner(E, P) if expert_owner is None else i64(expert_owner)
+    flats = [i64(x).reshape(-1) for x in ids_per_rank]
+    cnt = np.zeros((P, E), dtype=np.int64)
+    for i, f in enumerate(flats):
+        kept = f[f >= 0]
+        cnt[i] = np.bincount(kept, minlength=E)[:E]
+    recv = [[] for _ in range(P)]
+    for e in range(E):
+        j = int(owner[e])
+        for i, f in enumerate(flats):
+            for a in np.flatnonzero(f == e):
+                recv[j].append((i, int(a)))
+    R = np.array([len(r) for r in recv], dtype=np.int64)
+    cap = int(capacity) if capacity is not None else max(int(R.max()), 1)
+    dest = [np.full(len(f), -1, dtype=np.int64) for f in flats]
+    for j in range(P):
+        for row, (i, a) in enumerate(recv[j]):
+            if row < cap:
+                dest[i][a] = j * cap + row
+    n_tot = cnt.sum(axis=0)
+    owned, owner_n_e, owner_off = [], [], []
+    for j in range(P):
+        mine = [e for e in range(E) if owner[e] == j]
+        first, rows, run = [], [], 0
+        for e in mine:
+            f0 = min(run, cap)
+            first.append(f0)
+            rows.append(min(int(n_tot[e]), cap - f0))
+            run += int(n_tot[e])
+        owned.append(np.array(mine, dtype=np.int64))
+        owner_n_e.append(np.array(rows, dtype=np.int64))
+        owner_off.append(np.array(first + [min(run, cap)], dtype=np.int64))
+    return dict(cnt=cnt, recv=[np.array(r, dtype=np.int64).reshape(-1, 2) for r in recv], R=R, dest=dest,
+                capacity=cap, owned=owned, owner_n_e=owner_n_e, owner_off=owner_off)
+
+
 def imbalance(counts) -> float:
     """max / mean of a load vector ([EP-DeepEP] §4)."""
     c = np.asarray(counts, dtype=np.float64)

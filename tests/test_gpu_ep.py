@@ -1,0 +1,271 @@
+"""Expert parallelism across GPUs (moe_ep_*) with P ranks emulated on one device.
+
+Every rank has its own window and the window table holds all of them, so each rank's
+kernels store into and load from the other ranks' windows exactly as they would through
+peer mappings.  The ranks' calls are issued stage by stage on one stream (all notifies,
+then all layouts, dispatches, expert FFNs and combines), so every wait finds its flags
+already set: no kernel waits on another.
+
+Compared with the oracle element by element: the EP layout (destinations, owner rows),
+the count table, received rows and gates in every window (bit-exact), and y (float
+tolerance); and y against the one-GPU layer on the concatenated batch (bit-exact).
+"""
+import numpy as np
+import pytest
+import torch
+
+import dispatch_combine_grouped_b200 as moe
+from dispatch_combine_grouped_b200 import ep
+from moe_inputs import small_config
+from oracle import moe_oracle as O
+from tests.gpu_cases import assert_close_fro, gpu_inputs
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    (small_config("ep_bf16", cfg_id=90, N=512, d=256, E=16, S=1, k=4, I=128, P=4), None),
+    (small_config("ep_pairs", cfg_id=91, N=1024, d=4096, E=8, S=1, k=2, I=256, P=2), None),
+    (small_config("ep_f32", cfg_id=92, N=256, d=128, E=8, S=0, k=2, I=64, P=2, dtype="f32"), None),
+    (small_config("ep_grouped_owner", cfg_id=93, N=384, d=192, E=32, S=2, k=4, I=96, P=4, n_groups=4,
+                  topk_groups=2, score="sigmoid"), "random"),
+    (small_config("ep_unequal", cfg_id=94, N=512, d=256, E=16, S=1, k=4, I=128, P=4), [200, 0, 57, 255]),
+]
+
+
+def _owner(cfg, spec):
+    if spec != "random":
+        return None
+    g = torch.Generator().manual_seed(cfg.cfg_id)
+    return torch.randint(0, cfg.P, (cfg.E,), generator=g, dtype=torch.int32).cuda()
+
+
+def _shards(cfg, spec):
+    if isinstance(spec, list):
+        return spec
+    return [cfg.N // cfg.P] * cfg.P
+
+
+class Emulated:
+    """P ranks on one device: windows, groups, per-rank weights, workspaces and handles."""
+
+    def __init__(self, cfg, shards, owner=None, capacity=None):
+        self.cfg, self.shards, self.owner = cfg, shards, owner
+        self.capacity = capacity or cfg.N * cfg.k
+        self.rcfg = [cfg.replace(N=n) for n in shards]
+        self.groups, self.windows = ep.emulated_groups(self.rcfg[0], self.capacity, owner, rank_cfgs=self.rcfg)
+        self.owned = [ep.owned_experts(cfg.E, cfg.P, r, owner.cpu() if owner is not None else None)
+                      for r in range(cfg.P)]
+        self.ws = [ep.alloc_ws(c, self.capacity) for c in self.rcfg]
+        self.handles = [ep.Handle(c, len(o)) for c, o in zip(self.rcfg, self.owned)]
+        self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def weights(self, inp):
+        E, S = self.cfg.E, self.cfg.S
+        out = []
+        for o in self.owned:
+            idx = torch.tensor(list(o) + list(range(E, E + S)), dtype=torch.long, device="cuda")
+            out.append((inp["w13"].index_select(0, idx).contiguous(), inp["w2"].index_select(0, idx).contiguous()))
+        return out
+
+    def step(self, inp, epoch, ids=None, w=None):
+        cfg, P = self.cfg, self.cfg.P
+        starts = np.concatenate([[0], np.cumsum(self.shards)])
+        xs = [inp["x"][starts[r]:starts[r + 1]] for r in range(P)]
+        if ids is None:
+            routed = [moe.route(self.rcfg[r], xs[r], inp["w_gate"], inp["bias"]) for r in range(P)]
+            ids = [rt[1] for rt in routed]
+            w = [rt[2] for rt in routed]
+        wts = self.weights(inp)
+        for r in range(P):
+            ep.notify(self.rcfg[r], self.groups[r], epoch, ids[r], self.ws[r], self.status)
+        for r in range(P):
+            ep.layout(self.rcfg[r], self.groups[r], epoch, ids[r], self.handles[r], self.ws[r], self.owner,
+                      self.status)
+        for r in range(P):
+            ep.dispatch(self.rcfg[r], self.groups[r], epoch, xs[r], w[r], self.handles[r])
+        for r in range(P):
+            ep.expert_ffn(self.rcfg[r], self.groups[r], epoch, xs[r], wts[r][0], wts[r][1], self.handles[r],
+                          self.ws[r], self.status)
+        ys = [ep.combine(self.rcfg[r], self.groups[r], epoch, self.handles[r], status=self.status)
+              for r in range(P)]
+        torch.cuda.synchronize()
+        return dict(xs=xs, ids=ids, w=w, y=torch.cat(ys))
+
+
+def check_windows(em, res, lay):
+    """Count tables, received rows and gates in every window, bit-exact."""
+    cfg = em.cfg
+    for j in range(cfg.P):
+        v = ep.window_views(em.rcfg[j], em.capacity, em.windows[j])
+        assert np.array_equal(v["cnt_tab"].cpu().numpy(), lay["cnt"]), f"count table of rank {j}"
+        rows = lay["recv"][j][:em.capacity]
+        R = len(rows)
+        if R == 0:
+            continue
+        x_want = torch.stack([res["xs"][i][a // cfg.k] for i, a in rows])
+        g_want = torch.stack([res["w"][i].reshape(-1)[a] for i, a in rows])
+        assert torch.equal(v["x_recv"][:R], x_want), f"received rows of owner {j}"
+        assert torch.equal(v["gate"][:R], g_want), f"gates of owner {j}"
+
+
+def check_handles(em, lay):
+    for r in range(em.cfg.P):
+        h = em.handles[r].as_dict()
+        assert np.array_equal(h["dest"].cpu().numpy(), lay["dest"][r]), f"dest of rank {r}"
+        assert np.array_equal(h["owner_n_e"].cpu().numpy(), lay["owner_n_e"][r]), f"owner_n_e of rank {r}"
+        assert np.array_equal(h["owner_off"].cpu().numpy(), lay["owner_off"][r]), f"owner_off of rank {r}"
+
+
+def y_oracle(cfg, inp, ids_all, owner, routed_ids=None):
+    """routed_ids: the router's choice before any drop; the gates come from it (a kept
+    assignment keeps its gate), the rows from ids_all."""
+    ref = O.dispatch_layout(ids_all, cfg.E, cfg.P, owner, cfg.S)
+    g64 = O.gate_weights(O.gate_logits(cfg, inp["x"], inp["w_gate"], inp["bias"]),
+                         ids_all if routed_ids is None else routed_ids, cfg.score, cfg.renormalize)
+    xp = O.permute(inp["x"], ref, cfg.k)
+    o = O.experts_on_rows(xp, ref, inp["w13"], inp["w2"], cfg.E)
+    shared = [O.swiglu_expert(inp["x"], inp["w13"][cfg.E + s], inp["w2"][cfg.E + s]) for s in range(cfg.S)]
+    return O.combine(o, ref, g64, cfg.N, cfg.k, shared)
+
+
+@pytest.mark.parametrize("cfg,spec", CASES, ids=[c.name for c, _ in CASES])
+def test_ep_step_matches_oracle(cfg, spec):
+    inp = gpu_inputs(cfg)
+    owner = _owner(cfg, spec)
+    em = Emulated(cfg, _shards(cfg, spec), owner)
+    res = em.step(inp, epoch=1)
+    assert int(em.status.item()) == 0
+    own_np = owner.cpu().numpy() if owner is not None else None
+    lay = O.ep_layout([i.cpu().numpy() for i in res["ids"]], cfg.E, cfg.P, own_np, em.capacity)
+    check_handles(em, lay)
+    check_windows(em, res, lay)
+    ids_all = torch.cat(res["ids"]).cpu().numpy()
+    assert_close_fro(res["y"], y_oracle(cfg, inp, ids_all, own_np), what="EP y")
+    # the one-GPU layer on the concatenated batch gives the same y, bit for bit
+    y1 = moe.layer_forward(cfg, inp["x"], inp["w_gate"], inp["bias"], owner, inp["w13"], inp["w2"])
+    torch.cuda.synchronize()
+    assert torch.equal(res["y"], y1)
+
+
+def test_ep_epochs_reuse_windows():
+    """Three steps on the same windows with different inputs: flags only grow, nothing is reset."""
+    cfg, _ = CASES[0]
+    em = Emulated(cfg, _shards(cfg, None))
+    for epoch in (1, 2, 3):
+        inp = gpu_inputs(cfg, seed_offset=epoch)
+        res = em.step(inp, epoch=epoch)
+        assert int(em.status.item()) == 0
+        y1 = moe.layer_forward(cfg, inp["x"], inp["w_gate"], inp["bias"], None, inp["w13"], inp["w2"])
+        torch.cuda.synchronize()
+        assert torch.equal(res["y"], y1), f"epoch {epoch}"
+        flags = ep.window_views(em.rcfg[0], em.capacity, em.windows[0])
+        assert flags["cnt_flag"][:cfg.P].tolist() == [epoch] * cfg.P
+        assert flags["disp_flag"][:cfg.P].tolist() == [epoch] * cfg.P
+        assert flags["done_flag"][:cfg.P].tolist() == [epoch] * cfg.P
+
+
+def test_ep_capacity_overflow_drops_rows_in_bounds():
+    """capacity below an owner's load: rows past it are not received, every rank reports
+    MOE_ERR_WORKSPACE, and nothing outside the windows is written (guard bands)."""
+    cfg, _ = CASES[0]
+    inp = gpu_inputs(cfg)
+    rcfg = cfg.replace(N=cfg.N // cfg.P)
+    probe = Emulated(cfg, _shards(cfg, None))
+    res0 = probe.step(inp, epoch=1)
+    lay_full = O.ep_layout([i.cpu().numpy() for i in res0["ids"]], cfg.E, cfg.P)
+    cap = int(lay_full["R"].max()) - 7
+    em = Emulated(cfg, _shards(cfg, None), capacity=cap)
+    # windows with 4 KiB guard bands on both sides
+    nbytes, G = ep.window_bytes(rcfg, cap), 4096
+    raws = [torch.full((nbytes + 2 * G,), 0xA5, dtype=torch.uint8, device="cuda") for _ in range(cfg.P)]
+    for r in raws:
+        r[G:G + nbytes].zero_()
+    em.windows = [r[G:G + nbytes] for r in raws]
+    em.groups = [ep.Group(r, cap, len(em.owned[r]), [w.data_ptr() for w in em.windows]) for r in range(cfg.P)]
+    res = em.step(inp, epoch=1, ids=res0["ids"], w=res0["w"])
+    assert int(em.status.item()) == moe.binding.MOE_ERR_WORKSPACE
+    lay = O.ep_layout([i.cpu().numpy() for i in res["ids"]], cfg.E, cfg.P, None, cap)
+    check_handles(em, lay)
+    check_windows(em, res, lay)
+    for r in raws:
+        assert bool((r[:G] == 0xA5).all()) and bool((r[G + nbytes:] == 0xA5).all()), "guard band written"
+
+
+def test_ep_dropped_assignments():
+    """Capacity-factor drops (-1 ids) take no row anywhere and add nothing to y."""
+    cfg, _ = CASES[0]
+    inp = gpu_inputs(cfg)
+    em = Emulated(cfg, _shards(cfg, None))
+    n = cfg.N // cfg.P
+    routed = [moe.route(cfg.replace(N=n), inp["x"][r * n:(r + 1) * n], inp["w_gate"], inp["bias"])
+              for r in range(cfg.P)]
+    ids = [moe.capacity_drop(cfg.replace(N=n), rt[1], 20) for rt in routed]
+    w = [rt[2] for rt in routed]
+    res = em.step(inp, epoch=1, ids=ids, w=w)
+    assert int(em.status.item()) == 0
+    lay = O.ep_layout([i.cpu().numpy() for i in ids], cfg.E, cfg.P, None, em.capacity)
+    assert any((i.cpu().numpy() == -1).any() for i in ids)
+    check_handles(em, lay)
+    check_windows(em, res, lay)
+    ids_all = torch.cat(ids).cpu().numpy()
+    routed_all = torch.cat([rt[1] for rt in routed]).cpu().numpy()
+    assert_close_fro(res["y"], y_oracle(cfg, inp, ids_all, None, routed_all), what="EP y with drops")
+    # the one-GPU steps on the same kept ids and gates give the same y, bit for bit
+    lay1 = moe.dispatch_layout(cfg, torch.cat(ids))
+    xp = moe.permute(cfg, lay1, inp["x"])
+    _, out = moe.grouped_ffn(cfg, lay1, xp, inp["x"], inp["w13"], inp["w2"], topk_w=torch.cat(w))
+    y1 = moe.combine(cfg, lay1, out)
+    torch.cuda.synchronize()
+    assert torch.equal(res["y"], y1)
+
+
+def test_ep_one_rank_layer_forward_matches_one_gpu_layer():
+    """P = 1: moe_ep_layer_forward (router + the five steps in one call) equals moe_layer_forward."""
+    cfg = small_config("ep_p1", cfg_id=95, N=300, d=256, E=16, S=1, k=4, I=128, P=1)
+    inp = gpu_inputs(cfg)
+    cap = cfg.N * cfg.k
+    groups, windows = ep.emulated_groups(cfg, cap)
+    ws = ep.alloc_ws(cfg, cap)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    h = ep.Handle(cfg, cfg.E)
+    for epoch in (1, 2):
+        y = ep.layer_forward(cfg, groups[0], epoch, inp["x"], inp["w_gate"], inp["bias"], inp["w13"], inp["w2"], ws,
+                             handle=h, status=status)
+        y1 = moe.layer_forward(cfg, inp["x"], inp["w_gate"], inp["bias"], None, inp["w13"], inp["w2"])
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert torch.equal(y, y1), f"epoch {epoch}"
+
+
+def test_ep_wait_times_out_and_context_stays_usable():
+    """A layout for an epoch no rank has published: the bounded wait gives up (2 s),
+    MOE_ERR_TIMEOUT is reported, no destination is written, and the context still runs."""
+    cfg, _ = CASES[0]
+    inp = gpu_inputs(cfg)
+    em = Emulated(cfg, _shards(cfg, None))
+    res = em.step(inp, epoch=1)
+    assert int(em.status.item()) == 0
+    rc = em.rcfg[0]
+    ep.layout(rc, em.groups[0], 2, res["ids"][0], em.handles[0], em.ws[0], None, em.status)
+    torch.cuda.synchronize()
+    assert int(em.status.item()) == moe.binding.MOE_ERR_TIMEOUT
+    assert bool((em.handles[0].as_dict()["dest"] == -1).all())
+    z = torch.ones(1024, device="cuda") * 2
+    assert float(z.sum().item()) == 2048.0
+
+
+def test_ep_host_errors():
+    cfg, _ = CASES[0]
+    rc = cfg.replace(N=cfg.N // cfg.P)
+    em = Emulated(cfg, _shards(cfg, None))
+    ids = torch.zeros(rc.N, rc.k, dtype=torch.int32, device="cuda")
+    with pytest.raises(moe.MoEError):   # epoch 0
+        ep.notify(rc, em.groups[0], 0, ids, em.ws[0])
+    with pytest.raises(moe.MoEError):   # rank outside [0, P)
+        ep.notify(rc, ep.Group(cfg.P, em.capacity, 4, em.groups[0].windows), 1, ids, em.ws[0])
+    with pytest.raises(moe.MoEError):   # small workspace
+        ep.notify(rc, em.groups[0], 1, ids, em.ws[0][:16])
+    with pytest.raises(moe.MoEError):   # unaligned window
+        bad = list(em.groups[0].windows)
+        bad[1] += 16
+        ep.notify(rc, ep.Group(0, em.capacity, 4, bad), 1, ids, em.ws[0])
