@@ -43,6 +43,9 @@ def parse():
                          "(one JSON line with the curve)")
     ap.add_argument("--fp8", action="store_true",
                     help="the FP8 (e4m3) expert path: quantised dispatch payload and expert GEMMs")
+    ap.add_argument("--ep", type=int, default=0, metavar="P",
+                    help="expert parallelism with P ranks emulated on this GPU (moe_ep_*): per-stage times "
+                         "of all ranks, the one-GPU layer beside it, and the NVLink bytes a real P-GPU step moves")
     ap.add_argument("--eplb", type=int, default=0, metavar="R",
                     help="run the routed experts over E + R physical slots (redundant copies of the "
                          "hot experts, planned from the batch's own counts)")
@@ -344,6 +347,142 @@ def run_movement_sweep(args, cfg, local):
           flush=True)
 
 
+def run_ep(args, cfg, local):
+    """The expert-parallel layer (moe_ep_*) with P ranks emulated on this GPU: P windows,
+    each rank's stages issued for all ranks in turn on one stream (every wait finds its
+    flags set).  Times each stage summed over the ranks, L2 flushed before every step,
+    beside the one-GPU layer on the same batch, and counts the rows a real P-GPU step
+    sends across NVLink (assignments whose owner is not their source)."""
+    import torch
+    import dispatch_combine_grouped_b200 as moe
+    from dispatch_combine_grouped_b200 import ep
+    from moe_inputs import make_inputs
+
+    P = args.ep
+    if cfg.N % P or cfg.E % P:
+        raise SystemExit(f"--ep {P}: N and E of {cfg.name} must be multiples of P")
+    dev = torch.device("cuda", local)
+    gcfg = cfg.replace(P=P)
+    inp = make_inputs(gcfg, device=dev)
+    n = cfg.N // P
+    rc = gcfg.replace(N=n)
+    cap = 2 * -(-cfg.N * cfg.k // P)          # receive rows per owner: twice the mean load
+    groups, windows = ep.emulated_groups(rc, cap)
+    ws = [ep.alloc_ws(rc, cap) for _ in range(P)]
+    handles = [ep.Handle(rc, cfg.E // P) for _ in range(P)]
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    E, S = cfg.E, cfg.S
+    wts = []
+    for r in range(P):
+        idx = torch.tensor(list(range(r * E // P, (r + 1) * E // P)) + list(range(E, E + S)), device=dev)
+        wts.append((inp["w13"].index_select(0, idx), inp["w2"].index_select(0, idx)))
+    xs = [inp["x"][r * n:(r + 1) * n] for r in range(P)]
+    routed = [moe.route(rc, xs[r], inp["w_gate"], inp["bias"]) for r in range(P)]
+    ys = [torch.empty(n, cfg.d, dtype=cfg.torch_dtype, device=dev) for _ in range(P)]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stages = ["route", "notify", "layout", "dispatch", "ffn", "combine"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record()
+        mark(0)
+        for r in range(P):
+            moe.route(rc, xs[r], inp["w_gate"], inp["bias"], out=routed[r])
+        mark(1)
+        for r in range(P):
+            ep.notify(rc, groups[r], routed[r][1], ws[r], status)
+        mark(2)
+        for r in range(P):
+            ep.layout(rc, groups[r], routed[r][1], handles[r], ws[r], None, status)
+        mark(3)
+        for r in range(P):
+            ep.dispatch(rc, groups[r], xs[r], routed[r][2], handles[r])
+        mark(4)
+        for r in range(P):
+            ep.expert_ffn(rc, groups[r], xs[r], wts[r][0], wts[r][1], handles[r], ws[r], status)
+        mark(5)
+        for r in range(P):
+            ep.combine(rc, groups[r], handles[r], y=ys[r], status=status)
+        mark(6)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise SystemExit(f"EP step reported status {int(status.item())}")
+    # per-stage times (eager launches, events between the stages)
+    tot = [0.0] * len(stages)
+    for _ in range(args.steps):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+        step(ev)
+        torch.cuda.synchronize()
+        for i in range(len(stages)):
+            tot[i] += ev[i].elapsed_time(ev[i + 1])
+    # the whole step as one CUDA graph replay (no host launch gaps); each replay is a new
+    # step because the step number lives in the windows
+    cs = torch.cuda.Stream(device=dev)
+    cs.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cs):
+        step()
+    step_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        step_ms.append(a.elapsed_time(b))
+    if int(status.item()) != 0:
+        raise SystemExit(f"EP step reported status {int(status.item())}")
+    # the one-GPU layer on the same batch (same experts, one owner per E/P block)
+    ws1 = moe.alloc_workspace(gcfg, dev)
+    y1 = moe.layer_forward(gcfg, inp["x"], inp["w_gate"], inp["bias"], None, inp["w13"], inp["w2"], ws=ws1)
+    one = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        moe.layer_forward(gcfg, inp["x"], inp["w_gate"], inp["bias"], None, inp["w13"], inp["w2"], y=y1, ws=ws1)
+        b.record()
+        torch.cuda.synchronize()
+        one.append(a.elapsed_time(b))
+    same = bool(torch.equal(torch.cat(ys), y1))
+    # rows a real P-GPU step moves between GPUs (owner != source), per rank and direction
+    eb = 2 if cfg.dtype == "bf16" else 4
+    cross = []
+    for r in range(P):
+        dest = handles[r].as_dict()["dest"]
+        owner = torch.div(dest[dest >= 0], cap, rounding_mode="floor")
+        cross.append(int((owner != r).sum().item()))
+    row_bytes = cfg.d * eb
+    max_cross = max(cross) * row_bytes
+    med = sorted(step_ms)[len(step_ms) // 2]
+    stage_ms = {k: tot[i] / args.steps for i, k in enumerate(stages)}
+    x_bytes, rows_bytes = cfg.N * row_bytes, cfg.N * cfg.k * row_bytes
+    print(json.dumps({
+        "metric": "MoE-layer tokens/s, expert-parallel path with P ranks emulated on one GPU",
+        "value": cfg.N / (med / 1e3), "unit": "tokens/s", "n_gpus": 1, "ep_ranks_emulated": P,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": med, "dtype": cfg.dtype,
+        "config": {"workload": describe(gcfg), "tokens_per_rank": n, "capacity_rows_per_owner": cap,
+                   "l2": "flushed before every step"},
+        "how": "ms_per_step: the emulated step of all P ranks as one CUDA graph replay; stages: eager launches "
+               "with events between the stages (all ranks of a stage together)",
+        "stages_ms_all_ranks": stage_ms,
+        "dispatch_gbs_local": (x_bytes + rows_bytes) / (stage_ms["dispatch"] / 1e3) / 1e9,
+        "combine_gbs_local": (rows_bytes + S * x_bytes + x_bytes) / (stage_ms["combine"] / 1e3) / 1e9,
+        "one_gpu_layer_ms": sorted(one)[len(one) // 2],
+        "y_bit_identical_to_one_gpu_layer": same,
+        "nvlink": {"cross_rows_per_rank": cross, "max_bytes_per_rank_per_direction": max_cross,
+                   "roofline_us_at_770_gbs": max_cross / 770e9 * 1e6,
+                   "note": "bytes a real P-GPU step moves over NVLink each way; not measured here (one GPU)"},
+        "status": int(status.item()),
+    }), flush=True)
+
+
 def run_fp8(args, cfg, world, rank, local):
     """The layer with the FP8 expert path on one stream: route -> layout -> quantise x +
     FP8 permute -> FP8 grouped FFN (FC1, h quantisation, FC2) -> combine.  Weights are
@@ -501,6 +640,13 @@ def main():
     if args.movement_sweep:
         if rank == 0:
             run_movement_sweep(args, cfg, local)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    if args.ep:
+        if rank == 0:
+            run_ep(args, cfg, local)
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()

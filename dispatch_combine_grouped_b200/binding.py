@@ -114,7 +114,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_layer_forward_fp8_overlapped": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp,
                                                    vp]),
     }
-    grpp, hdp, u64 = ctypes.POINTER(CEpGroup), ctypes.POINTER(CEpHandle), ctypes.c_uint64
+    grpp, hdp = ctypes.POINTER(CEpGroup), ctypes.POINTER(CEpHandle)
     sig.update({
         "moe_ep_window_bytes": (sz, [cfgp, i32]),
         "moe_ep_window_layout": (i32, [cfgp, i32, vp]),
@@ -122,12 +122,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_ep_ipc_handle": (i32, [vp, vp, ctypes.POINTER(sz)]),
         "moe_ep_ipc_open": (i32, [vp, sz, ctypes.POINTER(vp)]),
         "moe_ep_ipc_close": (i32, [vp, sz]),
-        "moe_ep_notify": (i32, [cfgp, grpp, u64, vp, vp, vp, sz, vp]),
-        "moe_ep_layout": (i32, [cfgp, grpp, u64, vp, vp, hdp, vp, vp, sz, vp]),
-        "moe_ep_dispatch": (i32, [cfgp, grpp, u64, vp, vp, hdp, vp]),
-        "moe_ep_expert_ffn": (i32, [cfgp, grpp, u64, vp, vp, vp, hdp, vp, vp, sz, vp]),
-        "moe_ep_combine": (i32, [cfgp, grpp, u64, hdp, vp, vp, vp]),
-        "moe_ep_layer_forward": (i32, [cfgp, grpp, u64, vp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz, vp]),
+        "moe_ep_notify": (i32, [cfgp, grpp, vp, vp, vp, sz, vp]),
+        "moe_ep_layout": (i32, [cfgp, grpp, vp, vp, hdp, vp, vp, sz, vp]),
+        "moe_ep_dispatch": (i32, [cfgp, grpp, vp, vp, hdp, vp]),
+        "moe_ep_expert_ffn": (i32, [cfgp, grpp, vp, vp, vp, hdp, vp, vp, sz, vp]),
+        "moe_ep_combine": (i32, [cfgp, grpp, hdp, vp, vp, vp]),
+        "moe_ep_layer_forward": (i32, [cfgp, grpp, vp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz, vp]),
     })
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

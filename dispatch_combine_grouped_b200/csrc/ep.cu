@@ -20,8 +20,11 @@
 //            the last CTA to finish publishes the epoch to every owner
 //   combine  the gather-and-sum kernel with remote sources: the owners' output rows are
 //            loaded over NVLink and summed in slot order in fp32
-// Flags hold epochs (1, 2, 3, ... one per step) and only grow, so nothing is reset
-// between steps.  Every wait is bounded (MOE_WAIT_LIMIT_NS) and reports MOE_ERR_TIMEOUT.
+// Flags hold epochs: each rank counts its steps in its own window (the notify kernel
+// increments the count, later kernels of the step read it), so the epoch is never a
+// launch argument and a captured CUDA graph replays correctly.  Flags only grow, so
+// nothing is reset between steps.  Every wait is bounded (MOE_WAIT_LIMIT_NS) and
+// reports MOE_ERR_TIMEOUT.
 // No TMA and no multicast touches peer memory: peer traffic is plain 16-byte loads and
 // stores.
 #include "common.cuh"
@@ -64,16 +67,24 @@ __device__ __forceinline__ T* at(const char* base, size_t off) {
   return reinterpret_cast<T*>(const_cast<char*>(base) + off);
 }
 
+// This rank's current step (written by an earlier kernel on the same stream).
+__device__ __forceinline__ uint64_t step_of(const char* own, const EpOffsets& off) {
+  return *reinterpret_cast<const volatile uint64_t*>(own + off.step);
+}
+
 // ---------------------------------------------------------------- count exchange
 // Row `me` of every rank's count table = this rank's per-expert counts n_loc[E].
 __global__ void ep_push_counts_kernel(const __grid_constant__ EpPeers peers, EpOffsets off,
-                                      const int32_t* __restrict__ n_loc, int E, int P, int me, uint64_t epoch) {
+                                      const int32_t* __restrict__ n_loc, int E, int P, int me) {
   for (int p = 0; p < P; ++p) {
     int32_t* row = at<int32_t>(peers.base[p], off.cnt_tab) + (size_t)me * E;
     for (int e = threadIdx.x; e < E; e += blockDim.x) row[e] = n_loc[e];
   }
   __syncthreads();
   if (threadIdx.x == 0) {
+    uint64_t* step = at<uint64_t>(peers.base[me], off.step);
+    const uint64_t epoch = *step + 1;  // this step
+    *step = epoch;
     __threadfence_system();
     for (int p = 0; p < P; ++p) st_release_sys(at<uint64_t>(peers.base[p], off.cnt_flag) + me, epoch);
   }
@@ -88,7 +99,6 @@ struct EpLayoutArgs {
   int E, P, me, A, capacity, local_experts, per_owner;
   const char* win;            // this rank's window
   EpOffsets off;
-  uint64_t epoch;
   int32_t* dest;              // [A] owner * capacity + row, -1 = no row
   int32_t* own_n_e;           // [local_experts]
   int32_t* own_off;           // [local_experts + 1]
@@ -105,7 +115,7 @@ __global__ void __launch_bounds__(kEpLayoutThreads) ep_layout_kernel(EpLayoutArg
   __shared__ int own_of[kMaxSlots];
   __shared__ int R[kMaxP];
   const int tid = threadIdx.x;
-  if (tid == 0) s_ok = wait_epochs(at<uint64_t>(a.win, a.off.cnt_flag), a.P, a.epoch, a.status);
+  if (tid == 0) s_ok = wait_epochs(at<uint64_t>(a.win, a.off.cnt_flag), a.P, step_of(a.win, a.off), a.status);
   __syncthreads();
   const int32_t* cnt = at<int32_t>(a.win, a.off.cnt_tab);
   for (int e = tid; e < a.E; e += blockDim.x) {
@@ -195,8 +205,8 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_dispatch_kernel(const __grid
                                                                      EpOffsets off, const uint4* __restrict__ x,
                                                                      const int32_t* __restrict__ dest,
                                                                      const float* __restrict__ topk_w, int N,
-                                                                     int k, int vpr, int capacity, int P, int me,
-                                                                     uint64_t epoch) {
+                                                                     int k, int vpr, int capacity, int P,
+                                                                     int me) {
   const int lane = threadIdx.x & 31;
   for (int t = blockIdx.x * kEpWarps + (threadIdx.x >> 5); t < N; t += gridDim.x * kEpWarps) {
     const int my = lane < k ? dest[(size_t)t * k + lane] : -1;
@@ -242,6 +252,7 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_dispatch_kernel(const __grid
     uint32_t* ctr = at<uint32_t>(peers.base[me], off.disp_ctr);
     if (atomicAdd(ctr, 1u) == gridDim.x - 1) {
       *ctr = 0;  // ready for the next launch, which is stream-ordered after this one
+      const uint64_t epoch = step_of(peers.base[me], off);
       __threadfence_system();
       for (int p = 0; p < P; ++p) st_release_sys(at<uint64_t>(peers.base[p], off.disp_flag) + me, epoch);
     }
@@ -249,14 +260,15 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_dispatch_kernel(const __grid
 }
 
 // ---------------------------------------------------------------- waits and signals
-__global__ void ep_wait_kernel(const uint64_t* flags, int n, uint64_t epoch, int* status) {
-  if (threadIdx.x == 0) wait_epochs(flags, n, epoch, status);
+__global__ void ep_wait_kernel(const char* own, EpOffsets off, size_t flag_off, int n, int* status) {
+  if (threadIdx.x == 0) wait_epochs(at<uint64_t>(own, flag_off), n, step_of(own, off), status);
 }
 
 // flag[me] = epoch in every rank's window, after everything before this launch on the stream
-__global__ void ep_signal_kernel(const __grid_constant__ EpPeers peers, size_t flag_off, int P, int me,
-                                 uint64_t epoch) {
+__global__ void ep_signal_kernel(const __grid_constant__ EpPeers peers, EpOffsets off, size_t flag_off, int P,
+                                 int me) {
   if (threadIdx.x != 0) return;
+  const uint64_t epoch = step_of(peers.base[me], off);
   __threadfence_system();
   for (int p = 0; p < P; ++p) st_release_sys(at<uint64_t>(peers.base[p], flag_off) + me, epoch);
 }
@@ -311,9 +323,10 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_combine_kernel(const __grid_
                                                                     EpOffsets off, const int32_t* __restrict__ dest,
                                                                     uint4* __restrict__ y, int N, int k, int S,
                                                                     int vpr, int capacity, int P, int me,
-                                                                    uint64_t epoch, int* status) {
+                                                                    int* status) {
   __shared__ int s_ok;
-  if (threadIdx.x == 0) s_ok = wait_epochs(at<uint64_t>(peers.base[me], off.done_flag), P, epoch, status);
+  if (threadIdx.x == 0)
+    s_ok = wait_epochs(at<uint64_t>(peers.base[me], off.done_flag), P, step_of(peers.base[me], off), status);
   __syncthreads();
   if (!s_ok) return;
   const int lane = threadIdx.x & 31;
@@ -354,7 +367,8 @@ EpOffsets ep_offsets(const moe_config& c, int capacity) {
   o.cnt_flag = 0;
   o.disp_flag = o.cnt_flag + kMaxP * sizeof(uint64_t);
   o.done_flag = o.disp_flag + kMaxP * sizeof(uint64_t);
-  o.disp_ctr = o.done_flag + kMaxP * sizeof(uint64_t);
+  o.step = o.done_flag + kMaxP * sizeof(uint64_t);
+  o.disp_ctr = o.step + sizeof(uint64_t);
   o.cnt_tab = al256(o.disp_ctr + sizeof(uint32_t));
   o.gate = al256(o.cnt_tab + (size_t)c.P * c.E * sizeof(int32_t));
   o.x_recv = al256(o.gate + (size_t)capacity * sizeof(float));
@@ -371,15 +385,14 @@ static inline unsigned ep_grid(long long items, int per_cta) {
 }
 
 cudaError_t launch_ep_push_counts(const EpPeers& peers, const EpOffsets& off, const int32_t* n_loc, int E, int P,
-                                  int me, uint64_t epoch, cudaStream_t st) {
-  ep_push_counts_kernel<<<1, 256, 0, st>>>(peers, off, n_loc, E, P, me, epoch);
+                                  int me, cudaStream_t st) {
+  ep_push_counts_kernel<<<1, 256, 0, st>>>(peers, off, n_loc, E, P, me);
   return cudaGetLastError();
 }
 
 cudaError_t launch_ep_layout(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me, int capacity,
-                             int local_experts, uint64_t epoch, const int32_t* owner, const int32_t* ids,
-                             const moe_layout& loc, int32_t* dest, int32_t* own_n_e, int32_t* own_off, int* status,
-                             cudaStream_t st) {
+                             int local_experts, const int32_t* owner, const int32_t* ids, const moe_layout& loc,
+                             int32_t* dest, int32_t* own_n_e, int32_t* own_off, int* status, cudaStream_t st) {
   EpLayoutArgs a;
   a.ids = ids;
   a.tok2row = loc.tok2row;
@@ -394,7 +407,6 @@ cudaError_t launch_ep_layout(const moe_config& c, const EpPeers& peers, const Ep
   a.per_owner = c.E / c.P > 0 ? c.E / c.P : 1;
   a.win = peers.base[me];
   a.off = off;
-  a.epoch = epoch;
   a.dest = dest;
   a.own_n_e = own_n_e;
   a.own_off = own_off;
@@ -404,36 +416,37 @@ cudaError_t launch_ep_layout(const moe_config& c, const EpPeers& peers, const Ep
 }
 
 cudaError_t launch_ep_dispatch(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me,
-                               int capacity, uint64_t epoch, const void* x, const int32_t* dest,
-                               const float* topk_w, cudaStream_t st) {
+                               int capacity, const void* x, const int32_t* dest, const float* topk_w,
+                               cudaStream_t st) {
   const int vpr = c.d * (c.dtype == MOE_BF16 ? 2 : 4) / 16;
   ep_dispatch_kernel<<<ep_grid(c.N, kEpWarps), kEpWarps * 32, 0, st>>>(
-      peers, off, static_cast<const uint4*>(x), dest, topk_w, c.N, c.k, vpr, capacity, c.P, me, epoch);
+      peers, off, static_cast<const uint4*>(x), dest, topk_w, c.N, c.k, vpr, capacity, c.P, me);
   return cudaGetLastError();
 }
 
-cudaError_t launch_ep_wait(const uint64_t* flags, int n, uint64_t epoch, int* status, cudaStream_t st) {
-  ep_wait_kernel<<<1, 32, 0, st>>>(flags, n, epoch, status);
+cudaError_t launch_ep_wait(const char* own, const EpOffsets& off, size_t flag_off, int n, int* status,
+                           cudaStream_t st) {
+  ep_wait_kernel<<<1, 32, 0, st>>>(own, off, flag_off, n, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_ep_signal(const EpPeers& peers, size_t flag_off, int P, int me, uint64_t epoch,
+cudaError_t launch_ep_signal(const EpPeers& peers, const EpOffsets& off, size_t flag_off, int P, int me,
                              cudaStream_t st) {
-  ep_signal_kernel<<<1, 32, 0, st>>>(peers, flag_off, P, me, epoch);
+  ep_signal_kernel<<<1, 32, 0, st>>>(peers, off, flag_off, P, me);
   return cudaGetLastError();
 }
 
 cudaError_t launch_ep_combine(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me, int capacity,
-                              uint64_t epoch, const int32_t* dest, void* y, int* status, cudaStream_t st) {
+                              const int32_t* dest, void* y, int* status, cudaStream_t st) {
   const int vpr = c.d * (c.dtype == MOE_BF16 ? 2 : 4) / 16;
   const long long items = (long long)c.N * ((vpr + 31) / 32);
   const unsigned grid = ep_grid(items, kEpWarps);
   if (c.dtype == MOE_BF16)
     ep_combine_kernel<__nv_bfloat16><<<grid, kEpWarps * 32, 0, st>>>(
-        peers, off, dest, static_cast<uint4*>(y), c.N, c.k, c.n_shared, vpr, capacity, c.P, me, epoch, status);
+        peers, off, dest, static_cast<uint4*>(y), c.N, c.k, c.n_shared, vpr, capacity, c.P, me, status);
   else
     ep_combine_kernel<float><<<grid, kEpWarps * 32, 0, st>>>(
-        peers, off, dest, static_cast<uint4*>(y), c.N, c.k, c.n_shared, vpr, capacity, c.P, me, epoch, status);
+        peers, off, dest, static_cast<uint4*>(y), c.N, c.k, c.n_shared, vpr, capacity, c.P, me, status);
   return cudaGetLastError();
 }
 

@@ -115,6 +115,7 @@ moe_status eplb_plan(int E, int R, int P, const int64_t* load, int32_t* copies, 
 // allocates with the same size; its parts sit at the same offsets on every rank.
 struct EpOffsets {
   size_t cnt_flag, disp_flag, done_flag;  // [kMaxP] u64 epochs, indexed by the signalling rank
+  size_t step;                            // u64: this rank's steps so far (= the running step's epoch)
   size_t disp_ctr;                        // u32: this rank's dispatch CTAs finished in the running launch
   size_t cnt_tab;                         // [P, E] int32: row i = source i's expert counts
   size_t gate;                            // [capacity] fp32: gate of each received row
@@ -127,19 +128,19 @@ struct EpPeers {
 };
 EpOffsets ep_offsets(const moe_config& c, int capacity);
 cudaError_t launch_ep_push_counts(const EpPeers& peers, const EpOffsets& off, const int32_t* n_loc, int E, int P,
-                                  int me, uint64_t epoch, cudaStream_t st);
+                                  int me, cudaStream_t st);
 cudaError_t launch_ep_layout(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me, int capacity,
-                             int local_experts, uint64_t epoch, const int32_t* owner, const int32_t* ids,
-                             const moe_layout& loc, int32_t* dest, int32_t* own_n_e, int32_t* own_off, int* status,
-                             cudaStream_t st);
+                             int local_experts, const int32_t* owner, const int32_t* ids, const moe_layout& loc,
+                             int32_t* dest, int32_t* own_n_e, int32_t* own_off, int* status, cudaStream_t st);
 cudaError_t launch_ep_dispatch(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me,
-                               int capacity, uint64_t epoch, const void* x, const int32_t* dest,
-                               const float* topk_w, cudaStream_t st);
-cudaError_t launch_ep_wait(const uint64_t* flags, int n, uint64_t epoch, int* status, cudaStream_t st);
-cudaError_t launch_ep_signal(const EpPeers& peers, size_t flag_off, int P, int me, uint64_t epoch,
+                               int capacity, const void* x, const int32_t* dest, const float* topk_w,
+                               cudaStream_t st);
+cudaError_t launch_ep_wait(const char* own, const EpOffsets& off, size_t flag_off, int n, int* status,
+                           cudaStream_t st);
+cudaError_t launch_ep_signal(const EpPeers& peers, const EpOffsets& off, size_t flag_off, int P, int me,
                              cudaStream_t st);
 cudaError_t launch_ep_combine(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me, int capacity,
-                              uint64_t epoch, const int32_t* dest, void* y, int* status, cudaStream_t st);
+                              const int32_t* dest, void* y, int* status, cudaStream_t st);
 
 int sm_count();
 // TMA maps for bf16 K-major operands; box_k (64, 32 or 16) selects the 128/64/32-byte swizzle

@@ -358,7 +358,7 @@ EpWs carve_ep(const moe_config& c, int capacity, char* base) {
   return w;
 }
 
-moe_status check_ep(const moe_config* cfg, const moe_ep_group* g, uint64_t epoch, EpPeers* peers) {
+moe_status check_ep(const moe_config* cfg, const moe_ep_group* g, EpPeers* peers) {
   moe_status s = check_config(cfg);
   if (s != MOE_OK) return s;
   if (!g || !g->windows) return fail(MOE_ERR_INVALID_ARG, "EP group or its window table is NULL");
@@ -368,7 +368,6 @@ moe_status check_ep(const moe_config* cfg, const moe_ep_group* g, uint64_t epoch
       (long long)g->capacity + (long long)c.n_shared * c.N >= (1LL << 30))
     return fail(MOE_ERR_UNSUPPORTED, "need 1 <= capacity, capacity * P < 2^31 and capacity + S*N < 2^30");
   if (g->local_experts < 0 || g->local_experts > c.E) return fail(MOE_ERR_INVALID_ARG, "local_experts outside [0, E]");
-  if (epoch == 0) return fail(MOE_ERR_INVALID_ARG, "epochs start at 1");
   memset(peers, 0, sizeof(*peers));
   for (int p = 0; p < c.P; ++p) {
     if (!g->windows[p] || (reinterpret_cast<uintptr_t>(g->windows[p]) & 255) != 0)
@@ -386,32 +385,32 @@ moe_status check_ep_ws(const moe_config& c, const moe_ep_group* g, void* ws, siz
 
 bool handle_complete(const moe_ep_handle* h) { return h && h->dest && h->owner_n_e && h->owner_off; }
 
-moe_status ep_notify_impl(const moe_config& c, const moe_ep_group& g, const EpPeers& peers, uint64_t epoch,
+moe_status ep_notify_impl(const moe_config& c, const moe_ep_group& g, const EpPeers& peers,
                           const int32_t* ids, int32_t* status, const EpWs& w, cudaStream_t st) {
   moe_status s = cuda_status(launch_layout(one_owner(c), nullptr, ids, w.loc, status, w.lay_ws, st), "local layout");
   if (s != MOE_OK) return s;
   return cuda_status(
-      launch_ep_push_counts(peers, ep_offsets(c, g.capacity), w.loc.n_e, c.E, c.P, g.rank, epoch, st),
+      launch_ep_push_counts(peers, ep_offsets(c, g.capacity), w.loc.n_e, c.E, c.P, g.rank, st),
       "count exchange");
 }
 
-moe_status ep_layout_impl(const moe_config& c, const moe_ep_group& g, const EpPeers& peers, uint64_t epoch,
+moe_status ep_layout_impl(const moe_config& c, const moe_ep_group& g, const EpPeers& peers,
                           const int32_t* owner, const int32_t* ids, const moe_ep_handle& hd, int32_t* status,
                           const EpWs& w, cudaStream_t st) {
   return cuda_status(launch_ep_layout(c, peers, ep_offsets(c, g.capacity), g.rank, g.capacity, g.local_experts,
-                                      epoch, owner, ids, w.loc, hd.dest, hd.owner_n_e, hd.owner_off, status, st),
+                                      owner, ids, w.loc, hd.dest, hd.owner_n_e, hd.owner_off, status, st),
                      "EP layout");
 }
 
 // The owner's grouped FFN: routed groups = the owned experts over the received rows
 // (A_routed = capacity, no row map: row r's gate is gate[r]), shared groups over the
 // rank's own N tokens; outputs into the window's output rows.
-moe_status ep_ffn_impl(const moe_config& c, const moe_ep_group& g, const EpPeers& peers, uint64_t epoch,
+moe_status ep_ffn_impl(const moe_config& c, const moe_ep_group& g, const EpPeers& peers,
                        const void* x, const void* w13, const void* w2, const moe_ep_handle& hd, int32_t* status,
                        const EpWs& w, cudaStream_t st) {
   const EpOffsets off = ep_offsets(c, g.capacity);
   char* win = peers.base[g.rank];
-  cudaError_t e = launch_ep_wait(reinterpret_cast<const uint64_t*>(win + off.disp_flag), c.P, epoch, status, st);
+  cudaError_t e = launch_ep_wait(win, off, off.disp_flag, c.P, status, st);
   if (e != cudaSuccess) return cuda_status(e, "dispatch wait");
   moe_config co = c;
   co.E = g.local_experts;
@@ -436,7 +435,7 @@ moe_status ep_ffn_impl(const moe_config& c, const moe_ep_group& g, const EpPeers
     e = c.dtype == MOE_BF16 ? tc_grouped(g2, dec, g.capacity + S * c.N, 0, st) : launch_simt_gemm(g2, st);
     if (e != cudaSuccess) return cuda_status(e, "EP FC2 grouped GEMM");
   }
-  return cuda_status(launch_ep_signal(peers, off.done_flag, c.P, g.rank, epoch, st), "FFN done signal");
+  return cuda_status(launch_ep_signal(peers, off, off.done_flag, c.P, g.rank, st), "FFN done signal");
 }
 
 }  // namespace
@@ -870,7 +869,8 @@ moe_status moe_ep_window_layout(const moe_config* cfg, int32_t capacity, size_t*
   if (s != MOE_OK) return s;
   if (capacity < 1 || !offsets) return fail(MOE_ERR_INVALID_ARG, "capacity < 1 or NULL offsets");
   const EpOffsets o = ep_offsets(*cfg, capacity);
-  const size_t v[8] = {o.cnt_flag, o.disp_flag, o.done_flag, o.disp_ctr, o.cnt_tab, o.gate, o.x_recv, o.out_recv};
+  const size_t v[9] = {o.cnt_flag, o.disp_flag, o.done_flag, o.step, o.disp_ctr, o.cnt_tab, o.gate, o.x_recv,
+                       o.out_recv};
   memcpy(offsets, v, sizeof(v));
   return MOE_OK;
 }
@@ -913,72 +913,72 @@ moe_status moe_ep_ipc_close(void* window, size_t offset) {
   return cuda_status(cudaIpcCloseMemHandle(static_cast<char*>(window) - offset), "cudaIpcCloseMemHandle");
 }
 
-moe_status moe_ep_notify(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const int32_t* topk_ids,
+moe_status moe_ep_notify(const moe_config* cfg, const moe_ep_group* grp, const int32_t* topk_ids,
                          int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream) {
   EpPeers peers;
-  moe_status s = check_ep(cfg, grp, epoch, &peers);
+  moe_status s = check_ep(cfg, grp, &peers);
   if (s != MOE_OK) return s;
   if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes)) != MOE_OK) return s;
   if (cfg->N > 0 && !topk_ids) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
-  return ep_notify_impl(*cfg, *grp, peers, epoch, topk_ids, dev_status, carve_ep(*cfg, grp->capacity, (char*)ws),
+  return ep_notify_impl(*cfg, *grp, peers, topk_ids, dev_status, carve_ep(*cfg, grp->capacity, (char*)ws),
                         (cudaStream_t)stream);
 }
 
-moe_status moe_ep_layout(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const int32_t* expert_owner,
+moe_status moe_ep_layout(const moe_config* cfg, const moe_ep_group* grp, const int32_t* expert_owner,
                          const int32_t* topk_ids, const moe_ep_handle* handle, int32_t* dev_status, void* ws,
                          size_t ws_bytes, moe_stream_t stream) {
   EpPeers peers;
-  moe_status s = check_ep(cfg, grp, epoch, &peers);
+  moe_status s = check_ep(cfg, grp, &peers);
   if (s != MOE_OK) return s;
   if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
   if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes)) != MOE_OK) return s;
   if (!handle_complete(handle) || (cfg->N > 0 && !topk_ids)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
-  return ep_layout_impl(*cfg, *grp, peers, epoch, expert_owner, topk_ids, *handle, dev_status,
+  return ep_layout_impl(*cfg, *grp, peers, expert_owner, topk_ids, *handle, dev_status,
                         carve_ep(*cfg, grp->capacity, (char*)ws), (cudaStream_t)stream);
 }
 
-moe_status moe_ep_dispatch(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const void* x,
+moe_status moe_ep_dispatch(const moe_config* cfg, const moe_ep_group* grp, const void* x,
                            const float* topk_w, const moe_ep_handle* handle, moe_stream_t stream) {
   EpPeers peers;
-  moe_status s = check_ep(cfg, grp, epoch, &peers);
+  moe_status s = check_ep(cfg, grp, &peers);
   if (s != MOE_OK) return s;
   if (!handle_complete(handle) || (cfg->N > 0 && (!x || !topk_w))) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
-  return cuda_status(launch_ep_dispatch(*cfg, peers, ep_offsets(*cfg, grp->capacity), grp->rank, grp->capacity,
-                                        epoch, x, handle->dest, topk_w, (cudaStream_t)stream),
+  return cuda_status(launch_ep_dispatch(*cfg, peers, ep_offsets(*cfg, grp->capacity), grp->rank, grp->capacity, x,
+                                        handle->dest, topk_w, (cudaStream_t)stream),
                      "EP dispatch");
 }
 
-moe_status moe_ep_expert_ffn(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const void* x,
+moe_status moe_ep_expert_ffn(const moe_config* cfg, const moe_ep_group* grp, const void* x,
                              const void* w13, const void* w2, const moe_ep_handle* handle, int32_t* dev_status,
                              void* ws, size_t ws_bytes, moe_stream_t stream) {
   EpPeers peers;
-  moe_status s = check_ep(cfg, grp, epoch, &peers);
+  moe_status s = check_ep(cfg, grp, &peers);
   if (s != MOE_OK) return s;
   if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes)) != MOE_OK) return s;
   const bool any = grp->local_experts > 0 || (cfg->N > 0 && cfg->n_shared > 0);
   if (!handle_complete(handle) || (any && (!w13 || !w2)) || (cfg->N > 0 && cfg->n_shared > 0 && !x))
     return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
-  return ep_ffn_impl(*cfg, *grp, peers, epoch, x, w13, w2, *handle, dev_status,
+  return ep_ffn_impl(*cfg, *grp, peers, x, w13, w2, *handle, dev_status,
                      carve_ep(*cfg, grp->capacity, (char*)ws), (cudaStream_t)stream);
 }
 
-moe_status moe_ep_combine(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const moe_ep_handle* handle,
+moe_status moe_ep_combine(const moe_config* cfg, const moe_ep_group* grp, const moe_ep_handle* handle,
                           void* y, int32_t* dev_status, moe_stream_t stream) {
   EpPeers peers;
-  moe_status s = check_ep(cfg, grp, epoch, &peers);
+  moe_status s = check_ep(cfg, grp, &peers);
   if (s != MOE_OK) return s;
   if (!handle_complete(handle) || (cfg->N > 0 && !y)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
-  return cuda_status(launch_ep_combine(*cfg, peers, ep_offsets(*cfg, grp->capacity), grp->rank, grp->capacity, epoch,
+  return cuda_status(launch_ep_combine(*cfg, peers, ep_offsets(*cfg, grp->capacity), grp->rank, grp->capacity,
                                        handle->dest, y, dev_status, (cudaStream_t)stream),
                      "EP combine");
 }
 
-moe_status moe_ep_layer_forward(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const void* x,
+moe_status moe_ep_layer_forward(const moe_config* cfg, const moe_ep_group* grp, const void* x,
                                 const void* w_gate, const float* bias, const int32_t* expert_owner, const void* w13,
                                 const void* w2, void* y, const moe_ep_handle* handle_out, int32_t* dev_status,
                                 void* ws, size_t ws_bytes, moe_stream_t stream) {
   EpPeers peers;
-  moe_status s = check_ep(cfg, grp, epoch, &peers);
+  moe_status s = check_ep(cfg, grp, &peers);
   if (s != MOE_OK) return s;
   if ((s = check_router(*cfg)) != MOE_OK) return s;
   if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
@@ -991,15 +991,15 @@ moe_status moe_ep_layer_forward(const moe_config* cfg, const moe_ep_group* grp, 
   const moe_ep_handle& hd = handle_out ? *handle_out : w.hd;
   cudaStream_t st = (cudaStream_t)stream;
   if (c.N > 0 && (s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
-  if ((s = ep_notify_impl(c, *grp, peers, epoch, w.ids, dev_status, w, st)) != MOE_OK) return s;
-  if ((s = ep_layout_impl(c, *grp, peers, epoch, expert_owner, w.ids, hd, dev_status, w, st)) != MOE_OK) return s;
-  if ((s = cuda_status(launch_ep_dispatch(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, epoch,
-                                          x, hd.dest, w.w, st),
+  if ((s = ep_notify_impl(c, *grp, peers, w.ids, dev_status, w, st)) != MOE_OK) return s;
+  if ((s = ep_layout_impl(c, *grp, peers, expert_owner, w.ids, hd, dev_status, w, st)) != MOE_OK) return s;
+  if ((s = cuda_status(launch_ep_dispatch(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, x,
+                                          hd.dest, w.w, st),
                        "EP dispatch")) != MOE_OK)
     return s;
-  if ((s = ep_ffn_impl(c, *grp, peers, epoch, x, w13, w2, hd, dev_status, w, st)) != MOE_OK) return s;
-  return cuda_status(launch_ep_combine(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, epoch, hd.dest,
-                                       y, dev_status, st),
+  if ((s = ep_ffn_impl(c, *grp, peers, x, w13, w2, hd, dev_status, w, st)) != MOE_OK) return s;
+  return cuda_status(launch_ep_combine(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, hd.dest, y,
+                                       dev_status, st),
                      "EP combine");
 }
 

@@ -5,7 +5,6 @@ this module adds is the plumbing around them:
   - windows: one device buffer per rank, mapped into every other rank's address space
     (``ipc_group``: CUDA IPC handles exchanged over a torch.distributed process group),
     or, for P ranks emulated on one device, P buffers of one process (``emulated_groups``);
-  - the epoch of each step (the same on every rank, 1, 2, 3, ...);
   - host-side checks that every rank agrees on the shapes that fix the window layout.
 
 The EP layer follows the ep_deepep explainer §2-3 (each rank is a source of tokens and
@@ -20,8 +19,9 @@ import torch
 
 from . import binding as B
 
-N_OFFSETS = 8
-OFFSET_NAMES = ["cnt_flag", "disp_flag", "done_flag", "disp_ctr", "cnt_tab", "gate", "x_recv", "out_recv"]
+N_OFFSETS = 9
+OFFSET_NAMES = ["cnt_flag", "disp_flag", "done_flag", "step", "disp_ctr", "cnt_tab", "gate", "x_recv",
+                "out_recv"]
 MAX_RANKS = 32
 
 
@@ -74,6 +74,7 @@ def window_views(cfg, capacity: int, window: torch.Tensor) -> dict:
     return dict(cnt_flag=view(o["cnt_flag"], MAX_RANKS, torch.int64),
                 disp_flag=view(o["disp_flag"], MAX_RANKS, torch.int64),
                 done_flag=view(o["done_flag"], MAX_RANKS, torch.int64),
+                step=view(o["step"], 1, torch.int64),
                 cnt_tab=view(o["cnt_tab"], P * E, torch.int32).view(P, E),
                 gate=view(o["gate"], capacity, torch.float32),
                 x_recv=window[o["x_recv"]:o["x_recv"] + capacity * d * eb].view(dt).view(capacity, d),
@@ -189,50 +190,51 @@ def ipc_group(cfg, capacity: int, window: torch.Tensor, expert_owner=None, proce
     return grp, close
 
 
-def notify(cfg, grp: Group, epoch: int, topk_ids, ws, status=None):
+def notify(cfg, grp: Group, topk_ids, ws, status=None):
+    """Starts this rank's next step (moe_ep_notify)."""
     c = B.c_config(cfg)
-    B._check(B.load().moe_ep_notify(ctypes.byref(c), ctypes.byref(grp.c), epoch, B._p(topk_ids), B._p(status),
+    B._check(B.load().moe_ep_notify(ctypes.byref(c), ctypes.byref(grp.c), B._p(topk_ids), B._p(status),
                                     B._p(ws), ws.numel(), B._stream()), "moe_ep_notify")
 
 
-def layout(cfg, grp: Group, epoch: int, topk_ids, handle: Handle, ws, expert_owner=None, status=None):
+def layout(cfg, grp: Group, topk_ids, handle: Handle, ws, expert_owner=None, status=None):
     c = B.c_config(cfg)
-    B._check(B.load().moe_ep_layout(ctypes.byref(c), ctypes.byref(grp.c), epoch, B._p(expert_owner),
+    B._check(B.load().moe_ep_layout(ctypes.byref(c), ctypes.byref(grp.c), B._p(expert_owner),
                                     B._p(topk_ids), ctypes.byref(handle.c), B._p(status), B._p(ws), ws.numel(),
                                     B._stream()), "moe_ep_layout")
     return handle
 
 
-def dispatch(cfg, grp: Group, epoch: int, x, topk_w, handle: Handle):
+def dispatch(cfg, grp: Group, x, topk_w, handle: Handle):
     c = B.c_config(cfg)
-    B._check(B.load().moe_ep_dispatch(ctypes.byref(c), ctypes.byref(grp.c), epoch, B._p(x), B._p(topk_w),
+    B._check(B.load().moe_ep_dispatch(ctypes.byref(c), ctypes.byref(grp.c), B._p(x), B._p(topk_w),
                                       ctypes.byref(handle.c), B._stream()), "moe_ep_dispatch")
 
 
-def expert_ffn(cfg, grp: Group, epoch: int, x, w13, w2, handle: Handle, ws, status=None):
+def expert_ffn(cfg, grp: Group, x, w13, w2, handle: Handle, ws, status=None):
     c = B.c_config(cfg)
-    B._check(B.load().moe_ep_expert_ffn(ctypes.byref(c), ctypes.byref(grp.c), epoch, B._p(x), B._p(w13),
+    B._check(B.load().moe_ep_expert_ffn(ctypes.byref(c), ctypes.byref(grp.c), B._p(x), B._p(w13),
                                         B._p(w2), ctypes.byref(handle.c), B._p(status), B._p(ws), ws.numel(),
                                         B._stream()), "moe_ep_expert_ffn")
 
 
-def combine(cfg, grp: Group, epoch: int, handle: Handle, y=None, status=None, device="cuda"):
+def combine(cfg, grp: Group, handle: Handle, y=None, status=None, device="cuda"):
     c = B.c_config(cfg)
     if y is None:
         y = torch.empty(cfg.N, cfg.d, dtype=B._dtype(cfg), device=device)
-    B._check(B.load().moe_ep_combine(ctypes.byref(c), ctypes.byref(grp.c), epoch, ctypes.byref(handle.c), B._p(y),
+    B._check(B.load().moe_ep_combine(ctypes.byref(c), ctypes.byref(grp.c), ctypes.byref(handle.c), B._p(y),
                                      B._p(status), B._stream()), "moe_ep_combine")
     return y
 
 
-def layer_forward(cfg, grp: Group, epoch: int, x, w_gate, bias, w13, w2, ws, expert_owner=None, y=None,
+def layer_forward(cfg, grp: Group, x, w_gate, bias, w13, w2, ws, expert_owner=None, y=None,
                   handle: Handle | None = None, status=None):
     """The layer on this rank (moe_ep_layer_forward): route, notify, layout, dispatch,
-    expert FFN, combine.  With P > 1 every rank must call it for the same epoch."""
+    expert FFN, combine.  With P > 1 every rank must run the same sequence of steps."""
     c = B.c_config(cfg)
     if y is None:
         y = torch.empty(cfg.N, cfg.d, dtype=B._dtype(cfg), device=x.device)
-    B._check(B.load().moe_ep_layer_forward(ctypes.byref(c), ctypes.byref(grp.c), epoch, B._p(x), B._p(w_gate),
+    B._check(B.load().moe_ep_layer_forward(ctypes.byref(c), ctypes.byref(grp.c), B._p(x), B._p(w_gate),
                                            B._p(bias), B._p(expert_owner), B._p(w13), B._p(w2), B._p(y),
                                            ctypes.byref(handle.c) if handle is not None else None, B._p(status),
                                            B._p(ws), ws.numel(), B._stream()), "moe_ep_layer_forward")

@@ -486,16 +486,19 @@ moe_status moe_layer_forward_fp8_overlapped(const moe_config* cfg, const void* x
  * The window.  Every rank allocates one device buffer of moe_ep_window_bytes(cfg,
  * capacity) bytes, zeroes it, and maps every other rank's window into its address space
  * (moe_ep_ipc_handle on the owner's side, moe_ep_ipc_open on the others'), all before
- * any rank's first step.  It holds the epoch flags, the count table [P, E], the gate and
+ * any rank's first step.  It holds the step flags, the count table [P, E], the gate and
  * the row of each received assignment (capacity rows) and the expert output rows
  * (capacity routed rows, then S*N shared rows).  capacity = receive rows per owner, the
  * same on every rank; at most the layer's total assignments are ever needed.  When the
  * routing sends more than capacity rows to an owner, the rows beyond it are dropped and
  * MOE_ERR_WORKSPACE is written to *dev_status on every rank.
  *
- * epoch: 1, 2, 3, ... one per layer step, the same on every rank.  Each wait compares a
- * flag with it; flags only grow, so nothing is reset between steps.  Every wait is
- * bounded (2 s); on timeout MOE_ERR_TIMEOUT is written to *dev_status and the waiting
+ * Steps: every rank counts its layer steps in its own window (moe_ep_notify's kernel
+ * increments the count; the later calls of the step read it on the device), so the
+ * step number is never a call argument and a CUDA graph that captures a step replays
+ * correctly.  Every rank must run the same sequence of steps.  Each wait compares a flag
+ * with the step number; flags only grow, so nothing is reset between steps.  Every wait
+ * is bounded (2 s); on timeout MOE_ERR_TIMEOUT is written to *dev_status and the waiting
  * kernel skips its work, so outputs of that step are undefined but no access leaves its
  * buffer.
  *
@@ -541,10 +544,10 @@ typedef struct {
 /* Bytes of one rank's window (0 on an invalid configuration). */
 size_t moe_ep_window_bytes(const moe_config* cfg, int32_t capacity);
 /* Byte offsets of the window's parts (the same on every rank; a rank's own N only sizes
- * the shared rows at the end): offsets[0..7] = count flags [32] u64, dispatch flags [32]
- * u64, done flags [32] u64 (each indexed by the signalling rank), dispatch counter u32,
- * count table [P, E] int32, gates [capacity] fp32, received rows [capacity, d], output
- * rows [capacity + S*N, d]. */
+ * the shared rows at the end): offsets[0..8] = count flags [32] u64, dispatch flags [32]
+ * u64, done flags [32] u64 (each indexed by the signalling rank), step counter u64,
+ * dispatch counter u32, count table [P, E] int32, gates [capacity] fp32, received rows
+ * [capacity, d], output rows [capacity + S*N, d]. */
 moe_status moe_ep_window_layout(const moe_config* cfg, int32_t capacity, size_t* offsets);
 /* Bytes of scratch the EP calls of one step need (ws; the same ws for all calls of a step
  * and for moe_ep_layer_forward, which also keeps the router outputs and the handle there). */
@@ -560,28 +563,25 @@ moe_status moe_ep_ipc_open(const void* handle, size_t offset, void** window);
 moe_status moe_ep_ipc_close(void* window, size_t offset);
 
 /* Step 1: local layout + count exchange.  topk_ids [N, k] (-1 = dropped). */
-moe_status moe_ep_notify(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch,
-                         const int32_t* topk_ids, int32_t* dev_status, void* ws, size_t ws_bytes,
+moe_status moe_ep_notify(const moe_config* cfg, const moe_ep_group* grp, const int32_t* topk_ids, int32_t* dev_status, void* ws, size_t ws_bytes,
                          moe_stream_t stream);
 /* Step 2: destinations.  expert_owner [E] or NULL; fills *handle. */
-moe_status moe_ep_layout(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch,
-                         const int32_t* expert_owner, const int32_t* topk_ids, const moe_ep_handle* handle,
+moe_status moe_ep_layout(const moe_config* cfg, const moe_ep_group* grp, const int32_t* expert_owner, const int32_t* topk_ids, const moe_ep_handle* handle,
                          int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream);
 /* Step 3: dispatch.  x [N, d] dtype, topk_w [N, k] fp32 (the gates FC2 applies). */
-moe_status moe_ep_dispatch(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const void* x,
+moe_status moe_ep_dispatch(const moe_config* cfg, const moe_ep_group* grp, const void* x,
                            const float* topk_w, const moe_ep_handle* handle, moe_stream_t stream);
 /* Step 4: this owner's experts.  x [N, d] (the shared experts' rows); w13 [local_experts + S,
  * 2I, d] and w2 [local_experts + S, d, I]: the owned experts in ascending id, then the
  * shared experts (the layout of moe_grouped_ffn's weights restricted to this owner). */
-moe_status moe_ep_expert_ffn(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const void* x,
+moe_status moe_ep_expert_ffn(const moe_config* cfg, const moe_ep_group* grp, const void* x,
                              const void* w13, const void* w2, const moe_ep_handle* handle, int32_t* dev_status,
                              void* ws, size_t ws_bytes, moe_stream_t stream);
 /* Step 5: combine into y [N, d] dtype, in token order. */
-moe_status moe_ep_combine(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch,
-                          const moe_ep_handle* handle, void* y, int32_t* dev_status, moe_stream_t stream);
+moe_status moe_ep_combine(const moe_config* cfg, const moe_ep_group* grp, const moe_ep_handle* handle, void* y, int32_t* dev_status, moe_stream_t stream);
 /* The layer on this rank: moe_route on its N tokens, then steps 1-5.  handle_out (NULL ok)
  * receives the EP layout instead of the workspace. */
-moe_status moe_ep_layer_forward(const moe_config* cfg, const moe_ep_group* grp, uint64_t epoch, const void* x,
+moe_status moe_ep_layer_forward(const moe_config* cfg, const moe_ep_group* grp, const void* x,
                                 const void* w_gate, const float* bias, const int32_t* expert_owner,
                                 const void* w13, const void* w2, void* y, const moe_ep_handle* handle_out,
                                 int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream);

@@ -67,7 +67,22 @@ class Emulated:
             out.append((inp["w13"].index_select(0, idx).contiguous(), inp["w2"].index_select(0, idx).contiguous()))
         return out
 
-    def step(self, inp, epoch, ids=None, w=None):
+    def launch(self, xs, ids, w, wts, ys):
+        """One EP step of every rank, stage by stage (no synchronisation: capturable)."""
+        P = self.cfg.P
+        for r in range(P):
+            ep.notify(self.rcfg[r], self.groups[r], ids[r], self.ws[r], self.status)
+        for r in range(P):
+            ep.layout(self.rcfg[r], self.groups[r], ids[r], self.handles[r], self.ws[r], self.owner, self.status)
+        for r in range(P):
+            ep.dispatch(self.rcfg[r], self.groups[r], xs[r], w[r], self.handles[r])
+        for r in range(P):
+            ep.expert_ffn(self.rcfg[r], self.groups[r], xs[r], wts[r][0], wts[r][1], self.handles[r], self.ws[r],
+                          self.status)
+        for r in range(P):
+            ep.combine(self.rcfg[r], self.groups[r], self.handles[r], y=ys[r], status=self.status)
+
+    def step(self, inp, ids=None, w=None):
         cfg, P = self.cfg, self.cfg.P
         starts = np.concatenate([[0], np.cumsum(self.shards)])
         xs = [inp["x"][starts[r]:starts[r + 1]] for r in range(P)]
@@ -75,19 +90,8 @@ class Emulated:
             routed = [moe.route(self.rcfg[r], xs[r], inp["w_gate"], inp["bias"]) for r in range(P)]
             ids = [rt[1] for rt in routed]
             w = [rt[2] for rt in routed]
-        wts = self.weights(inp)
-        for r in range(P):
-            ep.notify(self.rcfg[r], self.groups[r], epoch, ids[r], self.ws[r], self.status)
-        for r in range(P):
-            ep.layout(self.rcfg[r], self.groups[r], epoch, ids[r], self.handles[r], self.ws[r], self.owner,
-                      self.status)
-        for r in range(P):
-            ep.dispatch(self.rcfg[r], self.groups[r], epoch, xs[r], w[r], self.handles[r])
-        for r in range(P):
-            ep.expert_ffn(self.rcfg[r], self.groups[r], epoch, xs[r], wts[r][0], wts[r][1], self.handles[r],
-                          self.ws[r], self.status)
-        ys = [ep.combine(self.rcfg[r], self.groups[r], epoch, self.handles[r], status=self.status)
-              for r in range(P)]
+        ys = [torch.empty(c.N, c.d, dtype=c.torch_dtype, device="cuda") for c in self.rcfg]
+        self.launch(xs, ids, w, self.weights(inp), ys)
         torch.cuda.synchronize()
         return dict(xs=xs, ids=ids, w=w, y=torch.cat(ys))
 
@@ -133,7 +137,7 @@ def test_ep_step_matches_oracle(cfg, spec):
     inp = gpu_inputs(cfg)
     owner = _owner(cfg, spec)
     em = Emulated(cfg, _shards(cfg, spec), owner)
-    res = em.step(inp, epoch=1)
+    res = em.step(inp)
     assert int(em.status.item()) == 0
     own_np = owner.cpu().numpy() if owner is not None else None
     lay = O.ep_layout([i.cpu().numpy() for i in res["ids"]], cfg.E, cfg.P, own_np, em.capacity)
@@ -153,7 +157,7 @@ def test_ep_epochs_reuse_windows():
     em = Emulated(cfg, _shards(cfg, None))
     for epoch in (1, 2, 3):
         inp = gpu_inputs(cfg, seed_offset=epoch)
-        res = em.step(inp, epoch=epoch)
+        res = em.step(inp)
         assert int(em.status.item()) == 0
         y1 = moe.layer_forward(cfg, inp["x"], inp["w_gate"], inp["bias"], None, inp["w13"], inp["w2"])
         torch.cuda.synchronize()
@@ -162,6 +166,7 @@ def test_ep_epochs_reuse_windows():
         assert flags["cnt_flag"][:cfg.P].tolist() == [epoch] * cfg.P
         assert flags["disp_flag"][:cfg.P].tolist() == [epoch] * cfg.P
         assert flags["done_flag"][:cfg.P].tolist() == [epoch] * cfg.P
+        assert flags["step"].tolist() == [epoch]
 
 
 def test_ep_capacity_overflow_drops_rows_in_bounds():
@@ -171,7 +176,7 @@ def test_ep_capacity_overflow_drops_rows_in_bounds():
     inp = gpu_inputs(cfg)
     rcfg = cfg.replace(N=cfg.N // cfg.P)
     probe = Emulated(cfg, _shards(cfg, None))
-    res0 = probe.step(inp, epoch=1)
+    res0 = probe.step(inp)
     lay_full = O.ep_layout([i.cpu().numpy() for i in res0["ids"]], cfg.E, cfg.P)
     cap = int(lay_full["R"].max()) - 7
     em = Emulated(cfg, _shards(cfg, None), capacity=cap)
@@ -182,7 +187,7 @@ def test_ep_capacity_overflow_drops_rows_in_bounds():
         r[G:G + nbytes].zero_()
     em.windows = [r[G:G + nbytes] for r in raws]
     em.groups = [ep.Group(r, cap, len(em.owned[r]), [w.data_ptr() for w in em.windows]) for r in range(cfg.P)]
-    res = em.step(inp, epoch=1, ids=res0["ids"], w=res0["w"])
+    res = em.step(inp, ids=res0["ids"], w=res0["w"])
     assert int(em.status.item()) == moe.binding.MOE_ERR_WORKSPACE
     lay = O.ep_layout([i.cpu().numpy() for i in res["ids"]], cfg.E, cfg.P, None, cap)
     check_handles(em, lay)
@@ -201,7 +206,7 @@ def test_ep_dropped_assignments():
               for r in range(cfg.P)]
     ids = [moe.capacity_drop(cfg.replace(N=n), rt[1], 20) for rt in routed]
     w = [rt[2] for rt in routed]
-    res = em.step(inp, epoch=1, ids=ids, w=w)
+    res = em.step(inp, ids=ids, w=w)
     assert int(em.status.item()) == 0
     lay = O.ep_layout([i.cpu().numpy() for i in ids], cfg.E, cfg.P, None, em.capacity)
     assert any((i.cpu().numpy() == -1).any() for i in ids)
@@ -229,7 +234,7 @@ def test_ep_one_rank_layer_forward_matches_one_gpu_layer():
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     h = ep.Handle(cfg, cfg.E)
     for epoch in (1, 2):
-        y = ep.layer_forward(cfg, groups[0], epoch, inp["x"], inp["w_gate"], inp["bias"], inp["w13"], inp["w2"], ws,
+        y = ep.layer_forward(cfg, groups[0], inp["x"], inp["w_gate"], inp["bias"], inp["w13"], inp["w2"], ws,
                              handle=h, status=status)
         y1 = moe.layer_forward(cfg, inp["x"], inp["w_gate"], inp["bias"], None, inp["w13"], inp["w2"])
         torch.cuda.synchronize()
@@ -238,15 +243,17 @@ def test_ep_one_rank_layer_forward_matches_one_gpu_layer():
 
 
 def test_ep_wait_times_out_and_context_stays_usable():
-    """A layout for an epoch no rank has published: the bounded wait gives up (2 s),
-    MOE_ERR_TIMEOUT is reported, no destination is written, and the context still runs."""
+    """Rank 0 starts a second step that no other rank starts: its layout's bounded wait for
+    the count rows gives up (2 s), MOE_ERR_TIMEOUT is reported, no destination is written,
+    and the context still runs."""
     cfg, _ = CASES[0]
     inp = gpu_inputs(cfg)
     em = Emulated(cfg, _shards(cfg, None))
-    res = em.step(inp, epoch=1)
+    res = em.step(inp)
     assert int(em.status.item()) == 0
     rc = em.rcfg[0]
-    ep.layout(rc, em.groups[0], 2, res["ids"][0], em.handles[0], em.ws[0], None, em.status)
+    ep.notify(rc, em.groups[0], res["ids"][0], em.ws[0], em.status)
+    ep.layout(rc, em.groups[0], res["ids"][0], em.handles[0], em.ws[0], None, em.status)
     torch.cuda.synchronize()
     assert int(em.status.item()) == moe.binding.MOE_ERR_TIMEOUT
     assert bool((em.handles[0].as_dict()["dest"] == -1).all())
@@ -259,13 +266,56 @@ def test_ep_host_errors():
     rc = cfg.replace(N=cfg.N // cfg.P)
     em = Emulated(cfg, _shards(cfg, None))
     ids = torch.zeros(rc.N, rc.k, dtype=torch.int32, device="cuda")
-    with pytest.raises(moe.MoEError):   # epoch 0
-        ep.notify(rc, em.groups[0], 0, ids, em.ws[0])
     with pytest.raises(moe.MoEError):   # rank outside [0, P)
-        ep.notify(rc, ep.Group(cfg.P, em.capacity, 4, em.groups[0].windows), 1, ids, em.ws[0])
+        ep.notify(rc, ep.Group(cfg.P, em.capacity, 4, em.groups[0].windows), ids, em.ws[0])
+    with pytest.raises(moe.MoEError):   # capacity 0
+        ep.notify(rc, ep.Group(0, 0, 4, em.groups[0].windows), ids, em.ws[0])
     with pytest.raises(moe.MoEError):   # small workspace
-        ep.notify(rc, em.groups[0], 1, ids, em.ws[0][:16])
+        ep.notify(rc, em.groups[0], ids, em.ws[0][:16])
     with pytest.raises(moe.MoEError):   # unaligned window
         bad = list(em.groups[0].windows)
         bad[1] += 16
-        ep.notify(rc, ep.Group(0, em.capacity, 4, bad), 1, ids, em.ws[0])
+        ep.notify(rc, ep.Group(0, em.capacity, 4, bad), ids, em.ws[0])
+    assert int(em.groups[0].windows[0]) and all(ep.window_views(rc, em.capacity, w)["step"].item() == 0
+                                                 for w in em.windows), "a refused call launched nothing"
+
+
+def test_ep_step_captured_in_cuda_graph():
+    """The emulated step of all ranks captured once and replayed with new inputs: the step
+    number lives in the windows, so each replay is a new step with correct waits."""
+    cfg, _ = CASES[0]
+    em = Emulated(cfg, _shards(cfg, None))
+    P, n = cfg.P, cfg.N // cfg.P
+    inp = gpu_inputs(cfg)
+    x = inp["x"].clone()
+    xs = [x[r * n:(r + 1) * n] for r in range(P)]
+    routed = [moe.route(em.rcfg[r], xs[r], inp["w_gate"], inp["bias"]) for r in range(P)]
+    ids, w = [rt[1] for rt in routed], [rt[2] for rt in routed]
+    wts = em.weights(inp)
+    ys = [torch.empty(n, cfg.d, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
+
+    def body():
+        for r in range(P):
+            moe.route(em.rcfg[r], xs[r], inp["w_gate"], inp["bias"], out=routed[r])
+        em.launch(xs, ids, w, wts, ys)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        body()  # eager step 1
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        body()
+    for rep in range(3):
+        new = gpu_inputs(cfg, seed_offset=10 + rep)["x"]
+        x.copy_(new)
+        g.replay()
+        torch.cuda.synchronize()
+        assert int(em.status.item()) == 0
+        y1 = moe.layer_forward(cfg, new, inp["w_gate"], inp["bias"], None, inp["w13"], inp["w2"])
+        torch.cuda.synchronize()
+        assert torch.equal(torch.cat(ys), y1), f"replay {rep}"
+    steps = [int(ep.window_views(em.rcfg[r], em.capacity, em.windows[r])["step"].item()) for r in range(P)]
+    assert steps == [4] * P   # one eager step + three replays (the capture itself launches nothing)
