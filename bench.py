@@ -367,16 +367,26 @@ def run_ep(args, cfg, local):
     n = cfg.N // P
     rc = gcfg.replace(N=n)
     cap = 2 * -(-cfg.N * cfg.k // P)          # receive rows per owner: twice the mean load
+    f8 = bool(args.fp8)
     groups, windows = ep.emulated_groups(rc, cap)
-    ws = [ep.alloc_ws(rc, cap) for _ in range(P)]
+    ws = [ep.alloc_ws(rc, cap, fp8=f8) for _ in range(P)]
     handles = [ep.Handle(rc, cfg.E // P) for _ in range(P)]
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     E, S = cfg.E, cfg.S
     wts = []
+    if f8:  # weights quantised once (a load-time step), then sliced per owner
+        w13_q, w13_s = moe.quantize_fp8(inp["w13"])
+        w2_q, w2_s = moe.quantize_fp8(inp["w2"])
+        del inp["w13"], inp["w2"]
     for r in range(P):
         idx = torch.tensor(list(range(r * E // P, (r + 1) * E // P)) + list(range(E, E + S)), device=dev)
-        wts.append((inp["w13"].index_select(0, idx), inp["w2"].index_select(0, idx)))
+        if f8:
+            wts.append(tuple(t.index_select(0, idx) for t in (w13_q, w13_s, w2_q, w2_s)))
+        else:
+            wts.append((inp["w13"].index_select(0, idx), inp["w2"].index_select(0, idx)))
     xs = [inp["x"][r * n:(r + 1) * n] for r in range(P)]
+    qs = [(torch.empty(n, cfg.d, dtype=torch.uint8, device=dev), torch.empty(n, dtype=torch.float32, device=dev))
+          for _ in range(P)] if f8 else None
     routed = [moe.route(rc, xs[r], inp["w_gate"], inp["bias"]) for r in range(P)]
     ys = [torch.empty(n, cfg.d, dtype=cfg.torch_dtype, device=dev) for _ in range(P)]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -389,6 +399,8 @@ def run_ep(args, cfg, local):
         mark(0)
         for r in range(P):
             moe.route(rc, xs[r], inp["w_gate"], inp["bias"], out=routed[r])
+            if f8:
+                moe.quantize_fp8(xs[r], out=qs[r][0], scale=qs[r][1])
         mark(1)
         for r in range(P):
             ep.notify(rc, groups[r], routed[r][1], ws[r], status)
@@ -397,10 +409,16 @@ def run_ep(args, cfg, local):
             ep.layout(rc, groups[r], routed[r][1], handles[r], ws[r], None, status)
         mark(3)
         for r in range(P):
-            ep.dispatch(rc, groups[r], xs[r], routed[r][2], handles[r])
+            if f8:
+                ep.dispatch_fp8(rc, groups[r], qs[r][0], qs[r][1], routed[r][2], handles[r])
+            else:
+                ep.dispatch(rc, groups[r], xs[r], routed[r][2], handles[r])
         mark(4)
         for r in range(P):
-            ep.expert_ffn(rc, groups[r], xs[r], wts[r][0], wts[r][1], handles[r], ws[r], status)
+            if f8:
+                ep.expert_ffn_fp8(rc, groups[r], qs[r][0], qs[r][1], *wts[r], handles[r], ws[r], status)
+            else:
+                ep.expert_ffn(rc, groups[r], xs[r], wts[r][0], wts[r][1], handles[r], ws[r], status)
         mark(5)
         for r in range(P):
             ep.combine(rc, groups[r], handles[r], y=ys[r], status=status)
@@ -439,14 +457,25 @@ def run_ep(args, cfg, local):
     if int(status.item()) != 0:
         raise SystemExit(f"EP step reported status {int(status.item())}")
     # the one-GPU layer on the same batch (same experts, one owner per E/P block)
-    ws1 = moe.alloc_workspace(gcfg, dev)
-    y1 = moe.layer_forward(gcfg, inp["x"], inp["w_gate"], inp["bias"], None, inp["w13"], inp["w2"], ws=ws1)
+    if f8:
+        ws1 = torch.empty(moe.workspace_bytes_fp8(gcfg), dtype=torch.uint8, device=dev)
+
+        def one_gpu(y=None):
+            return moe.layer_forward_fp8(gcfg, inp["x"], inp["w_gate"], inp["bias"], None, w13_q, w13_s, w2_q, w2_s,
+                                         y=y, ws=ws1)
+    else:
+        ws1 = moe.alloc_workspace(gcfg, dev)
+
+        def one_gpu(y=None):
+            return moe.layer_forward(gcfg, inp["x"], inp["w_gate"], inp["bias"], None, inp["w13"], inp["w2"], y=y,
+                                     ws=ws1)
+    y1 = one_gpu()
     one = []
     for _ in range(args.steps):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        moe.layer_forward(gcfg, inp["x"], inp["w_gate"], inp["bias"], None, inp["w13"], inp["w2"], y=y1, ws=ws1)
+        one_gpu(y1)
         b.record()
         torch.cuda.synchronize()
         one.append(a.elapsed_time(b))
@@ -458,27 +487,34 @@ def run_ep(args, cfg, local):
         dest = handles[r].as_dict()["dest"]
         owner = torch.div(dest[dest >= 0], cap, rounding_mode="floor")
         cross.append(int((owner != r).sum().item()))
-    row_bytes = cfg.d * eb
-    max_cross = max(cross) * row_bytes
+    row_bytes = cfg.d * eb                      # output rows (combine) and bf16 payload rows
+    pay_bytes = cfg.d * (1 if f8 else eb)       # dispatch payload rows (e4m3: d bytes)
+    max_cross = max(cross) * pay_bytes
     med = sorted(step_ms)[len(step_ms) // 2]
     stage_ms = {k: tot[i] / args.steps for i, k in enumerate(stages)}
     x_bytes, rows_bytes = cfg.N * row_bytes, cfg.N * cfg.k * row_bytes
+    pay_x, pay_rows = cfg.N * pay_bytes, cfg.N * cfg.k * pay_bytes
     print(json.dumps({
-        "metric": "MoE-layer tokens/s, expert-parallel path with P ranks emulated on one GPU",
+        "metric": "MoE-layer tokens/s, expert-parallel path with P ranks emulated on one GPU"
+                  + (" (FP8 dispatch and experts, bf16 combine)" if f8 else ""),
         "value": cfg.N / (med / 1e3), "unit": "tokens/s", "n_gpus": 1, "ep_ranks_emulated": P,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": med, "dtype": cfg.dtype,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": med,
+        "dtype": "e4m3 (scaled), bf16 out" if f8 else cfg.dtype,
         "config": {"workload": describe(gcfg), "tokens_per_rank": n, "capacity_rows_per_owner": cap,
                    "l2": "flushed before every step"},
         "how": "ms_per_step: the emulated step of all P ranks as one CUDA graph replay; stages: eager launches "
                "with events between the stages (all ranks of a stage together)",
         "stages_ms_all_ranks": stage_ms,
-        "dispatch_gbs_local": (x_bytes + rows_bytes) / (stage_ms["dispatch"] / 1e3) / 1e9,
+        "dispatch_gbs_local": (pay_x + pay_rows) / (stage_ms["dispatch"] / 1e3) / 1e9,
         "combine_gbs_local": (rows_bytes + S * x_bytes + x_bytes) / (stage_ms["combine"] / 1e3) / 1e9,
         "one_gpu_layer_ms": sorted(one)[len(one) // 2],
         "y_bit_identical_to_one_gpu_layer": same,
-        "nvlink": {"cross_rows_per_rank": cross, "max_bytes_per_rank_per_direction": max_cross,
-                   "roofline_us_at_770_gbs": max_cross / 770e9 * 1e6,
-                   "note": "bytes a real P-GPU step moves over NVLink each way; not measured here (one GPU)"},
+        "nvlink": {"cross_rows_per_rank": cross, "dispatch_bytes_per_rank": max_cross,
+                   "combine_bytes_per_rank": max(cross) * row_bytes,
+                   "roofline_us_at_770_gbs": (max_cross + max(cross) * row_bytes) / 770e9 * 1e6,
+                   "note": "bytes a real P-GPU step sends from (and receives into) each GPU in the dispatch and "
+                           "in the combine; the roofline time is their sum at the measured 770 GB/s peer copy; "
+                           "not measured here (one GPU)"},
         "status": int(status.item()),
     }), flush=True)
 

@@ -34,7 +34,8 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_con
             "moe_workspace_bytes_fp8", "moe_layer_forward_fp8", "moe_capacity_drop",
             "moe_layer_forward_fp8_overlapped", "moe_ep_window_bytes", "moe_ep_window_layout",
             "moe_ep_workspace_bytes", "moe_ep_ipc_handle", "moe_ep_ipc_open", "moe_ep_ipc_close", "moe_ep_notify",
-            "moe_ep_layout", "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ep_layer_forward"]
+            "moe_ep_layout", "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ep_layer_forward",
+            "moe_ep_workspace_bytes_fp8", "moe_ep_dispatch_fp8", "moe_ep_expert_ffn_fp8", "moe_ep_layer_forward_fp8"]
 
 
 class CConfig(ctypes.Structure):
@@ -128,6 +129,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_ep_expert_ffn": (i32, [cfgp, grpp, vp, vp, vp, hdp, vp, vp, sz, vp]),
         "moe_ep_combine": (i32, [cfgp, grpp, hdp, vp, vp, vp]),
         "moe_ep_layer_forward": (i32, [cfgp, grpp, vp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz, vp]),
+        "moe_ep_workspace_bytes_fp8": (sz, [cfgp, i32]),
+        "moe_ep_dispatch_fp8": (i32, [cfgp, grpp, vp, vp, vp, hdp, vp]),
+        "moe_ep_expert_ffn_fp8": (i32, [cfgp, grpp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz, vp]),
+        "moe_ep_layer_forward_fp8": (i32, [cfgp, grpp, vp, vp, vp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz, vp]),
     })
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

@@ -200,11 +200,13 @@ __device__ __forceinline__ uint4 ld_nc(const uint4* p) {
 }
 
 // Each token row of x is read once and stored into the receive rows of the owners of its
-// k experts; the gate of each assignment goes beside its row.  Grid-stride over tokens.
+// k experts; the gate of each assignment (and, for an FP8 payload, the token's scale)
+// goes beside its row.  Grid-stride over tokens.
 __global__ void __launch_bounds__(kEpWarps * 32) ep_dispatch_kernel(const __grid_constant__ EpPeers peers,
                                                                      EpOffsets off, const uint4* __restrict__ x,
                                                                      const int32_t* __restrict__ dest,
-                                                                     const float* __restrict__ topk_w, int N,
+                                                                     const float* __restrict__ topk_w,
+                                                                     const float* __restrict__ x_scale, int N,
                                                                      int k, int vpr, int capacity, int P,
                                                                      int me) {
   const int lane = threadIdx.x & 31;
@@ -213,6 +215,7 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_dispatch_kernel(const __grid
     if (my >= 0) {
       const int o = my / capacity;
       at<float>(peers.base[o], off.gate)[my - o * capacity] = topk_w[(size_t)t * k + lane];
+      if (x_scale) at<float>(peers.base[o], off.scale)[my - o * capacity] = x_scale[t];
     }
     uint4* rows[kMaxK];
 #pragma unroll
@@ -371,7 +374,8 @@ EpOffsets ep_offsets(const moe_config& c, int capacity) {
   o.disp_ctr = o.step + sizeof(uint64_t);
   o.cnt_tab = al256(o.disp_ctr + sizeof(uint32_t));
   o.gate = al256(o.cnt_tab + (size_t)c.P * c.E * sizeof(int32_t));
-  o.x_recv = al256(o.gate + (size_t)capacity * sizeof(float));
+  o.scale = al256(o.gate + (size_t)capacity * sizeof(float));
+  o.x_recv = al256(o.scale + (size_t)capacity * sizeof(float));
   o.out_recv = al256(o.x_recv + (size_t)capacity * c.d * eb);
   o.total = al256(o.out_recv + ((size_t)capacity + (size_t)c.n_shared * c.N) * c.d * eb);
   return o;
@@ -417,10 +421,9 @@ cudaError_t launch_ep_layout(const moe_config& c, const EpPeers& peers, const Ep
 
 cudaError_t launch_ep_dispatch(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me,
                                int capacity, const void* x, const int32_t* dest, const float* topk_w,
-                               cudaStream_t st) {
-  const int vpr = c.d * (c.dtype == MOE_BF16 ? 2 : 4) / 16;
+                               const float* x_scale, int row_bytes, cudaStream_t st) {
   ep_dispatch_kernel<<<ep_grid(c.N, kEpWarps), kEpWarps * 32, 0, st>>>(
-      peers, off, static_cast<const uint4*>(x), dest, topk_w, c.N, c.k, vpr, capacity, c.P, me);
+      peers, off, static_cast<const uint4*>(x), dest, topk_w, x_scale, c.N, c.k, row_bytes / 16, capacity, c.P, me);
   return cudaGetLastError();
 }
 

@@ -343,10 +343,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float* sb = nullptr;
         if (F8) {
           const int gz = p.g0 + td.g;
-          // token of the row: routed rows through row2tok; a shared expert's rows are the
-          // tokens in order, after A_routed and the earlier shared experts' blocks
+          // token of the row: routed rows through row2tok (or their own scale in
+          // a_scale_rows); a shared expert's rows are the tokens in order, after A_routed
+          // and the earlier shared experts' blocks
           if (row_ok)
-            ra = p.a_scale[gz < p.E ? p.row2tok[orow] / p.k : (int)(orow - p.A_routed - (long long)(gz - p.E) * p.N)];
+            ra = gz < p.E ? (p.a_scale_rows ? p.a_scale_rows[orow] : p.a_scale[p.row2tok[orow] / p.k])
+                          : p.a_scale[(int)(orow - p.A_routed - (long long)(gz - p.E) * p.N)];
           sb = p.b_scale + (size_t)gz * p.b_rows;
         }
 #pragma unroll 1

@@ -78,6 +78,7 @@ struct GemmArgs {
   int k;                // top-k (FC1: routed row -> token = row2tok / k)
   const float* a_scale; // FC1: per token [N]; FC2: per h row [A + S*N]
   const float* b_scale; // per weight row [groups, b_rows]
+  const float* a_scale_rows;  // FC1: when set, routed row r's scale is a_scale_rows[r] (no row map)
 };
 
 // Rows a launch covers, for grid sizing: routed rows if any routed group is in range,
@@ -119,6 +120,7 @@ struct EpOffsets {
   size_t disp_ctr;                        // u32: this rank's dispatch CTAs finished in the running launch
   size_t cnt_tab;                         // [P, E] int32: row i = source i's expert counts
   size_t gate;                            // [capacity] fp32: gate of each received row
+  size_t scale;                           // [capacity] fp32: FP8 dispatch: token scale of each received row
   size_t x_recv;                          // [capacity, d]: received rows, expert-major
   size_t out_recv;                        // [capacity + S*N, d]: FC2 rows (routed, then shared)
   size_t total;
@@ -132,9 +134,11 @@ cudaError_t launch_ep_push_counts(const EpPeers& peers, const EpOffsets& off, co
 cudaError_t launch_ep_layout(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me, int capacity,
                              int local_experts, const int32_t* owner, const int32_t* ids, const moe_layout& loc,
                              int32_t* dest, int32_t* own_n_e, int32_t* own_off, int* status, cudaStream_t st);
+// rows of row_bytes bytes (d * elem for bf16 / fp32, d for e4m3 codes); x_scale (FP8): each
+// token's scale, stored beside each of its received rows (NULL: none)
 cudaError_t launch_ep_dispatch(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me,
                                int capacity, const void* x, const int32_t* dest, const float* topk_w,
-                               cudaStream_t st);
+                               const float* x_scale, int row_bytes, cudaStream_t st);
 cudaError_t launch_ep_wait(const char* own, const EpOffsets& off, size_t flag_off, int n, int* status,
                            cudaStream_t st);
 cudaError_t launch_ep_signal(const EpPeers& peers, const EpOffsets& off, size_t flag_off, int P, int me,

@@ -315,6 +315,11 @@ struct EpWs {
   int32_t* ids;
   float* w;
   moe_ep_handle hd;
+  // FP8 only
+  void* h_q;        // [capacity + S*N, I] e4m3
+  float* h_scale;   // [capacity + S*N]
+  void* x_q;        // [N, d] e4m3 (moe_ep_layer_forward_fp8)
+  float* x_scale;   // [N]
   size_t total;
 };
 
@@ -324,7 +329,7 @@ moe_config one_owner(const moe_config& c) {
   return c1;
 }
 
-EpWs carve_ep(const moe_config& c, int capacity, char* base) {
+EpWs carve_ep(const moe_config& c, int capacity, char* base, bool fp8 = false) {
   EpWs w;
   memset(&w, 0, sizeof(w));
   const size_t A = (size_t)c.N * c.k, E = c.E, S = c.n_shared, eb = elem_bytes(c);
@@ -354,6 +359,13 @@ EpWs carve_ep(const moe_config& c, int capacity, char* base) {
   w.hd.dest = i32(A);
   w.hd.owner_n_e = i32(E);
   w.hd.owner_off = i32(E + 1);
+  if (fp8) {
+    const size_t rows = (size_t)capacity + S * c.N;
+    w.h_q = take(rows * c.I);
+    w.h_scale = reinterpret_cast<float*>(take(rows * 4));
+    w.x_q = take((size_t)c.N * c.d);
+    w.x_scale = reinterpret_cast<float*>(take((size_t)c.N * 4));
+  }
   w.total = off;
   return w;
 }
@@ -377,8 +389,9 @@ moe_status check_ep(const moe_config* cfg, const moe_ep_group* g, EpPeers* peers
   return MOE_OK;
 }
 
-moe_status check_ep_ws(const moe_config& c, const moe_ep_group* g, void* ws, size_t ws_bytes) {
-  if (!ws || ws_bytes < carve_ep(c, g->capacity, nullptr).total) return fail(MOE_ERR_WORKSPACE, "EP workspace too small");
+moe_status check_ep_ws(const moe_config& c, const moe_ep_group* g, void* ws, size_t ws_bytes, bool fp8 = false) {
+  if (!ws || ws_bytes < carve_ep(c, g->capacity, nullptr, fp8).total)
+    return fail(MOE_ERR_WORKSPACE, "EP workspace too small");
   if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return fail(MOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
   return MOE_OK;
 }
@@ -434,6 +447,61 @@ moe_status ep_ffn_impl(const moe_config& c, const moe_ep_group& g, const EpPeers
     g2.A_routed = g.capacity;
     e = c.dtype == MOE_BF16 ? tc_grouped(g2, dec, g.capacity + S * c.N, 0, st) : launch_simt_gemm(g2, st);
     if (e != cudaSuccess) return cuda_status(e, "EP FC2 grouped GEMM");
+  }
+  return cuda_status(launch_ep_signal(peers, off, off.done_flag, c.P, g.rank, st), "FFN done signal");
+}
+
+// The owner's FP8 expert FFN: FC1 on the received e4m3 rows (each row's token scale
+// received beside it) and on the rank's own e4m3 token rows for the shared experts,
+// per-row quantisation of h, FC2 on e4m3 h; outputs bf16 into the window.
+struct EpFp8 {
+  const void* x_q;
+  const float* x_scale;
+  const void* w13_q;
+  const float* w13_scale;
+  const void* w2_q;
+  const float* w2_scale;
+};
+
+moe_status ep_ffn_fp8_impl(const moe_config& c, const moe_ep_group& g, const EpPeers& peers, const EpFp8& f,
+                           const moe_ep_handle& hd, int32_t* status, const EpWs& w, cudaStream_t st) {
+  const EpOffsets off = ep_offsets(c, g.capacity);
+  char* win = peers.base[g.rank];
+  cudaError_t e = launch_ep_wait(win, off, off.disp_flag, c.P, status, st);
+  if (e != cudaSuccess) return cuda_status(e, "dispatch wait");
+  moe_config co = c;
+  co.E = g.local_experts;
+  moe_layout L;
+  memset(&L, 0, sizeof(L));
+  L.n_e = hd.owner_n_e;
+  L.expert_off = hd.owner_off;
+  const int S = c.N > 0 ? c.n_shared : 0;
+  const int G = g.local_experts + S;
+  moe_config dec = c;
+  dec.N = g.capacity > c.N ? g.capacity : c.N;
+  if (G > 0) {
+    GemmArgs g1 = fc1_args(co, L, win + off.x_recv, S > 0 ? f.x_q : nullptr, f.w13_q, w.h);
+    g1.G = G;
+    g1.A_routed = g.capacity;
+    g1.fp8 = 1;
+    g1.k = c.k;
+    g1.a_scale = f.x_scale;
+    g1.a_scale_rows = reinterpret_cast<const float*>(win + off.scale);
+    g1.b_scale = f.w13_scale;
+    e = tc_grouped(g1, dec, g.capacity, c.N, st);
+    if (e != cudaSuccess) return cuda_status(e, "EP FC1 grouped GEMM (fp8)");
+    const long long rows = (long long)g.capacity + (long long)S * c.N;
+    e = launch_quantize_rows(w.h, rows, c.I, w.h_q, w.h_scale, st);
+    if (e != cudaSuccess) return cuda_status(e, "h quantisation");
+    GemmArgs g2 = fc2_args(co, L, w.h_q, f.w2_q, reinterpret_cast<const float*>(win + off.gate), win + off.out_recv);
+    g2.G = G;
+    g2.A_routed = g.capacity;
+    g2.fp8 = 1;
+    g2.k = c.k;
+    g2.a_scale = w.h_scale;
+    g2.b_scale = f.w2_scale;
+    e = tc_grouped(g2, dec, (int)rows, 0, st);
+    if (e != cudaSuccess) return cuda_status(e, "EP FC2 grouped GEMM (fp8)");
   }
   return cuda_status(launch_ep_signal(peers, off, off.done_flag, c.P, g.rank, st), "FFN done signal");
 }
@@ -869,8 +937,8 @@ moe_status moe_ep_window_layout(const moe_config* cfg, int32_t capacity, size_t*
   if (s != MOE_OK) return s;
   if (capacity < 1 || !offsets) return fail(MOE_ERR_INVALID_ARG, "capacity < 1 or NULL offsets");
   const EpOffsets o = ep_offsets(*cfg, capacity);
-  const size_t v[9] = {o.cnt_flag, o.disp_flag, o.done_flag, o.step, o.disp_ctr, o.cnt_tab, o.gate, o.x_recv,
-                       o.out_recv};
+  const size_t v[10] = {o.cnt_flag, o.disp_flag, o.done_flag, o.step,   o.disp_ctr,
+                        o.cnt_tab,  o.gate,      o.scale,     o.x_recv, o.out_recv};
   memcpy(offsets, v, sizeof(v));
   return MOE_OK;
 }
@@ -944,7 +1012,8 @@ moe_status moe_ep_dispatch(const moe_config* cfg, const moe_ep_group* grp, const
   if (s != MOE_OK) return s;
   if (!handle_complete(handle) || (cfg->N > 0 && (!x || !topk_w))) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
   return cuda_status(launch_ep_dispatch(*cfg, peers, ep_offsets(*cfg, grp->capacity), grp->rank, grp->capacity, x,
-                                        handle->dest, topk_w, (cudaStream_t)stream),
+                                        handle->dest, topk_w, nullptr, cfg->d * elem_bytes(*cfg),
+                                        (cudaStream_t)stream),
                      "EP dispatch");
 }
 
@@ -994,10 +1063,84 @@ moe_status moe_ep_layer_forward(const moe_config* cfg, const moe_ep_group* grp, 
   if ((s = ep_notify_impl(c, *grp, peers, w.ids, dev_status, w, st)) != MOE_OK) return s;
   if ((s = ep_layout_impl(c, *grp, peers, expert_owner, w.ids, hd, dev_status, w, st)) != MOE_OK) return s;
   if ((s = cuda_status(launch_ep_dispatch(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, x,
-                                          hd.dest, w.w, st),
+                                          hd.dest, w.w, nullptr, c.d * elem_bytes(c), st),
                        "EP dispatch")) != MOE_OK)
     return s;
   if ((s = ep_ffn_impl(c, *grp, peers, x, w13, w2, hd, dev_status, w, st)) != MOE_OK) return s;
+  return cuda_status(launch_ep_combine(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, hd.dest, y,
+                                       dev_status, st),
+                     "EP combine");
+}
+
+size_t moe_ep_workspace_bytes_fp8(const moe_config* cfg, int32_t capacity) {
+  if (check_fp8(cfg) != MOE_OK || capacity < 1) return 0;
+  return carve_ep(*cfg, capacity, nullptr, true).total;
+}
+
+moe_status moe_ep_dispatch_fp8(const moe_config* cfg, const moe_ep_group* grp, const void* x_q, const float* x_scale,
+                               const float* topk_w, const moe_ep_handle* handle, moe_stream_t stream) {
+  moe_status s = check_fp8(cfg);
+  if (s != MOE_OK) return s;
+  EpPeers peers;
+  if ((s = check_ep(cfg, grp, &peers)) != MOE_OK) return s;
+  if (!handle_complete(handle) || (cfg->N > 0 && (!x_q || !x_scale || !topk_w)))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return cuda_status(launch_ep_dispatch(*cfg, peers, ep_offsets(*cfg, grp->capacity), grp->rank, grp->capacity, x_q,
+                                        handle->dest, topk_w, x_scale, cfg->d, (cudaStream_t)stream),
+                     "EP dispatch (fp8)");
+}
+
+moe_status moe_ep_expert_ffn_fp8(const moe_config* cfg, const moe_ep_group* grp, const void* x_q, const float* x_scale,
+                                 const void* w13_q, const float* w13_scale, const void* w2_q, const float* w2_scale,
+                                 const moe_ep_handle* handle, int32_t* dev_status, void* ws, size_t ws_bytes,
+                                 moe_stream_t stream) {
+  moe_status s = check_fp8(cfg);
+  if (s != MOE_OK) return s;
+  EpPeers peers;
+  if ((s = check_ep(cfg, grp, &peers)) != MOE_OK) return s;
+  if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes, true)) != MOE_OK) return s;
+  const bool any = grp->local_experts > 0 || (cfg->N > 0 && cfg->n_shared > 0);
+  if (!handle_complete(handle) || (any && (!w13_q || !w13_scale || !w2_q || !w2_scale)) ||
+      (cfg->N > 0 && cfg->n_shared > 0 && (!x_q || !x_scale)))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  const EpFp8 f = {x_q, x_scale, w13_q, w13_scale, w2_q, w2_scale};
+  return ep_ffn_fp8_impl(*cfg, *grp, peers, f, *handle, dev_status, carve_ep(*cfg, grp->capacity, (char*)ws, true),
+                         (cudaStream_t)stream);
+}
+
+moe_status moe_ep_layer_forward_fp8(const moe_config* cfg, const moe_ep_group* grp, const void* x, const void* w_gate,
+                                    const float* bias, const int32_t* expert_owner, const void* w13_q,
+                                    const float* w13_scale, const void* w2_q, const float* w2_scale, void* y,
+                                    const moe_ep_handle* handle_out, int32_t* dev_status, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream) {
+  moe_status s = check_fp8(cfg);
+  if (s != MOE_OK) return s;
+  EpPeers peers;
+  if ((s = check_ep(cfg, grp, &peers)) != MOE_OK) return s;
+  if ((s = check_router(*cfg)) != MOE_OK) return s;
+  if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
+  if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes, true)) != MOE_OK) return s;
+  if (handle_out && !handle_complete(handle_out)) return fail(MOE_ERR_INVALID_ARG, "incomplete handle_out");
+  const moe_config& c = *cfg;
+  const bool any = grp->local_experts > 0 || (c.N > 0 && c.n_shared > 0);
+  if ((c.N > 0 && (!x || !w_gate || !y)) || (any && (!w13_q || !w13_scale || !w2_q || !w2_scale)))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  const EpWs w = carve_ep(c, grp->capacity, static_cast<char*>(ws), true);
+  const moe_ep_handle& hd = handle_out ? *handle_out : w.hd;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (c.N > 0) {
+    if ((s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
+    if ((s = cuda_status(launch_quantize_rows(x, c.N, c.d, w.x_q, w.x_scale, st), "x quantisation")) != MOE_OK)
+      return s;
+  }
+  if ((s = ep_notify_impl(c, *grp, peers, w.ids, dev_status, w, st)) != MOE_OK) return s;
+  if ((s = ep_layout_impl(c, *grp, peers, expert_owner, w.ids, hd, dev_status, w, st)) != MOE_OK) return s;
+  if ((s = cuda_status(launch_ep_dispatch(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, w.x_q,
+                                          hd.dest, w.w, w.x_scale, c.d, st),
+                       "EP dispatch (fp8)")) != MOE_OK)
+    return s;
+  const EpFp8 f = {w.x_q, w.x_scale, w13_q, w13_scale, w2_q, w2_scale};
+  if ((s = ep_ffn_fp8_impl(c, *grp, peers, f, hd, dev_status, w, st)) != MOE_OK) return s;
   return cuda_status(launch_ep_combine(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, hd.dest, y,
                                        dev_status, st),
                      "EP combine");

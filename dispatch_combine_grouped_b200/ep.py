@@ -19,8 +19,8 @@ import torch
 
 from . import binding as B
 
-N_OFFSETS = 9
-OFFSET_NAMES = ["cnt_flag", "disp_flag", "done_flag", "step", "disp_ctr", "cnt_tab", "gate", "x_recv",
+N_OFFSETS = 10
+OFFSET_NAMES = ["cnt_flag", "disp_flag", "done_flag", "step", "disp_ctr", "cnt_tab", "gate", "scale", "x_recv",
                 "out_recv"]
 MAX_RANKS = 32
 
@@ -77,6 +77,8 @@ def window_views(cfg, capacity: int, window: torch.Tensor) -> dict:
                 step=view(o["step"], 1, torch.int64),
                 cnt_tab=view(o["cnt_tab"], P * E, torch.int32).view(P, E),
                 gate=view(o["gate"], capacity, torch.float32),
+                scale=view(o["scale"], capacity, torch.float32),
+                x_recv_fp8=window[o["x_recv"]:o["x_recv"] + capacity * d].view(capacity, d),
                 x_recv=window[o["x_recv"]:o["x_recv"] + capacity * d * eb].view(dt).view(capacity, d),
                 out_recv=window[o["out_recv"]:o["out_recv"] + (capacity + S * N) * d * eb].view(dt)
                 .view(capacity + S * N, d))
@@ -108,8 +110,14 @@ class Handle:
         return dict(dest=self.dest[:self.n_dest], owner_n_e=self.owner_n_e[:self.L], owner_off=self.owner_off)
 
 
-def alloc_ws(cfg, capacity: int, device="cuda") -> torch.Tensor:
-    return torch.empty(max(workspace_bytes(cfg, capacity), 1), dtype=torch.uint8, device=device)
+def workspace_bytes_fp8(cfg, capacity: int) -> int:
+    c = B.c_config(cfg)
+    return B.load().moe_ep_workspace_bytes_fp8(ctypes.byref(c), capacity)
+
+
+def alloc_ws(cfg, capacity: int, device="cuda", fp8=False) -> torch.Tensor:
+    n = workspace_bytes_fp8(cfg, capacity) if fp8 else workspace_bytes(cfg, capacity)
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=device)
 
 
 def emulated_groups(cfg, capacity: int, expert_owner=None, device="cuda", rank_cfgs=None):
@@ -238,4 +246,35 @@ def layer_forward(cfg, grp: Group, x, w_gate, bias, w13, w2, ws, expert_owner=No
                                            B._p(bias), B._p(expert_owner), B._p(w13), B._p(w2), B._p(y),
                                            ctypes.byref(handle.c) if handle is not None else None, B._p(status),
                                            B._p(ws), ws.numel(), B._stream()), "moe_ep_layer_forward")
+    return y
+
+
+def dispatch_fp8(cfg, grp: Group, x_q, x_scale, topk_w, handle: Handle):
+    """FP8 payload: e4m3 token rows (d bytes) with each token's scale beside its rows."""
+    c = B.c_config(cfg)
+    B._check(B.load().moe_ep_dispatch_fp8(ctypes.byref(c), ctypes.byref(grp.c), B._p(x_q), B._p(x_scale),
+                                          B._p(topk_w), ctypes.byref(handle.c), B._stream()), "moe_ep_dispatch_fp8")
+
+
+def expert_ffn_fp8(cfg, grp: Group, x_q, x_scale, w13_q, w13_scale, w2_q, w2_scale, handle: Handle, ws, status=None):
+    c = B.c_config(cfg)
+    B._check(B.load().moe_ep_expert_ffn_fp8(ctypes.byref(c), ctypes.byref(grp.c), B._p(x_q), B._p(x_scale),
+                                            B._p(w13_q), B._p(w13_scale), B._p(w2_q), B._p(w2_scale),
+                                            ctypes.byref(handle.c), B._p(status), B._p(ws), ws.numel(),
+                                            B._stream()), "moe_ep_expert_ffn_fp8")
+
+
+def layer_forward_fp8(cfg, grp: Group, x, w_gate, bias, w13_q, w13_scale, w2_q, w2_scale, ws, expert_owner=None,
+                      y=None, handle: Handle | None = None, status=None):
+    """The layer on this rank with FP8 dispatch and experts, bf16 combine
+    (moe_ep_layer_forward_fp8); ws from alloc_ws(..., fp8=True)."""
+    c = B.c_config(cfg)
+    if y is None:
+        y = torch.empty(cfg.N, cfg.d, dtype=torch.bfloat16, device=x.device)
+    B._check(B.load().moe_ep_layer_forward_fp8(ctypes.byref(c), ctypes.byref(grp.c), B._p(x), B._p(w_gate),
+                                               B._p(bias), B._p(expert_owner), B._p(w13_q), B._p(w13_scale),
+                                               B._p(w2_q), B._p(w2_scale), B._p(y),
+                                               ctypes.byref(handle.c) if handle is not None else None,
+                                               B._p(status), B._p(ws), ws.numel(), B._stream()),
+             "moe_ep_layer_forward_fp8")
     return y

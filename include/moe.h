@@ -544,10 +544,11 @@ typedef struct {
 /* Bytes of one rank's window (0 on an invalid configuration). */
 size_t moe_ep_window_bytes(const moe_config* cfg, int32_t capacity);
 /* Byte offsets of the window's parts (the same on every rank; a rank's own N only sizes
- * the shared rows at the end): offsets[0..8] = count flags [32] u64, dispatch flags [32]
+ * the shared rows at the end): offsets[0..9] = count flags [32] u64, dispatch flags [32]
  * u64, done flags [32] u64 (each indexed by the signalling rank), step counter u64,
- * dispatch counter u32, count table [P, E] int32, gates [capacity] fp32, received rows
- * [capacity, d], output rows [capacity + S*N, d]. */
+ * dispatch counter u32, count table [P, E] int32, gates [capacity] fp32, token scales
+ * [capacity] fp32 (FP8 dispatch), received rows [capacity, d] (of d bytes each for the FP8
+ * dispatch), output rows [capacity + S*N, d]. */
 moe_status moe_ep_window_layout(const moe_config* cfg, int32_t capacity, size_t* offsets);
 /* Bytes of scratch the EP calls of one step need (ws; the same ws for all calls of a step
  * and for moe_ep_layer_forward, which also keeps the router outputs and the handle there). */
@@ -585,6 +586,30 @@ moe_status moe_ep_layer_forward(const moe_config* cfg, const moe_ep_group* grp, 
                                 const void* w_gate, const float* bias, const int32_t* expert_owner,
                                 const void* w13, const void* w2, void* y, const moe_ep_handle* handle_out,
                                 int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* The EP layer with the FP8 expert path (FP8 dispatch, bf16 combine: the e4m3 payload is
+ * d bytes per row instead of 2d, so half the NVLink bytes of the dispatch; conventions of
+ * moe_quantize_fp8 / moe_grouped_ffn_fp8).  dtype = MOE_BF16, d % 16 == 0, I % 16 == 0.
+ *   moe_ep_dispatch_fp8: as moe_ep_dispatch, rows of e4m3 codes x_q [N, d] with each
+ *     token's scale x_scale [N] stored beside each of its received rows.
+ *   moe_ep_expert_ffn_fp8: as moe_ep_expert_ffn on e4m3 operands: x_q, x_scale are this
+ *     rank's own quantised tokens (the shared experts' rows); w13_q [local_experts + S, 2I,
+ *     d] e4m3 with w13_scale [local_experts + S, 2I], w2_q [local_experts + S, d, I] e4m3
+ *     with w2_scale [local_experts + S, d]; h is quantised per row between FC1 and FC2.
+ *   moe_ep_layer_forward_fp8: moe_route, moe_quantize_fp8(x), then the five EP steps with
+ *     the two above.  ws of moe_ep_workspace_bytes_fp8 bytes. */
+size_t moe_ep_workspace_bytes_fp8(const moe_config* cfg, int32_t capacity);
+moe_status moe_ep_dispatch_fp8(const moe_config* cfg, const moe_ep_group* grp, const void* x_q, const float* x_scale,
+                               const float* topk_w, const moe_ep_handle* handle, moe_stream_t stream);
+moe_status moe_ep_expert_ffn_fp8(const moe_config* cfg, const moe_ep_group* grp, const void* x_q, const float* x_scale,
+                                 const void* w13_q, const float* w13_scale, const void* w2_q, const float* w2_scale,
+                                 const moe_ep_handle* handle, int32_t* dev_status, void* ws, size_t ws_bytes,
+                                 moe_stream_t stream);
+moe_status moe_ep_layer_forward_fp8(const moe_config* cfg, const moe_ep_group* grp, const void* x, const void* w_gate,
+                                    const float* bias, const int32_t* expert_owner, const void* w13_q,
+                                    const float* w13_scale, const void* w2_q, const float* w2_scale, void* y,
+                                    const moe_ep_handle* handle_out, int32_t* dev_status, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -319,3 +319,80 @@ def test_ep_step_captured_in_cuda_graph():
         assert torch.equal(torch.cat(ys), y1), f"replay {rep}"
     steps = [int(ep.window_views(em.rcfg[r], em.capacity, em.windows[r])["step"].item()) for r in range(P)]
     assert steps == [4] * P   # one eager step + three replays (the capture itself launches nothing)
+
+
+FP8_CASES = [
+    (small_config("ep_f8", cfg_id=96, N=512, d=256, E=16, S=1, k=4, I=128, P=4), None),
+    (small_config("ep_f8_pairs", cfg_id=97, N=1024, d=4096, E=8, S=1, k=2, I=256, P=2), None),
+    (small_config("ep_f8_owner", cfg_id=98, N=384, d=192, E=32, S=2, k=4, I=96, P=4, n_groups=4, topk_groups=2,
+                  score="sigmoid"), "random"),
+]
+
+
+@pytest.mark.parametrize("cfg,spec", FP8_CASES, ids=[c.name for c, _ in FP8_CASES])
+def test_ep_fp8_step_matches_one_gpu_fp8_layer(cfg, spec):
+    """FP8 dispatch (e4m3 rows + token scales over the peer windows), FP8 expert FFN on the
+    owners, bf16 combine: the received codes and scales are the quantised token rows bit
+    for bit, and y equals the one-GPU FP8 layer bit for bit."""
+    inp = gpu_inputs(cfg)
+    owner = _owner(cfg, spec)
+    em = Emulated(cfg, _shards(cfg, spec), owner)
+    em.ws = [ep.alloc_ws(c, em.capacity, fp8=True) for c in em.rcfg]
+    P, n = cfg.P, cfg.N // cfg.P
+    w13_q, w13_s = moe.quantize_fp8(inp["w13"])
+    w2_q, w2_s = moe.quantize_fp8(inp["w2"])
+    xs = [inp["x"][r * n:(r + 1) * n] for r in range(P)]
+    routed = [moe.route(em.rcfg[r], xs[r], inp["w_gate"], inp["bias"]) for r in range(P)]
+    ids, w = [rt[1] for rt in routed], [rt[2] for rt in routed]
+    qs = [moe.quantize_fp8(x) for x in xs]
+    E, S = cfg.E, cfg.S
+    ys = []
+    for r in range(P):
+        ep.notify(em.rcfg[r], em.groups[r], ids[r], em.ws[r], em.status)
+    for r in range(P):
+        ep.layout(em.rcfg[r], em.groups[r], ids[r], em.handles[r], em.ws[r], owner, em.status)
+    for r in range(P):
+        ep.dispatch_fp8(em.rcfg[r], em.groups[r], qs[r][0], qs[r][1], w[r], em.handles[r])
+    for r in range(P):
+        idx = torch.tensor(list(em.owned[r]) + list(range(E, E + S)), dtype=torch.long, device="cuda")
+        ep.expert_ffn_fp8(em.rcfg[r], em.groups[r], qs[r][0], qs[r][1], w13_q.index_select(0, idx),
+                          w13_s.index_select(0, idx), w2_q.index_select(0, idx), w2_s.index_select(0, idx),
+                          em.handles[r], em.ws[r], em.status)
+    for r in range(P):
+        ys.append(ep.combine(em.rcfg[r], em.groups[r], em.handles[r], status=em.status))
+    torch.cuda.synchronize()
+    assert int(em.status.item()) == 0
+    own_np = owner.cpu().numpy() if owner is not None else None
+    lay = O.ep_layout([i.cpu().numpy() for i in ids], cfg.E, cfg.P, own_np, em.capacity)
+    check_handles(em, lay)
+    for j in range(P):
+        v = ep.window_views(em.rcfg[j], em.capacity, em.windows[j])
+        rows = lay["recv"][j]
+        R = len(rows)
+        if R == 0:
+            continue
+        assert torch.equal(v["x_recv_fp8"][:R], torch.stack([qs[i][0][a // cfg.k] for i, a in rows]))
+        assert torch.equal(v["scale"][:R], torch.stack([qs[i][1][a // cfg.k] for i, a in rows]))
+        assert torch.equal(v["gate"][:R], torch.stack([w[i].reshape(-1)[a] for i, a in rows]))
+    y1 = moe.layer_forward_fp8(cfg, inp["x"], inp["w_gate"], inp["bias"], owner, w13_q, w13_s, w2_q, w2_s)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(ys), y1)
+
+
+def test_ep_fp8_layer_forward_one_rank():
+    """P = 1: moe_ep_layer_forward_fp8 equals moe_layer_forward_fp8, over two steps."""
+    cfg = small_config("ep_f8_p1", cfg_id=99, N=300, d=256, E=16, S=1, k=4, I=128, P=1)
+    inp = gpu_inputs(cfg)
+    cap = cfg.N * cfg.k
+    groups, windows = ep.emulated_groups(cfg, cap)
+    ws = ep.alloc_ws(cfg, cap, fp8=True)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    w13_q, w13_s = moe.quantize_fp8(inp["w13"])
+    w2_q, w2_s = moe.quantize_fp8(inp["w2"])
+    for _ in range(2):
+        y = ep.layer_forward_fp8(cfg, groups[0], inp["x"], inp["w_gate"], inp["bias"], w13_q, w13_s, w2_q, w2_s, ws,
+                                 status=status)
+        y1 = moe.layer_forward_fp8(cfg, inp["x"], inp["w_gate"], inp["bias"], None, w13_q, w13_s, w2_q, w2_s)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert torch.equal(y, y1)
