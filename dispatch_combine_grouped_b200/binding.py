@@ -35,7 +35,8 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_con
             "moe_layer_forward_fp8_overlapped", "moe_ep_window_bytes", "moe_ep_window_layout",
             "moe_ep_workspace_bytes", "moe_ep_ipc_handle", "moe_ep_ipc_open", "moe_ep_ipc_close", "moe_ep_notify",
             "moe_ep_layout", "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ep_layer_forward",
-            "moe_ep_workspace_bytes_fp8", "moe_ep_dispatch_fp8", "moe_ep_expert_ffn_fp8", "moe_ep_layer_forward_fp8"]
+            "moe_ep_workspace_bytes_fp8", "moe_ep_dispatch_fp8", "moe_ep_expert_ffn_fp8", "moe_ep_layer_forward_fp8",
+            "moe_ep_layer_forward_overlapped", "moe_ep_layer_forward_fp8_overlapped"]
 
 
 class CConfig(ctypes.Structure):
@@ -133,6 +134,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_ep_dispatch_fp8": (i32, [cfgp, grpp, vp, vp, vp, hdp, vp]),
         "moe_ep_expert_ffn_fp8": (i32, [cfgp, grpp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz, vp]),
         "moe_ep_layer_forward_fp8": (i32, [cfgp, grpp, vp, vp, vp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz, vp]),
+        "moe_ep_layer_forward_overlapped": (i32, [cfgp, grpp, vp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz, vp, vp]),
+        "moe_ep_layer_forward_fp8_overlapped": (i32, [cfgp, grpp, vp, vp, vp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz,
+                                                      vp, vp]),
     })
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

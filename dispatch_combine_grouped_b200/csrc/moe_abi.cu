@@ -415,16 +415,24 @@ moe_status ep_layout_impl(const moe_config& c, const moe_ep_group& g, const EpPe
                      "EP layout");
 }
 
-// The owner's grouped FFN: routed groups = the owned experts over the received rows
-// (A_routed = capacity, no row map: row r's gate is gate[r]), shared groups over the
-// rank's own N tokens; outputs into the window's output rows.
-moe_status ep_ffn_impl(const moe_config& c, const moe_ep_group& g, const EpPeers& peers,
-                       const void* x, const void* w13, const void* w2, const moe_ep_handle& hd, int32_t* status,
-                       const EpWs& w, cudaStream_t st) {
-  const EpOffsets off = ep_offsets(c, g.capacity);
-  char* win = peers.base[g.rank];
-  cudaError_t e = launch_ep_wait(win, off, off.disp_flag, c.P, status, st);
-  if (e != cudaSuccess) return cuda_status(e, "dispatch wait");
+// The owner's expert GEMMs over groups [g0, g0+G): groups [0, local_experts) are the
+// owned experts over the received rows (A_routed = capacity, no row map: row r's gate is
+// gate[r], and with FP8 its token scale is scale[r]); the S shared groups run over the
+// rank's own N tokens.  Outputs go to the window's output rows.  FP8: FC1 on e4m3 rows,
+// per-row quantisation of the h rows of the range, FC2 on e4m3 h.
+struct EpFfn {
+  bool fp8;
+  const void* x;  // bf16 tokens, or e4m3 codes with x_scale
+  const float* x_scale;
+  const void* w13;
+  const float* w13_scale;
+  const void* w2;
+  const float* w2_scale;
+};
+
+moe_status ep_gemms(const moe_config& c, const moe_ep_group& g, char* win, const EpOffsets& off, const EpFfn& f,
+                    const moe_ep_handle& hd, const EpWs& w, cudaStream_t st, int g0, int G) {
+  if (G <= 0) return MOE_OK;
   moe_config co = c;
   co.E = g.local_experts;
   moe_layout L;
@@ -432,78 +440,113 @@ moe_status ep_ffn_impl(const moe_config& c, const moe_ep_group& g, const EpPeers
   L.n_e = hd.owner_n_e;
   L.expert_off = hd.owner_off;
   const int S = c.N > 0 ? c.n_shared : 0;  // the shared experts have no rows without tokens
-  const int G = g.local_experts + S;
+  const long long cap = g.capacity;
   // pair tiles pay for wide rows when a group can exceed 128 rows
   moe_config dec = c;
   dec.N = g.capacity > c.N ? g.capacity : c.N;
-  if (G > 0) {
-    GemmArgs g1 = fc1_args(co, L, win + off.x_recv, S > 0 ? x : nullptr, w13, w.h);
-    g1.G = G;
-    g1.A_routed = g.capacity;
-    e = c.dtype == MOE_BF16 ? tc_grouped(g1, dec, g.capacity, c.N, st) : launch_simt_gemm(g1, st);
-    if (e != cudaSuccess) return cuda_status(e, "EP FC1 grouped GEMM");
-    GemmArgs g2 = fc2_args(co, L, w.h, w2, reinterpret_cast<const float*>(win + off.gate), win + off.out_recv);
-    g2.G = G;
-    g2.A_routed = g.capacity;
-    e = c.dtype == MOE_BF16 ? tc_grouped(g2, dec, g.capacity + S * c.N, 0, st) : launch_simt_gemm(g2, st);
-    if (e != cudaSuccess) return cuda_status(e, "EP FC2 grouped GEMM");
-  }
-  return cuda_status(launch_ep_signal(peers, off, off.done_flag, c.P, g.rank, st), "FFN done signal");
-}
-
-// The owner's FP8 expert FFN: FC1 on the received e4m3 rows (each row's token scale
-// received beside it) and on the rank's own e4m3 token rows for the shared experts,
-// per-row quantisation of h, FC2 on e4m3 h; outputs bf16 into the window.
-struct EpFp8 {
-  const void* x_q;
-  const float* x_scale;
-  const void* w13_q;
-  const float* w13_scale;
-  const void* w2_q;
-  const float* w2_scale;
-};
-
-moe_status ep_ffn_fp8_impl(const moe_config& c, const moe_ep_group& g, const EpPeers& peers, const EpFp8& f,
-                           const moe_ep_handle& hd, int32_t* status, const EpWs& w, cudaStream_t st) {
-  const EpOffsets off = ep_offsets(c, g.capacity);
-  char* win = peers.base[g.rank];
-  cudaError_t e = launch_ep_wait(win, off, off.disp_flag, c.P, status, st);
-  if (e != cudaSuccess) return cuda_status(e, "dispatch wait");
-  moe_config co = c;
-  co.E = g.local_experts;
-  moe_layout L;
-  memset(&L, 0, sizeof(L));
-  L.n_e = hd.owner_n_e;
-  L.expert_off = hd.owner_off;
-  const int S = c.N > 0 ? c.n_shared : 0;
-  const int G = g.local_experts + S;
-  moe_config dec = c;
-  dec.N = g.capacity > c.N ? g.capacity : c.N;
-  if (G > 0) {
-    GemmArgs g1 = fc1_args(co, L, win + off.x_recv, S > 0 ? f.x_q : nullptr, f.w13_q, w.h);
-    g1.G = G;
-    g1.A_routed = g.capacity;
+  GemmArgs g1 = fc1_args(co, L, win + off.x_recv, S > 0 ? f.x : nullptr, f.w13, w.h);
+  g1.g0 = g0;
+  g1.G = G;
+  g1.A_routed = g.capacity;
+  g1.max_ctas = shared_cap(co, g0);
+  if (f.fp8) {
     g1.fp8 = 1;
     g1.k = c.k;
     g1.a_scale = f.x_scale;
     g1.a_scale_rows = reinterpret_cast<const float*>(win + off.scale);
     g1.b_scale = f.w13_scale;
-    e = tc_grouped(g1, dec, g.capacity, c.N, st);
-    if (e != cudaSuccess) return cuda_status(e, "EP FC1 grouped GEMM (fp8)");
-    const long long rows = (long long)g.capacity + (long long)S * c.N;
-    e = launch_quantize_rows(w.h, rows, c.I, w.h_q, w.h_scale, st);
+  }
+  cudaError_t e = c.dtype == MOE_BF16 ? tc_grouped(g1, dec, g.capacity, c.N, st) : launch_simt_gemm(g1, st);
+  if (e != cudaSuccess) return cuda_status(e, "EP FC1 grouped GEMM");
+  const long long rows = cap + (long long)S * c.N;
+  if (f.fp8) {  // h rows of this range: the routed rows [0, capacity), then N per shared group
+    const int Lx = g.local_experts;
+    const long long r0 = g0 < Lx ? 0 : cap + (long long)(g0 - Lx) * c.N;
+    const long long r1 = g0 + G <= Lx ? cap : cap + (long long)(g0 + G - Lx) * c.N;
+    e = launch_quantize_rows(static_cast<const uint16_t*>(w.h) + r0 * c.I, r1 - r0, c.I,
+                             static_cast<uint8_t*>(w.h_q) + r0 * c.I, w.h_scale + r0, st);
     if (e != cudaSuccess) return cuda_status(e, "h quantisation");
-    GemmArgs g2 = fc2_args(co, L, w.h_q, f.w2_q, reinterpret_cast<const float*>(win + off.gate), win + off.out_recv);
-    g2.G = G;
-    g2.A_routed = g.capacity;
+  }
+  GemmArgs g2 = fc2_args(co, L, f.fp8 ? w.h_q : w.h, f.w2, reinterpret_cast<const float*>(win + off.gate),
+                         win + off.out_recv);
+  g2.g0 = g0;
+  g2.G = G;
+  g2.A_routed = g.capacity;
+  g2.max_ctas = shared_cap(co, g0);
+  if (f.fp8) {
     g2.fp8 = 1;
     g2.k = c.k;
     g2.a_scale = w.h_scale;
     g2.b_scale = f.w2_scale;
-    e = tc_grouped(g2, dec, (int)rows, 0, st);
-    if (e != cudaSuccess) return cuda_status(e, "EP FC2 grouped GEMM (fp8)");
   }
+  e = c.dtype == MOE_BF16 ? tc_grouped(g2, dec, (int)rows, 0, st) : launch_simt_gemm(g2, st);
+  return cuda_status(e, "EP FC2 grouped GEMM");
+}
+
+// wait for every source's dispatch, the expert GEMMs of groups [0, G), "done" to every source
+moe_status ep_ffn_impl(const moe_config& c, const moe_ep_group& g, const EpPeers& peers, const EpFfn& f,
+                       const moe_ep_handle& hd, int32_t* status, const EpWs& w, cudaStream_t st, int G) {
+  const EpOffsets off = ep_offsets(c, g.capacity);
+  char* win = peers.base[g.rank];
+  cudaError_t e = launch_ep_wait(win, off, off.disp_flag, c.P, status, st);
+  if (e != cudaSuccess) return cuda_status(e, "dispatch wait");
+  moe_status s = ep_gemms(c, g, win, off, f, hd, w, st, 0, G);
+  if (s != MOE_OK) return s;
   return cuda_status(launch_ep_signal(peers, off, off.done_flag, c.P, g.rank, st), "FFN done signal");
+}
+
+int ep_groups(const moe_config& c, const moe_ep_group& g) { return g.local_experts + (c.N > 0 ? c.n_shared : 0); }
+
+// One rank's layer.  With a side stream (and shared experts), the shared experts' GEMMs
+// run there from right after the router, beside the count exchange, the dispatch, the
+// wait for the other ranks' rows and the routed GEMMs; the combine waits for them.
+moe_status ep_forward(const moe_config& c, const moe_ep_group& g, const EpPeers& peers, const void* x,
+                      const void* w_gate, const float* bias, const int32_t* owner, const EpFfn& fin, void* y,
+                      const moe_ep_handle* handle_out, int32_t* status, const EpWs& w, cudaStream_t st,
+                      cudaStream_t side) {
+  const moe_ep_handle& hd = handle_out ? *handle_out : w.hd;
+  const EpOffsets off = ep_offsets(c, g.capacity);
+  EpFfn f = fin;
+  moe_status s = MOE_OK;
+  if (c.N > 0) {
+    if ((s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
+    if (f.fp8) {
+      s = cuda_status(launch_quantize_rows(x, c.N, c.d, w.x_q, w.x_scale, st), "x quantisation");
+      if (s != MOE_OK) return s;
+      f.x = w.x_q;
+      f.x_scale = w.x_scale;
+    } else {
+      f.x = x;
+    }
+  }
+  const bool overlap = side && side != st && c.N > 0 && c.n_shared > 0;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  if (overlap) {
+    cudaError_t e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
+    if (e == cudaSuccess) {
+      s = ep_gemms(c, g, peers.base[g.rank], off, f, hd, w, side, g.local_experts, c.n_shared);
+      e = cudaEventRecord(join, side);
+    }
+    if (e != cudaSuccess && s == MOE_OK) s = cuda_status(e, "fork");
+  }
+  const int G = overlap ? g.local_experts : ep_groups(c, g);
+  if (s == MOE_OK) s = ep_notify_impl(c, g, peers, w.ids, status, w, st);
+  if (s == MOE_OK) s = ep_layout_impl(c, g, peers, owner, w.ids, hd, status, w, st);
+  if (s == MOE_OK)
+    s = cuda_status(launch_ep_dispatch(c, peers, off, g.rank, g.capacity, f.x, hd.dest, w.w,
+                                       f.fp8 ? f.x_scale : nullptr, c.d * (f.fp8 ? 1 : elem_bytes(c)), st),
+                    "EP dispatch");
+  if (s == MOE_OK) s = ep_ffn_impl(c, g, peers, f, hd, status, w, st, G);
+  if (overlap) {
+    if (join) cudaStreamWaitEvent(st, join, 0);  // join even after an error
+    if (fork) cudaEventDestroy(fork);
+    if (join) cudaEventDestroy(join);
+  }
+  if (s != MOE_OK) return s;
+  return cuda_status(launch_ep_combine(c, peers, off, g.rank, g.capacity, hd.dest, y, status, st), "EP combine");
 }
 
 }  // namespace
@@ -1027,8 +1070,9 @@ moe_status moe_ep_expert_ffn(const moe_config* cfg, const moe_ep_group* grp, con
   const bool any = grp->local_experts > 0 || (cfg->N > 0 && cfg->n_shared > 0);
   if (!handle_complete(handle) || (any && (!w13 || !w2)) || (cfg->N > 0 && cfg->n_shared > 0 && !x))
     return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
-  return ep_ffn_impl(*cfg, *grp, peers, x, w13, w2, *handle, dev_status,
-                     carve_ep(*cfg, grp->capacity, (char*)ws), (cudaStream_t)stream);
+  const EpFfn f = {false, x, nullptr, w13, nullptr, w2, nullptr};
+  return ep_ffn_impl(*cfg, *grp, peers, f, *handle, dev_status, carve_ep(*cfg, grp->capacity, (char*)ws),
+                     (cudaStream_t)stream, ep_groups(*cfg, *grp));
 }
 
 moe_status moe_ep_combine(const moe_config* cfg, const moe_ep_group* grp, const moe_ep_handle* handle,
@@ -1042,34 +1086,45 @@ moe_status moe_ep_combine(const moe_config* cfg, const moe_ep_group* grp, const 
                      "EP combine");
 }
 
+static moe_status ep_layer(const moe_config* cfg, const moe_ep_group* grp, const void* x, const void* w_gate,
+                           const float* bias, const int32_t* expert_owner, const EpFfn& f, void* y,
+                           const moe_ep_handle* handle_out, int32_t* dev_status, void* ws, size_t ws_bytes,
+                           moe_stream_t stream, moe_stream_t side) {
+  moe_status s = f.fp8 ? check_fp8(cfg) : check_config(cfg);
+  if (s != MOE_OK) return s;
+  EpPeers peers;
+  if ((s = check_ep(cfg, grp, &peers)) != MOE_OK) return s;
+  if ((s = check_router(*cfg)) != MOE_OK) return s;
+  if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
+  if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes, f.fp8)) != MOE_OK) return s;
+  if (handle_out && !handle_complete(handle_out)) return fail(MOE_ERR_INVALID_ARG, "incomplete handle_out");
+  const moe_config& c = *cfg;
+  const bool any = grp->local_experts > 0 || (c.N > 0 && c.n_shared > 0);
+  if ((c.N > 0 && (!x || !w_gate || !y)) || (any && (!f.w13 || !f.w2)) ||
+      (any && f.fp8 && (!f.w13_scale || !f.w2_scale)))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return ep_forward(c, *grp, peers, x, w_gate, bias, expert_owner, f, y, handle_out, dev_status,
+                    carve_ep(c, grp->capacity, static_cast<char*>(ws), f.fp8), (cudaStream_t)stream,
+                    (cudaStream_t)side);
+}
+
 moe_status moe_ep_layer_forward(const moe_config* cfg, const moe_ep_group* grp, const void* x,
                                 const void* w_gate, const float* bias, const int32_t* expert_owner, const void* w13,
                                 const void* w2, void* y, const moe_ep_handle* handle_out, int32_t* dev_status,
                                 void* ws, size_t ws_bytes, moe_stream_t stream) {
-  EpPeers peers;
-  moe_status s = check_ep(cfg, grp, &peers);
-  if (s != MOE_OK) return s;
-  if ((s = check_router(*cfg)) != MOE_OK) return s;
-  if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
-  if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes)) != MOE_OK) return s;
-  if (handle_out && !handle_complete(handle_out)) return fail(MOE_ERR_INVALID_ARG, "incomplete handle_out");
-  const moe_config& c = *cfg;
-  const bool any = grp->local_experts > 0 || (c.N > 0 && c.n_shared > 0);
-  if ((c.N > 0 && (!x || !w_gate || !y)) || (any && (!w13 || !w2))) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
-  const EpWs w = carve_ep(c, grp->capacity, static_cast<char*>(ws));
-  const moe_ep_handle& hd = handle_out ? *handle_out : w.hd;
-  cudaStream_t st = (cudaStream_t)stream;
-  if (c.N > 0 && (s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
-  if ((s = ep_notify_impl(c, *grp, peers, w.ids, dev_status, w, st)) != MOE_OK) return s;
-  if ((s = ep_layout_impl(c, *grp, peers, expert_owner, w.ids, hd, dev_status, w, st)) != MOE_OK) return s;
-  if ((s = cuda_status(launch_ep_dispatch(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, x,
-                                          hd.dest, w.w, nullptr, c.d * elem_bytes(c), st),
-                       "EP dispatch")) != MOE_OK)
-    return s;
-  if ((s = ep_ffn_impl(c, *grp, peers, x, w13, w2, hd, dev_status, w, st)) != MOE_OK) return s;
-  return cuda_status(launch_ep_combine(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, hd.dest, y,
-                                       dev_status, st),
-                     "EP combine");
+  const EpFfn f = {false, nullptr, nullptr, w13, nullptr, w2, nullptr};
+  return ep_layer(cfg, grp, x, w_gate, bias, expert_owner, f, y, handle_out, dev_status, ws, ws_bytes, stream,
+                  nullptr);
+}
+
+moe_status moe_ep_layer_forward_overlapped(const moe_config* cfg, const moe_ep_group* grp, const void* x,
+                                           const void* w_gate, const float* bias, const int32_t* expert_owner,
+                                           const void* w13, const void* w2, void* y, const moe_ep_handle* handle_out,
+                                           int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                           moe_stream_t side_stream) {
+  const EpFfn f = {false, nullptr, nullptr, w13, nullptr, w2, nullptr};
+  return ep_layer(cfg, grp, x, w_gate, bias, expert_owner, f, y, handle_out, dev_status, ws, ws_bytes, stream,
+                  side_stream);
 }
 
 size_t moe_ep_workspace_bytes_fp8(const moe_config* cfg, int32_t capacity) {
@@ -1103,9 +1158,9 @@ moe_status moe_ep_expert_ffn_fp8(const moe_config* cfg, const moe_ep_group* grp,
   if (!handle_complete(handle) || (any && (!w13_q || !w13_scale || !w2_q || !w2_scale)) ||
       (cfg->N > 0 && cfg->n_shared > 0 && (!x_q || !x_scale)))
     return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
-  const EpFp8 f = {x_q, x_scale, w13_q, w13_scale, w2_q, w2_scale};
-  return ep_ffn_fp8_impl(*cfg, *grp, peers, f, *handle, dev_status, carve_ep(*cfg, grp->capacity, (char*)ws, true),
-                         (cudaStream_t)stream);
+  const EpFfn f = {true, x_q, x_scale, w13_q, w13_scale, w2_q, w2_scale};
+  return ep_ffn_impl(*cfg, *grp, peers, f, *handle, dev_status, carve_ep(*cfg, grp->capacity, (char*)ws, true),
+                     (cudaStream_t)stream, ep_groups(*cfg, *grp));
 }
 
 moe_status moe_ep_layer_forward_fp8(const moe_config* cfg, const moe_ep_group* grp, const void* x, const void* w_gate,
@@ -1113,37 +1168,20 @@ moe_status moe_ep_layer_forward_fp8(const moe_config* cfg, const moe_ep_group* g
                                     const float* w13_scale, const void* w2_q, const float* w2_scale, void* y,
                                     const moe_ep_handle* handle_out, int32_t* dev_status, void* ws, size_t ws_bytes,
                                     moe_stream_t stream) {
-  moe_status s = check_fp8(cfg);
-  if (s != MOE_OK) return s;
-  EpPeers peers;
-  if ((s = check_ep(cfg, grp, &peers)) != MOE_OK) return s;
-  if ((s = check_router(*cfg)) != MOE_OK) return s;
-  if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
-  if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes, true)) != MOE_OK) return s;
-  if (handle_out && !handle_complete(handle_out)) return fail(MOE_ERR_INVALID_ARG, "incomplete handle_out");
-  const moe_config& c = *cfg;
-  const bool any = grp->local_experts > 0 || (c.N > 0 && c.n_shared > 0);
-  if ((c.N > 0 && (!x || !w_gate || !y)) || (any && (!w13_q || !w13_scale || !w2_q || !w2_scale)))
-    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
-  const EpWs w = carve_ep(c, grp->capacity, static_cast<char*>(ws), true);
-  const moe_ep_handle& hd = handle_out ? *handle_out : w.hd;
-  cudaStream_t st = (cudaStream_t)stream;
-  if (c.N > 0) {
-    if ((s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
-    if ((s = cuda_status(launch_quantize_rows(x, c.N, c.d, w.x_q, w.x_scale, st), "x quantisation")) != MOE_OK)
-      return s;
-  }
-  if ((s = ep_notify_impl(c, *grp, peers, w.ids, dev_status, w, st)) != MOE_OK) return s;
-  if ((s = ep_layout_impl(c, *grp, peers, expert_owner, w.ids, hd, dev_status, w, st)) != MOE_OK) return s;
-  if ((s = cuda_status(launch_ep_dispatch(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, w.x_q,
-                                          hd.dest, w.w, w.x_scale, c.d, st),
-                       "EP dispatch (fp8)")) != MOE_OK)
-    return s;
-  const EpFp8 f = {w.x_q, w.x_scale, w13_q, w13_scale, w2_q, w2_scale};
-  if ((s = ep_ffn_fp8_impl(c, *grp, peers, f, hd, dev_status, w, st)) != MOE_OK) return s;
-  return cuda_status(launch_ep_combine(c, peers, ep_offsets(c, grp->capacity), grp->rank, grp->capacity, hd.dest, y,
-                                       dev_status, st),
-                     "EP combine");
+  const EpFfn f = {true, nullptr, nullptr, w13_q, w13_scale, w2_q, w2_scale};
+  return ep_layer(cfg, grp, x, w_gate, bias, expert_owner, f, y, handle_out, dev_status, ws, ws_bytes, stream,
+                  nullptr);
+}
+
+moe_status moe_ep_layer_forward_fp8_overlapped(const moe_config* cfg, const moe_ep_group* grp, const void* x,
+                                               const void* w_gate, const float* bias, const int32_t* expert_owner,
+                                               const void* w13_q, const float* w13_scale, const void* w2_q,
+                                               const float* w2_scale, void* y, const moe_ep_handle* handle_out,
+                                               int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                               moe_stream_t side_stream) {
+  const EpFfn f = {true, nullptr, nullptr, w13_q, w13_scale, w2_q, w2_scale};
+  return ep_layer(cfg, grp, x, w_gate, bias, expert_owner, f, y, handle_out, dev_status, ws, ws_bytes, stream,
+                  side_stream);
 }
 
 moe_status moe_capacity_drop(const moe_config* cfg, const int32_t* topk_ids, int32_t capacity, int32_t* kept_ids,

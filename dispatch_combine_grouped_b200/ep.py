@@ -236,16 +236,22 @@ def combine(cfg, grp: Group, handle: Handle, y=None, status=None, device="cuda")
 
 
 def layer_forward(cfg, grp: Group, x, w_gate, bias, w13, w2, ws, expert_owner=None, y=None,
-                  handle: Handle | None = None, status=None):
+                  handle: Handle | None = None, status=None, side_stream=None):
     """The layer on this rank (moe_ep_layer_forward): route, notify, layout, dispatch,
-    expert FFN, combine.  With P > 1 every rank must run the same sequence of steps."""
+    expert FFN, combine; with side_stream (a torch.cuda.Stream) the shared experts run
+    there (moe_ep_layer_forward_overlapped).  With P > 1 every rank must run the same
+    sequence of steps."""
     c = B.c_config(cfg)
     if y is None:
         y = torch.empty(cfg.N, cfg.d, dtype=B._dtype(cfg), device=x.device)
-    B._check(B.load().moe_ep_layer_forward(ctypes.byref(c), ctypes.byref(grp.c), B._p(x), B._p(w_gate),
-                                           B._p(bias), B._p(expert_owner), B._p(w13), B._p(w2), B._p(y),
-                                           ctypes.byref(handle.c) if handle is not None else None, B._p(status),
-                                           B._p(ws), ws.numel(), B._stream()), "moe_ep_layer_forward")
+    args = [ctypes.byref(c), ctypes.byref(grp.c), B._p(x), B._p(w_gate), B._p(bias), B._p(expert_owner), B._p(w13),
+            B._p(w2), B._p(y), ctypes.byref(handle.c) if handle is not None else None, B._p(status), B._p(ws),
+            ws.numel(), B._stream()]
+    if side_stream is None:
+        B._check(B.load().moe_ep_layer_forward(*args), "moe_ep_layer_forward")
+    else:
+        B._check(B.load().moe_ep_layer_forward_overlapped(*args, ctypes.c_void_p(side_stream.cuda_stream)),
+                 "moe_ep_layer_forward_overlapped")
     return y
 
 
@@ -265,16 +271,19 @@ def expert_ffn_fp8(cfg, grp: Group, x_q, x_scale, w13_q, w13_scale, w2_q, w2_sca
 
 
 def layer_forward_fp8(cfg, grp: Group, x, w_gate, bias, w13_q, w13_scale, w2_q, w2_scale, ws, expert_owner=None,
-                      y=None, handle: Handle | None = None, status=None):
+                      y=None, handle: Handle | None = None, status=None, side_stream=None):
     """The layer on this rank with FP8 dispatch and experts, bf16 combine
-    (moe_ep_layer_forward_fp8); ws from alloc_ws(..., fp8=True)."""
+    (moe_ep_layer_forward_fp8, or ..._overlapped with side_stream); ws from
+    alloc_ws(..., fp8=True)."""
     c = B.c_config(cfg)
     if y is None:
         y = torch.empty(cfg.N, cfg.d, dtype=torch.bfloat16, device=x.device)
-    B._check(B.load().moe_ep_layer_forward_fp8(ctypes.byref(c), ctypes.byref(grp.c), B._p(x), B._p(w_gate),
-                                               B._p(bias), B._p(expert_owner), B._p(w13_q), B._p(w13_scale),
-                                               B._p(w2_q), B._p(w2_scale), B._p(y),
-                                               ctypes.byref(handle.c) if handle is not None else None,
-                                               B._p(status), B._p(ws), ws.numel(), B._stream()),
-             "moe_ep_layer_forward_fp8")
+    args = [ctypes.byref(c), ctypes.byref(grp.c), B._p(x), B._p(w_gate), B._p(bias), B._p(expert_owner),
+            B._p(w13_q), B._p(w13_scale), B._p(w2_q), B._p(w2_scale), B._p(y),
+            ctypes.byref(handle.c) if handle is not None else None, B._p(status), B._p(ws), ws.numel(), B._stream()]
+    if side_stream is None:
+        B._check(B.load().moe_ep_layer_forward_fp8(*args), "moe_ep_layer_forward_fp8")
+    else:
+        B._check(B.load().moe_ep_layer_forward_fp8_overlapped(*args, ctypes.c_void_p(side_stream.cuda_stream)),
+                 "moe_ep_layer_forward_fp8_overlapped")
     return y

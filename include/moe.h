@@ -587,6 +587,19 @@ moe_status moe_ep_layer_forward(const moe_config* cfg, const moe_ep_group* grp, 
                                 const void* w13, const void* w2, void* y, const moe_ep_handle* handle_out,
                                 int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_ep_layer_forward with the shared experts overlapped ([MoE-IV] §4 and [EP-DeepEP]
+ * §7: hide the dispatch behind independent compute): after the router on `stream`, the
+ * shared experts' GEMMs over this rank's own tokens run on `side_stream` while the count
+ * exchange, the dispatch, the wait for the other ranks' rows and the routed GEMMs run on
+ * `stream`; `stream` waits for `side_stream` before the combine.  Same y, bit for bit; two
+ * events are created and destroyed per call.  With n_shared == 0, N == 0 or side_stream
+ * == stream this is moe_ep_layer_forward. */
+moe_status moe_ep_layer_forward_overlapped(const moe_config* cfg, const moe_ep_group* grp, const void* x,
+                                           const void* w_gate, const float* bias, const int32_t* expert_owner,
+                                           const void* w13, const void* w2, void* y, const moe_ep_handle* handle_out,
+                                           int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                           moe_stream_t side_stream);
+
 /* The EP layer with the FP8 expert path (FP8 dispatch, bf16 combine: the e4m3 payload is
  * d bytes per row instead of 2d, so half the NVLink bytes of the dispatch; conventions of
  * moe_quantize_fp8 / moe_grouped_ffn_fp8).  dtype = MOE_BF16, d % 16 == 0, I % 16 == 0.
@@ -610,6 +623,14 @@ moe_status moe_ep_layer_forward_fp8(const moe_config* cfg, const moe_ep_group* g
                                     const float* w13_scale, const void* w2_q, const float* w2_scale, void* y,
                                     const moe_ep_handle* handle_out, int32_t* dev_status, void* ws, size_t ws_bytes,
                                     moe_stream_t stream);
+/* moe_ep_layer_forward_fp8 with the shared experts on side_stream (as
+ * moe_ep_layer_forward_overlapped; bit for bit the same y). */
+moe_status moe_ep_layer_forward_fp8_overlapped(const moe_config* cfg, const moe_ep_group* grp, const void* x,
+                                               const void* w_gate, const float* bias, const int32_t* expert_owner,
+                                               const void* w13_q, const float* w13_scale, const void* w2_q,
+                                               const float* w2_scale, void* y, const moe_ep_handle* handle_out,
+                                               int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                               moe_stream_t side_stream);
 
 #ifdef __cplusplus
 }

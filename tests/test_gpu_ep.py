@@ -225,7 +225,8 @@ def test_ep_dropped_assignments():
 
 
 def test_ep_one_rank_layer_forward_matches_one_gpu_layer():
-    """P = 1: moe_ep_layer_forward (router + the five steps in one call) equals moe_layer_forward."""
+    """P = 1: moe_ep_layer_forward (router + the five steps in one call), and its overlapped
+    form (shared experts on a side stream), equal moe_layer_forward."""
     cfg = small_config("ep_p1", cfg_id=95, N=300, d=256, E=16, S=1, k=4, I=128, P=1)
     inp = gpu_inputs(cfg)
     cap = cfg.N * cfg.k
@@ -233,13 +234,15 @@ def test_ep_one_rank_layer_forward_matches_one_gpu_layer():
     ws = ep.alloc_ws(cfg, cap)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     h = ep.Handle(cfg, cfg.E)
-    for epoch in (1, 2):
+    side = torch.cuda.Stream()
+    for epoch in (1, 2, 3):
         y = ep.layer_forward(cfg, groups[0], inp["x"], inp["w_gate"], inp["bias"], inp["w13"], inp["w2"], ws,
-                             handle=h, status=status)
+                             handle=h, status=status, side_stream=side if epoch == 3 else None)
         y1 = moe.layer_forward(cfg, inp["x"], inp["w_gate"], inp["bias"], None, inp["w13"], inp["w2"])
         torch.cuda.synchronize()
         assert int(status.item()) == 0
         assert torch.equal(y, y1), f"epoch {epoch}"
+    assert int(ep.window_views(cfg, cap, windows[0])["step"].item()) == 3
 
 
 def test_ep_wait_times_out_and_context_stays_usable():
@@ -380,7 +383,7 @@ def test_ep_fp8_step_matches_one_gpu_fp8_layer(cfg, spec):
 
 
 def test_ep_fp8_layer_forward_one_rank():
-    """P = 1: moe_ep_layer_forward_fp8 equals moe_layer_forward_fp8, over two steps."""
+    """P = 1: moe_ep_layer_forward_fp8 and its overlapped form equal moe_layer_forward_fp8."""
     cfg = small_config("ep_f8_p1", cfg_id=99, N=300, d=256, E=16, S=1, k=4, I=128, P=1)
     inp = gpu_inputs(cfg)
     cap = cfg.N * cfg.k
@@ -389,9 +392,10 @@ def test_ep_fp8_layer_forward_one_rank():
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     w13_q, w13_s = moe.quantize_fp8(inp["w13"])
     w2_q, w2_s = moe.quantize_fp8(inp["w2"])
-    for _ in range(2):
+    side = torch.cuda.Stream()
+    for step in range(3):
         y = ep.layer_forward_fp8(cfg, groups[0], inp["x"], inp["w_gate"], inp["bias"], w13_q, w13_s, w2_q, w2_s, ws,
-                                 status=status)
+                                 status=status, side_stream=side if step == 2 else None)
         y1 = moe.layer_forward_fp8(cfg, inp["x"], inp["w_gate"], inp["bias"], None, w13_q, w13_s, w2_q, w2_s)
         torch.cuda.synchronize()
         assert int(status.item()) == 0
