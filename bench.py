@@ -205,7 +205,8 @@ def whole_job_tokens_per_s(tokens_per_rank: int, world: int, slowest_ms_per_step
 # ------------------------------------------------------------------------------ oracle arm
 def oracle_tokens_per_s(cfg, seconds, inputs=None):
     """Time the float64 oracle (as it stands) on consecutive 128-token slices of the
-    workload until about ``seconds`` have passed.  Returns (tokens/s, tokens, seconds, threads)."""
+    workload until about ``seconds`` have passed.  Returns (tokens/s, tokens, seconds, threads,
+    seconds spent in each step of the layer: routing + layout, permute, experts, combine)."""
     import numpy as np
     import torch
     from moe_inputs import make_inputs
@@ -219,16 +220,32 @@ def oracle_tokens_per_s(cfg, seconds, inputs=None):
     owner = inp["expert_owner"].cpu() if inp["expert_owner"] is not None else None
     bias = inp["bias"].cpu() if inp["bias"] is not None else None
     n_slice = 128
-    sub = cfg.replace(N=n_slice)
+    wg = inp["w_gate"].cpu()
+    phases = {"routing_layout": 0.0, "permute": 0.0, "ffn": 0.0, "combine": 0.0}
     done, t0 = 0, time.perf_counter()
     while True:
         s0 = done % cfg.N
         xs = x[s0:s0 + n_slice]
-        O.moe_layer(sub.replace(N=xs.shape[0]), xs, inp["w_gate"].cpu(), bias, w13, w2, owner)
+        c = cfg.replace(N=xs.shape[0])
+        # the oracle's layer (moe_layer), its steps timed one by one in the same order
+        ta = time.perf_counter()
+        ids = O.select_experts(O.router_logits(xs, wg, bias), c.k, c.n_groups, c.topk_groups)
+        g = O.gate_weights(O.gate_logits(c, xs, wg, bias), ids, c.score, c.renormalize)
+        lay = O.dispatch_layout(ids, c.E, c.P, owner, c.S)
+        tb = time.perf_counter()
+        xp = O.permute(xs, lay, c.k)
+        tc = time.perf_counter()
+        o = O.experts_on_rows(xp, lay, w13, w2, c.E)
+        shared = [O.swiglu_expert(xs, w13[c.E + s], w2[c.E + s]) for s in range(c.S)]
+        td = time.perf_counter()
+        O.combine(o, lay, g, c.N, c.k, shared)
+        te = time.perf_counter()
+        for k_, v_ in zip(phases, (tb - ta, tc - tb, td - tc, te - td)):
+            phases[k_] += v_
         done += xs.shape[0]
         el = time.perf_counter() - t0
         if el >= seconds:
-            return done / el, done, el, threads
+            return done / el, done, el, threads, {k_: round(v_, 3) for k_, v_ in phases.items()}
 
 
 def run_reference(args, cfg, rank):
@@ -239,11 +256,12 @@ def run_reference(args, cfg, rank):
     per_step = max(1.0, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_tokens_per_s(cfg, per_step / 4, inp)
-    tot_tok, tot_s, threads = 0, 0.0, 1
+    tot_tok, tot_s, threads, phases = 0, 0.0, 1, {}
     for _ in range(args.steps):
-        _, tok, s, threads = oracle_tokens_per_s(cfg, per_step, inp)
+        _, tok, s, threads, ph = oracle_tokens_per_s(cfg, per_step, inp)
         tot_tok += tok
         tot_s += s
+        phases = {k: round(phases.get(k, 0.0) + v, 3) for k, v in ph.items()}
     v = tot_tok / tot_s
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
@@ -251,7 +269,8 @@ def run_reference(args, cfg, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": describe(cfg)},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{tot_tok} tokens of the workload in 128-token slices, whole layer in float64"},
+                         "sample": f"{tot_tok} tokens of the workload in 128-token slices, whole layer in float64",
+                         "phases_s": phases},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -949,11 +968,12 @@ def main():
             "wall_s_timed": wall,
         }
         if not args.no_cpu_baseline and world == 1:
-            v, tok, s, threads = oracle_tokens_per_s(cfg, args.cpu_seconds, {k: (t.cpu() if t is not None else None)
-                                                                             for k, t in inp.items()})
+            v, tok, s, threads, phases = oracle_tokens_per_s(
+                cfg, args.cpu_seconds, {k: (t.cpu() if t is not None else None) for k, t in inp.items()})
             line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                     "sample": f"{tok} tokens of the workload in 128-token slices, "
-                                              f"whole layer in float64, {s:.1f} s"}
+                                              f"whole layer in float64, {s:.1f} s",
+                                    "phases_s": phases}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
