@@ -385,24 +385,50 @@ def run_ep(args, cfg, local):
     inp = make_inputs(gcfg, device=dev)
     n = cfg.N // P
     rc = gcfg.replace(N=n)
-    cap = 2 * -(-cfg.N * cfg.k // P)          # receive rows per owner: twice the mean load
     f8 = bool(args.fp8)
-    groups, windows = ep.emulated_groups(rc, cap)
-    ws = [ep.alloc_ws(rc, cap, fp8=f8) for _ in range(P)]
-    handles = [ep.Handle(rc, cfg.E // P) for _ in range(P)]
+    E, S, R = cfg.E, cfg.S, args.eplb
+    if R and f8:
+        raise SystemExit("--ep with --eplb runs the bf16 path")
+    # the workload's placement (e.g. the hot-spot table), else contiguous; with EPLB the
+    # copies are planned from this batch's counts and the slot weights placed once
+    # (load-time steps); each rank maps its assignments to slots inside the step
+    _, ids0, _ = moe.route(gcfg, inp["x"], inp["w_gate"], inp["bias"])
+    n_e0 = torch.bincount(ids0.reshape(-1).long(), minlength=E).cpu().numpy()
+    pc, owner_t, w13_ep, w2_ep = rc, inp["expert_owner"], inp["w13"], inp["w2"]
+    own0 = owner_t.cpu().numpy() if owner_t is not None else np.arange(E) // (E // P)
+    slots_of = [[e for e in range(E) if own0[e] == r] for r in range(P)]
+    load = np.bincount(own0, weights=n_e0, minlength=P)
+    if R:
+        plan = moe.eplb_plan(n_e0, R, P)
+        load = np.asarray(plan["owner_load"], dtype=np.float64)
+        pc = moe.physical_config(rc, R)
+        owner_t = torch.tensor(plan["slot_owner"], dtype=torch.int32, device=dev)
+        rep_off = torch.tensor(plan["replica_off"], dtype=torch.int32, device=dev)
+        rep_slots = torch.tensor(plan["replica_slots"], dtype=torch.int32, device=dev)
+        slots_of = [[q for q in range(E + R) if plan["slot_owner"][q] == r] for r in range(P)]
+        w13_ep = moe.eplb_place_weights(plan["slot_expert"], E, S, inp["w13"])
+        w2_ep = moe.eplb_place_weights(plan["slot_expert"], E, S, inp["w2"])
+        phys = [torch.empty(n, cfg.k, dtype=torch.int32, device=dev) for _ in range(P)]
+        eplb_ws = torch.empty(max(moe.eplb_workspace_bytes(rc), 1), dtype=torch.uint8, device=dev)
+    E_slots = pc.E
+    # receive rows per owner, sized from this batch's counts as the pages size receive
+    # buffers from the exchanged counts (+ k*P rows for the per-rank split of copies)
+    cap = int(-(-(int(load.max()) + cfg.k * P) // 128) * 128)
+    groups, windows = ep.emulated_groups(pc, cap, owner_t)
+    ws = [ep.alloc_ws(pc, cap, fp8=f8) for _ in range(P)]
+    handles = [ep.Handle(pc, len(slots_of[r])) for r in range(P)]
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    E, S = cfg.E, cfg.S
     wts = []
     if f8:  # weights quantised once (a load-time step), then sliced per owner
         w13_q, w13_s = moe.quantize_fp8(inp["w13"])
         w2_q, w2_s = moe.quantize_fp8(inp["w2"])
         del inp["w13"], inp["w2"]
     for r in range(P):
-        idx = torch.tensor(list(range(r * E // P, (r + 1) * E // P)) + list(range(E, E + S)), device=dev)
+        idx = torch.tensor(slots_of[r] + list(range(E_slots, E_slots + S)), device=dev)
         if f8:
             wts.append(tuple(t.index_select(0, idx) for t in (w13_q, w13_s, w2_q, w2_s)))
         else:
-            wts.append((inp["w13"].index_select(0, idx), inp["w2"].index_select(0, idx)))
+            wts.append((w13_ep.index_select(0, idx), w2_ep.index_select(0, idx)))
     xs = [inp["x"][r * n:(r + 1) * n] for r in range(P)]
     qs = [(torch.empty(n, cfg.d, dtype=torch.uint8, device=dev), torch.empty(n, dtype=torch.float32, device=dev))
           for _ in range(P)] if f8 else None
@@ -411,7 +437,7 @@ def run_ep(args, cfg, local):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stages = ["route", "notify", "layout", "dispatch", "ffn", "combine"]
 
-    def step(ev=None):
+    def step(ev=None, fev=None):
         def mark(i):
             if ev is not None:
                 ev[i].record()
@@ -420,27 +446,34 @@ def run_ep(args, cfg, local):
             moe.route(rc, xs[r], inp["w_gate"], inp["bias"], out=routed[r])
             if f8:
                 moe.quantize_fp8(xs[r], out=qs[r][0], scale=qs[r][1])
+            if R:
+                moe.eplb_assign(rc, routed[r][1], rep_off, rep_slots, E + R, status=status, out=phys[r], ws=eplb_ws)
+        ids_ep = phys if R else [rt[1] for rt in routed]
         mark(1)
         for r in range(P):
-            ep.notify(rc, groups[r], routed[r][1], ws[r], status)
+            ep.notify(pc, groups[r], ids_ep[r], ws[r], status)
         mark(2)
         for r in range(P):
-            ep.layout(rc, groups[r], routed[r][1], handles[r], ws[r], None, status)
+            ep.layout(pc, groups[r], ids_ep[r], handles[r], ws[r], owner_t, status)
         mark(3)
         for r in range(P):
             if f8:
-                ep.dispatch_fp8(rc, groups[r], qs[r][0], qs[r][1], routed[r][2], handles[r])
+                ep.dispatch_fp8(pc, groups[r], qs[r][0], qs[r][1], routed[r][2], handles[r])
             else:
-                ep.dispatch(rc, groups[r], xs[r], routed[r][2], handles[r])
+                ep.dispatch(pc, groups[r], xs[r], routed[r][2], handles[r])
         mark(4)
         for r in range(P):
+            if fev is not None:
+                fev[r][0].record()
             if f8:
-                ep.expert_ffn_fp8(rc, groups[r], qs[r][0], qs[r][1], *wts[r], handles[r], ws[r], status)
+                ep.expert_ffn_fp8(pc, groups[r], qs[r][0], qs[r][1], *wts[r], handles[r], ws[r], status)
             else:
-                ep.expert_ffn(rc, groups[r], xs[r], wts[r][0], wts[r][1], handles[r], ws[r], status)
+                ep.expert_ffn(pc, groups[r], xs[r], wts[r][0], wts[r][1], handles[r], ws[r], status)
+            if fev is not None:
+                fev[r][1].record()
         mark(5)
         for r in range(P):
-            ep.combine(rc, groups[r], handles[r], y=ys[r], status=status)
+            ep.combine(pc, groups[r], handles[r], y=ys[r], status=status)
         mark(6)
 
     for _ in range(args.warmup):
@@ -450,13 +483,17 @@ def run_ep(args, cfg, local):
         raise SystemExit(f"EP step reported status {int(status.item())}")
     # per-stage times (eager launches, events between the stages)
     tot = [0.0] * len(stages)
+    ffn_owner = [0.0] * P   # each owner's expert FFN (the critical path of a real P-GPU step)
     for _ in range(args.steps):
         flush.zero_()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
-        step(ev)
+        fev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(P)]
+        step(ev, fev)
         torch.cuda.synchronize()
         for i in range(len(stages)):
             tot[i] += ev[i].elapsed_time(ev[i + 1])
+        for r in range(P):
+            ffn_owner[r] += fev[r][0].elapsed_time(fev[r][1]) / args.steps
     # the whole step as one CUDA graph replay (no host launch gaps); each replay is a new
     # step because the step number lives in the windows
     cs = torch.cuda.Stream(device=dev)
@@ -480,14 +517,14 @@ def run_ep(args, cfg, local):
         ws1 = torch.empty(moe.workspace_bytes_fp8(gcfg), dtype=torch.uint8, device=dev)
 
         def one_gpu(y=None):
-            return moe.layer_forward_fp8(gcfg, inp["x"], inp["w_gate"], inp["bias"], None, w13_q, w13_s, w2_q, w2_s,
-                                         y=y, ws=ws1)
+            return moe.layer_forward_fp8(gcfg, inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], w13_q,
+                                         w13_s, w2_q, w2_s, y=y, ws=ws1)
     else:
         ws1 = moe.alloc_workspace(gcfg, dev)
 
         def one_gpu(y=None):
-            return moe.layer_forward(gcfg, inp["x"], inp["w_gate"], inp["bias"], None, inp["w13"], inp["w2"], y=y,
-                                     ws=ws1)
+            return moe.layer_forward(gcfg, inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], inp["w13"],
+                                     inp["w2"], y=y, ws=ws1)
     y1 = one_gpu()
     one = []
     for _ in range(args.steps):
@@ -506,6 +543,7 @@ def run_ep(args, cfg, local):
         dest = handles[r].as_dict()["dest"]
         owner = torch.div(dest[dest >= 0], cap, rounding_mode="floor")
         cross.append(int((owner != r).sum().item()))
+    owner_rows = [int(h.as_dict()["owner_off"][-1].item()) for h in handles]
     row_bytes = cfg.d * eb                      # output rows (combine) and bf16 payload rows
     pay_bytes = cfg.d * (1 if f8 else eb)       # dispatch payload rows (e4m3: d bytes)
     max_cross = max(cross) * pay_bytes
@@ -534,6 +572,11 @@ def run_ep(args, cfg, local):
                    "note": "bytes a real P-GPU step sends from (and receives into) each GPU in the dispatch and "
                            "in the combine; the roofline time is their sum at the measured 770 GB/s peer copy; "
                            "not measured here (one GPU)"},
+        "owner_receive_rows": owner_rows,
+        "ffn_ms_per_owner": [round(v, 4) for v in ffn_owner],
+        "ffn_ms_slowest_owner": max(ffn_owner),
+        "owner_rows_max_over_mean": max(owner_rows) / (sum(owner_rows) / P) if sum(owner_rows) else None,
+        **({"eplb": {"copies": R, "slots": E + R}} if R else {}),
         "status": int(status.item()),
     }), flush=True)
 

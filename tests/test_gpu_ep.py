@@ -400,3 +400,43 @@ def test_ep_fp8_layer_forward_one_rank():
         torch.cuda.synchronize()
         assert int(status.item()) == 0
         assert torch.equal(y, y1)
+
+
+def test_ep_with_redundant_expert_slots():
+    """EPLB across ranks (Wide EP: redundant copies of hot experts balance the owners'
+    receive load): each rank maps its logical ids to physical slots (moe_eplb_assign on
+    its own assignments), the EP path runs over the E + R slots with the plan's slot
+    owners and slot weights, and y equals the one-GPU layer over the logical experts bit
+    for bit (copies hold identical weights)."""
+    cfg = small_config("ep_eplb", cfg_id=110, N=512, d=256, E=16, S=1, k=4, I=128, P=4, bias="zipf",
+                       bias_alpha=0.6)
+    inp = gpu_inputs(cfg)
+    R, P, n = 4, cfg.P, cfg.N // cfg.P
+    _, ids_all, _ = moe.route(cfg, inp["x"], inp["w_gate"], inp["bias"])
+    n_e = torch.bincount(ids_all.reshape(-1).long(), minlength=cfg.E).cpu().numpy()
+    plan = moe.eplb_plan(n_e, R, P)
+    pcfg = moe.physical_config(cfg, R)
+    owner = torch.tensor(plan["slot_owner"], dtype=torch.int32, device="cuda")
+    rep_off = torch.tensor(plan["replica_off"], dtype=torch.int32, device="cuda")
+    rep_slots = torch.tensor(plan["replica_slots"], dtype=torch.int32, device="cuda")
+    phys_inp = dict(inp, w13=moe.eplb_place_weights(plan["slot_expert"], cfg.E, cfg.S, inp["w13"]),
+                    w2=moe.eplb_place_weights(plan["slot_expert"], cfg.E, cfg.S, inp["w2"]))
+    em = Emulated(pcfg, [n] * P, owner)
+    rcfg = cfg.replace(N=n)
+    ids, w = [], []
+    for r in range(P):
+        _, i_r, w_r = moe.route(rcfg, inp["x"][r * n:(r + 1) * n], inp["w_gate"], inp["bias"])
+        ids.append(moe.eplb_assign(rcfg, i_r, rep_off, rep_slots, cfg.E + R))
+        w.append(w_r)
+    res = em.step(phys_inp, ids=ids, w=w)
+    assert int(em.status.item()) == 0
+    lay = O.ep_layout([i.cpu().numpy() for i in ids], pcfg.E, P, owner.cpu().numpy(), em.capacity)
+    check_handles(em, lay)
+    check_windows(em, res, lay)
+    y1 = moe.layer_forward(cfg, inp["x"], inp["w_gate"], inp["bias"], None, inp["w13"], inp["w2"])
+    torch.cuda.synchronize()
+    assert torch.equal(res["y"], y1)
+    # the plan balances the owners' receive rows at least as well as the contiguous placement
+    base = O.ep_layout([ids_all[r * n:(r + 1) * n].cpu().numpy() for r in range(P)], cfg.E, P)
+    print("owner receive rows, contiguous:", base["R"].tolist(), "with", R, "copies:", lay["R"].tolist())
+    assert lay["R"].max() <= base["R"].max()
