@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--ep", type=int, default=0, metavar="P",
                     help="expert parallelism with P ranks emulated on this GPU (moe_ep_*): per-stage times "
                          "of all ranks, the one-GPU layer beside it, and the NVLink bytes a real P-GPU step moves")
+    ap.add_argument("--ep-real", action="store_true",
+                    help="under torchrun (2+ GPUs): the expert-parallel layer across the ranks over NVLink "
+                         "(moe_ep_layer_forward_overlapped, windows mapped through CUDA IPC)")
     ap.add_argument("--eplb", type=int, default=0, metavar="R",
                     help="run the routed experts over E + R physical slots (redundant copies of the "
                          "hot experts, planned from the batch's own counts)")
@@ -581,6 +584,89 @@ def run_ep(args, cfg, local):
     }), flush=True)
 
 
+def run_ep_real(args, cfg, world, rank, local):
+    """The expert-parallel layer across the torchrun ranks, one GPU each (moe_ep_*): every
+    rank holds the workload's N tokens (its own draw) and E / world experts of one shared
+    weight draw, maps every other rank's window through CUDA IPC, and runs each step as
+    moe_ep_layer_forward_overlapped (shared experts on a side stream).  Timed like the main
+    bench: W warm-up steps, K timed steps between a barrier + synchronize on both sides, L2
+    flushed before every step, the max over ranks."""
+    import torch
+    import torch.distributed as dist
+    import dispatch_combine_grouped_b200 as moe
+    from dispatch_combine_grouped_b200 import ep
+    from moe_inputs import make_inputs
+
+    if world < 2 or cfg.E % world:
+        raise SystemExit("--ep-real needs torchrun with 2 or more ranks dividing E")
+    dev = torch.device("cuda", local)
+    rc = cfg.replace(P=world)
+    inp = make_inputs(rc, device=dev)                                     # weights: one draw for all ranks
+    x = make_inputs(rc, device=dev, seed_offset=rank, with_experts=False)["x"]  # tokens: this rank's own
+    E, S = cfg.E, cfg.S
+    owner = inp["expert_owner"]
+    own = owner.cpu().numpy() if owner is not None else np.arange(E) // (E // world)
+    mine = [e for e in range(E) if own[e] == rank]
+    idx = torch.tensor(mine + list(range(E, E + S)), device=dev)
+    w13, w2 = inp["w13"].index_select(0, idx), inp["w2"].index_select(0, idx)
+    del inp["w13"], inp["w2"]
+    torch.cuda.empty_cache()
+    cap = int(-(-cfg.N * cfg.k * min(world, 4) // 128) * 128)   # receive rows per owner: up to 4x the mean
+    window = ep.alloc_window(rc, cap)
+    ws = ep.alloc_ws(rc, cap)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    y = torch.empty_like(x)
+    side = torch.cuda.Stream(device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    dist.barrier()
+    grp, close = ep.ipc_group(rc, cap, window, owner)
+    dist.barrier()
+
+    def step():
+        ep.layer_forward(rc, grp, x, inp["w_gate"], inp["bias"], w13, w2, ws, expert_owner=owner, y=y,
+                         status=status, side_stream=side)
+
+    try:
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        bad = torch.tensor([int(status.item())], device=dev)
+        dist.all_reduce(bad, op=dist.ReduceOp.MAX)
+        if int(bad.item()) != 0:
+            raise SystemExit(f"EP step reported status {int(bad.item())} on some rank")
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            torch.cuda.synchronize()
+            dist.barrier()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            step()
+            b.record()
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        dist.barrier()
+        med = sorted(ms)[len(ms) // 2]
+        slowest = max_over_ranks(med, world, dev)
+        st = torch.tensor([int(status.item())], device=dev)
+        dist.all_reduce(st, op=dist.ReduceOp.MAX)
+        if rank == 0:
+            print(json.dumps({
+                "metric": "MoE-layer tokens/s, expert-parallel across GPUs (moe_ep_layer_forward_overlapped)",
+                "value": whole_job_tokens_per_s(cfg.N, world, slowest), "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": slowest, "higher_is_better": True,
+                "scaling": "weak", "dtype": cfg.dtype, "data": "synthetic",
+                "config": {"workload": describe(rc), "tokens_per_gpu": cfg.N, "experts_per_gpu": len(mine),
+                           "capacity_rows_per_owner": cap, "l2": "flushed before every step"},
+                "status": int(st.item()),
+            }), flush=True)
+    finally:
+        torch.cuda.synchronize()
+        dist.barrier()
+        close()
+
+
 def run_fp8(args, cfg, world, rank, local):
     """The layer with the FP8 expert path on one stream: route -> layout -> quantise x +
     FP8 permute -> FP8 grouped FFN (FC1, h quantisation, FC2) -> combine.  Weights are
@@ -741,6 +827,11 @@ def main():
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()
+        return
+    if args.ep_real:
+        run_ep_real(args, cfg, world, rank, local)
+        dist.barrier()
+        dist.destroy_process_group()
         return
     if args.ep:
         if rank == 0:
