@@ -440,3 +440,33 @@ def test_ep_with_redundant_expert_slots():
     base = O.ep_layout([ids_all[r * n:(r + 1) * n].cpu().numpy() for r in range(P)], cfg.E, P)
     print("owner receive rows, contiguous:", base["R"].tolist(), "with", R, "copies:", lay["R"].tolist())
     assert lay["R"].max() <= base["R"].max()
+
+
+@pytest.mark.parametrize("cfg", [
+    small_config("ep_p32", cfg_id=111, N=32 * 24, d=128, E=64, S=1, k=4, I=64, P=32),
+    small_config("ep_e512", cfg_id=112, N=256, d=128, E=512, S=0, k=8, I=64, P=8),
+], ids=["P32", "E512"])
+def test_ep_at_size_limits(cfg):
+    """The largest rank count (P = 32) and the largest expert-slot count (E = 512, ids and
+    gates given directly, as a caller mapping to physical slots would): EP layout and
+    windows against the oracle, y bit-identical to the one-GPU steps on the same ids."""
+    inp = gpu_inputs(cfg)
+    P, n = cfg.P, cfg.N // cfg.P
+    g = torch.Generator(device="cuda").manual_seed(cfg.cfg_id)
+    ids_all = torch.stack([torch.randperm(cfg.E, generator=g, device="cuda")[:cfg.k] for _ in range(cfg.N)])
+    ids_all = ids_all.to(torch.int32).contiguous()
+    w_all = torch.rand(cfg.N, cfg.k, generator=g, device="cuda")
+    ids = [ids_all[r * n:(r + 1) * n].contiguous() for r in range(P)]
+    w = [w_all[r * n:(r + 1) * n].contiguous() for r in range(P)]
+    em = Emulated(cfg, [n] * P)
+    res = em.step(inp, ids=ids, w=w)
+    assert int(em.status.item()) == 0
+    lay = O.ep_layout([i.cpu().numpy() for i in ids], cfg.E, P, None, em.capacity)
+    check_handles(em, lay)
+    check_windows(em, res, lay)
+    lay1 = moe.dispatch_layout(cfg, ids_all)
+    xp = moe.permute(cfg, lay1, inp["x"])
+    _, out = moe.grouped_ffn(cfg, lay1, xp, inp["x"], inp["w13"], inp["w2"], topk_w=w_all)
+    y1 = moe.combine(cfg, lay1, out)
+    torch.cuda.synchronize()
+    assert torch.equal(res["y"], y1)
