@@ -278,6 +278,20 @@ def dispatch_layout(ids, E: int, P: int, expert_owner=None, S: int = 0) -> dict:
                 row2tok=row2tok, tile_off=tile_off)
 
 
+def _ep_receive_lists(flats, owner, E: int, P: int) -> list:
+    """Owner j's receive rows as (source i, local a): the experts j owns in ascending id,
+    each expert's assignments from source 0, then source 1, ..., each source's in ascending
+    local index a ([DeepEP] §2: blocks arrive in source order; the expert-local order is
+    ascending (t, slot))."""
+    recv = [[] for _ in range(P)]
+    for e in range(E):
+        j = int(owner[e])
+        for i, f in enumerate(flats):
+            for a in np.flatnonzero(f == e):
+                recv[j].append((i, int(a)))
+    return recv
+
+
 def ep_layout(ids_per_rank, E: int, P: int, expert_owner=None, capacity=None) -> dict:
     """The dispatch across P ranks, each rank one source of tokens and the owner of some
     experts ([EP-DeepEP] §3: tokens go to the owner of their expert and come back to
@@ -303,12 +317,7 @@ def ep_layout(ids_per_rank, E: int, P: int, expert_owner=None, capacity=None) ->
     for i, f in enumerate(flats):
         kept = f[f >= 0]
         cnt[i] = np.bincount(kept, minlength=E)[:E]
-    recv = [[] for _ in range(P)]
-    for e in range(E):
-        j = int(owner[e])
-        for i, f in enumerate(flats):
-            for a in np.flatnonzero(f == e):
-                recv[j].append((i, int(a)))
+    recv = _ep_receive_lists(flats, owner, E, P)
     R = np.array([len(r) for r in recv], dtype=np.int64)
     cap = int(capacity) if capacity is not None else max(int(R.max()), 1)
     dest = [np.full(len(f), -1, dtype=np.int64) for f in flats]

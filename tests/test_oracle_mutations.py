@@ -184,3 +184,43 @@ def test_dropped_rows_leaking_into_combine_are_caught(monkeypatch):
         return orig(o_rows, lay, gates, N, k, shared_out)
     monkeypatch.setattr(O, "combine", leaky)
     _fails(cap_pins.check_layout_path_with_drops, 0.8)
+
+
+# ---- the expert-parallel receive order (oracle.ep_layout): each planted order mistake
+# must fail one of the EP pins in tests/test_ep_oracle.py
+import tests.test_ep_oracle as ep_pins  # noqa: E402
+
+
+def _ep_pins_fail():
+    failed = 0
+    for check, args in [(ep_pins.test_worked_example_two_ranks, ()),
+                        (ep_pins.test_equal_shards_match_one_gpu_layout, (1,)),
+                        (ep_pins.test_equal_shards_match_one_gpu_layout, (4,)),
+                        (ep_pins.test_unequal_shards_and_capacity, (0,))]:
+        try:
+            check(*args)
+        except AssertionError:
+            failed += 1
+    return failed
+
+
+def _receive_lists(order_sources, order_experts, order_a):
+    def lists(flats, owner, E, P):
+        recv = [[] for _ in range(P)]
+        for e in order_experts(range(E)):
+            for i, f in order_sources(list(enumerate(flats))):
+                for a in order_a(np.flatnonzero(f == e)):
+                    recv[int(owner[e])].append((i, int(a)))
+        return recv
+    return lists
+
+
+@pytest.mark.parametrize("name,mut", [
+    ("sources reversed", _receive_lists(lambda s: s[::-1], lambda e: e, lambda a: a)),
+    ("experts descending", _receive_lists(lambda s: s, lambda e: list(e)[::-1], lambda a: a)),
+    ("local index descending", _receive_lists(lambda s: s, lambda e: e, lambda a: a[::-1])),
+])
+def test_ep_receive_order_mistakes_are_caught(monkeypatch, name, mut):
+    assert _ep_pins_fail() == 0, "the unmodified oracle passes its EP pins"
+    monkeypatch.setattr(O, "_ep_receive_lists", mut)
+    assert _ep_pins_fail() >= 1, name
