@@ -140,7 +140,7 @@ def _agree(values: dict, process_group=None) -> list:
     world = dist.get_world_size(process_group)
     got = [None] * world
     dist.all_gather_object(got, values, group=process_group)
-    keys = [k for k in values if k not in ("rank", "handle", "offset")]
+    keys = [k for k in values if k not in ("rank", "handle", "offset", "error")]
     for r, v in enumerate(got):
         for k in keys:
             if v[k] != values[k]:
@@ -150,16 +150,49 @@ def _agree(values: dict, process_group=None) -> list:
     return got
 
 
-def exchange_windows(cfg, capacity: int, rank: int, handle: bytes, offset: int, process_group=None) -> list:
+def exchange_windows(cfg, capacity: int, rank: int, handle, offset: int, process_group=None,
+                     error: str | None = None) -> list:
     """Gather every rank's (IPC handle, offset) after checking that all ranks agree on the
-    shapes that fix the window layout (P, E, d, dtype, S, capacity).  Host logic only."""
+    shapes that fix the window layout (P, E, d, dtype, S, capacity).  A rank that could not
+    get its handle passes error=...: every rank then raises with it.  Host logic only."""
     c = B.c_config(cfg)
     mine = dict(rank=rank, P=c.P, E=c.E, d=c.d, dtype=c.dtype, S=c.n_shared, capacity=capacity,
-                handle=bytes(handle), offset=int(offset))
+                handle=bytes(handle) if handle is not None else None, offset=int(offset), error=error)
     got = _agree(mine, process_group)
+    errors = [g["error"] for g in got if g["error"]]
+    if errors:
+        raise RuntimeError("; ".join(errors))
     if len(got) != c.P:
         raise ValueError(f"process group has {len(got)} ranks, the configuration P = {c.P}")
     return [(g["handle"], g["offset"]) for g in got]
+
+
+def map_windows(table, rank: int, own_ptr: int, open_fn, close_fn, process_group=None):
+    """Map every other rank's window: open_fn(handle, offset) -> address (raises on
+    failure), close_fn(address, offset) unmaps.  Collective: every rank learns whether
+    every rank mapped every window, and if one failed all ranks unmap what they mapped and
+    raise, so that no rank goes on to a collective the others have abandoned.  Returns
+    (addresses in rank order, [(address, offset) opened here])."""
+    import torch.distributed as dist
+    ptrs, opened, failed = [], [], None
+    for r, (hb, o) in enumerate(table):
+        if r == rank:
+            ptrs.append(own_ptr)
+            continue
+        try:
+            p = open_fn(hb, o)
+        except Exception as e:  # noqa: BLE001  (reported to every rank below)
+            failed = f"rank {rank} could not map the window of rank {r}: {e}"
+            break
+        opened.append((p, o))
+        ptrs.append(p)
+    reports = [None] * dist.get_world_size(process_group)
+    dist.all_gather_object(reports, failed, group=process_group)
+    if any(reports):
+        for p, o in opened:
+            close_fn(p, o)
+        raise RuntimeError("; ".join(m for m in reports if m))
+    return ptrs, opened
 
 
 def ipc_group(cfg, capacity: int, window: torch.Tensor, expert_owner=None, process_group=None):
@@ -171,23 +204,22 @@ def ipc_group(cfg, capacity: int, window: torch.Tensor, expert_owner=None, proce
     rank = dist.get_rank(process_group)
     h = (ctypes.c_char * 64)()
     off = ctypes.c_size_t(0)
-    B._check(lib.moe_ep_ipc_handle(ctypes.c_void_p(window.data_ptr()), h, ctypes.byref(off)), "moe_ep_ipc_handle")
-    table = exchange_windows(cfg, capacity, rank, bytes(h), off.value, process_group)
-    ptrs, opened = [], []
-    try:
-        for r, (hb, o) in enumerate(table):
-            if r == rank:
-                ptrs.append(window.data_ptr())
-                continue
-            buf = (ctypes.c_char * 64).from_buffer_copy(hb)
-            p = ctypes.c_void_p(0)
-            B._check(lib.moe_ep_ipc_open(buf, o, ctypes.byref(p)), "moe_ep_ipc_open")
-            opened.append((p.value, o))
-            ptrs.append(p.value)
-    except Exception:
-        for p, o in opened:
-            lib.moe_ep_ipc_close(ctypes.c_void_p(p), o)
-        raise
+    err = None
+    if lib.moe_ep_ipc_handle(ctypes.c_void_p(window.data_ptr()), h, ctypes.byref(off)) != B.MOE_OK:
+        err = f"rank {rank}: moe_ep_ipc_handle: {lib.moe_last_error().decode()}"
+    table = exchange_windows(cfg, capacity, rank, None if err else bytes(h), off.value, process_group, error=err)
+
+    def open_fn(hb, o):
+        buf = (ctypes.c_char * 64).from_buffer_copy(hb)
+        p = ctypes.c_void_p(0)
+        if lib.moe_ep_ipc_open(buf, o, ctypes.byref(p)) != B.MOE_OK:
+            raise RuntimeError(lib.moe_last_error().decode())
+        return p.value
+
+    def close_fn(p, o):
+        lib.moe_ep_ipc_close(ctypes.c_void_p(p), o)
+
+    ptrs, opened = map_windows(table, rank, window.data_ptr(), open_fn, close_fn, process_group)
 
     def close():
         for p, o in opened:
