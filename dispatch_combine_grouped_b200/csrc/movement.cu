@@ -234,7 +234,9 @@ __global__ void __launch_bounds__(kMoveWarps * 32) combine_kernel(const uint4* _
 }
 
 // The combine with 32-byte vectors (rows whose size is a multiple of 32 bytes): one
-// vector per lane per item, k (+S) loads in flight per lane.
+// vector per lane per item, k (+S) loads in flight per lane; grid-stride over items with
+// a grid of a few CTAs per SM (measured 10-16% faster on B200 than one short-lived CTA
+// per 8 items).
 template <typename T>
 __global__ void __launch_bounds__(kMoveWarps * 32) combine_kernel32(const V32* __restrict__ routed,
                                                                      const V32* __restrict__ shared,
@@ -244,61 +246,62 @@ __global__ void __launch_bounds__(kMoveWarps * 32) combine_kernel32(const V32* _
                                                                      int vpr) {
   const int lane = threadIdx.x & 31;
   const int chunks = (vpr + 31) / 32;
-  const long long item = (long long)blockIdx.x * kMoveWarps + (threadIdx.x >> 5);
-  if (item >= (long long)N * chunks) return;
-  const int t = (int)(item / chunks);
-  const int v = (int)(item - (long long)t * chunks) * 32 + lane;
-  const int my_row = lane < k ? map[(size_t)t * k + lane] : 0;
-  const float my_g = (lane < k && gates) ? gates[(size_t)t * k + lane] : 1.0f;
-  int rows[kMaxK];
-  float gs[kMaxK];
+  for (long long item = (long long)blockIdx.x * kMoveWarps + (threadIdx.x >> 5); item < (long long)N * chunks;
+       item += (long long)gridDim.x * kMoveWarps) {
+    const int t = (int)(item / chunks);
+    const int v = (int)(item - (long long)t * chunks) * 32 + lane;
+    const int my_row = lane < k ? map[(size_t)t * k + lane] : 0;
+    const float my_g = (lane < k && gates) ? gates[(size_t)t * k + lane] : 1.0f;
+    int rows[kMaxK];
+    float gs[kMaxK];
 #pragma unroll
-  for (int j = 0; j < kMaxK; ++j) {
-    rows[j] = __shfl_sync(0xffffffffu, my_row, j);
-    gs[j] = __shfl_sync(0xffffffffu, my_g, j);
-  }
-  if (v >= vpr) return;
-  V32 q[kMaxK];
-#pragma unroll
-  for (int j = 0; j < kMaxK; ++j)
-    if (j < k && rows[j] >= 0) q[j] = ld_stream32(routed + (size_t)rows[j] * vpr + v);
-  constexpr int n = Vec<T>::n;  // elements per 16 bytes
-  float acc[2 * 8];
-#pragma unroll
-  for (int i = 0; i < 2 * n; ++i) acc[i] = 0.f;
-#pragma unroll
-  for (int j = 0; j < kMaxK; ++j) {
-    if (j < k && rows[j] >= 0) {  // a dropped assignment adds nothing
-      float f[8];
-      Vec<T>::unpack(make_uint4(q[j].w[0], q[j].w[1], q[j].w[2], q[j].w[3]), f);
-#pragma unroll
-      for (int i = 0; i < n; ++i) acc[i] = fmaf(gs[j], f[i], acc[i]);
-      Vec<T>::unpack(make_uint4(q[j].w[4], q[j].w[5], q[j].w[6], q[j].w[7]), f);
-#pragma unroll
-      for (int i = 0; i < n; ++i) acc[n + i] = fmaf(gs[j], f[i], acc[n + i]);
+    for (int j = 0; j < kMaxK; ++j) {
+      rows[j] = __shfl_sync(0xffffffffu, my_row, j);
+      gs[j] = __shfl_sync(0xffffffffu, my_g, j);
     }
-  }
-  for (int s = 0; s < S; ++s) {
-    const V32 sv = ld_stream32(shared + ((size_t)s * N + t) * vpr + v);
-    float f[8];
-    Vec<T>::unpack(make_uint4(sv.w[0], sv.w[1], sv.w[2], sv.w[3]), f);
+    if (v >= vpr) continue;
+    V32 q[kMaxK];
 #pragma unroll
-    for (int i = 0; i < n; ++i) acc[i] += f[i];
-    Vec<T>::unpack(make_uint4(sv.w[4], sv.w[5], sv.w[6], sv.w[7]), f);
+    for (int j = 0; j < kMaxK; ++j)
+      if (j < k && rows[j] >= 0) q[j] = ld_stream32(routed + (size_t)rows[j] * vpr + v);
+    constexpr int n = Vec<T>::n;  // elements per 16 bytes
+    float acc[2 * 8];
 #pragma unroll
-    for (int i = 0; i < n; ++i) acc[n + i] += f[i];
-  }
-  float lo[8], hi[8];
+    for (int i = 0; i < 2 * n; ++i) acc[i] = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    lo[i] = i < n ? acc[i] : 0.f;
-    hi[i] = i < n ? acc[n + i] : 0.f;
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j < k && rows[j] >= 0) {  // a dropped assignment adds nothing
+        float f[8];
+        Vec<T>::unpack(make_uint4(q[j].w[0], q[j].w[1], q[j].w[2], q[j].w[3]), f);
+#pragma unroll
+        for (int i = 0; i < n; ++i) acc[i] = fmaf(gs[j], f[i], acc[i]);
+        Vec<T>::unpack(make_uint4(q[j].w[4], q[j].w[5], q[j].w[6], q[j].w[7]), f);
+#pragma unroll
+        for (int i = 0; i < n; ++i) acc[n + i] = fmaf(gs[j], f[i], acc[n + i]);
+      }
+    }
+    for (int s = 0; s < S; ++s) {
+      const V32 sv = ld_stream32(shared + ((size_t)s * N + t) * vpr + v);
+      float f[8];
+      Vec<T>::unpack(make_uint4(sv.w[0], sv.w[1], sv.w[2], sv.w[3]), f);
+#pragma unroll
+      for (int i = 0; i < n; ++i) acc[i] += f[i];
+      Vec<T>::unpack(make_uint4(sv.w[4], sv.w[5], sv.w[6], sv.w[7]), f);
+#pragma unroll
+      for (int i = 0; i < n; ++i) acc[n + i] += f[i];
+    }
+    float lo[8], hi[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      lo[i] = i < n ? acc[i] : 0.f;
+      hi[i] = i < n ? acc[n + i] : 0.f;
+    }
+    const uint4 a = Vec<T>::pack(lo), b = Vec<T>::pack(hi);
+    V32 o;
+    o.w[0] = a.x; o.w[1] = a.y; o.w[2] = a.z; o.w[3] = a.w;
+    o.w[4] = b.x; o.w[5] = b.y; o.w[6] = b.z; o.w[7] = b.w;
+    st32(y + (size_t)t * vpr + v, o);
   }
-  const uint4 a = Vec<T>::pack(lo), b = Vec<T>::pack(hi);
-  V32 o;
-  o.w[0] = a.x; o.w[1] = a.y; o.w[2] = a.z; o.w[3] = a.w;
-  o.w[4] = b.x; o.w[5] = b.y; o.w[6] = b.z; o.w[7] = b.w;
-  st32(y + (size_t)t * vpr + v, o);
 }
 
 static inline int elem_bytes(const moe_config& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
@@ -344,7 +347,8 @@ static void combine_launch(const moe_config& c, const uint4* routed, const uint4
   if (row_bytes % 32 == 0) {
     const int vpr32 = row_bytes / 32;
     const long long items = (long long)c.N * ((vpr32 + 31) / 32);
-    combine_kernel32<T><<<blocks_for(items), kMoveWarps * 32, 0, st>>>(
+    const long long nb = blocks_for(items), cap = 4LL * sm_count();  // grid-stride: 4 CTAs per SM
+    combine_kernel32<T><<<(unsigned)(nb < cap ? nb : cap), kMoveWarps * 32, 0, st>>>(
         reinterpret_cast<const V32*>(routed), reinterpret_cast<const V32*>(shared), map, gates,
         reinterpret_cast<V32*>(y), c.N, c.k, c.n_shared, vpr32);
     return;
