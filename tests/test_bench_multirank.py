@@ -7,6 +7,8 @@ import sys
 import pytest
 import torch.multiprocessing as mp
 
+from tests.ports import free_port
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
@@ -26,7 +28,7 @@ def _rank(rank, world, port, out):
 
 
 def test_max_over_ranks_and_whole_job_rate_gloo():
-    world, port = 2, 29517 + os.getpid() % 1000
+    world, port = 2, free_port()
     with mp.Manager() as m:
         out = m.dict()
         mp.spawn(_rank, args=(world, port, out), nprocs=world, join=True)

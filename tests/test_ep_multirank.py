@@ -10,6 +10,8 @@ import sys
 
 import torch.multiprocessing as mp
 
+from tests.ports import free_port
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
@@ -35,7 +37,7 @@ def _rank(rank, world, port, out, case):
 
 
 def _run(case):
-    world, port = 2, 29617 + os.getpid() % 1000 + hash(case) % 50
+    world, port = 2, free_port()
     with mp.Manager() as m:
         out = m.dict()
         mp.spawn(_rank, args=(world, port, out, case), nprocs=world, join=True)
@@ -97,7 +99,7 @@ def _map_rank(rank, world, port, out, case):
 
 
 def _run_map(case):
-    world, port = 2, 29667 + os.getpid() % 1000 + hash(case) % 50
+    world, port = 2, free_port()
     with mp.Manager() as m:
         out = m.dict()
         mp.spawn(_map_rank, args=(world, port, out, case), nprocs=world, join=True)

@@ -14,6 +14,8 @@ import sys
 import pytest
 import torch.multiprocessing as mp
 
+from tests.ports import free_port
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 pytestmark = pytest.mark.gpu
@@ -82,7 +84,7 @@ def _proc(rank, port, out):
 
 
 def test_ipc_mapped_window_receives_counts_and_rows():
-    port = 29717 + os.getpid() % 1000
+    port = free_port()
     ctx = mp.get_context("spawn")
     with ctx.Manager() as m:
         out = m.dict()
