@@ -52,7 +52,7 @@ typedef struct CUstream_st* moe_stream_t; /* same type as cudaStream_t */
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1, /* NULL pointer, negative or inconsistent size */
-  MOE_ERR_UNSUPPORTED = 2, /* valid request outside the sizes this build supports */
+  MOE_ERR_UNSUPPORTED = 2, /* valid request outside the sizes this library supports */
   MOE_ERR_WORKSPACE = 3,   /* workspace smaller than the matching *_workspace_bytes() */
   MOE_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed (launch, tensor map) */
   MOE_ERR_BAD_INDEX = 5,   /* device: an expert id outside [0, E) (other than -1) was seen */
