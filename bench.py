@@ -16,7 +16,6 @@ import argparse
 import hashlib
 import json
 import os
-import subprocess
 import sys
 import time
 

@@ -17,7 +17,6 @@ from __future__ import annotations
 
 import dataclasses
 import math
-from typing import Optional
 
 import torch
 

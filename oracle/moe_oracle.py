@@ -48,7 +48,6 @@ Readings where the pages are silent (each is listed in the design notes):
 from __future__ import annotations
 
 import itertools
-import math
 
 import numpy as np
 

@@ -12,7 +12,6 @@ import os
 
 import numpy as np
 import pytest
-import torch
 
 from moe_inputs import make_inputs, small_config
 from oracle import eplb as EP

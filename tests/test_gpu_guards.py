@@ -6,7 +6,6 @@ covered.
 """
 import math
 
-import numpy as np
 import pytest
 import torch
 

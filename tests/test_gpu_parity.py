@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import dispatch_combine_grouped_b200 as moe
-from moe_inputs import CONFIGS, MoEConfig, small_config
+from moe_inputs import CONFIGS, small_config
 from oracle import moe_oracle as O
 from tests.gpu_cases import (assert_close_fro, assert_close_rel, assert_layout_equal, check_route, gpu_inputs,
                              layout_to_numpy, run_steps)
