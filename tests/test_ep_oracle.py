@@ -99,3 +99,31 @@ def test_unequal_shards_and_capacity(seed):
         assert got == list(range(received))
     assert np.array_equal(lay["cnt"].sum(axis=0),
                           np.bincount(np.concatenate([x.reshape(-1) for x in ids]), minlength=E))
+
+
+def test_cross_rank_volume_matches_the_pages_estimate():
+    """ep_deepep explainer, the EP communication estimate: with experts spread evenly over P
+    ranks and routing independent of the token's rank, a fraction (P-1)/P of each rank's
+    k assignments per token leaves the rank, each way.  Uniform random routing on 8 ranks."""
+    rng = np.random.default_rng(7)
+    P, E, k, n = 8, 64, 6, 512
+    ids = [np.stack([rng.choice(E, size=k, replace=False) for _ in range(n)]) for _ in range(P)]
+    lay = O.ep_layout(ids, E, P)
+    cap = lay["capacity"]
+    for r in range(P):
+        dest = lay["dest"][r]
+        leaving = int(((dest >= 0) & (dest // cap != r)).sum())   # rows the oracle sends to other owners
+        assert abs(leaving / (n * k) - (P - 1) / P) < 0.03
+    # and every assignment is received exactly once
+    assert int(lay["R"].sum()) == P * n * k
+
+
+def test_wide_ep_slot_arithmetic():
+    """Wide EP page, 'why make EP wide': 256 experts + 32 redundant copies = 288 slots, 9 per
+    rank on 32 ranks; the oracle's placement gives every owner exactly that many slots."""
+    from oracle import eplb as L
+    load = np.random.default_rng(3).integers(1, 1000, size=256)
+    plan = L.plan(load, R=32, P=32)
+    assert len(plan["slot_expert"]) == 288
+    assert np.bincount(plan["slot_owner"], minlength=32).tolist() == [9] * 32
+    assert sorted(np.bincount(plan["slot_expert"], minlength=256).tolist())[-1] >= 2  # hot experts copied
