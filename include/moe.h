@@ -519,6 +519,16 @@ moe_status moe_layer_forward_fp8_overlapped(const moe_config* cfg, const void* x
  * another rank's window only after that rank's previous step has finished with the
  * buffer it writes, so one window serves every step.  moe_ep_layer_forward runs the
  * router and the five calls in this order.  The calls of one step take the same ws.
+ *
+ * Errors (host, before any launch): grp or grp->windows NULL, rank outside [0, P),
+ * local_experts outside [0, E], a window that is NULL or not 256-byte aligned, a NULL
+ * array the call needs -> MOE_ERR_INVALID_ARG; capacity < 1, capacity * P >= 2^31 or
+ * capacity + S*N >= 2^30 -> MOE_ERR_UNSUPPORTED; ws smaller than the matching
+ * moe_ep_workspace_bytes*() -> MOE_ERR_WORKSPACE; plus the moe_config checks.  On the
+ * device (*dev_status): an expert id outside [0, E) other than -1 or an owner outside
+ * [0, P) -> MOE_ERR_BAD_INDEX; a rank owning another number of experts than
+ * local_experts -> MOE_ERR_INVALID_ARG; a routing that overflows capacity ->
+ * MOE_ERR_WORKSPACE; a wait that ran out -> MOE_ERR_TIMEOUT.
  * ========================================================================== */
 
 typedef struct {
