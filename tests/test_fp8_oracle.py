@@ -77,3 +77,46 @@ def test_gemm_is_the_product_of_the_dequantised_operands():
     np.testing.assert_allclose(d, brute, rtol=1e-12, atol=1e-12)
     # and close to the unquantised product (relative error of e4m3 operands)
     assert np.linalg.norm(d - a @ b.T) / np.linalg.norm(a @ b.T) < 0.05
+
+
+def test_fp8_ffn_equals_the_bf16_oracle_when_quantisation_is_exact():
+    """The FP8 expert FFN (fc1 then fc2) reduces to the float64 SwiGLU expert of the main
+    oracle when every operand is an e4m3 value under a scale of 1: then the codes carry the
+    values exactly and only the operand path differs (codes + scales vs plain floats)."""
+    from oracle import moe_oracle as O
+    rng = np.random.default_rng(0)
+    finite = F.e4m3_decode(np.arange(0x00, 0x7F))        # every finite non-negative e4m3 value
+    small = finite[(finite > 0) & (finite <= 2.0)]
+    R, d, I = 5, 32, 16
+
+    def pick(shape):
+        v = rng.choice(small, size=shape) * rng.choice([-1.0, 1.0], size=shape)
+        return v, F.e4m3_encode(v)
+
+    x, qx = pick((R, d))
+    w13, qw13 = pick((2 * I, d))
+    w2, qw2 = pick((d, I))
+    h = F.fc1(qx, np.ones(R), qw13, np.ones(2 * I), I)
+    assert np.allclose(h, O.silu(x @ w13[:I].T) * (x @ w13[I:].T), rtol=1e-15, atol=0)
+    # FC2 on an h that is itself exactly representable, then the whole expert
+    hv, qh = pick((R, I))
+    np.testing.assert_allclose(F.fc2(qh, np.ones(R), qw2, np.ones(d)), hv @ w2.T, rtol=1e-15, atol=0)
+    y_ref = O.swiglu_expert(x, w13, w2)
+    np.testing.assert_allclose(h @ w2.T, y_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_fp8_gemm_scale_properties():
+    """Properties of a scaled product that a transposed, dropped or misplaced scale breaks:
+    swapping the operands transposes the result, and doubling one row's scale doubles
+    exactly that row."""
+    rng = np.random.default_rng(1)
+    qa = rng.integers(0, 0x7F, size=(4, 8)).astype(np.uint8)
+    qb = rng.integers(0, 0x7F, size=(3, 8)).astype(np.uint8)
+    sa, sb = rng.uniform(0.5, 2.0, 4), rng.uniform(0.5, 2.0, 3)
+    d = F.gemm_rows(qa, sa, qb, sb)
+    np.testing.assert_allclose(F.gemm_rows(qb, sb, qa, sa), d.T, rtol=1e-15)
+    sa2 = sa.copy()
+    sa2[2] *= 2
+    d2 = F.gemm_rows(qa, sa2, qb, sb)
+    np.testing.assert_allclose(d2[2], 2 * d[2], rtol=1e-15)
+    np.testing.assert_array_equal(np.delete(d2, 2, axis=0), np.delete(d, 2, axis=0))
