@@ -1,14 +1,18 @@
 """Benchmark: one MoE layer forward (router -> top-k -> dispatch layout -> permute ->
 grouped SwiGLU experts -> combine) per step, on synthetic seeded inputs.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload fine] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wide] [--impl reference]
 
-Default workload: the fine-grained MoE layer (N=4096 tokens, d=2048, 64 routed + 2
-shared experts, top-6, I=1408, bf16).  Each step runs through the library's C ABI;
-inputs are resident in HBM when the timed region starts and L2 is flushed (a 256 MiB
-write) before every step, outside the step's CUDA-event bracket.  Under torchrun each
-rank runs its own independent batch (weak scaling, no collective on the data path);
-the time is the max over ranks.  Prints one JSON line on rank 0.
+Default workload: the wide-expert prefill layer (N=8192 tokens, d=7168, 256 routed + 1
+shared expert, top-8 of 4 of 8 groups, I=2048, bf16), the largest single-GPU workload and
+the one the grouped-GEMM target is stated on.  Each step runs through the library's C
+ABI; inputs are resident in HBM when the timed region starts and L2 is flushed (a 256 MiB
+write) before every step, outside the step's CUDA-event bracket.  On one GPU the default
+run then measures the other workloads (fine, decode, hot, hot_cal, tiny) the same way,
+with fewer steps, and reports each one's times, rates and roofline fractions under
+"workloads".  Under torchrun each rank runs its own independent batch (weak scaling, no
+collective on the data path); the time is the max over ranks.  Prints one JSON line on
+rank 0.
 """
 from __future__ import annotations
 
@@ -33,7 +37,9 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="fine")
+    ap.add_argument("--workload", default="wide")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-workload summary of the other workloads (one GPU, default workload)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -76,6 +82,45 @@ def algorithmic(cfg, n_e_touched=None):
         combine_bytes=(A + S * N + N) * d * b,
         router_flops=2.0 * N * d * E,
     )
+
+
+SPEC_BF16_TFLOPS = 2250.0   # B200 dense bf16 tensor rate (nominal, no sparsity)
+SPEC_SM_MHZ = 1965.0        # the SM clock that nominal rate is quoted at (clocks.max.sm)
+
+
+def config_dict(cfg, world: int) -> dict:
+    """The workload description both arms print (identical keys, so the lines compare)."""
+    return {"workload": describe(cfg), "tokens_per_gpu": cfg.N,
+            "l2": "flushed before every step (256 MiB write, outside the step's event bracket)",
+            "parallelism": f"{world} independent replicas (one batch per GPU)"}
+
+
+def touched_weight_bytes(cfg, touched: int) -> float:
+    """W13 and W2 bytes of the experts that received rows plus the shared experts."""
+    b = 2 if cfg.dtype == "bf16" else 4
+    return (touched + cfg.S) * 3.0 * cfg.d * cfg.I * b
+
+
+def roofline_layer_ms(cfg, touched: int, hbm_gbs: float, tensor_tflops: float) -> dict:
+    """Roofline time of each step of one layer and their sum: the router, permute and
+    combine at HBM bandwidth (their algorithmic bytes), the FFN at the slower of its FLOPs
+    at the tensor peak and its touched weight bytes at HBM bandwidth."""
+    alg = algorithmic(cfg, touched)
+    b = 2 if cfg.dtype == "bf16" else 4
+    bw = hbm_gbs * 1e9
+    router_bytes = (cfg.N * cfg.d + cfg.E * cfg.d) * b + cfg.N * cfg.E * 4 + cfg.N * cfg.k * 8
+    ffn_tc = alg["ffn_flops"] / (tensor_tflops * 1e12)
+    ffn_hbm = touched_weight_bytes(cfg, touched) / bw
+    parts = {"router": max(router_bytes / bw, alg["router_flops"] / (tensor_tflops * 1e12)),
+             "permute": alg["permute_bytes"] / bw, "ffn": max(ffn_tc, ffn_hbm),
+             "combine": alg["combine_bytes"] / bw}
+    return {"ms": 1e3 * sum(parts.values()), "parts_ms": {k: 1e3 * v for k, v in parts.items()},
+            "ffn_bound": "tensor" if ffn_tc >= ffn_hbm else "hbm"}
+
+
+def spec_at_clock(sm_mhz) -> float:
+    """The nominal dense bf16 rate scaled to the SM clock the kernels ran at."""
+    return SPEC_BF16_TFLOPS * (float(sm_mhz) / SPEC_SM_MHZ if sm_mhz else 1.0)
 
 
 def load_peaks():
@@ -205,75 +250,116 @@ def whole_job_tokens_per_s(tokens_per_rank: int, world: int, slowest_ms_per_step
 
 
 # ------------------------------------------------------------------------------ oracle arm
-def oracle_tokens_per_s(cfg, seconds, inputs=None):
-    """Time the float64 oracle (as it stands) on consecutive 128-token slices of the
-    workload until about ``seconds`` have passed.  Returns (tokens/s, tokens, seconds, threads,
-    seconds spent in each step of the layer: routing + layout, permute, experts, combine)."""
-    import numpy as np
-    import torch
-    from moe_inputs import make_inputs
+def cpu_slice_tokens(cfg) -> int:
+    """Tokens per oracle slice: the oracle converts every touched expert's weights to
+    float64 once per slice, which dominates on the 7168-wide experts (about 0.15 s per
+    expert), so those workloads take 16-token slices; the others 128."""
+    return min(cfg.N, 16 if cfg.d >= 7168 else 128)
+
+
+def oracle_slice(cfg, inp, s0, n_tok):
+    """The float64 oracle (as it stands) on tokens [s0, s0 + n_tok) of the workload, its
+    layer steps timed one by one in the pages' order.  Returns (tokens, seconds, seconds
+    per step: routing + layout, permute, experts, combine)."""
     from oracle import moe_oracle as O
+    xs = inp["x"][s0:s0 + n_tok]
+    c = cfg.replace(N=xs.shape[0])
+    w13, w2, wg, bias, owner = inp["w13"], inp["w2"], inp["w_gate"], inp["bias"], inp["expert_owner"]
+    ta = time.perf_counter()
+    ids = O.select_experts(O.router_logits(xs, wg, bias), c.k, c.n_groups, c.topk_groups)
+    g = O.gate_weights(O.gate_logits(c, xs, wg, bias), ids, c.score, c.renormalize)
+    lay = O.dispatch_layout(ids, c.E, c.P, owner, c.S)
+    tb = time.perf_counter()
+    xp = O.permute(xs, lay, c.k)
+    tc = time.perf_counter()
+    o = O.experts_on_rows(xp, lay, w13, w2, c.E)
+    shared = [O.swiglu_expert(xs, w13[c.E + s], w2[c.E + s]) for s in range(c.S)]
+    td = time.perf_counter()
+    O.combine(o, lay, g, c.N, c.k, shared)
+    te = time.perf_counter()
+    return xs.shape[0], te - ta, (tb - ta, tc - tb, td - tc, te - td)
+
+
+PHASES = ("routing_layout", "permute", "ffn", "combine")
+
+
+def cpu_inputs(inp):
+    return {k: (t.cpu() if t is not None else None) for k, t in inp.items()}
+
+
+def oracle_tokens_per_s(cfg, seconds, inputs, slice_tokens=None):
+    """Time the oracle on consecutive slices of the workload until about ``seconds`` have
+    passed (at least one slice).  Returns (tokens/s, tokens, seconds, threads, seconds spent
+    in each step of the layer)."""
+    import torch
     threads = len(os.sched_getaffinity(0))
     torch.set_num_threads(threads)
-    inp = inputs if inputs is not None else make_inputs(cfg, device="cpu")
-    w13 = inp["w13"].cpu()
-    w2 = inp["w2"].cpu()
-    x = inp["x"].cpu()
-    owner = inp["expert_owner"].cpu() if inp["expert_owner"] is not None else None
-    bias = inp["bias"].cpu() if inp["bias"] is not None else None
-    n_slice = 128
-    wg = inp["w_gate"].cpu()
-    phases = {"routing_layout": 0.0, "permute": 0.0, "ffn": 0.0, "combine": 0.0}
-    done, t0 = 0, time.perf_counter()
+    n_slice = slice_tokens or cpu_slice_tokens(cfg)
+    phases = dict.fromkeys(PHASES, 0.0)
+    done, el = 0, 0.0
     while True:
-        s0 = done % cfg.N
-        xs = x[s0:s0 + n_slice]
-        c = cfg.replace(N=xs.shape[0])
-        # the oracle's layer (moe_layer), its steps timed one by one in the same order
-        ta = time.perf_counter()
-        ids = O.select_experts(O.router_logits(xs, wg, bias), c.k, c.n_groups, c.topk_groups)
-        g = O.gate_weights(O.gate_logits(c, xs, wg, bias), ids, c.score, c.renormalize)
-        lay = O.dispatch_layout(ids, c.E, c.P, owner, c.S)
-        tb = time.perf_counter()
-        xp = O.permute(xs, lay, c.k)
-        tc = time.perf_counter()
-        o = O.experts_on_rows(xp, lay, w13, w2, c.E)
-        shared = [O.swiglu_expert(xs, w13[c.E + s], w2[c.E + s]) for s in range(c.S)]
-        td = time.perf_counter()
-        O.combine(o, lay, g, c.N, c.k, shared)
-        te = time.perf_counter()
-        for k_, v_ in zip(phases, (tb - ta, tc - tb, td - tc, te - td)):
+        tok, sec, ph = oracle_slice(cfg, inputs, done % cfg.N, n_slice)
+        for k_, v_ in zip(PHASES, ph):
             phases[k_] += v_
-        done += xs.shape[0]
-        el = time.perf_counter() - t0
+        done += tok
+        el += sec
         if el >= seconds:
             return done / el, done, el, threads, {k_: round(v_, 3) for k_, v_ in phases.items()}
 
 
+def cpu_baseline_entry(cfg, seconds, inputs):
+    v, tok, s, threads, phases = oracle_tokens_per_s(cfg, seconds, inputs)
+    return {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{tok} tokens of the workload in {cpu_slice_tokens(cfg)}-token slices, whole layer in "
+                      f"float64, {s:.1f} s", "phases_s": phases}
+
+
 def run_reference(args, cfg, rank):
+    """The reference arm: the float64 oracle as it stands, on the host cores.  Each step
+    is one slice of the workload (its tokens in order, wrapping around), sized so that
+    the W + K steps end within a few minutes; the line reports the steps and tokens that
+    actually ran and their measured time."""
     if rank != 0:
         return
+    import torch
     from moe_inputs import make_inputs
-    inp = make_inputs(cfg, device="cpu")
-    per_step = max(1.0, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    threads = len(os.sched_getaffinity(0))
+    torch.set_num_threads(threads)
+    # the same draw as the GPU arm (its CUDA generators) when a GPU is present
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = cpu_inputs(make_inputs(cfg, device=dev))
+    if dev == "cuda":
+        torch.cuda.empty_cache()
+    # slice size: one trial slice, then scaled so that a step takes about budget seconds
+    budget = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    n = cpu_slice_tokens(cfg)
+    _, t_trial, _ = oracle_slice(cfg, inp, 0, n)
+    n = int(max(1, min(cfg.N, round(n * min(1.0, budget / max(t_trial, 1e-6))))))
+    pos = 0
     for _ in range(args.warmup):
-        oracle_tokens_per_s(cfg, per_step / 4, inp)
-    tot_tok, tot_s, threads, phases = 0, 0.0, 1, {}
+        tok, _, _ = oracle_slice(cfg, inp, pos % cfg.N, n)
+        pos += tok
+    tot_tok, tot_s, phases = 0, 0.0, dict.fromkeys(PHASES, 0.0)
     for _ in range(args.steps):
-        _, tok, s, threads, ph = oracle_tokens_per_s(cfg, per_step, inp)
+        tok, sec, ph = oracle_slice(cfg, inp, pos % cfg.N, n)
+        pos += tok
         tot_tok += tok
-        tot_s += s
-        phases = {k: round(phases.get(k, 0.0) + v, 3) for k, v in ph.items()}
+        tot_s += sec
+        for k_, v_ in zip(PHASES, ph):
+            phases[k_] += v_
     v = tot_tok / tot_s
+    sample = (f"{args.steps} steps of {n} tokens each ({tot_tok} tokens, consecutive slices of the workload), "
+              f"whole layer in float64, {tot_s:.1f} s")
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * cfg.N / v,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": describe(cfg)},
-        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{tot_tok} tokens of the workload in 128-token slices, whole layer in float64",
-                         "phases_s": phases},
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * tot_s / args.steps,
+        "tokens_per_step": n, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded normal inputs, random-init weights)",
+        "config": config_dict(cfg, args.gpus),
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample,
+                         "phases_s": {k: round(x, 3) for k, x in phases.items()}},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": "each step is one bounded slice of the workload (tokens_per_step tokens), not the whole batch",
     }
     print(json.dumps(line), flush=True)
 
@@ -804,48 +890,14 @@ def run_fp8(args, cfg, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def main():
-    args = parse()
-    from moe_inputs import CONFIGS, PROFILE_CASES
-    cfg = CONFIGS[args.workload] if args.workload in CONFIGS else PROFILE_CASES[args.workload]
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
-        return run_reference(args, cfg, rank)
-
+def bench_layer(args, cfg, world, rank, local, steps, warmup, headline=True):
+    """One workload: W warm-up steps, K timed steps (the product's overlapped order, CUDA
+    events between the stages), a one-stream pass for the per-stage breakdown, the movement
+    kernels timed on their own, the fused entry point and (headline only) the end-to-end
+    measurement through the public call; the oracle's CPU baseline on rank 0 at N=1.
+    Returns the JSON line (rank 0) or None."""
     import torch
     import torch.distributed as dist
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    if args.movement_sweep:
-        if rank == 0:
-            run_movement_sweep(args, cfg, local)
-        if world > 1:
-            dist.barrier()
-            dist.destroy_process_group()
-        return
-    if args.ep_real:
-        run_ep_real(args, cfg, world, rank, local)
-        dist.barrier()
-        dist.destroy_process_group()
-        return
-    if args.ep:
-        if rank == 0:
-            run_ep(args, cfg, local)
-        if world > 1:
-            dist.barrier()
-            dist.destroy_process_group()
-        return
-    if args.fp8:
-        run_fp8(args, cfg, world, rank, local)
-        if world > 1:
-            dist.barrier()
-            dist.destroy_process_group()
-        return
-
     import dispatch_combine_grouped_b200 as moe
     from moe_inputs import make_inputs
 
@@ -946,10 +998,10 @@ def main():
         return [torch.cuda.Event(enable_timing=True) for _ in range(7)]
 
     clocks = ClockSampler(local)
-    evs = [new_events() for _ in range(args.steps)]
+    evs = [new_events() for _ in range(steps)]
     clocks.start()
     torch.cuda.nvtx.range_push("warmup")
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush.zero_()
         step(new_events())
     torch.cuda.synchronize()
@@ -960,7 +1012,7 @@ def main():
     torch.cuda.nvtx.range_push("timed")
     clocks.mark_timed()
     wall0 = time.perf_counter()
-    for i in range(args.steps):
+    for i in range(steps):
         flush.zero_()
         step(evs[i])
     torch.cuda.synchronize()
@@ -978,18 +1030,18 @@ def main():
         for j, n in enumerate(names):
             stage_ms[n] += ev[j].elapsed_time(ev[j + 1])
         step_ms += ev[0].elapsed_time(ev[6])
-    step_ms_max = max_over_ranks(step_ms, world, dev) / args.steps
+    step_ms_max = max_over_ranks(step_ms, world, dev) / steps
     for n in names:
-        stage_ms[n] /= args.steps
+        stage_ms[n] /= steps
 
     # diagnostic: the same kernels one after another on one stream (per-stage breakdown)
-    seq_evs = [new_events() for _ in range(args.steps)]
-    for i in range(args.steps):
+    seq_evs = [new_events() for _ in range(steps)]
+    for i in range(steps):
         flush.zero_()
         step_sequential(seq_evs[i])
     torch.cuda.synchronize()
-    seq_ms = {n: sum(ev[j].elapsed_time(ev[j + 1]) for ev in seq_evs) / args.steps for j, n in enumerate(names)}
-    seq_step_ms = sum(ev[0].elapsed_time(ev[6]) for ev in seq_evs) / args.steps
+    seq_ms = {n: sum(ev[j].elapsed_time(ev[j + 1]) for ev in seq_evs) / steps for j, n in enumerate(names)}
+    seq_step_ms = sum(ev[0].elapsed_time(ev[6]) for ev in seq_evs) / steps
 
     # the movement kernels timed on their own (L2 flushed, events around the one launch),
     # after an idle pause: in the steps the GPU runs at its power cap and the SM clock sits
@@ -999,7 +1051,7 @@ def main():
 
     def kernel_ms(fn):
         pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for _ in range(max(args.steps, 5))]
+                 for _ in range(max(steps, 5))]
         for a, b in pairs:
             flush.zero_()
             a.record()
@@ -1011,20 +1063,22 @@ def main():
     permute_ms = kernel_ms(lambda: moe.permute(pcfg, layout, x, out=x_perm))
     combine_ms = kernel_ms(lambda: moe.combine(pcfg, layout, out, y=y))
 
-    # the fused entry point (one C call per step, same kernels and order as the timed step)
-    fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.zero_()
-        fev[i][0].record()
-        moe.layer_forward_overlapped(cfg, x, wg, bias, owner, w13, w2, side, y=y, ws=ws, status=status)
-        fev[i][1].record()
-    torch.cuda.synchronize()
-    fused_ms = sum(a.elapsed_time(b) for a, b in fev) / args.steps
+    fused_ms, e2e_ms = None, None
+    if headline:
+        # the fused entry point (one C call per step, same kernels and order as the timed step)
+        fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            fev[i][0].record()
+            moe.layer_forward_overlapped(cfg, x, wg, bias, owner, w13, w2, side, y=y, ws=ws, status=status)
+            fev[i][1].record()
+        torch.cuda.synchronize()
+        fused_ms = sum(a.elapsed_time(b) for a, b in fev) / steps
 
-    # end to end: pinned host input -> device, layer, result -> pinned host, every step
-    e2e_ms = max_over_ranks(e2e_pipelined(
-        lambda xd, yd: moe.layer_forward_overlapped(cfg, xd, wg, bias, owner, w13, w2, side, y=yd, ws=ws,
-                                                    status=status), x, y, flush, max(args.steps, 8)), world, dev)
+        # end to end: pinned host input -> device, layer, result -> pinned host, every step
+        e2e_ms = max_over_ranks(e2e_pipelined(
+            lambda xd, yd: moe.layer_forward_overlapped(cfg, xd, wg, bias, owner, w13, w2, side, y=yd, ws=ws,
+                                                        status=status), x, y, flush, max(steps, 8)), world, dev)
 
     n_e = layout["n_e"].cpu()
     touched = int((n_e > 0).sum())
@@ -1033,80 +1087,174 @@ def main():
     alg = algorithmic(cfg, touched)
     peaks, peak_src = load_peaks()
     tpeak, tkind = tensor_peak(peaks, clock_rec)
+    sm_mhz = (clock_rec or {}).get("sm_mhz")
+    spec = spec_at_clock(sm_mhz)
     A_rows = cfg.N * cfg.k
     routed_fc1_flops = 4.0 * A_rows * cfg.d * cfg.I
     routed_ffn_flops = 6.0 * A_rows * cfg.d * cfg.I
     fc1_tflops = routed_fc1_flops / (stage_ms["fc1"] / 1e3) / 1e12
-    ffn_seq_tflops = alg["ffn_flops"] / ((seq_ms["fc1"] + seq_ms["fc2"]) / 1e3) / 1e12
+    ffn_seq_ms = seq_ms["fc1"] + seq_ms["fc2"]
+    ffn_seq_tflops = alg["ffn_flops"] / (ffn_seq_ms / 1e3) / 1e12
+    ffn_weight_gbs = touched_weight_bytes(cfg, touched) / (ffn_seq_ms / 1e3) / 1e9
+    roof = roofline_layer_ms(cfg, touched, peaks["hbm_gbs"], tpeak)
     # movement bandwidth from the kernels timed on their own (median launch, full clock)
     permute_gbs = alg["permute_bytes"] / (permute_ms / 1e3) / 1e9
     combine_gbs = alg["combine_bytes"] / (combine_ms / 1e3) / 1e9
     src = source_hash("dispatch_combine_grouped_b200/csrc/gemm_tc.cu", "dispatch_combine_grouped_b200/csrc/gemm_tc2.cu",
                       "dispatch_combine_grouped_b200/csrc/common.cuh")
     traffic = recorded_traffic("fc1_routed", cfg.name, src)
-    tokens_total = cfg.N * world
     value = whole_job_tokens_per_s(cfg.N, world, step_ms_max)
-    gl = 2 if (cfg.dtype == "bf16" and cfg.N > 128 and cfg.d >= 4096) else 1   # pair + tail launches
-    launches_per_step = 2 + 3 + 1 + 2 * gl + (2 * gl if S else 0) + 1 + (4 if R else 0)
+    launches_per_step = kernel_launches_per_step(cfg, R)
     if R:
         R_after = np.diff(layout["recv_off"].cpu().numpy())
         eplb_info["owner_max_over_mean_after"] = float(R_after.max() / R_after.mean())
         eplb_info["note"] = ("stages_ms.layout includes the replica assignment; the fused and e2e "
                              "numbers run the layer without copies")
+    if rank != 0:
+        return None
+    ffn_rec = {"tflops": ffn_seq_tflops, "ms": ffn_seq_ms, "frac_of_peak": ffn_seq_tflops / tpeak, "peak_kind": tkind,
+               "frac_of_burst_peak": ffn_seq_tflops / peaks["bf16_tflops"],
+               "frac_of_sustained_peak": ffn_seq_tflops / peaks["bf16_tflops_sustained"],
+               "frac_of_spec_at_clock": ffn_seq_tflops / spec,
+               "weight_gbs": ffn_weight_gbs, "weight_frac_of_hbm": ffn_weight_gbs / peaks["hbm_gbs"],
+               "bound": roof["ffn_bound"],
+               "frac_of_roofline": roof["parts_ms"]["ffn"] / ffn_seq_ms,
+               "routed_tflops_overlapped": routed_ffn_flops / ((stage_ms["fc1"] + stage_ms["fc2"]) / 1e3) / 1e12}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": step_ms_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded normal inputs, random-init weights)",
+        "config": config_dict(cfg, world),
+        "roofline": {"kernel": "routed grouped FC1 + SwiGLU (tcgen05; CTA-pair and one-CTA tiles)",
+                     "bound": "tensor", "achieved": fc1_tflops, "peak": tpeak, "unit": "TFLOP/s",
+                     "frac": fc1_tflops / tpeak,
+                     "peak_source": f"{peak_src} bf16 {tkind} (median SM clock during the timed steps "
+                                    f"{sm_mhz} MHz)",
+                     "frac_of_burst": fc1_tflops / peaks["bf16_tflops"],
+                     "frac_of_sustained": fc1_tflops / peaks["bf16_tflops_sustained"],
+                     "frac_of_spec_at_clock": fc1_tflops / spec,
+                     "spec_at_clock_tflops": spec,
+                     "traffic": traffic, "flops_per_launch": routed_fc1_flops, "ms_per_launch": stage_ms["fc1"],
+                     "note": "timed inside the step, with the shared experts running on a side stream; "
+                             "frac_of_spec_at_clock divides by 2250 TFLOP/s scaled to the median SM clock"},
+        "layer_roofline": {"ms": roof["ms"], "parts_ms": roof["parts_ms"], "frac": roof["ms"] / step_ms_max,
+                           "how": "router, permute, combine: algorithmic bytes at the measured HBM copy rate; "
+                                  "FFN: max(FLOPs at the tensor peak, touched weight bytes at HBM)"},
+        "stages_ms": stage_ms,
+        "sequential": {"ms_per_step": seq_step_ms, "stages_ms": seq_ms,
+                       "ffn_tflops": ffn_seq_tflops, "ffn_frac_of_peak": ffn_seq_tflops / tpeak},
+        "ffn": ffn_rec,
+        "permute": {"gbs": permute_gbs, "ms": permute_ms, "frac_of_hbm": permute_gbs / peaks["hbm_gbs"],
+                    "frac_of_8tbs": permute_gbs / 8000.0,
+                    "gbs_in_step": alg["permute_bytes"] / (seq_ms["permute"] / 1e3) / 1e9},
+        "combine": {"gbs": combine_gbs, "ms": combine_ms, "frac_of_hbm": combine_gbs / peaks["hbm_gbs"],
+                    "frac_of_8tbs": combine_gbs / 8000.0,
+                    "gbs_in_step": alg["combine_bytes"] / (seq_ms["combine"] / 1e3) / 1e9},
+        "imbalance": {"max_over_mean_n_e": float(n_e.max()) / float(n_e.float().mean()),
+                      "experts_empty": int((n_e == 0).sum()),
+                      "max_over_mean_owner_rows": owner_imb},
+        "gpu_launches": launches_per_step * steps,
+        **({"eplb": eplb_info} if R else {}),
+        "clocks": clock_rec,
+        "wall_s_timed": wall,
+    }
+    if headline:
+        line["fused_ms_per_step"] = fused_ms
+        line["e2e"] = {"value": whole_job_tokens_per_s(cfg.N, world, e2e_ms), "unit": "tokens/s",
+                       "h2d_bytes_per_step": x.numel() * x.element_size(),
+                       "d2h_bytes_per_step": y.numel() * y.element_size(), "ms_per_step": e2e_ms,
+                       "how": "moe_layer_forward_overlapped per step, input copied in from pinned host memory and "
+                              "result copied out, on their own streams so that step i overlaps the copies of "
+                              "steps i+1 and i-1 (two device buffers each way); device-timed from the first "
+                              "copy-in to the last copy-out"}
+    if not args.no_cpu_baseline and world == 1:
+        cpu_s = args.cpu_seconds if headline else min(args.cpu_seconds, 6.0)
+        line["cpu_baseline"] = cpu_baseline_entry(cfg, cpu_s, cpu_inputs(inp))
+    return line
 
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": step_ms_max, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded normal inputs, random-init weights)",
-            "config": {"workload": describe(cfg), "tokens_per_gpu": cfg.N, "l2": "flushed before every step "
-                       "(256 MiB write, outside the step's event bracket)", "parallelism": f"{world} independent "
-                       "replicas (one batch per GPU)"},
-            "roofline": {"kernel": "routed grouped FC1 + SwiGLU (tcgen05)", "bound": "tensor",
-                         "achieved": fc1_tflops, "peak": tpeak, "unit": "TFLOP/s",
-                         "frac": fc1_tflops / tpeak,
-                         "peak_source": f"{peak_src} bf16 {tkind} (median SM clock during the timed steps "
-                                        f"{(clock_rec or {}).get('sm_mhz')} MHz)",
-                         "frac_of_burst": fc1_tflops / peaks["bf16_tflops"],
-                         "frac_of_sustained": fc1_tflops / peaks["bf16_tflops_sustained"],
-                         "traffic": traffic, "flops_per_launch": routed_fc1_flops, "ms_per_launch": stage_ms["fc1"],
-                         "note": "timed inside the step, with the shared experts running on a side stream"},
-            "stages_ms": stage_ms,
-            "sequential": {"ms_per_step": seq_step_ms, "stages_ms": seq_ms,
-                           "ffn_tflops": ffn_seq_tflops, "ffn_frac_of_peak": ffn_seq_tflops / tpeak},
-            "ffn": {"tflops": ffn_seq_tflops, "frac_of_peak": ffn_seq_tflops / tpeak, "peak_kind": tkind,
-                    "frac_of_burst_peak": ffn_seq_tflops / peaks["bf16_tflops"],
-                    "frac_of_sustained_peak": ffn_seq_tflops / peaks["bf16_tflops_sustained"],
-                    "routed_tflops_overlapped": routed_ffn_flops / ((stage_ms["fc1"] + stage_ms["fc2"]) / 1e3) / 1e12},
-            "permute": {"gbs": permute_gbs, "ms": permute_ms, "frac_of_hbm": permute_gbs / peaks["hbm_gbs"],
-                        "frac_of_8tbs": permute_gbs / 8000.0,
-                        "gbs_in_step": alg["permute_bytes"] / (seq_ms["permute"] / 1e3) / 1e9},
-            "combine": {"gbs": combine_gbs, "ms": combine_ms, "frac_of_hbm": combine_gbs / peaks["hbm_gbs"],
-                        "frac_of_8tbs": combine_gbs / 8000.0,
-                        "gbs_in_step": alg["combine_bytes"] / (seq_ms["combine"] / 1e3) / 1e9},
-            "fused_ms_per_step": fused_ms,
-            "imbalance": {"max_over_mean_n_e": float(n_e.max()) / float(n_e.float().mean()),
-                          "experts_empty": int((n_e == 0).sum()),
-                          "max_over_mean_owner_rows": owner_imb},
-            "e2e": {"value": whole_job_tokens_per_s(cfg.N, world, e2e_ms), "unit": "tokens/s",
-                    "h2d_bytes_per_step": x.numel() * x.element_size(),
-                    "d2h_bytes_per_step": y.numel() * y.element_size(), "ms_per_step": e2e_ms,
-                    "how": "moe_layer_forward* per step, input copied in from pinned host memory and result "
-                           "copied out, on their own streams so that step i overlaps the copies of steps "
-                           "i+1 and i-1 (two device buffers each way); device-timed from the first copy-in "
-                           "to the last copy-out"},
-            "gpu_launches": launches_per_step * args.steps,
-            **({"eplb": eplb_info} if R else {}),
-            "clocks": clock_rec,
-            "wall_s_timed": wall,
-        }
-        if not args.no_cpu_baseline and world == 1:
-            v, tok, s, threads, phases = oracle_tokens_per_s(
-                cfg, args.cpu_seconds, {k: (t.cpu() if t is not None else None) for k, t in inp.items()})
-            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                                    "sample": f"{tok} tokens of the workload in 128-token slices, "
-                                              f"whole layer in float64, {s:.1f} s",
-                                    "phases_s": phases}
+
+def kernel_launches_per_step(cfg, R=0):
+    """This library's kernels in one timed step: router (GEMM + top-k), three layout
+    kernels, permute, FC1 and FC2 per group range (a pair-tile and a tail launch each on
+    the CTA-pair path), combine, and the replica assignment's four with redundant slots."""
+    gl = 2 if (cfg.dtype == "bf16" and cfg.N > 128 and cfg.d >= 4096) else 1
+    return 2 + 3 + 1 + 2 * gl + (2 * gl if cfg.S else 0) + 1 + (4 if R else 0)
+
+
+def summarize(line) -> dict:
+    """The per-workload record of the default run's "workloads" field."""
+    keep = {"ms_per_step": line["ms_per_step"], "tokens_per_s": line["value"], "config": line["config"]["workload"],
+            "layer_roofline_ms": line["layer_roofline"]["ms"], "frac_of_layer_roofline": line["layer_roofline"]["frac"],
+            "ffn": {k: line["ffn"][k] for k in ("tflops", "ms", "bound", "frac_of_roofline", "frac_of_burst_peak",
+                                                 "frac_of_sustained_peak", "frac_of_spec_at_clock", "weight_gbs",
+                                                 "weight_frac_of_hbm")},
+            "routed_fc1": {"tflops": line["roofline"]["achieved"], "frac": line["roofline"]["frac"],
+                           "frac_of_burst": line["roofline"]["frac_of_burst"], "traffic": line["roofline"]["traffic"]},
+            "permute": {k: line["permute"][k] for k in ("gbs", "frac_of_hbm", "frac_of_8tbs", "gbs_in_step")},
+            "combine": {k: line["combine"][k] for k in ("gbs", "frac_of_hbm", "frac_of_8tbs", "gbs_in_step")},
+            "imbalance": line["imbalance"], "clocks": line["clocks"], "steps": line["steps"],
+            "gpu_launches": line["gpu_launches"]}
+    if "cpu_baseline" in line:
+        keep["cpu_baseline"] = line["cpu_baseline"]
+    return keep
+
+
+def main():
+    args = parse()
+    from moe_inputs import CONFIGS, PROFILE_CASES
+    cfg = CONFIGS[args.workload] if args.workload in CONFIGS else PROFILE_CASES[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, cfg, rank)
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.movement_sweep:
+        if rank == 0:
+            run_movement_sweep(args, cfg, local)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    if args.ep_real:
+        run_ep_real(args, cfg, world, rank, local)
+        dist.barrier()
+        dist.destroy_process_group()
+        return
+    if args.ep:
+        if rank == 0:
+            run_ep(args, cfg, local)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    if args.fp8:
+        run_fp8(args, cfg, world, rank, local)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    line = bench_layer(args, cfg, world, rank, local, args.steps, args.warmup, headline=True)
+    if line is not None and world == 1 and not args.no_workloads and args.workload == "wide" and not args.eplb:
+        # the other workloads, measured the same way with fewer steps (one GPU only: under
+        # torchrun the ranks would hold all GPUs for the sweep)
+        import torch
+        torch.cuda.empty_cache()
+        sweep = {"wide": summarize(line)}
+        for name in ("fine", "decode", "hot", "hot_cal", "tiny"):
+            w_line = bench_layer(args, CONFIGS[name], world, rank, local, min(args.steps, 10), 3, headline=False)
+            sweep[name] = summarize(w_line)
+            del w_line
+            torch.cuda.empty_cache()
+        line["workloads"] = sweep
+    if rank == 0 and line is not None:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -31,7 +31,7 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_con
             "moe_combine", "moe_combine_staged",
             "moe_layer_forward", "moe_eplb_plan", "moe_eplb_workspace_bytes", "moe_eplb_assign",
             "moe_eplb_place_weights", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8",
-            "moe_workspace_bytes_fp8", "moe_layer_forward_fp8", "moe_capacity_drop",
+            "moe_workspace_bytes_fp8", "moe_layer_forward_fp8", "moe_capacity_drop", "moe_capacity_rows",
             "moe_layer_forward_fp8_overlapped", "moe_ep_window_bytes", "moe_ep_window_layout",
             "moe_ep_workspace_bytes", "moe_ep_ipc_handle", "moe_ep_ipc_open", "moe_ep_ipc_close", "moe_ep_notify",
             "moe_ep_layout", "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ep_layer_forward",
@@ -113,6 +113,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_workspace_bytes_fp8": (sz, [cfgp]),
         "moe_layer_forward_fp8": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp]),
         "moe_capacity_drop": (i32, [cfgp, vp, i32, vp, vp, vp, sz, vp]),
+        "moe_capacity_rows": (i32, [cfgp, ctypes.c_double, ctypes.POINTER(i32)]),
         "moe_layer_forward_fp8_overlapped": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp,
                                                    vp]),
     }
@@ -514,9 +515,12 @@ def layer_forward_fp8(cfg, x, w_gate, bias, expert_owner, w13_q, w13_scale, w2_q
 
 # ---------------------------------------------------------------- capacity factor
 def capacity_of(factor: float, cfg) -> int:
-    """ceil(factor * N * k / E): the uniform share of one expert times the factor."""
-    import math
-    return int(math.ceil(factor * cfg.N * cfg.k / cfg.E))
+    """moe_capacity_rows: ceil(factor * N * k / E), the uniform share of one expert times
+    the factor (computed by the library)."""
+    c = c_config(cfg)
+    out = ctypes.c_int32(0)
+    _check(load().moe_capacity_rows(ctypes.byref(c), float(factor), ctypes.byref(out)), "moe_capacity_rows")
+    return int(out.value)
 
 
 def capacity_drop(cfg, topk_ids, capacity: int, status=None, out=None, ws=None):

@@ -24,7 +24,13 @@
 // increments the count, later kernels of the step read it), so the epoch is never a
 // launch argument and a captured CUDA graph replays correctly.  Flags only grow, so
 // nothing is reset between steps.  Every wait is bounded (MOE_WAIT_LIMIT_NS) and
-// reports MOE_ERR_TIMEOUT.
+// reports MOE_ERR_TIMEOUT.  A failed wait also fails the step on every rank: the rank
+// records the step in its window (err_step), and the flags it publishes later in that
+// step (its dispatch to the owners, its "done" to the sources) carry an error mark (the
+// top bit) beside the epoch; a wait that finds the mark for its epoch reports
+// MOE_ERR_TIMEOUT and fails the step there too, so no combine sums rows of an owner
+// whose inputs did not all arrive.  The mark is tied to its epoch: the next step's flags
+// are plain again.
 // No TMA and no multicast touches peer memory: peer traffic is plain 16-byte loads and
 // stores.
 #include "common.cuh"
@@ -45,21 +51,30 @@ __device__ __forceinline__ uint64_t ld_acquire_sys(const uint64_t* p) {
   return v;
 }
 
-// One thread: wait until flags[0..n) all hold at least epoch.  Gives up after
-// MOE_WAIT_LIMIT_NS (or 2^32 polls), reports MOE_ERR_TIMEOUT and returns false.
+// Error mark on a published flag: the epoch's step failed on the publishing rank.
+constexpr uint64_t kEpErr = 1ull << 63;
+
+// One thread: wait until flags[0..n) all hold at least epoch (error marks aside).  Gives
+// up after MOE_WAIT_LIMIT_NS (or 2^32 polls), reports MOE_ERR_TIMEOUT and returns false;
+// also returns false with MOE_ERR_TIMEOUT when a flag carries the error mark of this
+// epoch (a wait failed on the rank that published it).
 __device__ bool wait_epochs(const uint64_t* flags, int n, uint64_t epoch, int* status) {
   const uint64_t t0 = global_timer_ns();
   uint64_t polls = 0;
+  bool ok = true;
   for (int i = 0; i < n; ++i) {
-    while (ld_acquire_sys(flags + i) < epoch) {
+    uint64_t v;
+    while (((v = ld_acquire_sys(flags + i)) & ~kEpErr) < epoch) {
       if ((++polls & 31u) == 0u && (global_timer_ns() - t0 > MOE_WAIT_LIMIT_NS || polls > 0xffffffffull)) {
         report(status, MOE_ERR_TIMEOUT);
         return false;
       }
       __nanosleep(64);
     }
+    if (v == (epoch | kEpErr)) ok = false;
   }
-  return true;
+  if (!ok) report(status, MOE_ERR_TIMEOUT);
+  return ok;
 }
 
 template <typename T>
@@ -70,6 +85,19 @@ __device__ __forceinline__ T* at(const char* base, size_t off) {
 // This rank's current step (written by an earlier kernel on the same stream).
 __device__ __forceinline__ uint64_t step_of(const char* own, const EpOffsets& off) {
   return *reinterpret_cast<const volatile uint64_t*>(own + off.step);
+}
+
+// The running step failed on this rank (a wait of one of its kernels gave up or met an
+// error mark); later kernels of the step, on the same stream, see it.
+__device__ __forceinline__ void fail_step(const char* own, const EpOffsets& off) {
+  *reinterpret_cast<volatile uint64_t*>(const_cast<char*>(own) + off.err_step) = step_of(own, off);
+}
+__device__ __forceinline__ bool step_failed(const char* own, const EpOffsets& off) {
+  return *reinterpret_cast<const volatile uint64_t*>(own + off.err_step) == step_of(own, off);
+}
+// The value this rank publishes for the running step: its epoch, marked if it failed.
+__device__ __forceinline__ uint64_t published_epoch(const char* own, const EpOffsets& off) {
+  return step_of(own, off) | (step_failed(own, off) ? kEpErr : 0ull);
 }
 
 // ---------------------------------------------------------------- count exchange
@@ -115,7 +143,10 @@ __global__ void __launch_bounds__(kEpLayoutThreads) ep_layout_kernel(EpLayoutArg
   __shared__ int own_of[kMaxSlots];
   __shared__ int R[kMaxP];
   const int tid = threadIdx.x;
-  if (tid == 0) s_ok = wait_epochs(at<uint64_t>(a.win, a.off.cnt_flag), a.P, step_of(a.win, a.off), a.status);
+  if (tid == 0) {
+    s_ok = wait_epochs(at<uint64_t>(a.win, a.off.cnt_flag), a.P, step_of(a.win, a.off), a.status);
+    if (!s_ok) fail_step(a.win, a.off);
+  }
   __syncthreads();
   const int32_t* cnt = at<int32_t>(a.win, a.off.cnt_tab);
   for (int e = tid; e < a.E; e += blockDim.x) {
@@ -255,7 +286,7 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_dispatch_kernel(const __grid
     uint32_t* ctr = at<uint32_t>(peers.base[me], off.disp_ctr);
     if (atomicAdd(ctr, 1u) == gridDim.x - 1) {
       *ctr = 0;  // ready for the next launch, which is stream-ordered after this one
-      const uint64_t epoch = step_of(peers.base[me], off);
+      const uint64_t epoch = published_epoch(peers.base[me], off);
       __threadfence_system();
       for (int p = 0; p < P; ++p) st_release_sys(at<uint64_t>(peers.base[p], off.disp_flag) + me, epoch);
     }
@@ -264,14 +295,16 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_dispatch_kernel(const __grid
 
 // ---------------------------------------------------------------- waits and signals
 __global__ void ep_wait_kernel(const char* own, EpOffsets off, size_t flag_off, int n, int* status) {
-  if (threadIdx.x == 0) wait_epochs(at<uint64_t>(own, flag_off), n, step_of(own, off), status);
+  if (threadIdx.x == 0 && !wait_epochs(at<uint64_t>(own, flag_off), n, step_of(own, off), status))
+    fail_step(own, off);
 }
 
-// flag[me] = epoch in every rank's window, after everything before this launch on the stream
+// flag[me] = epoch in every rank's window (with the error mark if the step failed on this
+// rank), after everything before this launch on the stream
 __global__ void ep_signal_kernel(const __grid_constant__ EpPeers peers, EpOffsets off, size_t flag_off, int P,
                                  int me) {
   if (threadIdx.x != 0) return;
-  const uint64_t epoch = step_of(peers.base[me], off);
+  const uint64_t epoch = published_epoch(peers.base[me], off);
   __threadfence_system();
   for (int p = 0; p < P; ++p) st_release_sys(at<uint64_t>(peers.base[p], flag_off) + me, epoch);
 }
@@ -328,10 +361,17 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_combine_kernel(const __grid_
                                                                     int vpr, int capacity, int P, int me,
                                                                     int* status) {
   __shared__ int s_ok;
-  if (threadIdx.x == 0)
-    s_ok = wait_epochs(at<uint64_t>(peers.base[me], off.done_flag), P, step_of(peers.base[me], off), status);
+  if (threadIdx.x == 0) {
+    const char* own = peers.base[me];
+    s_ok = wait_epochs(at<uint64_t>(own, off.done_flag), P, step_of(own, off), status);
+    if (s_ok && step_failed(own, off)) {  // an earlier wait of this rank's step gave up
+      report(status, MOE_ERR_TIMEOUT);
+      s_ok = 0;
+    }
+    if (!s_ok) fail_step(own, off);
+  }
   __syncthreads();
-  if (!s_ok) return;
+  if (!s_ok) return;  // y is not written
   const int lane = threadIdx.x & 31;
   const int chunks = (vpr + 31) / 32;
   const uint4* shared = at<uint4>(peers.base[me], off.out_recv) + (size_t)capacity * vpr;
@@ -372,7 +412,8 @@ EpOffsets ep_offsets(const moe_config& c, int capacity) {
   o.done_flag = o.disp_flag + kMaxP * sizeof(uint64_t);
   o.step = o.done_flag + kMaxP * sizeof(uint64_t);
   o.disp_ctr = o.step + sizeof(uint64_t);
-  o.cnt_tab = al256(o.disp_ctr + sizeof(uint32_t));
+  o.err_step = o.disp_ctr + sizeof(uint64_t);
+  o.cnt_tab = al256(o.err_step + sizeof(uint64_t));
   o.gate = al256(o.cnt_tab + (size_t)c.P * c.E * sizeof(int32_t));
   o.scale = al256(o.gate + (size_t)capacity * sizeof(float));
   o.x_recv = al256(o.scale + (size_t)capacity * sizeof(float));

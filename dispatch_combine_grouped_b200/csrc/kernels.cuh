@@ -20,6 +20,10 @@ constexpr int kMaxShared = 8;     // shared experts
 constexpr int kLayoutChunk = 1024;  // assignments per counting chunk
 constexpr int kTileRows = 128;      // rows per block in tile_off
 
+// ---- moe_abi.cu : the text moe_last_error returns, for entry points in other files
+moe_status record_error(moe_status s, const char* what);
+moe_status record_cuda_error(cudaError_t e, const char* where);
+
 // ---- layout.cu
 size_t layout_ws_bytes(int A, int E, int P, int nchunks);
 cudaError_t launch_layout(const moe_config& cfg, const int32_t* owner, const int32_t* ids, const moe_layout& L,
@@ -118,6 +122,7 @@ struct EpOffsets {
   size_t cnt_flag, disp_flag, done_flag;  // [kMaxP] u64 epochs, indexed by the signalling rank
   size_t step;                            // u64: this rank's steps so far (= the running step's epoch)
   size_t disp_ctr;                        // u32: this rank's dispatch CTAs finished in the running launch
+  size_t err_step;                        // u64: the last step in which a wait of this rank failed
   size_t cnt_tab;                         // [P, E] int32: row i = source i's expert counts
   size_t gate;                            // [capacity] fp32: gate of each received row
   size_t scale;                           // [capacity] fp32: FP8 dispatch: token scale of each received row

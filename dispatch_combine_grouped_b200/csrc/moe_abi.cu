@@ -1,6 +1,7 @@
 // C entry points of libmoe: argument validation, workspace carving and the launch order
 // of the layer's steps.  Every step runs in this library's CUDA kernels; nothing here
 // computes on the host.
+#include <math.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -551,9 +552,16 @@ moe_status ep_forward(const moe_config& c, const moe_ep_group& g, const EpPeers&
 
 }  // namespace
 
+namespace moe {
+// The error recorder for entry points defined in other files of this library (the text
+// moe_last_error returns).
+moe_status record_error(moe_status s, const char* what) { return fail(s, what); }
+moe_status record_cuda_error(cudaError_t e, const char* where) { return cuda_status(e, where); }
+}  // namespace moe
+
 extern "C" {
 
-int32_t moe_version(void) { return 100; }
+int32_t moe_version(void) { return 101; }
 
 const char* moe_status_string(int32_t s) {
   switch (s) {
@@ -980,7 +988,7 @@ moe_status moe_ep_window_layout(const moe_config* cfg, int32_t capacity, size_t*
   if (s != MOE_OK) return s;
   if (capacity < 1 || !offsets) return fail(MOE_ERR_INVALID_ARG, "capacity < 1 or NULL offsets");
   const EpOffsets o = ep_offsets(*cfg, capacity);
-  const size_t v[10] = {o.cnt_flag, o.disp_flag, o.done_flag, o.step,   o.disp_ctr,
+  const size_t v[11] = {o.cnt_flag, o.disp_flag, o.done_flag, o.step,   o.disp_ctr, o.err_step,
                         o.cnt_tab,  o.gate,      o.scale,     o.x_recv, o.out_recv};
   memcpy(offsets, v, sizeof(v));
   return MOE_OK;
@@ -1182,6 +1190,18 @@ moe_status moe_ep_layer_forward_fp8_overlapped(const moe_config* cfg, const moe_
   const EpFfn f = {true, nullptr, nullptr, w13_q, w13_scale, w2_q, w2_scale};
   return ep_layer(cfg, grp, x, w_gate, bias, expert_owner, f, y, handle_out, dev_status, ws, ws_bytes, stream,
                   side_stream);
+}
+
+moe_status moe_capacity_rows(const moe_config* cfg, double factor, int32_t* capacity) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (!capacity) return fail(MOE_ERR_INVALID_ARG, "capacity is NULL");
+  if (!(factor > 0.0) || !isfinite(factor)) return fail(MOE_ERR_INVALID_ARG, "factor must be finite and > 0");
+  // the uniform share N*k/E times the factor, rounded up (evaluated left to right in double)
+  const double c = ceil(factor * (double)cfg->N * (double)cfg->k / (double)cfg->E);
+  if (c > 2147483647.0) return fail(MOE_ERR_UNSUPPORTED, "capacity exceeds int32");
+  *capacity = (int32_t)c;
+  return MOE_OK;
 }
 
 moe_status moe_capacity_drop(const moe_config* cfg, const int32_t* topk_ids, int32_t capacity, int32_t* kept_ids,

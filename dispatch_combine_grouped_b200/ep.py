@@ -19,9 +19,9 @@ import torch
 
 from . import binding as B
 
-N_OFFSETS = 10
-OFFSET_NAMES = ["cnt_flag", "disp_flag", "done_flag", "step", "disp_ctr", "cnt_tab", "gate", "scale", "x_recv",
-                "out_recv"]
+N_OFFSETS = 11
+OFFSET_NAMES = ["cnt_flag", "disp_flag", "done_flag", "step", "disp_ctr", "err_step", "cnt_tab", "gate", "scale",
+                "x_recv", "out_recv"]
 MAX_RANKS = 32
 
 
@@ -75,6 +75,7 @@ def window_views(cfg, capacity: int, window: torch.Tensor) -> dict:
                 disp_flag=view(o["disp_flag"], MAX_RANKS, torch.int64),
                 done_flag=view(o["done_flag"], MAX_RANKS, torch.int64),
                 step=view(o["step"], 1, torch.int64),
+                err_step=view(o["err_step"], 1, torch.int64),
                 cnt_tab=view(o["cnt_tab"], P * E, torch.int32).view(P, E),
                 gate=view(o["gate"], capacity, torch.float32),
                 scale=view(o["scale"], capacity, torch.float32),

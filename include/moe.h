@@ -179,7 +179,11 @@ moe_status moe_dispatch_layout(const moe_config* cfg, const int32_t* expert_owne
  *          with E <= 256, P <= 32); larger configurations return MOE_ERR_UNSUPPORTED.
  *   Set-up: the first call on each device looks up the array's device address
  *          (cudaGetSymbolAddress, with that device current) and caches it; make that
- *          first call before any stream capture.
+ *          first call before any stream capture.  The cache is tied to the device's
+ *          context: after a device reset (cudaDeviceReset, or anything else that
+ *          destroys the primary context) the array is reloaded at another address and
+ *          the next call looks it up again, so that call, too, should come before any
+ *          capture.  The scratch contents do not survive a reset.
  *   Sharing: all calls on a device use the same array, so calls that overlap on the GPU
  *          (different streams, or different host threads) race and corrupt each other's
  *          results; serialise them.  Contents left by an earlier call are harmless:
@@ -375,6 +379,15 @@ moe_status moe_eplb_plan(int32_t E, int32_t R, int32_t P, const int64_t* load, i
 moe_status moe_capacity_drop(const moe_config* cfg, const int32_t* topk_ids, int32_t capacity, int32_t* kept_ids,
                              int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/*
+ * The capacity of a capacity factor ([EP-DeepEP] §4: an expert's share of one round's
+ * assignments, N*k/E, times the factor): *capacity = ceil(factor * N * k / E), evaluated
+ * in double precision left to right (host only, launches nothing).
+ * Errors: factor not finite or <= 0, or capacity NULL -> MOE_ERR_INVALID_ARG; a result
+ * above INT32_MAX -> MOE_ERR_UNSUPPORTED; an invalid cfg as moe_check_config.
+ */
+moe_status moe_capacity_rows(const moe_config* cfg, double factor, int32_t* capacity);
+
 /* Bytes of scratch moe_eplb_assign and moe_capacity_drop need (a one-owner dispatch
  * layout of the logical ids). */
 size_t moe_eplb_workspace_bytes(const moe_config* cfg);
@@ -554,11 +567,12 @@ typedef struct {
 /* Bytes of one rank's window (0 on an invalid configuration). */
 size_t moe_ep_window_bytes(const moe_config* cfg, int32_t capacity);
 /* Byte offsets of the window's parts (the same on every rank; a rank's own N only sizes
- * the shared rows at the end): offsets[0..9] = count flags [32] u64, dispatch flags [32]
+ * the shared rows at the end): offsets[0..10] = count flags [32] u64, dispatch flags [32]
  * u64, done flags [32] u64 (each indexed by the signalling rank), step counter u64,
- * dispatch counter u32, count table [P, E] int32, gates [capacity] fp32, token scales
- * [capacity] fp32 (FP8 dispatch), received rows [capacity, d] (of d bytes each for the FP8
- * dispatch), output rows [capacity + S*N, d]. */
+ * dispatch counter u32, failed-step word u64 (the last step in which a wait of this rank
+ * gave up), count table [P, E] int32, gates [capacity] fp32, token scales [capacity] fp32
+ * (FP8 dispatch), received rows [capacity, d] (of d bytes each for the FP8 dispatch),
+ * output rows [capacity + S*N, d].  (ABI version 101 added the failed-step word.) */
 moe_status moe_ep_window_layout(const moe_config* cfg, int32_t capacity, size_t* offsets);
 /* Bytes of scratch the EP calls of one step need (ws; the same ws for all calls of a step
  * and for moe_ep_layer_forward, which also keeps the router outputs and the handle there). */

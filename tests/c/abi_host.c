@@ -59,10 +59,10 @@ int main(void) {
   CHECK(moe_workspace_bytes(&bad) == 0);
 
   /* the expert-parallel window: parts in order, inside the window */
-  size_t off[10];
+  size_t off[11];
   CHECK(moe_ep_window_layout(&c, 6144, off) == MOE_OK);
-  for (int i = 1; i < 10; ++i) CHECK(off[i] > off[i - 1]);
-  CHECK(moe_ep_window_bytes(&c, 6144) > off[9]);
+  for (int i = 1; i < 11; ++i) CHECK(off[i] > off[i - 1]);
+  CHECK(moe_ep_window_bytes(&c, 6144) > off[10]);
   CHECK(moe_ep_window_bytes(&c, 0) == 0);
 
   /* EPLB plan on the host: 8 experts, 4 extra copies, 4 owners */

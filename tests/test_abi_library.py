@@ -116,3 +116,36 @@ def test_eplb_calls_reject_bad_arguments_without_launching():
     assert lib.moe_eplb_place_weights(ctypes.c_void_p(se.ctypes.data), 3, 8, 0, 16, ctypes.c_void_p(16),
                                       ctypes.c_void_p(16), None) == binding.MOE_ERR_INVALID_ARG
 
+
+
+def test_capacity_rows_matches_the_oracle():
+    """moe_capacity_rows (host) equals the oracle's ceil(factor * N * k / E)."""
+    from oracle import moe_oracle as O
+    for name in ("fine", "wide", "hot", "hot_cal", "tiny"):
+        cfg = CONFIGS[name]
+        for factor in (0.5, 0.8, 1.0, 1.25, 1.3333, 2.0, 7.77):
+            assert moe.capacity_of(factor, cfg) == O.capacity(factor, cfg.N, cfg.k, cfg.E), (name, factor)
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        with pytest.raises(moe.MoEError) as e:
+            moe.capacity_of(bad, CONFIGS["fine"])
+        assert e.value.status == binding.MOE_ERR_INVALID_ARG
+
+
+def test_noalloc_layout_refusals_say_why():
+    """moe_dispatch_layout_noalloc refuses on the host (nothing is launched) and records
+    the reason for moe_last_error, like the other entry points."""
+    lib = binding.load()
+    fake = ctypes.c_void_p(256)  # never dereferenced: every case below is refused first
+    lay = binding.CLayout(*([256] * len(binding.LAYOUT_FIELDS)))
+    big = binding.c_config(small_config(N=40000, d=64, E=256, S=0, k=8, I=64, P=32))
+    assert lib.moe_dispatch_layout_noalloc(ctypes.byref(big), None, fake, ctypes.byref(lay), None, None) \
+        == binding.MOE_ERR_UNSUPPORTED
+    assert b"2 MiB" in lib.moe_last_error()
+    small = binding.c_config(small_config(N=8, d=64, E=8, S=0, k=2, I=64, P=3))
+    assert lib.moe_dispatch_layout_noalloc(ctypes.byref(small), None, fake, ctypes.byref(lay), None, None) \
+        == binding.MOE_ERR_INVALID_ARG
+    assert b"E % P" in lib.moe_last_error()
+    small = binding.c_config(small_config(N=8, d=64, E=8, S=0, k=2, I=64, P=2))
+    assert lib.moe_dispatch_layout_noalloc(ctypes.byref(small), None, fake, ctypes.byref(binding.CLayout()), None,
+                                           None) == binding.MOE_ERR_INVALID_ARG
+    assert b"non-NULL" in lib.moe_last_error()

@@ -56,3 +56,46 @@ def test_whole_job_rate_and_max_over_ranks():
     assert bench.whole_job_tokens_per_s(4096, 1, 0.5) == pytest.approx(4096 / 0.5e-3)
     assert bench.whole_job_tokens_per_s(4096, 8, 0.5) == pytest.approx(8 * 4096 / 0.5e-3)
     assert bench.max_over_ranks(2.5, 1) == 2.5
+
+
+def test_layer_roofline_per_workload():
+    """Layer roofline: router, permute and combine at HBM bandwidth, the FFN at the slower
+    of its FLOPs at the tensor peak and its touched weights at HBM.  With the measured
+    peaks the wide FFN is tensor-bound (near the ridge) and the decode FFN weight-bound."""
+    hbm, tc = 6454.3, 1693.9
+    wide = bench.roofline_layer_ms(CONFIGS["wide"], 256, hbm, tc)
+    assert wide["ffn_bound"] == "tensor"
+    assert wide["parts_ms"]["ffn"] == pytest.approx(6494e9 / 1693.9e12 * 1e3, rel=2e-3)
+    assert wide["parts_ms"]["permute"] == pytest.approx(1.057e9 / 6454.3e9 * 1e3, rel=2e-3)
+    assert wide["ms"] == pytest.approx(sum(wide["parts_ms"].values()))
+    dec = bench.roofline_layer_ms(CONFIGS["decode"], 252, hbm, tc)
+    assert dec["ffn_bound"] == "hbm"
+    assert dec["parts_ms"]["ffn"] == pytest.approx(253 * 3 * 7168 * 2048 * 2 / 6454.3e9 * 1e3, rel=1e-9)
+
+
+def test_both_arms_describe_the_workload_identically():
+    for name in ("wide", "fine", "tiny"):
+        assert bench.config_dict(CONFIGS[name], 1) == bench.config_dict(CONFIGS[name], 1)
+        assert set(bench.config_dict(CONFIGS[name], 1)) == {"workload", "tokens_per_gpu", "l2", "parallelism"}
+
+
+def test_spec_peak_scales_with_the_clock():
+    assert bench.spec_at_clock(1965) == pytest.approx(2250.0)
+    assert bench.spec_at_clock(1455) == pytest.approx(2250.0 * 1455 / 1965)
+
+
+def test_default_workload_is_the_wide_layer():
+    import sys as _sys
+    old = _sys.argv
+    _sys.argv = ["bench.py"]
+    try:
+        assert bench.parse().workload == "wide"
+    finally:
+        _sys.argv = old
+
+
+def test_launch_count_per_step():
+    # wide: router 2, layout 3, permute 1, routed FC1/FC2 pair + tail (4), shared (4), combine 1
+    assert bench.kernel_launches_per_step(CONFIGS["wide"]) == 15
+    assert bench.kernel_launches_per_step(CONFIGS["fine"]) == 2 + 3 + 1 + 2 + 2 + 1
+    assert bench.kernel_launches_per_step(CONFIGS["hot"]) == 2 + 3 + 1 + 4 + 0 + 1

@@ -16,7 +16,7 @@ def test_window_parts_in_order_and_sized(dtype, eb):
     names = ep.OFFSET_NAMES
     assert [o[n] for n in names] == sorted(o[n] for n in names)
     sizes = {"cnt_flag": 8 * ep.MAX_RANKS, "disp_flag": 8 * ep.MAX_RANKS, "done_flag": 8 * ep.MAX_RANKS, "step": 8,
-             "disp_ctr": 4, "cnt_tab": 4 * cfg.P * cfg.E, "gate": 4 * cap, "scale": 4 * cap,
+             "disp_ctr": 4, "err_step": 8, "cnt_tab": 4 * cfg.P * cfg.E, "gate": 4 * cap, "scale": 4 * cap,
              "x_recv": cap * cfg.d * eb, "out_recv": (cap + cfg.S * cfg.N) * cfg.d * eb}
     for a, b in zip(names, names[1:]):
         assert o[a] + sizes[a] <= o[b], (a, b)

@@ -264,6 +264,42 @@ def test_ep_wait_times_out_and_context_stays_usable():
     assert float(z.sum().item()) == 2048.0
 
 
+def test_ep_failed_dispatch_fails_the_step_on_every_rank():
+    """Rank 1 skips its dispatch in one step: every owner's bounded wait for it gives up,
+    each owner publishes its "done" with the error mark, and every rank's combine reports
+    MOE_ERR_TIMEOUT on its own status and leaves y unwritten, instead of summing rows of
+    owners whose inputs did not all arrive.  The next step runs normally again."""
+    cfg, _ = CASES[0]
+    inp = gpu_inputs(cfg)
+    em = Emulated(cfg, _shards(cfg, None))
+    res = em.step(inp)
+    assert int(em.status.item()) == 0
+    P, wts = cfg.P, em.weights(inp)
+    st = [torch.zeros(1, dtype=torch.int32, device="cuda") for _ in range(P)]
+    ys = [torch.full((c.N, c.d), 7.0, dtype=c.torch_dtype, device="cuda") for c in em.rcfg]
+    for r in range(P):
+        ep.notify(em.rcfg[r], em.groups[r], res["ids"][r], em.ws[r], st[r])
+    for r in range(P):
+        ep.layout(em.rcfg[r], em.groups[r], res["ids"][r], em.handles[r], em.ws[r], None, st[r])
+    for r in range(P):
+        if r != 1:
+            ep.dispatch(em.rcfg[r], em.groups[r], res["xs"][r], res["w"][r], em.handles[r])
+    for r in range(P):
+        ep.expert_ffn(em.rcfg[r], em.groups[r], res["xs"][r], wts[r][0], wts[r][1], em.handles[r], em.ws[r], st[r])
+    for r in range(P):
+        ep.combine(em.rcfg[r], em.groups[r], em.handles[r], y=ys[r], status=st[r])
+    torch.cuda.synchronize()
+    for r in range(P):
+        assert int(st[r].item()) == moe.binding.MOE_ERR_TIMEOUT, f"status of rank {r}"
+        assert bool((ys[r] == 7.0).all()), f"y of rank {r} was written"
+        v = ep.window_views(em.rcfg[r], em.capacity, em.windows[r])
+        assert int(v["err_step"].item()) == int(v["step"].item()) == 2
+        assert int(v["done_flag"][r].item()) == 2 - 2 ** 63   # epoch 2 with the error mark (int64 view)
+    again = em.step(inp)
+    assert int(em.status.item()) == 0
+    assert torch.equal(again["y"], res["y"])
+
+
 def test_ep_host_errors():
     cfg, _ = CASES[0]
     rc = cfg.replace(N=cfg.N // cfg.P)

@@ -1,8 +1,12 @@
 """GPU parity at the five full workload sizes (the bench's launch configuration).
 
 Routing and layout are checked completely (bit-exact against the oracle run on the
-GPU's fp32 logits); expert outputs and y are checked on sampled tokens that the
-oracle computes one by one from the output equation.
+GPU's fp32 logits).  The grouped GEMMs are checked on rows chosen so that every tile
+they run is compared with the oracle: for every routed expert and every shared expert,
+the first and the last row of each 128-row block of its rows (so every 256-row CTA-pair
+tile, both CTAs of it, and every 0..128-row tail tile), element by element, for h (the
+SwiGLU activations after FC1) and for the gate-scaled FC2 rows.  y is checked on sampled
+tokens that the oracle computes one by one from the output equation.
 """
 import numpy as np
 import pytest
@@ -11,12 +15,52 @@ import torch
 import dispatch_combine_grouped_b200 as moe
 from moe_inputs import CONFIGS
 from oracle import moe_oracle as O
-from tests.gpu_cases import assert_close_fro, assert_layout_equal, check_route, gpu_inputs, layout_to_numpy, run_steps
+from tests.gpu_cases import (assert_close_fro, assert_close_rel, assert_layout_equal, check_route, gpu_inputs,
+                             layout_to_numpy, run_steps)
 
 pytestmark = pytest.mark.gpu
 
 FULL = ["fine", "wide", "decode", "hot", "hot_cal"]
 SAMPLE_TOKENS = {"fine": 8, "wide": 4, "decode": 4, "hot": 8, "hot_cal": 8}
+BLOCK = 128  # row block of the grouped GEMM tiles (a CTA-pair tile spans two)
+
+
+def block_edge_rows(r0, n):
+    """The first and the last row of every 128-row block of the rows [r0, r0 + n)."""
+    rows = []
+    for b0 in range(r0, r0 + n, BLOCK):
+        rows += [b0, min(b0 + BLOCK, r0 + n) - 1]
+    return sorted(set(rows))
+
+
+def check_every_tile(cfg, inp, res, ref, gates):
+    """h and gate-scaled FC2 rows of every group's block edges against the float64 SwiGLU
+    expert ([EP-DeepEP] §2 Expert_e; [MoE-IV] §4.1 FC1, activation, FC2)."""
+    A, N, k, I = cfg.N * cfg.k, cfg.N, cfg.k, cfg.I
+    x64 = O.f64(inp["x"])
+    g_flat = gates.reshape(-1)
+    checked, experts = 0, 0
+    groups = [(e, int(ref["expert_off"][e]), int(ref["n_e"][e])) for e in range(cfg.E)]
+    groups += [(cfg.E + s, A + s * N, N) for s in range(cfg.S)]
+    for e, r0, n in groups:
+        if n == 0:
+            continue
+        rows = np.array(block_edge_rows(r0, n))
+        if e < cfg.E:
+            a = ref["row2tok"][rows]              # assignment of each row
+            tok, gate = a // k, g_flat[a]
+        else:
+            tok, gate = rows - r0, np.ones(len(rows))
+        w13 = O.f64(inp["w13"][e])
+        xr = x64[tok]
+        h_ref = O.silu(xr @ w13[:I].T) * (xr @ w13[I:].T)
+        o_ref = (h_ref @ O.f64(inp["w2"][e]).T) * gate[:, None]
+        idx = torch.tensor(rows, device="cuda")
+        assert_close_rel(res["h"][idx], h_ref, what=f"{cfg.name} h of group {e}")
+        assert_close_fro(res["out"][idx], o_ref, what=f"{cfg.name} FC2 x gate of group {e}")
+        checked += len(rows)
+        experts += 1
+    return checked, experts
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -38,6 +82,13 @@ def test_full_config(name):
     a_s = rng.choice(A, size=min(A, 2048), replace=False)
     xp = res["x_perm"][torch.tensor(ref["tok2row"][a_s], device="cuda")]
     assert torch.equal(xp, inp["x"][torch.tensor(a_s // cfg.k, device="cuda")]), "permute rows"
+
+    # every tile of the grouped GEMMs: block-edge rows of every group, element by element
+    g_all = O.gate_weights(O.gate_logits(cfg, inp["x"], inp["w_gate"], inp["bias"]), ids, cfg.score,
+                           cfg.renormalize)
+    n_rows, n_groups = check_every_tile(cfg, inp, res, ref, g_all)
+    print(f"{name}: {n_rows} rows of h and FC2 output checked over {n_groups} groups")
+    assert n_groups == int((ref["n_e"] > 0).sum()) + cfg.S
 
     tokens = np.sort(rng.choice(cfg.N, size=SAMPLE_TOKENS[name], replace=False))
     z64 = O.gate_logits(cfg, inp["x"][torch.tensor(tokens, device="cuda")], inp["w_gate"], inp["bias"])
