@@ -14,7 +14,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoe.so")
+# MOE_LIB=checked selects the bounds-checked build (libmoe_checked.so, see moe_checks_*)
+LIB_PATH = os.path.join(_HERE, "libmoe_checked.so" if os.environ.get("MOE_LIB") == "checked" else "libmoe.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_BAD_INDEX, \
     MOE_ERR_TIMEOUT = range(7)
@@ -23,7 +24,8 @@ MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
 GROUPS = {"all": 0, "routed": 1, "shared": 2}
 
 # every symbol include/moe.h declares
-EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_check_config",
+EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_checks_enabled", "moe_checks_register",
+            "moe_check_config",
             "moe_layout_workspace_bytes", "moe_workspace_bytes", "moe_route", "moe_dispatch_layout",
             "moe_dispatch_layout_noalloc",
             "moe_permute", "moe_permute_staged", "moe_grouped_ffn", "moe_expert_fc1", "moe_expert_fc2",
@@ -85,6 +87,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_version": (i32, []),
         "moe_status_string": (ctypes.c_char_p, [i32]),
         "moe_last_error": (ctypes.c_char_p, []),
+        "moe_checks_enabled": (i32, []),
+        "moe_checks_register": (i32, [vp]),
         "moe_check_config": (i32, [cfgp]),
         "moe_layout_workspace_bytes": (sz, [cfgp]),
         "moe_workspace_bytes": (sz, [cfgp]),
@@ -209,6 +213,17 @@ def selftest_bounded_wait(status, limit_ns=20_000_000):
 
 def version() -> int:
     return load().moe_version()
+
+
+def checks_enabled() -> bool:
+    """True when the loaded library is the bounds-checked build."""
+    return bool(load().moe_checks_enabled())
+
+
+def checks_register(word):
+    """Register a device int32 tensor (or None) that the bounds-checked build records
+    failed index checks into (MOE_ERR_BAD_INDEX)."""
+    _check(load().moe_checks_register(_p(word)), "moe_checks_register")
 
 
 def check_config(cfg):

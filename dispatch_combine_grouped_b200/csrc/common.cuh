@@ -21,6 +21,29 @@ __device__ __forceinline__ void report(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Bounds-checked build (compiled with -DMOE_CHECKS, the library libmoe_checked.so): the
+// kernels verify every index they read from a caller-visible map or table before using
+// it; a value outside its range is recorded as MOE_ERR_BAD_INDEX in the registered check
+// word (moe_checks_register) and the access is skipped.  Nothing traps.  In the normal
+// build the checks compile away.
+#ifdef MOE_CHECKS
+constexpr bool kChecks = true;
+#else
+constexpr bool kChecks = false;
+#endif
+
+// true when lo <= v < hi; otherwise (checked builds only) records MOE_ERR_BAD_INDEX in
+// *word and returns false, so that the caller skips the access.
+__device__ __forceinline__ bool check_range(long long v, long long lo, long long hi, int* word) {
+  if constexpr (kChecks) {
+    if (v < lo || v >= hi) {
+      report(word, MOE_ERR_BAD_INDEX);
+      return false;
+    }
+  }
+  return true;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -239,10 +239,11 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_dispatch_kernel(const __grid
                                                                      const float* __restrict__ topk_w,
                                                                      const float* __restrict__ x_scale, int N,
                                                                      int k, int vpr, int capacity, int P,
-                                                                     int me) {
+                                                                     int me, int* check) {
   const int lane = threadIdx.x & 31;
   for (int t = blockIdx.x * kEpWarps + (threadIdx.x >> 5); t < N; t += gridDim.x * kEpWarps) {
-    const int my = lane < k ? dest[(size_t)t * k + lane] : -1;
+    int my = lane < k ? dest[(size_t)t * k + lane] : -1;
+    if (!check_range(my, -1, (long long)P * capacity, check)) my = -1;  // bounds-checked build
     if (my >= 0) {
       const int o = my / capacity;
       at<float>(peers.base[o], off.gate)[my - o * capacity] = topk_w[(size_t)t * k + lane];
@@ -359,7 +360,7 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_combine_kernel(const __grid_
                                                                     EpOffsets off, const int32_t* __restrict__ dest,
                                                                     uint4* __restrict__ y, int N, int k, int S,
                                                                     int vpr, int capacity, int P, int me,
-                                                                    int* status) {
+                                                                    int* status, int* check) {
   __shared__ int s_ok;
   if (threadIdx.x == 0) {
     const char* own = peers.base[me];
@@ -379,7 +380,8 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_combine_kernel(const __grid_
        item += (long long)gridDim.x * kEpWarps) {
     const int t = (int)(item / chunks);
     const int v = (int)(item - (long long)t * chunks) * 32 + lane;
-    const int my = lane < k ? dest[(size_t)t * k + lane] : -1;
+    int my = lane < k ? dest[(size_t)t * k + lane] : -1;
+    if (!check_range(my, -1, (long long)P * capacity, check)) my = -1;  // bounds-checked build
     int rows[kMaxK];
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) rows[j] = __shfl_sync(0xffffffffu, my, j);
@@ -464,7 +466,8 @@ cudaError_t launch_ep_dispatch(const moe_config& c, const EpPeers& peers, const 
                                int capacity, const void* x, const int32_t* dest, const float* topk_w,
                                const float* x_scale, int row_bytes, cudaStream_t st) {
   ep_dispatch_kernel<<<ep_grid(c.N, kEpWarps), kEpWarps * 32, 0, st>>>(
-      peers, off, static_cast<const uint4*>(x), dest, topk_w, x_scale, c.N, c.k, row_bytes / 16, capacity, c.P, me);
+      peers, off, static_cast<const uint4*>(x), dest, topk_w, x_scale, c.N, c.k, row_bytes / 16, capacity, c.P, me,
+      check_word());
   return cudaGetLastError();
 }
 
@@ -487,10 +490,12 @@ cudaError_t launch_ep_combine(const moe_config& c, const EpPeers& peers, const E
   const unsigned grid = ep_grid(items, kEpWarps);
   if (c.dtype == MOE_BF16)
     ep_combine_kernel<__nv_bfloat16><<<grid, kEpWarps * 32, 0, st>>>(
-        peers, off, dest, static_cast<uint4*>(y), c.N, c.k, c.n_shared, vpr, capacity, c.P, me, status);
+        peers, off, dest, static_cast<uint4*>(y), c.N, c.k, c.n_shared, vpr, capacity, c.P, me, status,
+        check_word());
   else
     ep_combine_kernel<float><<<grid, kEpWarps * 32, 0, st>>>(
-        peers, off, dest, static_cast<uint4*>(y), c.N, c.k, c.n_shared, vpr, capacity, c.P, me, status);
+        peers, off, dest, static_cast<uint4*>(y), c.N, c.k, c.n_shared, vpr, capacity, c.P, me, status,
+        check_word());
   return cudaGetLastError();
 }
 

@@ -26,6 +26,12 @@ __global__ void __launch_bounds__(kSimtThreads) simt_gemm_kernel(const GemmArgs 
     if (gg < p.E) {
       rows = p.n_e[gg];
       arow = orow = p.expert_off[gg];
+      // bounds-checked build: a group must lie inside the routed rows
+      if (kChecks && (rows < 0 || arow < 0 || (long long)arow + rows > p.A_routed)) {
+        report(p.check, MOE_ERR_BAD_INDEX);
+        rows = 0;
+        arow = orow = 0;
+      }
     } else {
       const int s = gg - p.E;
       rows = p.N;
@@ -138,7 +144,10 @@ __global__ void __launch_bounds__(kSimtThreads) simt_gemm_kernel(const GemmArgs 
       if (r >= rows) continue;
       const long long orow = (long long)s_orow[g] + r;
       float scale = 1.0f;
-      if (MODE == MODE_FC2 && p.gate_w && gz < p.E) scale = p.gate_w[p.row2tok ? p.row2tok[orow] : orow];
+      if (MODE == MODE_FC2 && p.gate_w && gz < p.E) {
+          const int gi = p.row2tok ? p.row2tok[orow] : (int)orow;
+          scale = check_range(gi, 0, p.A_routed, p.check) ? p.gate_w[gi] : 0.0f;
+        }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int col = n0 + tx * 4 + j;

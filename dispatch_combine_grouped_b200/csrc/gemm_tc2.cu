@@ -99,6 +99,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     if (gg < p.E) {
       rows = p.n_e[gg];
       arow = orow = p.expert_off[gg];
+      // bounds-checked build: a group must lie inside the routed rows
+      if (kChecks && (rows < 0 || arow < 0 || (long long)arow + rows > p.A_routed)) {
+        report(p.check, MOE_ERR_BAD_INDEX);
+        rows = 0;
+        arow = orow = 0;
+      }
     } else {
       const int s = gg - p.E;
       rows = p.N;
@@ -279,7 +285,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           // a_scale_rows); a shared expert's rows are the tokens in order, after A_routed
           // and the earlier shared experts' blocks
           if (row_ok)
-            ra = gz < p.E ? (p.a_scale_rows ? p.a_scale_rows[orow] : p.a_scale[p.row2tok[orow] / p.k])
+            ra = gz < p.E ? (p.a_scale_rows ? p.a_scale_rows[orow] : token_scale(p, orow))
                           : p.a_scale[(int)(orow - p.A_routed - (long long)(gz - p.E) * p.N)];
           sb = p.b_scale + (size_t)gz * p.b_rows;
         }
@@ -317,7 +323,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
       } else {
         float scale = 1.0f;
-        if (row_ok && p.gate_w && p.g0 + g < p.E) scale = p.gate_w[p.row2tok ? p.row2tok[orow] : orow];
+        if (row_ok && p.gate_w && p.g0 + g < p.E) {
+          const int gi = p.row2tok ? p.row2tok[orow] : (int)orow;
+          scale = check_range(gi, 0, p.A_routed, p.check) ? p.gate_w[gi] : 0.0f;
+        }
         const float* sb = nullptr;
         if (F8) {
           if (row_ok) scale *= p.a_scale[orow];  // FP8: scale of this h row

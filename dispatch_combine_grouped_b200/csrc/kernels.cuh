@@ -6,6 +6,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "common.cuh"
 #include "moe.h"
 
 namespace moe {
@@ -23,6 +24,8 @@ constexpr int kTileRows = 128;      // rows per block in tile_off
 // ---- moe_abi.cu : the text moe_last_error returns, for entry points in other files
 moe_status record_error(moe_status s, const char* what);
 moe_status record_cuda_error(cudaError_t e, const char* where);
+// the device word a bounds-checked build records failed checks into (NULL: none registered)
+int* check_word();
 
 // ---- layout.cu
 size_t layout_ws_bytes(int A, int E, int P, int nchunks);
@@ -83,7 +86,21 @@ struct GemmArgs {
   const float* a_scale; // FC1: per token [N]; FC2: per h row [A + S*N]
   const float* b_scale; // per weight row [groups, b_rows]
   const float* a_scale_rows;  // FC1: when set, routed row r's scale is a_scale_rows[r] (no row map)
+  int* check;           // bounds-checked build: where failed checks are recorded (NULL: nowhere)
 };
+
+#ifdef __CUDACC__
+// FP8 FC1: the scale of a routed row's token (row -> assignment -> token); in the
+// bounds-checked build an assignment outside [0, A_routed) is recorded and scales by 0.
+__device__ __forceinline__ float token_scale(const GemmArgs& p, long long orow) {
+  const int a = p.row2tok[orow];
+  if (kChecks && (a < 0 || a >= p.A_routed)) {
+    if (p.check) atomicCAS(p.check, 0, MOE_ERR_BAD_INDEX);
+    return 0.0f;
+  }
+  return p.a_scale[a / p.k];
+}
+#endif
 
 // Rows a launch covers, for grid sizing: routed rows if any routed group is in range,
 // plus N rows per shared group in range.

@@ -176,6 +176,7 @@ GemmArgs fc1_args(const moe_config& c, const moe_layout& L, const void* x_perm, 
   g.a1 = c.n_shared > 0 ? x : nullptr;
   g.b = w13;
   g.b_rows = 2LL * c.I;
+  g.check = check_word();
   return g;
 }
 
@@ -201,6 +202,7 @@ GemmArgs fc2_args(const moe_config& c, const moe_layout& L, const void* h, const
   g.a0 = h;
   g.b = w2;
   g.b_rows = c.d;
+  g.check = check_word();
   return g;
 }
 
@@ -553,6 +555,10 @@ moe_status ep_forward(const moe_config& c, const moe_ep_group& g, const EpPeers&
 }  // namespace
 
 namespace moe {
+// Bounds-checked build: the caller's device word failed checks are recorded into.
+static int32_t* g_check_word = nullptr;
+int* check_word() { return g_check_word; }
+
 // The error recorder for entry points defined in other files of this library (the text
 // moe_last_error returns).
 moe_status record_error(moe_status s, const char* what) { return fail(s, what); }
@@ -562,6 +568,13 @@ moe_status record_cuda_error(cudaError_t e, const char* where) { return cuda_sta
 extern "C" {
 
 int32_t moe_version(void) { return 101; }
+
+int32_t moe_checks_enabled(void) { return kChecks ? 1 : 0; }
+
+moe_status moe_checks_register(int32_t* dev_word) {
+  g_check_word = dev_word;
+  return MOE_OK;
+}
 
 const char* moe_status_string(int32_t s) {
   switch (s) {
@@ -1196,7 +1209,7 @@ moe_status moe_capacity_rows(const moe_config* cfg, double factor, int32_t* capa
   moe_status s = check_config(cfg);
   if (s != MOE_OK) return s;
   if (!capacity) return fail(MOE_ERR_INVALID_ARG, "capacity is NULL");
-  if (!(factor > 0.0) || !isfinite(factor)) return fail(MOE_ERR_INVALID_ARG, "factor must be finite and > 0");
+  if (!(factor >= 0.0) || !isfinite(factor)) return fail(MOE_ERR_INVALID_ARG, "factor must be finite and >= 0");
   // the uniform share N*k/E times the factor, rounded up (evaluated left to right in double)
   const double c = ceil(factor * (double)cfg->N * (double)cfg->k / (double)cfg->E);
   if (c > 2147483647.0) return fail(MOE_ERR_UNSUPPORTED, "capacity exceeds int32");

@@ -30,11 +30,12 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 __global__ void __launch_bounds__(kMoveWarps * 32) scatter_token_rows(const uint4* __restrict__ src,
                                                                        uint4* __restrict__ dst,
                                                                        const int32_t* __restrict__ map, int N,
-                                                                       int k, int vpr) {
+                                                                       int k, int vpr, int dst_rows, int* check) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kMoveWarps + (threadIdx.x >> 5);
   if (t >= N) return;
-  const int my = lane < k ? map[(size_t)t * k + lane] : 0;
+  int my = lane < k ? map[(size_t)t * k + lane] : 0;
+  if (!check_range(my, -1, dst_rows, check)) my = -1;  // bounds-checked build: skip a bad row
   int rows[kMaxK];
 #pragma unroll
   for (int j = 0; j < kMaxK; ++j) rows[j] = __shfl_sync(0xffffffffu, my, j);
@@ -84,11 +85,12 @@ __device__ __forceinline__ void st32(V32* p, const V32& v) {
 __global__ void __launch_bounds__(kMoveWarps * 32) scatter_token_rows32(const V32* __restrict__ src,
                                                                          V32* __restrict__ dst,
                                                                          const int32_t* __restrict__ map, int N,
-                                                                         int k, int vpr) {
+                                                                         int k, int vpr, int dst_rows, int* check) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kMoveWarps + (threadIdx.x >> 5);
   if (t >= N) return;
-  const int my = lane < k ? map[(size_t)t * k + lane] : 0;
+  int my = lane < k ? map[(size_t)t * k + lane] : 0;
+  if (!check_range(my, -1, dst_rows, check)) my = -1;  // bounds-checked build: skip a bad row
   int rows[kMaxK];
 #pragma unroll
   for (int j = 0; j < kMaxK; ++j) rows[j] = __shfl_sync(0xffffffffu, my, j);
@@ -118,12 +120,14 @@ __global__ void __launch_bounds__(kMoveWarps * 32) scatter_token_rows32(const V3
 // Row scatter: dst[map[i]] = src[i]
 template <bool kScatter>
 __global__ void __launch_bounds__(kMoveWarps * 32) move_rows(const uint4* __restrict__ src, uint4* __restrict__ dst,
-                                                              const int32_t* __restrict__ map, int rows, int vpr) {
+                                                              const int32_t* __restrict__ map, int rows, int vpr,
+                                                              int* check) {
   const int lane = threadIdx.x & 31;
   const int i = blockIdx.x * kMoveWarps + (threadIdx.x >> 5);
   if (i >= rows) return;
   const int m = map[i];
   if (m < 0) return;  // an unused slot / a dropped assignment
+  if (!check_range(m, 0, rows, check)) return;  // bounds-checked build: skip a bad row
   const uint4* s = src + (size_t)(kScatter ? i : m) * vpr;
   uint4* d = dst + (size_t)(kScatter ? m : i) * vpr;
   for (int v0 = 0; v0 < vpr; v0 += 32 * kMoveUnroll) {
@@ -185,14 +189,15 @@ __global__ void __launch_bounds__(kMoveWarps * 32) combine_kernel(const uint4* _
                                                                    const int32_t* __restrict__ map,
                                                                    const float* __restrict__ gates,
                                                                    uint4* __restrict__ y, int N, int k, int S,
-                                                                   int vpr) {
+                                                                   int vpr, int* check) {
   const int lane = threadIdx.x & 31;
   const int chunks = (vpr + 32 * kCombVec - 1) / (32 * kCombVec);
   const long long item = (long long)blockIdx.x * kMoveWarps + (threadIdx.x >> 5);
   if (item >= (long long)N * chunks) return;
   const int t = (int)(item / chunks);
   const int v0 = (int)(item - (long long)t * chunks) * 32 * kCombVec + lane;
-  const int my_row = lane < k ? map[(size_t)t * k + lane] : 0;
+  int my_row = lane < k ? map[(size_t)t * k + lane] : 0;
+  if (!check_range(my_row, -1, (long long)N * k, check)) my_row = -1;  // bounds-checked build
   const float my_g = (lane < k && gates) ? gates[(size_t)t * k + lane] : 1.0f;
   int rows[kMaxK];
   float gs[kMaxK];
@@ -243,14 +248,15 @@ __global__ void __launch_bounds__(kMoveWarps * 32) combine_kernel32(const V32* _
                                                                      const int32_t* __restrict__ map,
                                                                      const float* __restrict__ gates,
                                                                      V32* __restrict__ y, int N, int k, int S,
-                                                                     int vpr) {
+                                                                     int vpr, int* check) {
   const int lane = threadIdx.x & 31;
   const int chunks = (vpr + 31) / 32;
   for (long long item = (long long)blockIdx.x * kMoveWarps + (threadIdx.x >> 5); item < (long long)N * chunks;
        item += (long long)gridDim.x * kMoveWarps) {
     const int t = (int)(item / chunks);
     const int v = (int)(item - (long long)t * chunks) * 32 + lane;
-    const int my_row = lane < k ? map[(size_t)t * k + lane] : 0;
+    int my_row = lane < k ? map[(size_t)t * k + lane] : 0;
+    if (!check_range(my_row, -1, (long long)N * k, check)) my_row = -1;  // bounds-checked build
     const float my_g = (lane < k && gates) ? gates[(size_t)t * k + lane] : 1.0f;
     int rows[kMaxK];
     float gs[kMaxK];
@@ -314,11 +320,13 @@ cudaError_t launch_permute_bytes(const moe_config& c, const moe_layout& L, const
   if (c.N == 0) return cudaSuccess;
   if (row_bytes % 32 == 0) {
     scatter_token_rows32<<<blocks_for(c.N), kMoveWarps * 32, 0, st>>>(
-        static_cast<const V32*>(x), static_cast<V32*>(x_perm), L.tok2row, c.N, c.k, row_bytes / 32);
+        static_cast<const V32*>(x), static_cast<V32*>(x_perm), L.tok2row, c.N, c.k, row_bytes / 32, c.N * c.k,
+        check_word());
     return cudaGetLastError();
   }
   scatter_token_rows<<<blocks_for(c.N), kMoveWarps * 32, 0, st>>>(
-      static_cast<const uint4*>(x), static_cast<uint4*>(x_perm), L.tok2row, c.N, c.k, row_bytes / 16);
+      static_cast<const uint4*>(x), static_cast<uint4*>(x_perm), L.tok2row, c.N, c.k, row_bytes / 16, c.N * c.k,
+      check_word());
   return cudaGetLastError();
 }
 
@@ -333,10 +341,10 @@ cudaError_t launch_permute_staged(const moe_config& c, const moe_layout& L, cons
   const int A = c.N * c.k;
   // hop 1: each source buckets its rows by destination owner (send buffer)
   scatter_token_rows<<<blocks_for(c.N), kMoveWarps * 32, 0, st>>>(
-      static_cast<const uint4*>(x), static_cast<uint4*>(send_buf), L.tok2send, c.N, c.k, vpr);
+      static_cast<const uint4*>(x), static_cast<uint4*>(send_buf), L.tok2send, c.N, c.k, vpr, A, check_word());
   // hop 2: the transpose to the owners plus the expert-local order
-  move_rows<true><<<blocks_for(A), kMoveWarps * 32, 0, st>>>(static_cast<const uint4*>(send_buf),
-                                                             static_cast<uint4*>(x_perm), L.send2row, A, vpr);
+  move_rows<true><<<blocks_for(A), kMoveWarps * 32, 0, st>>>(
+      static_cast<const uint4*>(send_buf), static_cast<uint4*>(x_perm), L.send2row, A, vpr, check_word());
   return cudaGetLastError();
 }
 
@@ -350,13 +358,13 @@ static void combine_launch(const moe_config& c, const uint4* routed, const uint4
     const long long nb = blocks_for(items), cap = 4LL * sm_count();  // grid-stride: 4 CTAs per SM
     combine_kernel32<T><<<(unsigned)(nb < cap ? nb : cap), kMoveWarps * 32, 0, st>>>(
         reinterpret_cast<const V32*>(routed), reinterpret_cast<const V32*>(shared), map, gates,
-        reinterpret_cast<V32*>(y), c.N, c.k, c.n_shared, vpr32);
+        reinterpret_cast<V32*>(y), c.N, c.k, c.n_shared, vpr32, check_word());
     return;
   }
   const int vpr = vecs_per_row(c);
   const long long items = (long long)c.N * ((vpr + 32 * kCombVec - 1) / (32 * kCombVec));
   combine_kernel<T><<<blocks_for(items), kMoveWarps * 32, 0, st>>>(routed, shared, map, gates, y, c.N, c.k,
-                                                                    c.n_shared, vpr);
+                                                                    c.n_shared, vpr, check_word());
 }
 
 cudaError_t launch_combine(const moe_config& c, const moe_layout& L, const void* out, const float* topk_w, void* y,
@@ -379,7 +387,8 @@ cudaError_t launch_combine_staged(const moe_config& c, const moe_layout& L, cons
   const int A = c.N * c.k;
   const uint4* o = static_cast<const uint4*>(out);
   // hop 1: owners return rows in send-slot order (reverse transpose): ret[s] = out[send2row[s]]
-  move_rows<false><<<blocks_for(A), kMoveWarps * 32, 0, st>>>(o, static_cast<uint4*>(ret_buf), L.send2row, A, vpr);
+  move_rows<false><<<blocks_for(A), kMoveWarps * 32, 0, st>>>(o, static_cast<uint4*>(ret_buf), L.send2row, A, vpr,
+                                                              check_word());
   // hop 2: unpermute + weighted sum at the source through tok2send
   const uint4* sh = o + (size_t)A * vpr;
   if (c.dtype == MOE_BF16)

@@ -122,6 +122,25 @@ const char* moe_status_string(int32_t status);
 /* Host-side description of the last error returned on this thread ("" if none). */
 const char* moe_last_error(void);
 
+/*
+ * Bounds-checked build (no counterpart in the pages; the survey's substitute for a race /
+ * bounds sanitizer, which is closed on this GPU pool).  The same sources compiled with
+ * -DMOE_CHECKS give libmoe_checked.so, whose kernels check every index they read from a
+ * caller-visible map or table before using it: token -> row maps (tok2row, send2row,
+ * tok2send) in the permute and combine, row -> assignment (row2tok) in the FC2 gate and
+ * the FP8 token scales, each group's rows (n_e, expert_off) in the grouped GEMMs, and the
+ * expert-parallel destinations (dest).  A value outside its range is skipped (no read or
+ * write through it) and MOE_ERR_BAD_INDEX is recorded in the registered device word with
+ * an atomic compare-and-swap (the first error is kept).  Nothing traps.  The ids given to
+ * the layout are checked in every build (moe_dispatch_layout's dev_status).
+ *   moe_checks_enabled: 1 in the checked build, 0 otherwise.
+ *   moe_checks_register: the caller's device int32 the checked kernels record into, for
+ *     every later call on any thread (NULL: record nowhere); the normal build accepts
+ *     and ignores it.  Launches nothing.
+ */
+int32_t moe_checks_enabled(void);
+moe_status moe_checks_register(int32_t* dev_word);
+
 /* Validate a configuration on the host (the same checks every call makes). */
 moe_status moe_check_config(const moe_config* cfg);
 
@@ -383,7 +402,7 @@ moe_status moe_capacity_drop(const moe_config* cfg, const int32_t* topk_ids, int
  * The capacity of a capacity factor ([EP-DeepEP] §4: an expert's share of one round's
  * assignments, N*k/E, times the factor): *capacity = ceil(factor * N * k / E), evaluated
  * in double precision left to right (host only, launches nothing).
- * Errors: factor not finite or <= 0, or capacity NULL -> MOE_ERR_INVALID_ARG; a result
+ * Errors: factor not finite or < 0, or capacity NULL -> MOE_ERR_INVALID_ARG; a result
  * above INT32_MAX -> MOE_ERR_UNSUPPORTED; an invalid cfg as moe_check_config.
  */
 moe_status moe_capacity_rows(const moe_config* cfg, double factor, int32_t* capacity);

@@ -123,9 +123,9 @@ def test_capacity_rows_matches_the_oracle():
     from oracle import moe_oracle as O
     for name in ("fine", "wide", "hot", "hot_cal", "tiny"):
         cfg = CONFIGS[name]
-        for factor in (0.5, 0.8, 1.0, 1.25, 1.3333, 2.0, 7.77):
+        for factor in (0.0, 0.5, 0.8, 1.0, 1.25, 1.3333, 2.0, 7.77):
             assert moe.capacity_of(factor, cfg) == O.capacity(factor, cfg.N, cfg.k, cfg.E), (name, factor)
-    for bad in (0.0, -1.0, float("nan"), float("inf")):
+    for bad in (-1.0, -1e-9, float("nan"), float("inf")):
         with pytest.raises(moe.MoEError) as e:
             moe.capacity_of(bad, CONFIGS["fine"])
         assert e.value.status == binding.MOE_ERR_INVALID_ARG
@@ -149,3 +149,27 @@ def test_noalloc_layout_refusals_say_why():
     assert lib.moe_dispatch_layout_noalloc(ctypes.byref(small), None, fake, ctypes.byref(binding.CLayout()), None,
                                            None) == binding.MOE_ERR_INVALID_ARG
     assert b"non-NULL" in lib.moe_last_error()
+
+
+def test_checked_build_loads_and_says_so():
+    """libmoe_checked.so (-DMOE_CHECKS) exports the same symbols and reports itself as the
+    bounds-checked build; the normal library does not."""
+    import sys
+    spec_root = ROOT
+    b = __import__("importlib").util.spec_from_file_location(
+        "_moe_build", os.path.join(spec_root, "dispatch_combine_grouped_b200", "build.py"))
+    mod = __import__("importlib").util.module_from_spec(b)
+    b.loader.exec_module(mod)
+    path = mod.build(checked=True)
+    lib = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    lib.moe_checks_enabled.restype = ctypes.c_int32
+    assert lib.moe_checks_enabled() == 1
+    assert binding.load().moe_checks_enabled() == 0
+    assert lib.moe_checks_register(None) == binding.MOE_OK
+    code = ("import dispatch_combine_grouped_b200 as m; import sys; "
+            "sys.exit(0 if m.checks_enabled() and m.binding.LIB_PATH.endswith('libmoe_checked.so') else 3)")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=dict(os.environ, MOE_LIB="checked"),
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
