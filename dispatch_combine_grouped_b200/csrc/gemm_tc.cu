@@ -465,13 +465,13 @@ static CUtensorMapSwizzle swizzle_for(int row_bytes) {
 
 // 2D map over [rows, K] (K contiguous; bf16, or bytes when u8), box [128 rows, box_k
 // elements], swizzle = the box's row bytes.
-bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K, int box_k, bool u8) {
+bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K, int box_k, bool u8, int box_rows) {
   auto enc = get_encode();
   if (!enc) return false;
   const int es = u8 ? 1 : 2;
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)(rows > 0 ? rows : 1)};
   cuuint64_t strides[1] = {(cuuint64_t)K * es};
-  cuuint32_t box[2] = {(cuuint32_t)box_k, BM};
+  cuuint32_t box[2] = {(cuuint32_t)box_k, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(box_k * es),

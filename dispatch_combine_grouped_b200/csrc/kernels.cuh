@@ -170,7 +170,8 @@ cudaError_t launch_ep_combine(const moe_config& c, const EpPeers& peers, const E
 
 int sm_count();
 // TMA maps for bf16 K-major operands; box_k (64, 32 or 16) selects the 128/64/32-byte swizzle
-bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K, int box_k = 64, bool u8 = false);
+bool make_map_a(CUtensorMap* m, const void* base, long long rows, long long K, int box_k = 64, bool u8 = false,
+                int box_rows = 128);
 bool make_map_b(CUtensorMap* m, const void* base, long long G, long long R, long long K, int box_rows,
                 int box_k = 64, bool u8 = false);
 

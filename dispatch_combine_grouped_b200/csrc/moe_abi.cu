@@ -206,17 +206,13 @@ GemmArgs fc2_args(const moe_config& c, const moe_layout& L, const void* h, const
   return g;
 }
 
-// bf16: 256-row pair tiles on CTA pairs first, then the 0..128-row tails on single CTAs.
-// Pairs are used for wide hidden sizes (d >= 4096), where they measured faster on B200
-// (they halve each SM's weight-tile traffic and deepen the load ring); with d = 2048 the
-// one-CTA tiles measured faster.  A group has at most N rows, so with N <= 128 every row
-// is a tail.
+// Tensor-core grouped GEMM: on CTA pairs for wide hidden sizes (d >= 4096), where every
+// row of a group runs in one pass over its weights (256-row blocks, the 1..128 rows past
+// the last block carried on it, or one 128-row tile for a group of at most 128 rows); with
+// d = 2048 the one-CTA 128-row tiles measured faster.  A group has at most N rows, so with
+// N <= 128 the one-CTA kernel runs.
 cudaError_t tc_grouped(GemmArgs g, const moe_config& c, int a0_rows, int a1_rows, cudaStream_t st) {
-  if (c.N > 128 && c.d >= 4096) {
-    cudaError_t e = launch_tc_gemm_pair(g, a0_rows, a1_rows, st);
-    if (e != cudaSuccess) return e;
-    g.tail_only = 1;
-  }
+  if (c.N > 128 && c.d >= 4096) return launch_tc_gemm_pair(g, a0_rows, a1_rows, st);
   return launch_tc_gemm(g, a0_rows, a1_rows, st);
 }
 
