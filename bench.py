@@ -854,10 +854,9 @@ def run_fp8(args, cfg, world, rank, local):
     fp8_peak = 2.0 * bpeak
     ffn_tflops = alg["ffn_flops"] / (stage_ms["ffn"] / 1e3) / 1e12
     # launches of one fused step: router 2, x quantisation 1, layout 3, permute 1, combine 1,
-    # and per FFN group range FC1 + h quantisation + FC2 (FC1 / FC2 as pair + tail launches
-    # on the CTA-pair path), once for the routed experts and once for the shared ones
-    gl = 2 if (cfg.N > 128 and cfg.d >= 4096) else 1
-    launches = 2 + 1 + 3 + 1 + 1 + (2 * gl + 1) * (2 if S else 1)
+    # and per FFN group range FC1 + h quantisation + FC2, once for the routed experts and
+    # once for the shared ones
+    launches = 2 + 1 + 3 + 1 + 1 + 3 * (2 if S else 1)
     if rank == 0:
         line = {
             "metric": METRIC, "value": whole_job_tokens_per_s(cfg.N, world, step_ms), "unit": "tokens/s",
@@ -1125,7 +1124,7 @@ def bench_layer(args, cfg, world, rank, local, steps, warmup, headline=True):
         "warmup": warmup, "ms_per_step": step_ms_max, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded normal inputs, random-init weights)",
         "config": config_dict(cfg, world),
-        "roofline": {"kernel": "routed grouped FC1 + SwiGLU (tcgen05; CTA-pair and one-CTA tiles)",
+        "roofline": {"kernel": "routed grouped FC1 + SwiGLU (tcgen05)",
                      "bound": "tensor", "achieved": fc1_tflops, "peak": tpeak, "unit": "TFLOP/s",
                      "frac": fc1_tflops / tpeak,
                      "peak_source": f"{peak_src} bf16 {tkind} (median SM clock during the timed steps "
@@ -1175,10 +1174,9 @@ def bench_layer(args, cfg, world, rank, local, steps, warmup, headline=True):
 
 def kernel_launches_per_step(cfg, R=0):
     """This library's kernels in one timed step: router (GEMM + top-k), three layout
-    kernels, permute, FC1 and FC2 per group range (a pair-tile and a tail launch each on
-    the CTA-pair path), combine, and the replica assignment's four with redundant slots."""
-    gl = 2 if (cfg.dtype == "bf16" and cfg.N > 128 and cfg.d >= 4096) else 1
-    return 2 + 3 + 1 + 2 * gl + (2 * gl if cfg.S else 0) + 1 + (4 if R else 0)
+    kernels, permute, FC1 and FC2 per group range (routed, then shared), combine, and the
+    replica assignment's four with redundant slots."""
+    return 2 + 3 + 1 + 2 + (2 if cfg.S else 0) + 1 + (4 if R else 0)
 
 
 def summarize(line) -> dict:

@@ -95,7 +95,7 @@ def test_default_workload_is_the_wide_layer():
 
 
 def test_launch_count_per_step():
-    # wide: router 2, layout 3, permute 1, routed FC1/FC2 pair + tail (4), shared (4), combine 1
-    assert bench.kernel_launches_per_step(CONFIGS["wide"]) == 15
+    # wide: router 2, layout 3, permute 1, routed FC1/FC2 2, shared FC1/FC2 2, combine 1
+    assert bench.kernel_launches_per_step(CONFIGS["wide"]) == 11
     assert bench.kernel_launches_per_step(CONFIGS["fine"]) == 2 + 3 + 1 + 2 + 2 + 1
-    assert bench.kernel_launches_per_step(CONFIGS["hot"]) == 2 + 3 + 1 + 4 + 0 + 1
+    assert bench.kernel_launches_per_step(CONFIGS["hot"]) == 2 + 3 + 1 + 2 + 0 + 1
