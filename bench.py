@@ -1063,6 +1063,37 @@ def bench_layer(args, cfg, world, rank, local, steps, warmup, headline=True):
     combine_ms = kernel_ms(lambda: moe.combine(pcfg, layout, out, y=y))
 
     fused_ms, e2e_ms = None, None
+    chunked = None
+    if headline or cfg.name == "hot_cal":
+        # the chunked pipeline (moe_layer_forward_chunked) beside the unchunked overlapped
+        # forward, same steps and flushes
+        chunked = {}
+        for nc in (1, 2, 4):
+            cws = torch.empty(max(moe.workspace_bytes_chunked(cfg, nc), 1), dtype=torch.uint8, device=dev)
+            moe.layer_forward_chunked(cfg, nc, x, wg, bias, owner, w13, w2, side, y=y, ws=cws, status=status)
+            cev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(min(steps, 10))]
+            for a, b in cev:
+                flush.zero_()
+                a.record()
+                moe.layer_forward_chunked(cfg, nc, x, wg, bias, owner, w13, w2, side, y=y, ws=cws, status=status)
+                b.record()
+            torch.cuda.synchronize()
+            chunked[str(nc)] = sorted(a.elapsed_time(b) for a, b in cev)[len(cev) // 2]
+            del cws
+        uev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(min(steps, 10))]
+        for a, b in uev:
+            flush.zero_()
+            a.record()
+            moe.layer_forward_overlapped(cfg, x, wg, bias, owner, w13, w2, side, y=y, ws=ws, status=status)
+            b.record()
+        torch.cuda.synchronize()
+        chunked = {"ms_per_step_by_chunks": chunked,
+                   "unchunked_overlapped_ms": sorted(a.elapsed_time(b) for a, b in uev)[len(uev) // 2],
+                   "how": "moe_layer_forward_chunked with 1, 2, 4 token chunks (layout and permute of chunk c "
+                          "beside the experts of chunk c-1 on a side stream) against moe_layer_forward_overlapped, "
+                          "median of the steps, L2 flushed before each"}
     if headline:
         # the fused entry point (one C call per step, same kernels and order as the timed step)
         fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
@@ -1157,6 +1188,8 @@ def bench_layer(args, cfg, world, rank, local, steps, warmup, headline=True):
         "clocks": clock_rec,
         "wall_s_timed": wall,
     }
+    if chunked is not None:
+        line["chunked"] = chunked
     if headline:
         line["fused_ms_per_step"] = fused_ms
         line["e2e"] = {"value": whole_job_tokens_per_s(cfg.N, world, e2e_ms), "unit": "tokens/s",
@@ -1194,6 +1227,8 @@ def summarize(line) -> dict:
             "gpu_launches": line["gpu_launches"]}
     if "cpu_baseline" in line:
         keep["cpu_baseline"] = line["cpu_baseline"]
+    if "chunked" in line:
+        keep["chunked"] = line["chunked"]
     return keep
 
 

@@ -10,7 +10,8 @@ from .binding import (EXPORTED, Layout, MoEError, alloc_workspace, c_config, che
                       expert_fc2, grouped_ffn, layer_forward, layer_forward_overlapped, layout_workspace_bytes,
                       load, permute, permute_staged, route, routed_ffn, selftest_bounded_wait, shared_ffn, version,
                       workspace_bytes, quantize_fp8, permute_fp8, grouped_ffn_fp8, workspace_bytes_fp8,
-                      layer_forward_fp8, capacity_drop, capacity_of, checks_enabled, checks_register)
+                      layer_forward_fp8, capacity_drop, capacity_of, checks_enabled, checks_register,
+                      layer_forward_chunked, workspace_bytes_chunked)
 
 from . import ep  # noqa: F401,E402  (expert parallelism across GPUs: moe_ep_*)
 

@@ -34,7 +34,8 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_checks_en
             "moe_layer_forward", "moe_eplb_plan", "moe_eplb_workspace_bytes", "moe_eplb_assign",
             "moe_eplb_place_weights", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8",
             "moe_workspace_bytes_fp8", "moe_layer_forward_fp8", "moe_capacity_drop", "moe_capacity_rows",
-            "moe_layer_forward_fp8_overlapped", "moe_ep_window_bytes", "moe_ep_window_layout",
+            "moe_layer_forward_fp8_overlapped", "moe_workspace_bytes_chunked", "moe_layer_forward_chunked",
+            "moe_ep_window_bytes", "moe_ep_window_layout",
             "moe_ep_workspace_bytes", "moe_ep_ipc_handle", "moe_ep_ipc_open", "moe_ep_ipc_close", "moe_ep_notify",
             "moe_ep_layout", "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ep_layer_forward",
             "moe_ep_workspace_bytes_fp8", "moe_ep_dispatch_fp8", "moe_ep_expert_ffn_fp8", "moe_ep_layer_forward_fp8",
@@ -118,6 +119,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_layer_forward_fp8": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp]),
         "moe_capacity_drop": (i32, [cfgp, vp, i32, vp, vp, vp, sz, vp]),
         "moe_capacity_rows": (i32, [cfgp, ctypes.c_double, ctypes.POINTER(i32)]),
+        "moe_workspace_bytes_chunked": (sz, [cfgp, i32]),
+        "moe_layer_forward_chunked": (i32, [cfgp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]),
         "moe_layer_forward_fp8_overlapped": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp,
                                                    vp]),
     }
@@ -388,6 +391,27 @@ def layer_forward_overlapped(cfg, x, w_gate, bias, expert_owner, w13, w2, side_s
                                                _p(w13), _p(w2), _p(y), lay, _p(status), _p(ws), ws.numel(), _stream(),
                                                ctypes.c_void_p(side_stream.cuda_stream)),
            "moe_layer_forward_overlapped")
+    return y
+
+
+def workspace_bytes_chunked(cfg, n_chunks: int) -> int:
+    c = c_config(cfg)
+    return load().moe_workspace_bytes_chunked(ctypes.byref(c), int(n_chunks))
+
+
+def layer_forward_chunked(cfg, n_chunks, x, w_gate, bias, expert_owner, w13, w2, side_stream, y=None, ws=None,
+                          status=None):
+    """moe_layer_forward_chunked: the layer as a pipeline over n_chunks token chunks (layout
+    and permute on the current stream, expert FFN on ``side_stream``)."""
+    c = c_config(cfg)
+    if ws is None:
+        ws = torch.empty(max(workspace_bytes_chunked(cfg, n_chunks), 1), dtype=torch.uint8, device=x.device)
+    if y is None:
+        y = torch.empty(cfg.N, cfg.d, dtype=x.dtype, device=x.device)
+    _check(load().moe_layer_forward_chunked(ctypes.byref(c), int(n_chunks), _p(x), _p(w_gate), _p(bias),
+                                            _p(expert_owner), _p(w13), _p(w2), _p(y), _p(status), _p(ws), ws.numel(),
+                                            _stream(), ctypes.c_void_p(side_stream.cuda_stream)),
+           "moe_layer_forward_chunked")
     return y
 
 

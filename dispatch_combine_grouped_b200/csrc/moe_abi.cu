@@ -810,6 +810,121 @@ moe_status moe_layer_forward_overlapped(const moe_config* cfg, const void* x, co
   return cuda_status(launch_combine(c, L, w.out, nullptr, y, st), "combine");
 }
 
+}  // extern "C"
+
+namespace {
+
+// ------------------------------------------------------------------ chunked pipeline
+// The tokens in n_chunks contiguous chunks, each a layer of its own after one router
+// launch over all of them ([EP-DeepEP] §7: T = T_warm + sum over chunks of max(T_disp,
+// T_exp, T_comb) + T_drain).  Chunk c's layout and permute run on `stream` beside chunk
+// c-1's expert FFN on `side_stream`; chunk c-1's combine follows on `stream`.
+constexpr int kMaxChunks = 16;
+
+struct ChunkPlan {
+  int n_chunks, per;  // tokens per chunk (the last one may hold fewer)
+  moe_config cc[kMaxChunks];
+  size_t off[kMaxChunks];  // workspace offset of each chunk's buffers
+  size_t route_bytes, total;
+};
+
+ChunkPlan plan_chunks(const moe_config& c, int n_chunks) {
+  ChunkPlan pl;
+  memset(&pl, 0, sizeof(pl));
+  pl.n_chunks = n_chunks;
+  pl.per = (c.N + n_chunks - 1) / n_chunks;
+  // routing of all tokens: logits, ids, gates
+  const size_t A = (size_t)c.N * c.k;
+  pl.route_bytes = align256((size_t)c.N * c.E * 4) + 2 * align256(A * 4 ? A * 4 : 1);
+  size_t off = pl.route_bytes;
+  for (int i = 0; i < n_chunks; ++i) {
+    pl.cc[i] = c;
+    const int t0 = i * pl.per;
+    pl.cc[i].N = t0 >= c.N ? 0 : (c.N - t0 < pl.per ? c.N - t0 : pl.per);
+    pl.off[i] = off;
+    off += carve_forward(pl.cc[i], nullptr).total;
+  }
+  pl.total = off;
+  return pl;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_bytes_chunked(const moe_config* cfg, int32_t n_chunks) {
+  if (check_config(cfg) != MOE_OK || n_chunks < 1 || n_chunks > kMaxChunks) return 0;
+  return plan_chunks(*cfg, n_chunks).total;
+}
+
+moe_status moe_layer_forward_chunked(const moe_config* cfg, int32_t n_chunks, const void* x, const void* w_gate,
+                                     const float* bias, const int32_t* expert_owner, const void* w13, const void* w2,
+                                     void* y, int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                     moe_stream_t side_stream) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if ((s = check_router(*cfg)) != MOE_OK) return s;
+  if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
+  if (n_chunks < 1 || n_chunks > kMaxChunks) return fail(MOE_ERR_INVALID_ARG, "n_chunks must be in [1, 16]");
+  const moe_config& c = *cfg;
+  const ChunkPlan pl = plan_chunks(c, n_chunks);
+  if (!ws || ws_bytes < pl.total) return fail(MOE_ERR_WORKSPACE, "chunked forward workspace too small");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return fail(MOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if (c.N == 0) return MOE_OK;
+  if (!x || !w_gate || !w13 || !w2 || !y) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  cudaStream_t st = (cudaStream_t)stream, side = (cudaStream_t)side_stream;
+  char* base = static_cast<char*>(ws);
+  const size_t A = (size_t)c.N * c.k;
+  float* logits = reinterpret_cast<float*>(base);
+  int32_t* ids = reinterpret_cast<int32_t*>(base + align256((size_t)c.N * c.E * 4));
+  float* gates = reinterpret_cast<float*>(reinterpret_cast<char*>(ids) + align256(A * 4));
+  if ((s = route_impl(c, x, w_gate, bias, logits, ids, gates, st)) != MOE_OK) return s;
+  const size_t xrow = (size_t)c.d * elem_bytes(c);
+  cudaEvent_t ev[2 * kMaxChunks];
+  int n_ev = 0;
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < 2 * n_chunks && e == cudaSuccess; ++i) {
+    e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+    if (e == cudaSuccess) ++n_ev;
+  }
+  FwdWs w[kMaxChunks];
+  const char* xs[kMaxChunks];
+  auto combine_chunk = [&](int i) -> moe_status {  // on `stream`, after chunk i's FFN
+    if (pl.cc[i].N == 0) return MOE_OK;
+    cudaError_t ee = cudaStreamWaitEvent(st, ev[n_chunks + i], 0);
+    if (ee != cudaSuccess) return cuda_status(ee, "chunk join");
+    return cuda_status(launch_combine(pl.cc[i], w[i].lay, w[i].out, nullptr,
+                                      static_cast<char*>(y) + (size_t)i * pl.per * xrow, st),
+                       "combine");
+  };
+  s = e == cudaSuccess ? MOE_OK : cuda_status(e, "chunk events");
+  for (int i = 0; i < n_chunks && s == MOE_OK; ++i) {
+    const moe_config& cc = pl.cc[i];
+    w[i] = carve_forward(cc, base + pl.off[i]);
+    xs[i] = static_cast<const char*>(x) + (size_t)i * pl.per * xrow;
+    if (cc.N > 0) {
+      // stream: this chunk's layout and permute (beside the FFN of the chunk before)
+      const int32_t* ids_i = ids + (size_t)i * pl.per * c.k;
+      s = cuda_status(launch_layout(cc, expert_owner, ids_i, w[i].lay, dev_status, w[i].lay_ws, st), "layout");
+      if (s == MOE_OK) s = cuda_status(launch_permute(cc, w[i].lay, xs[i], w[i].x_perm, st), "permute");
+      if (s == MOE_OK) s = cuda_status(cudaEventRecord(ev[i], st), "chunk fork");
+      // side stream: its experts (routed rows, then the shared experts over its tokens)
+      if (s == MOE_OK) s = cuda_status(cudaStreamWaitEvent(side, ev[i], 0), "chunk fork");
+      if (s == MOE_OK)
+        s = ffn_impl(cc, w[i].lay, w[i].x_perm, xs[i], w13, w2, gates + (size_t)i * pl.per * c.k, w[i].h,
+                     w[i].out, side);
+    }
+    if (s == MOE_OK) s = cuda_status(cudaEventRecord(ev[n_chunks + i], side), "chunk done");
+    // stream: the combine of the chunk before, now that this chunk's movement is queued
+    if (s == MOE_OK && i > 0) s = combine_chunk(i - 1);
+  }
+  if (s == MOE_OK) s = combine_chunk(n_chunks - 1);
+  // whatever happened, `stream` orders after all the side stream's work
+  if (n_ev == 2 * n_chunks && cudaEventRecord(ev[0], side) == cudaSuccess) cudaStreamWaitEvent(st, ev[0], 0);
+  for (int i = 0; i < n_ev; ++i) cudaEventDestroy(ev[i]);
+  return s;
+}
+
 size_t moe_eplb_workspace_bytes(const moe_config* cfg) {
   if (check_config(cfg) != MOE_OK) return 0;
   return eplb_ws_bytes(*cfg);

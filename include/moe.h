@@ -341,6 +341,30 @@ moe_status moe_layer_forward_overlapped(const moe_config* cfg, const void* x, co
                                         moe_stream_t stream, moe_stream_t side_stream);
 
 /*
+ * The layer as a pipeline over token chunks ([EP-DeepEP] §7, pipelined overlap: the layer
+ * time approaches T_warm + sum over chunks of max(T_disp, T_exp, T_comb) + T_drain).  The
+ * N tokens are split into n_chunks contiguous chunks of ceil(N / n_chunks) tokens (the last
+ * may hold fewer, and chunks past the end hold none).  One router launch covers all tokens;
+ * then each chunk is a layer of its own: its layout (its own counts, offsets and maps over
+ * its tokens) and permute on `stream`, its expert FFN (routed, then shared experts) on
+ * `side_stream`, and its combine on `stream` again, so that chunk c's layout and permute
+ * and chunk c-2's combine run beside chunk c-1's experts.  Each token's output rows are
+ * computed exactly as in moe_layer_forward (the same kernels, the same k order), so y is
+ * the same.  On one GPU the experts' weights are streamed once per chunk; the form pays
+ * off where the movement is long against the experts (the all-to-all of an EP layer).
+ *   n_chunks        1 .. 16
+ *   ws, ws_bytes    at least moe_workspace_bytes_chunked(cfg, n_chunks), 256-byte aligned
+ *   stream, side_stream  two different streams; when the call returns, `stream` orders
+ *                   after all the work and `side_stream` may be reused immediately
+ * Errors as moe_layer_forward; n_chunks outside [1, 16] -> MOE_ERR_INVALID_ARG.
+ */
+size_t moe_workspace_bytes_chunked(const moe_config* cfg, int32_t n_chunks);
+moe_status moe_layer_forward_chunked(const moe_config* cfg, int32_t n_chunks, const void* x, const void* w_gate,
+                                     const float* bias, const int32_t* expert_owner, const void* w13, const void* w2,
+                                     void* y, int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                     moe_stream_t side_stream);
+
+/*
  * Redundant expert slots, EPLB ([WideEP] "为什么要把 EP 做宽": E logical experts plus R
  * copies make E + R physical experts, (E + R) / P per owner; "DeepSeek-V3/R1 的两个具体
  * 布局": 256 + 32 = 288 slots; "Expert 副本在 Wide EP 中还有整除作用": hot experts are
