@@ -111,7 +111,7 @@ inline long long launch_rows(const GemmArgs& g) {
 
 // tensor-core (tcgen05) path, bf16 operands, fp32 accumulation: one CTA per tile
 cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStream_t st);
-// the same over CTA pairs (cta_group::2, 256 x 256 tiles) for the rows pair_rows() covers
+// the same over CTA pairs (cta_group::2): every row of a group in one pass over its weights
 cudaError_t launch_tc_gemm_pair(const GemmArgs& g, int a0_rows, int a1_rows, cudaStream_t st);
 // CUDA-core path, fp32 operands (the fp32 configurations)
 cudaError_t launch_simt_gemm(const GemmArgs& g, cudaStream_t st);
