@@ -20,6 +20,19 @@ notes):
   * GEMMs: D = (sum_k qa_k qb_k) * s_row * s_col; the combine is unchanged (fp32
     accumulation, bf16 output); h is rounded to bf16 before its own quantisation, as the
     CUDA path stores it.
+
+The block-scaled (MX) form.  "MoE我们喜欢你（四）" names MXFP8 beside FP8 as the low-precision
+expert compute; the pages do not define the format, so the reading is the published
+microscaling (MX) format for FP8 elements:
+  * a block is 32 consecutive values along the reduction dimension (K) of one row;
+  * its shared scale is a power of two X = 2^e stored as one unbiased-exponent byte
+    (E8M0: byte b means 2^(b-127); 255 is NaN and never written);
+  * e = floor(log2(max |v| of the block)) - 8, where 8 is the exponent of the largest power
+    of two e4m3 holds (256), clamped to [-127, 127]; an all-zero block takes e = -127;
+  * each element's code is the e4m3 round-to-nearest-even of v / X, saturating at +-448
+    (so the largest element, whose v / X lies in [256, 512), may clip to 448);
+  * a GEMM on MX operands is D = sum_k (qa_k * Xa(k // 32)) * (qb_k * Xb(k // 32)).
+v / X is exact (a power-of-two scaling), so the codes are a function of the stored values.
 """
 from __future__ import annotations
 
@@ -91,3 +104,61 @@ def fc1(qx_rows, sx_rows, qw13, sw13, I: int) -> np.ndarray:
 
 def fc2(qh_rows, sh_rows, qw2, sw2) -> np.ndarray:
     return gemm_rows(qh_rows, sh_rows, qw2, sw2)
+
+
+# ---------------------------------------------------------------------------------------
+# Block-scaled (MX) e4m3: 32-value blocks along K, one E8M0 power-of-two scale per block.
+# ---------------------------------------------------------------------------------------
+MX_BLOCK = 32
+E4M3_EMAX = 8  # 2^8 = 256 is the largest power of two e4m3 represents
+
+
+def e8m0_decode(b) -> np.ndarray:
+    """Scale of every E8M0 byte: 2^(b - 127); 255 is NaN."""
+    b = np.asarray(b, dtype=np.int64)
+    return np.where(b == 255, np.nan, np.ldexp(1.0, (b - 127).clip(-127, 127)))
+
+
+def mx_block_exponent(amax) -> np.ndarray:
+    """e of a block with largest magnitude amax (float64 array): floor(log2 amax) - 8,
+    clamped to [-127, 127]; -127 for amax == 0.  np.frexp writes amax = m 2^f with m in
+    [0.5, 1), so floor(log2 amax) = f - 1 exactly (subnormal amax included)."""
+    amax = np.asarray(amax, dtype=np.float64)
+    _, f = np.frexp(amax)
+    e = np.where(amax > 0, f.astype(np.int64) - 1 - E4M3_EMAX, -127)
+    return np.clip(e, -127, 127)
+
+
+def quantize_mx(x):
+    """MX quantisation of rows (the reading above).  x: [R, C] values exactly representable
+    in fp32 (bf16 or fp32 storage), C % 32 == 0.  Returns (codes uint8 [R, C], scale bytes
+    uint8 [R, C // 32])."""
+    x64 = np.asarray(x, dtype=np.float32).astype(np.float64)
+    R, C = x64.shape
+    assert C % MX_BLOCK == 0
+    blocks = x64.reshape(R, C // MX_BLOCK, MX_BLOCK)
+    e = mx_block_exponent(np.abs(blocks).max(axis=2) if C else np.zeros((R, 0)))
+    q = e4m3_encode(blocks * np.ldexp(1.0, -e)[:, :, None])  # exact scaling in float64
+    return q.reshape(R, C), (e + 127).astype(np.uint8)
+
+
+def dequantize_mx(codes, sf) -> np.ndarray:
+    """Values of MX rows: code value times its block's scale (float64)."""
+    scale = np.repeat(e8m0_decode(sf), MX_BLOCK, axis=1)
+    return e4m3_decode(codes) * scale
+
+
+def gemm_mx(qa, sa, qb, sb) -> np.ndarray:
+    """D[i, j] = sum_k (qa_ik Xa_i,k//32) (qb_jk Xb_j,k//32) in float64 (the products are
+    exact; only the sum rounds)."""
+    return dequantize_mx(qa, sa) @ dequantize_mx(qb, sb).T
+
+
+def fc1_mx(qx_rows, sx_rows, qw13, sw13, I: int) -> np.ndarray:
+    """SwiGLU activations of one expert's rows from MX operands (float64)."""
+    z = gemm_mx(qx_rows, sx_rows, qw13, sw13)
+    return silu(z[:, :I]) * z[:, I:]
+
+
+def fc2_mx(qh_rows, sh_rows, qw2, sw2) -> np.ndarray:
+    return gemm_mx(qh_rows, sh_rows, qw2, sw2)

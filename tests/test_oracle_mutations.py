@@ -224,3 +224,32 @@ def test_ep_receive_order_mistakes_are_caught(monkeypatch, name, mut):
     assert _ep_pins_fail() == 0, "the unmodified oracle passes its EP pins"
     monkeypatch.setattr(O, "_ep_receive_lists", mut)
     assert _ep_pins_fail() >= 1, name
+
+
+import tests.test_mx_oracle as mx_pins
+
+
+def test_mx_exponent_off_by_one_is_caught(monkeypatch):
+    orig = F8.mx_block_exponent
+    monkeypatch.setattr(F8, "mx_block_exponent", lambda amax: np.clip(orig(amax) + 1, -127, 127))
+    _fails(mx_pins.test_block_exponent_against_brute_force)
+    _fails(mx_pins.test_hand_values)
+
+
+def test_mx_scale_by_column_instead_of_block_is_caught(monkeypatch):
+    # a scale looked up by k % (K/32) instead of k // 32
+    def tiled(codes, sf):
+        return F8.e4m3_decode(codes) * np.tile(F8.e8m0_decode(sf), (1, F8.MX_BLOCK))
+    monkeypatch.setattr(F8, "dequantize_mx", tiled)
+    _fails(mx_pins.test_gemm_brute_force_and_block_indexing)
+
+
+def test_mx_ceil_exponent_is_caught(monkeypatch):
+    # the other common reading, 2^ceil(log2(amax / 448)): no saturation, a different scale
+    def ceil_exp(amax):
+        amax = np.asarray(amax, dtype=np.float64)
+        with np.errstate(divide="ignore"):
+            e = np.where(amax > 0, np.ceil(np.log2(np.where(amax > 0, amax, 1.0) / 448.0)), -127)
+        return np.clip(e, -127, 127).astype(np.int64)
+    monkeypatch.setattr(F8, "mx_block_exponent", ceil_exp)
+    _fails(mx_pins.test_hand_values)
