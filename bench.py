@@ -48,6 +48,9 @@ def parse():
                          "(one JSON line with the curve)")
     ap.add_argument("--fp8", action="store_true",
                     help="the FP8 (e4m3) expert path: quantised dispatch payload and expert GEMMs")
+    ap.add_argument("--mx", action="store_true",
+                    help="the block-scaled (MX) e4m3 expert path: E8M0 scales per 32 K values, applied "
+                         "by the tensor cores")
     ap.add_argument("--ep", type=int, default=0, metavar="P",
                     help="expert parallelism with P ranks emulated on this GPU (moe_ep_*): per-stage times "
                          "of all ranks, the one-GPU layer beside it, and the NVLink bytes a real P-GPU step moves")
@@ -889,6 +892,129 @@ def run_fp8(args, cfg, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_mx(args, cfg, world, rank, local):
+    """The layer with the MX (block-scaled e4m3) expert path on one stream: route -> layout
+    -> MX quantisation of x + permute of codes and scale rows -> MX grouped FFN (FC1, h
+    quantisation, FC2) -> combine.  Weights are quantised once, before timing."""
+    import torch
+    import dispatch_combine_grouped_b200 as moe
+    from moe_inputs import make_inputs
+
+    dev = torch.device("cuda", local)
+    inp = make_inputs(cfg, device=dev, seed_offset=rank)
+    A, S = cfg.N * cfg.k, cfg.S
+    rows = A + S * cfg.N
+    x, wg, bias, owner = inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"]
+    w13_q, w13_sf = moe.quantize_mx(inp["w13"])
+    w2_q, w2_sf = moe.quantize_mx(inp["w2"])
+    del inp
+    logits = torch.empty(cfg.N, cfg.E, dtype=torch.float32, device=dev)
+    ids = torch.empty(cfg.N, cfg.k, dtype=torch.int32, device=dev)
+    w = torch.empty(cfg.N, cfg.k, dtype=torch.float32, device=dev)
+    layout = moe.Layout(cfg, dev)
+    lay_ws = torch.empty(max(moe.layout_workspace_bytes(cfg), 1), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    x_q = torch.empty(cfg.N, cfg.d, dtype=torch.uint8, device=dev)
+    x_sf = torch.empty(cfg.N, cfg.d // 32, dtype=torch.uint8, device=dev)
+    x_perm = torch.empty(A, cfg.d, dtype=torch.uint8, device=dev)
+    x_sf_perm = torch.empty(A, cfg.d // 32, dtype=torch.uint8, device=dev)
+    h = torch.empty(rows, cfg.I, dtype=torch.bfloat16, device=dev)
+    h_q = torch.empty(rows, cfg.I, dtype=torch.uint8, device=dev)
+    h_sf = torch.empty(rows, cfg.I // 32, dtype=torch.uint8, device=dev)
+    out = torch.empty(rows, cfg.d, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(cfg.N, cfg.d, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(moe.workspace_bytes_mx(cfg), 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def events(n):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    def step(ev):
+        ev[0].record()
+        moe.route(cfg, x, wg, bias, out=(logits, ids, w))
+        ev[1].record()
+        moe.dispatch_layout(cfg, ids, owner, status=status, layout=layout, ws=lay_ws)
+        ev[2].record()
+        moe.quantize_mx(x, out=x_q, sf=x_sf)
+        moe.permute_mx(cfg, layout, x_q, x_sf, out=x_perm, sf_out=x_sf_perm)
+        ev[3].record()
+        moe.grouped_ffn_mx(cfg, layout, x_perm, x_sf_perm, x_q, x_sf, w13_q, w13_sf, w2_q, w2_sf, topk_w=w, h=h,
+                           h_q=h_q, h_sf=h_sf, out=out)
+        ev[4].record()
+        moe.combine(cfg, layout, out, y=y)
+        ev[5].record()
+
+    def fused(ev):
+        ev[0].record()
+        moe.layer_forward_mx(cfg, x, wg, bias, owner, w13_q, w13_sf, w2_q, w2_sf, y=y, ws=ws, status=status)
+        ev[1].record()
+
+    clocks = ClockSampler(local)
+    evs = [events(2) for _ in range(args.steps)]
+    clocks.start()
+    for _ in range(args.warmup):
+        flush.zero_()
+        fused(events(2))
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.mark_timed()
+    for i in range(args.steps):
+        flush.zero_()
+        fused(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clock_rec = clocks.stop()
+    assert status.item() == 0, f"device status {status.item()}"
+    step_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world, dev)
+    sev = [events(6) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        step(sev[i])
+    torch.cuda.synchronize()
+    names = ["route", "layout", "quantize_permute", "ffn", "combine"]
+    stage_ms = {n: sum(ev[j].elapsed_time(ev[j + 1]) for ev in sev) / args.steps for j, n in enumerate(names)}
+    e2e_ms = max_over_ranks(e2e_pipelined(
+        lambda xd, yd: moe.layer_forward_mx(cfg, xd, wg, bias, owner, w13_q, w13_sf, w2_q, w2_sf, y=yd, ws=ws,
+                                            status=status), x, y, flush, max(args.steps, 8)), world, dev)
+    alg = algorithmic(cfg)
+    peaks, peak_src = load_peaks()
+    bpeak, tkind = tensor_peak(peaks, clock_rec)
+    fp8_peak = 2.0 * bpeak
+    ffn_tflops = alg["ffn_flops"] / (stage_ms["ffn"] / 1e3) / 1e12
+    # launches of one fused step: router 2, x quantisation 1, layout 3, permute 2 (codes and
+    # scale rows), FC1 + h quantisation + FC2 3, combine 1
+    launches = 2 + 1 + 3 + 2 + 3 + 1
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": whole_job_tokens_per_s(cfg.N, world, step_ms), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "MX e4m3 expert GEMM operands (E8M0 scale per 32 K values) and dispatch payload, "
+                     "fp32 accumulate, bf16 activations",
+            "data": "synthetic (seeded normal inputs, random-init weights)",
+            "config": {"workload": describe(cfg) + " with the MX expert path", "tokens_per_gpu": cfg.N,
+                       "l2": "flushed before every step (256 MiB write, outside the step's event bracket)",
+                       "parallelism": f"{world} independent replicas (one batch per GPU)"},
+            "roofline": {"kernel": "MX grouped FFN (FC1 + h quantisation + FC2, tcgen05 kind::mxf8f6f4.block_scale)",
+                         "bound": "tensor", "achieved": ffn_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": ffn_tflops / fp8_peak,
+                         "peak_source": f"{peak_src} bf16 {tkind} x 2 (nominal e4m3 / bf16 ratio)",
+                         "traffic": None, "flops_per_launch": alg["ffn_flops"], "ms_per_launch": stage_ms["ffn"]},
+            "stages_ms": stage_ms,
+            "ffn": {"tflops": ffn_tflops, "frac_of_fp8_peak": ffn_tflops / fp8_peak,
+                    "frac_of_bf16_peak": ffn_tflops / bpeak},
+            "e2e": {"value": whole_job_tokens_per_s(cfg.N, world, e2e_ms), "unit": "tokens/s",
+                    "h2d_bytes_per_step": x.numel() * x.element_size(),
+                    "d2h_bytes_per_step": y.numel() * y.element_size(), "ms_per_step": e2e_ms},
+            "gpu_launches": launches * args.steps,
+            "clocks": clock_rec,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def bench_layer(args, cfg, world, rank, local, steps, warmup, headline=True):
     """One workload: W warm-up steps, K timed steps (the product's overlapped order, CUDA
     events between the stages), a one-stream pass for the per-stage breakdown, the movement
@@ -1267,8 +1393,8 @@ def main():
             dist.barrier()
             dist.destroy_process_group()
         return
-    if args.fp8:
-        run_fp8(args, cfg, world, rank, local)
+    if args.fp8 or args.mx:
+        (run_mx if args.mx else run_fp8)(args, cfg, world, rank, local)
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()

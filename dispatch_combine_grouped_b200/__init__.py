@@ -11,7 +11,8 @@ from .binding import (EXPORTED, Layout, MoEError, alloc_workspace, c_config, che
                       load, permute, permute_staged, route, routed_ffn, selftest_bounded_wait, shared_ffn, version,
                       workspace_bytes, quantize_fp8, permute_fp8, grouped_ffn_fp8, workspace_bytes_fp8,
                       layer_forward_fp8, capacity_drop, capacity_of, checks_enabled, checks_register,
-                      layer_forward_chunked, workspace_bytes_chunked)
+                      layer_forward_chunked, workspace_bytes_chunked, quantize_mx, permute_mx,
+                      grouped_ffn_mx, workspace_bytes_mx, layer_forward_mx)
 
 from . import ep  # noqa: F401,E402  (expert parallelism across GPUs: moe_ep_*)
 

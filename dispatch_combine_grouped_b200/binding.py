@@ -39,7 +39,9 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_checks_en
             "moe_ep_workspace_bytes", "moe_ep_ipc_handle", "moe_ep_ipc_open", "moe_ep_ipc_close", "moe_ep_notify",
             "moe_ep_layout", "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ep_layer_forward",
             "moe_ep_workspace_bytes_fp8", "moe_ep_dispatch_fp8", "moe_ep_expert_ffn_fp8", "moe_ep_layer_forward_fp8",
-            "moe_ep_layer_forward_overlapped", "moe_ep_layer_forward_fp8_overlapped"]
+            "moe_ep_layer_forward_overlapped", "moe_ep_layer_forward_fp8_overlapped",
+            "moe_quantize_mx", "moe_permute_mx", "moe_grouped_ffn_mx", "moe_workspace_bytes_mx",
+            "moe_layer_forward_mx"]
 
 
 class CConfig(ctypes.Structure):
@@ -116,6 +118,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_permute_fp8": (i32, [cfgp, layp, vp, vp, vp]),
         "moe_grouped_ffn_fp8": (i32, [cfgp, layp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_workspace_bytes_fp8": (sz, [cfgp]),
+        "moe_quantize_mx": (i32, [vp, ctypes.c_int64, i32, vp, vp, vp]),
+        "moe_permute_mx": (i32, [cfgp, layp, vp, vp, vp, vp, vp]),
+        "moe_grouped_ffn_mx": (i32, [cfgp, layp] + [vp] * 14),
+        "moe_workspace_bytes_mx": (sz, [cfgp]),
+        "moe_layer_forward_mx": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp]),
         "moe_layer_forward_fp8": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp]),
         "moe_capacity_drop": (i32, [cfgp, vp, i32, vp, vp, vp, sz, vp]),
         "moe_capacity_rows": (i32, [cfgp, ctypes.c_double, ctypes.POINTER(i32)]),
@@ -549,6 +556,68 @@ def layer_forward_fp8(cfg, x, w_gate, bias, expert_owner, w13_q, w13_scale, w2_q
     else:
         _check(load().moe_layer_forward_fp8_overlapped(*args, ctypes.c_void_p(side_stream.cuda_stream)),
                "moe_layer_forward_fp8_overlapped")
+    return y
+
+
+# ---------------------------------------------------------------- MX (block-scaled e4m3) expert path
+def quantize_mx(src, out=None, sf=None):
+    """moe_quantize_mx: e4m3 codes (uint8, same shape) and E8M0 scale bytes (uint8, last
+    dimension / 32) of a bf16 tensor whose last dimension is the row."""
+    rows = src.numel() // src.shape[-1]
+    cols = src.shape[-1]
+    if out is None:
+        out = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+    if sf is None:
+        sf = torch.empty(src.shape[:-1] + (cols // 32,), dtype=torch.uint8, device=src.device)
+    _check(load().moe_quantize_mx(_p(src), rows, cols, _p(out), _p(sf), _stream()), "moe_quantize_mx")
+    return out, sf
+
+
+def permute_mx(cfg, layout, x_q, x_sf, out=None, sf_out=None):
+    c = c_config(cfg)
+    A = cfg.N * cfg.k
+    if out is None:
+        out = torch.empty(A, cfg.d, dtype=torch.uint8, device=x_q.device)
+    if sf_out is None:
+        sf_out = torch.empty(A, cfg.d // 32, dtype=torch.uint8, device=x_q.device)
+    _check(load().moe_permute_mx(ctypes.byref(c), ctypes.byref(layout.c), _p(x_q), _p(x_sf), _p(out), _p(sf_out),
+                                 _stream()), "moe_permute_mx")
+    return out, sf_out
+
+
+def grouped_ffn_mx(cfg, layout, x_q_perm, x_sf_perm, x_q, x_sf, w13_q, w13_sf, w2_q, w2_sf, topk_w=None,
+                   h=None, h_q=None, h_sf=None, out=None):
+    """-> (h bf16, h_q e4m3, h_sf E8M0, out bf16) over [A + S*N] rows."""
+    c = c_config(cfg)
+    dev = x_q_perm.device
+    rows = cfg.N * cfg.k + cfg.S * cfg.N
+    h = h if h is not None else torch.empty(rows, cfg.I, dtype=torch.bfloat16, device=dev)
+    h_q = h_q if h_q is not None else torch.empty(rows, cfg.I, dtype=torch.uint8, device=dev)
+    h_sf = h_sf if h_sf is not None else torch.empty(rows, cfg.I // 32, dtype=torch.uint8, device=dev)
+    out = out if out is not None else torch.empty(rows, cfg.d, dtype=torch.bfloat16, device=dev)
+    _check(load().moe_grouped_ffn_mx(ctypes.byref(c), ctypes.byref(layout.c), _p(x_q_perm), _p(x_sf_perm), _p(x_q),
+                                     _p(x_sf), _p(w13_q), _p(w13_sf), _p(w2_q), _p(w2_sf), _p(topk_w), _p(h),
+                                     _p(h_q), _p(h_sf), _p(out), _stream()), "moe_grouped_ffn_mx")
+    return h, h_q, h_sf, out
+
+
+def workspace_bytes_mx(cfg) -> int:
+    c = c_config(cfg)
+    return load().moe_workspace_bytes_mx(ctypes.byref(c))
+
+
+def layer_forward_mx(cfg, x, w_gate, bias, expert_owner, w13_q, w13_sf, w2_q, w2_sf, y=None, ws=None, layout=None,
+                     status=None):
+    """moe_layer_forward_mx: the layer with the MX expert path on the current stream."""
+    c = c_config(cfg)
+    if y is None:
+        y = torch.empty(cfg.N, cfg.d, dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = torch.empty(max(workspace_bytes_mx(cfg), 1), dtype=torch.uint8, device=x.device)
+    _check(load().moe_layer_forward_mx(ctypes.byref(c), _p(x), _p(w_gate), _p(bias), _p(expert_owner), _p(w13_q),
+                                       _p(w13_sf), _p(w2_q), _p(w2_sf), _p(y),
+                                       ctypes.byref(layout.c) if layout is not None else None, _p(status), _p(ws),
+                                       ws.numel(), _stream()), "moe_layer_forward_mx")
     return y
 
 

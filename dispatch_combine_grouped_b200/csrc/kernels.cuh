@@ -87,6 +87,11 @@ struct GemmArgs {
   const float* b_scale; // per weight row [groups, b_rows]
   const float* a_scale_rows;  // FC1: when set, routed row r's scale is a_scale_rows[r] (no row map)
   int* check;           // bounds-checked build: where failed checks are recorded (NULL: nowhere)
+  // block-scaled (MX) e4m3 operands: E8M0 scale bytes, row-major [rows, K/32]
+  const uint8_t* a0_sf;  // rows of A map 0
+  const uint8_t* a1_sf;  // rows of A map 1 (FC1: the tokens, for the shared experts)
+  const uint8_t* b_sf;   // [groups, b_rows, K/32]
+  long long a0_rows, a1_rows;  // rows of the A tensors (the last row is read for rows past them)
 };
 
 #ifdef __CUDACC__
@@ -113,6 +118,8 @@ inline long long launch_rows(const GemmArgs& g) {
 cudaError_t launch_tc_gemm(const GemmArgs& g, int a0_rows, int a1_rows, cudaStream_t st);
 // the same over CTA pairs (cta_group::2): every row of a group in one pass over its weights
 cudaError_t launch_tc_gemm_pair(const GemmArgs& g, int a0_rows, int a1_rows, cudaStream_t st);
+// block-scaled (MX) e4m3 operands with E8M0 scales per 32 K values (FC1 / FC2 only)
+cudaError_t launch_tc_gemm_mx(const GemmArgs& g, cudaStream_t st);
 // CUDA-core path, fp32 operands (the fp32 configurations)
 cudaError_t launch_simt_gemm(const GemmArgs& g, cudaStream_t st);
 
@@ -122,6 +129,8 @@ cudaError_t launch_permute_bytes(const moe_config& c, const moe_layout& L, const
 // FP8 (fp8.cu): per-row e4m3 quantisation of bf16 rows, scale = amax / 448
 cudaError_t launch_quantize_rows(const void* src, long long rows, int cols, void* dst, float* scale,
                                  cudaStream_t st);
+// MX (fp8.cu): e4m3 codes and one E8M0 scale byte per 32 values of a bf16 row; cols % 32 == 0
+cudaError_t launch_quantize_mx(const void* src, long long rows, int cols, void* dst, uint8_t* sf, cudaStream_t st);
 
 // redundant expert slots (eplb.cu)
 size_t eplb_ws_bytes(const moe_config& c);

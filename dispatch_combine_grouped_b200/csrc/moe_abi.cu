@@ -87,11 +87,17 @@ struct FwdWs {
   float* x_scale;
   void* h_q;
   float* h_scale;
+  // MX forward only: E8M0 scale bytes, one per 32 values of a row
+  uint8_t* x_sf;       // [N, d/32]
+  uint8_t* x_sf_perm;  // [A, d/32]
+  uint8_t* h_sf;       // [A + S*N, I/32]
   size_t total;
 };
 
 // fp8: the FP8 forward's buffers (x_perm holds e4m3 rows, plus x_q, h_q and the scales)
-FwdWs carve_forward(const moe_config& c, char* base, bool fp8 = false) {
+// mx: the MX forward's buffers (those of the FP8 forward plus the scale bytes)
+FwdWs carve_forward(const moe_config& c, char* base, bool fp8 = false, bool mx = false) {
+  fp8 = fp8 || mx;
   FwdWs w;
   memset(&w, 0, sizeof(w));
   const size_t A = (size_t)c.N * c.k, E = c.E, P = c.P, S = c.n_shared, eb = elem_bytes(c);
@@ -124,6 +130,11 @@ FwdWs carve_forward(const moe_config& c, char* base, bool fp8 = false) {
     w.x_scale = reinterpret_cast<float*>(take((size_t)c.N * 4));
     w.h_q = take((A + S * c.N) * c.I);
     w.h_scale = reinterpret_cast<float*>(take((A + S * c.N) * 4));
+  }
+  if (mx) {
+    w.x_sf = reinterpret_cast<uint8_t*>(take((size_t)c.N * (c.d / 32)));
+    w.x_sf_perm = reinterpret_cast<uint8_t*>(take(A * (c.d / 32)));
+    w.h_sf = reinterpret_cast<uint8_t*>(take((A + S * c.N) * (c.I / 32)));
   }
   w.total = off;
   return w;
@@ -294,6 +305,56 @@ moe_status ffn_fp8_impl(const moe_config& c, const moe_layout& L, const Fp8Ffn& 
   g2.a_scale = f.h_scale;
   g2.b_scale = f.w2_scale;
   return cuda_status(tc_grouped(g2, c, (int)(A + (long long)c.n_shared * c.N), 0, st), "FC2 grouped GEMM (fp8)");
+}
+
+// MX expert FFN over groups [g0, g0+G): FC1 on block-scaled e4m3 rows -> h (bf16) -> MX
+// quantisation of h -> FC2 on block-scaled rows, on the block-scaled tile kernel.
+struct MxFfn {
+  const void* x_q_perm;
+  const uint8_t* x_sf_perm;
+  const void* x_q;
+  const uint8_t* x_sf;
+  const void* w13_q;
+  const uint8_t* w13_sf;
+  const void* w2_q;
+  const uint8_t* w2_sf;
+  const float* topk_w;
+  void* h;
+  void* h_q;
+  uint8_t* h_sf;
+  void* out;
+};
+
+moe_status ffn_mx_impl(const moe_config& c, const moe_layout& L, const MxFfn& f, cudaStream_t st, int g0 = 0,
+                       int G = -1) {
+  if (G < 0) G = c.E + c.n_shared - g0;
+  if (G == 0) return MOE_OK;
+  const long long A = (long long)c.N * c.k;
+  GemmArgs g = fc1_args(c, L, f.x_q_perm, f.x_q, f.w13_q, f.h);
+  g.g0 = g0;
+  g.G = G;
+  g.max_ctas = shared_cap(c, g0);
+  g.a0_sf = f.x_sf_perm;
+  g.a1_sf = f.x_sf;
+  g.b_sf = f.w13_sf;
+  g.a0_rows = A > 0 ? A : 1;
+  g.a1_rows = c.N;
+  cudaError_t e = launch_tc_gemm_mx(g, st);
+  if (e != cudaSuccess) return cuda_status(e, "FC1 grouped GEMM (mx)");
+  const long long r0 = g0 < c.E ? 0 : A + (long long)(g0 - c.E) * c.N;
+  const long long r1 = (g0 + G <= c.E) ? A : A + (long long)(g0 + G - c.E) * c.N;
+  e = launch_quantize_mx(static_cast<const uint16_t*>(f.h) + r0 * c.I, r1 - r0, c.I,
+                         static_cast<uint8_t*>(f.h_q) + r0 * c.I, f.h_sf + r0 * (c.I / 32), st);
+  if (e != cudaSuccess) return cuda_status(e, "h quantisation (mx)");
+  GemmArgs g2 = fc2_args(c, L, f.h_q, f.w2_q, f.topk_w, f.out);
+  g2.g0 = g0;
+  g2.G = G;
+  g2.max_ctas = shared_cap(c, g0);
+  g2.a0_sf = f.h_sf;
+  g2.b_sf = f.w2_sf;
+  g2.a0_rows = A + (long long)c.n_shared * c.N;
+  g2.a1_rows = g2.a0_rows;
+  return cuda_status(launch_tc_gemm_mx(g2, st), "FC2 grouped GEMM (mx)");
 }
 
 moe_status ffn_impl(const moe_config& c, const moe_layout& L, const void* x_perm, const void* x, const void* w13,
@@ -1095,6 +1156,90 @@ moe_status moe_layer_forward_fp8_overlapped(const moe_config* cfg, const void* x
                                             size_t ws_bytes, moe_stream_t stream, moe_stream_t side_stream) {
   return forward_fp8(cfg, x, w_gate, bias, expert_owner, w13_q, w13_scale, w2_q, w2_scale, y, layout_out,
                      dev_status, ws, ws_bytes, (cudaStream_t)stream, (cudaStream_t)side_stream);
+}
+
+moe_status moe_quantize_mx(const void* src, int64_t rows, int32_t cols, void* dst, uint8_t* sf,
+                           moe_stream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 32 != 0) return fail(MOE_ERR_INVALID_ARG, "need rows >= 0, cols % 32 == 0");
+  if (rows > 0 && (!src || !dst || !sf)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (rows > 0 && ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) != 0)
+    return fail(MOE_ERR_INVALID_ARG, "src and dst must be 16-byte aligned");
+  return cuda_status(launch_quantize_mx(src, rows, cols, dst, sf, (cudaStream_t)stream), "mx quantisation");
+}
+
+static moe_status check_mx(const moe_config* cfg) {
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "the MX path takes a bf16 configuration");
+  if (cfg->d % 512 != 0 || cfg->I % 128 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "the MX path needs d % 512 == 0 and I % 128 == 0");
+  return MOE_OK;
+}
+
+moe_status moe_permute_mx(const moe_config* cfg, const moe_layout* layout, const void* x_q, const uint8_t* x_sf,
+                          void* x_q_perm, uint8_t* x_sf_perm, moe_stream_t stream) {
+  moe_status s = check_mx(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->N == 0) return MOE_OK;
+  if (!layout || !layout->tok2row || !x_q || !x_sf || !x_q_perm || !x_sf_perm)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  const cudaStream_t st = (cudaStream_t)stream;
+  s = cuda_status(launch_permute_bytes(*cfg, *layout, x_q, x_q_perm, cfg->d, st), "permute (mx codes)");
+  if (s != MOE_OK) return s;
+  return cuda_status(launch_permute_bytes(*cfg, *layout, x_sf, x_sf_perm, cfg->d / 32, st), "permute (mx scales)");
+}
+
+moe_status moe_grouped_ffn_mx(const moe_config* cfg, const moe_layout* layout, const void* x_q_perm,
+                              const uint8_t* x_sf_perm, const void* x_q, const uint8_t* x_sf, const void* w13_q,
+                              const uint8_t* w13_sf, const void* w2_q, const uint8_t* w2_sf, const float* topk_w,
+                              void* h, void* h_q, uint8_t* h_sf, void* out, moe_stream_t stream) {
+  moe_status s = check_mx(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->N == 0) return MOE_OK;
+  if (!layout || !layout_complete(layout) || !x_q_perm || !x_sf_perm || !w13_q || !w13_sf || !w2_q || !w2_sf ||
+      !h || !h_q || !h_sf || !out || (cfg->n_shared > 0 && (!x_q || !x_sf)))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  MxFfn f{x_q_perm, x_sf_perm, x_q, x_sf, w13_q, w13_sf, w2_q, w2_sf, topk_w, h, h_q, h_sf, out};
+  return ffn_mx_impl(*cfg, *layout, f, (cudaStream_t)stream);
+}
+
+size_t moe_workspace_bytes_mx(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return carve_forward(*cfg, nullptr, true, true).total;
+}
+
+moe_status moe_layer_forward_mx(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
+                                const int32_t* expert_owner, const void* w13_q, const uint8_t* w13_sf,
+                                const void* w2_q, const uint8_t* w2_sf, void* y, const moe_layout* layout_out,
+                                int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status s = check_mx(cfg);
+  if (s != MOE_OK) return s;
+  if ((s = check_router(*cfg)) != MOE_OK) return s;
+  if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
+  const moe_config& c = *cfg;
+  FwdWs w = carve_forward(c, nullptr, true, true);
+  if (!ws || ws_bytes < w.total) return fail(MOE_ERR_WORKSPACE, "forward workspace too small");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return fail(MOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if (layout_out && !layout_complete(layout_out)) return fail(MOE_ERR_INVALID_ARG, "incomplete layout_out");
+  if (c.N > 0 && (!x || !w_gate || !w13_q || !w13_sf || !w2_q || !w2_sf || !y))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (c.N == 0) return MOE_OK;
+  w = carve_forward(c, static_cast<char*>(ws), true, true);
+  const moe_layout& L = layout_out ? *layout_out : w.lay;
+  const cudaStream_t st = (cudaStream_t)stream;
+  if ((s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
+  if ((s = cuda_status(launch_quantize_mx(x, c.N, c.d, w.x_q, w.x_sf, st), "x quantisation (mx)")) != MOE_OK)
+    return s;
+  if ((s = cuda_status(launch_layout(c, expert_owner, w.ids, L, dev_status, w.lay_ws, st), "layout")) != MOE_OK)
+    return s;
+  if ((s = cuda_status(launch_permute_bytes(c, L, w.x_q, w.x_perm, c.d, st), "permute (mx codes)")) != MOE_OK)
+    return s;
+  if ((s = cuda_status(launch_permute_bytes(c, L, w.x_sf, w.x_sf_perm, c.d / 32, st), "permute (mx scales)")) !=
+      MOE_OK)
+    return s;
+  MxFfn f{w.x_perm, w.x_sf_perm, w.x_q, w.x_sf, w13_q, w13_sf, w2_q, w2_sf, w.w, w.h, w.h_q, w.h_sf, w.out};
+  if ((s = ffn_mx_impl(c, L, f, st)) != MOE_OK) return s;
+  return cuda_status(launch_combine(c, L, w.out, nullptr, y, st), "combine");
 }
 
 size_t moe_ep_window_bytes(const moe_config* cfg, int32_t capacity) {

@@ -525,6 +525,57 @@ moe_status moe_layer_forward_fp8_overlapped(const moe_config* cfg, const void* x
                                             const moe_layout* layout_out, int32_t* dev_status, void* ws,
                                             size_t ws_bytes, moe_stream_t stream, moe_stream_t side_stream);
 
+/*
+ * Block-scaled (MX) e4m3 expert path ([MoE-IV] names MXFP8 as the low-precision expert
+ * compute; the format read as the published microscaling format for FP8 elements).
+ * Every 32 consecutive values of a row along the reduction dimension share one power-of-
+ * two scale X = 2^e, stored as one E8M0 byte (e + 127; 255 is never written):
+ * e = floor(log2(amax of the 32 values)) - 8, clamped to [-127, 127] (-127 for an
+ * all-zero block); code = e4m3 round-to-nearest-even of v / X, saturating at +-448.
+ * Scale bytes are row-major [rows, cols / 32] beside the codes [rows, cols].  A GEMM on
+ * MX operands computes sum_k (qa_k Xa(k/32)) (qb_k Xb(k/32)) with fp32 accumulation; the
+ * scales are applied by the tensor cores (tcgen05 kind::mxf8f6f4.block_scale).  The
+ * configuration stays bf16 (dtype = MOE_BF16) and needs d % 512 == 0, I % 128 == 0; x, y,
+ * h, the expert outputs and the combine are bf16 / fp32 as in the bf16 path.  Buffers are
+ * device memory, 16-byte aligned, owned by the caller.
+ */
+
+/* MX quantisation: src [rows, cols] bf16 -> dst [rows, cols] e4m3 codes, sf [rows, cols/32]
+ * E8M0 bytes.  cols % 32 == 0.  Used for the weights (once), x and h (per step). */
+moe_status moe_quantize_mx(const void* src, int64_t rows, int32_t cols, void* dst, uint8_t* sf,
+                           moe_stream_t stream);
+
+/* MX dispatch payload: x_q_perm[tok2row[a]] = x_q[a / k] (d bytes) and x_sf_perm[tok2row[a]]
+ * = x_sf[a / k] (d / 32 bytes): the permute of moe_permute on codes and scale rows. */
+moe_status moe_permute_mx(const moe_config* cfg, const moe_layout* layout, const void* x_q, const uint8_t* x_sf,
+                          void* x_q_perm, uint8_t* x_sf_perm, moe_stream_t stream);
+
+/*
+ * MX grouped SwiGLU FFN, routed and shared experts:
+ *   h = SiLU(X W_gate^T) * (X W_up^T) on MX operands         (bf16 [A + S*N, I])
+ *   h_q, h_sf = moe_quantize_mx(h)                          (e4m3 [A + S*N, I], E8M0 [A + S*N, I/32])
+ *   out = (h W2^T on MX operands) * gate(row)               (bf16 [A + S*N, d])
+ *   x_q_perm [A, d] + x_sf_perm [A, d/32] (moe_permute_mx); x_q [N, d] + x_sf [N, d/32]
+ *   (the shared experts' rows; NULL when n_shared == 0); w13_q [E+S, 2I, d] + w13_sf
+ *   [E+S, 2I, d/32]; w2_q [E+S, d, I] + w2_sf [E+S, d, I/32]; topk_w as in moe_grouped_ffn.
+ */
+moe_status moe_grouped_ffn_mx(const moe_config* cfg, const moe_layout* layout, const void* x_q_perm,
+                              const uint8_t* x_sf_perm, const void* x_q, const uint8_t* x_sf, const void* w13_q,
+                              const uint8_t* w13_sf, const void* w2_q, const uint8_t* w2_sf, const float* topk_w,
+                              void* h, void* h_q, uint8_t* h_sf, void* out, moe_stream_t stream);
+
+/* Bytes of scratch moe_layer_forward_mx needs (0 for an invalid configuration). */
+size_t moe_workspace_bytes_mx(const moe_config* cfg);
+
+/* The whole layer with the MX expert path, one stream: moe_route -> moe_dispatch_layout ->
+ * moe_quantize_mx(x) -> moe_permute_mx -> moe_grouped_ffn_mx -> moe_combine.  The weights
+ * come quantised (moe_quantize_mx of W13 and W2, once).  ws: 256-byte aligned, of
+ * moe_workspace_bytes_mx bytes. */
+moe_status moe_layer_forward_mx(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
+                                const int32_t* expert_owner, const void* w13_q, const uint8_t* w13_sf,
+                                const void* w2_q, const uint8_t* w2_sf, void* y, const moe_layout* layout_out,
+                                int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* ============================================================================
  * Expert parallelism across GPUs ([EP-DeepEP] §2-3: every rank is a source of tokens
  * and the owner of some experts; dispatch sends each assignment to the owner of its
