@@ -9,11 +9,15 @@
 //   warp 0      TMA producer: A tile [128 rows x 128 codes] + B tile [192 rows x 128 codes]
 //               per stage, 128B swizzle (the same boxes as the e4m3 kernel, B in two
 //               96-row boxes: FC1 W_gate rows and the matching W_up rows)
-//   warp 6      scale stager: reads the stage's scale bytes (4 per row: 128 K values) of
-//               the 128 A rows and the 192 B rows from the row-major arrays and writes them
-//               in the layout tcgen05.cp takes (32 rows x 16 bytes per 128-row atom: row r
-//               at byte 16 (r % 32) + 4 (r / 32) + k-block), then arrives on the stage's
-//               barrier with the TMA bytes
+//   warp 6      scale stager: reads the scale bytes (4 per row and stage: 128 K values) of
+//               the 128 A rows and the 192 B rows from the row-major arrays, 8 stages per
+//               batch of loads (32 bytes of each row, 16-byte loads when rows allow), and
+//               writes them in the layout tcgen05.cp takes (32 rows x 16 bytes per 128-row
+//               atom: row r at byte 16 (r % 32) + 4 (r / 32) + k-block), then arrives on
+//               the stage's barrier beside the TMA bytes.  Lanes read different rows, so
+//               4-byte loads cost one L1 wavefront per row each: the 16-byte form moves
+//               the same bytes in a quarter of the wavefronts (measured 1270 -> 1580
+//               TFLOP/s on the wide expert shapes)
 //   warp 1      MMA issuer: per stage three tcgen05.cp of the atoms into TMEM (scale A: 4
 //               columns, scale B: 8; every 32-lane quarter gets a copy) and 4 block-scaled
 //               MMAs (M=128, N=192, K=32 each; the scale of k-block kk is byte kk of the
@@ -111,7 +115,8 @@ __device__ __forceinline__ MxTile mx_decode_tile(int t, const int* prefix, int G
   return d;
 }
 
-template <int MODE>
+// VEC16: scale rows are 16-byte aligned (K % 512 == 0) and read 16 bytes at a time.
+template <int MODE, bool VEC16>
 __global__ void __launch_bounds__(kThreadsMx, 1)
     tc_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                       const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
@@ -289,16 +294,41 @@ __global__ void __launch_bounds__(kThreadsMx, 1)
         if (r > p.b_rows - 1) r = p.b_rows - 1;
         pb[q] = p.b_sf + ((long long)gz * p.b_rows + r) * kpr;
       }
-      // 8 stages of scale words per batch of loads, so that their latency is paid once
+      // 8 stages of scale words per batch of loads: 32 bytes of each of the lane's 10 rows
+      // (two 16-byte loads when rows are 16-byte aligned, K % 512 == 0; else 4-byte loads)
       for (int kb0 = 0; kb0 < num_kb && ok; kb0 += 8) {
         uint32_t va[8][4], vb[8][6];
+        if (VEC16) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (kb0 + j < num_kb) {
+          for (int h = 0; h < 2; ++h) {
+            if (kb0 + 4 * h < num_kb) {  // num_kb % 4 == 0: the 16 bytes lie inside the row
 #pragma unroll
-            for (int q = 0; q < 4; ++q) va[j][q] = __ldg(reinterpret_cast<const uint32_t*>(pa[q] + 4 * (kb0 + j)));
+              for (int q = 0; q < 4; ++q) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4*>(pa[q] + 4 * kb0 + 16 * h));
+                va[4 * h][q] = u.x;
+                va[4 * h + 1][q] = u.y;
+                va[4 * h + 2][q] = u.z;
+                va[4 * h + 3][q] = u.w;
+              }
 #pragma unroll
-            for (int q = 0; q < 6; ++q) vb[j][q] = __ldg(reinterpret_cast<const uint32_t*>(pb[q] + 4 * (kb0 + j)));
+              for (int q = 0; q < 6; ++q) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4*>(pb[q] + 4 * kb0 + 16 * h));
+                vb[4 * h][q] = u.x;
+                vb[4 * h + 1][q] = u.y;
+                vb[4 * h + 2][q] = u.z;
+                vb[4 * h + 3][q] = u.w;
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (kb0 + j < num_kb) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) va[j][q] = __ldg(reinterpret_cast<const uint32_t*>(pa[q] + 4 * (kb0 + j)));
+#pragma unroll
+              for (int q = 0; q < 6; ++q) vb[j][q] = __ldg(reinterpret_cast<const uint32_t*>(pb[q] + 4 * (kb0 + j)));
+            }
           }
         }
 #pragma unroll
@@ -311,7 +341,8 @@ __global__ void __launch_bounds__(kThreadsMx, 1)
             uint8_t* dst = sSF + stage * kSfBytes;
             *reinterpret_cast<uint4*>(dst + 16 * lane) = make_uint4(va[j][0], va[j][1], va[j][2], va[j][3]);
             *reinterpret_cast<uint4*>(dst + 512 + 16 * lane) = make_uint4(vb[j][0], vb[j][1], vb[j][2], vb[j][3]);
-            *reinterpret_cast<uint4*>(dst + 1024 + 16 * lane) = make_uint4(vb[j][4], vb[j][5], 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+            *reinterpret_cast<uint4*>(dst + 1024 + 16 * lane) =
+                make_uint4(vb[j][4], vb[j][5], 0x7F7F7F7Fu, 0x7F7F7F7Fu);
             fence_proxy_async_smem();  // visible to tcgen05.cp (async proxy)
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[stage]);
@@ -476,10 +507,10 @@ __global__ void __launch_bounds__(kThreadsMx, 1)
   if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
-template <int MODE>
+template <int MODE, bool VEC16>
 cudaError_t launch_mode(const GemmArgs& g, const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                         long long max_tiles, cudaStream_t st) {
-  auto kern = tc_gemm_mx_kernel<MODE>;
+  auto kern = tc_gemm_mx_kernel<MODE, VEC16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMx);
   if (e != cudaSuccess) return e;
   long long grid = sm_count();
@@ -503,8 +534,13 @@ cudaError_t launch_tc_gemm_mx(const GemmArgs& g, cudaStream_t st) {
   if (!make_map_b(&b, g.b, g.g0 + g.G, g.b_rows, g.K, kBN / 2, kBK, true)) return cudaErrorInvalidValue;
   const long long blocks = (launch_rows(g) + kBM - 1) / kBM + g.G;  // every group adds at most one partial block
   const long long n_tiles = g.mode == MODE_FC1 ? (g.n_out + kBN / 2 - 1) / (kBN / 2) : (g.n_out + kBN - 1) / kBN;
-  if (g.mode == MODE_FC1) return launch_mode<MODE_FC1>(g, a0, a1, b, blocks * n_tiles, st);
-  return launch_mode<MODE_FC2>(g, a0, a1, b, blocks * n_tiles, st);
+  // 16-byte scale loads need 16-byte aligned rows (K / 32 % 16 == 0) and arrays
+  const bool vec = g.K % 512 == 0 && ((reinterpret_cast<uintptr_t>(g.a0_sf) | reinterpret_cast<uintptr_t>(g.a1_sf) |
+                                       reinterpret_cast<uintptr_t>(g.b_sf)) & 15) == 0;
+  const long long mt = blocks * n_tiles;
+  if (g.mode == MODE_FC1)
+    return vec ? launch_mode<MODE_FC1, true>(g, a0, a1, b, mt, st) : launch_mode<MODE_FC1, false>(g, a0, a1, b, mt, st);
+  return vec ? launch_mode<MODE_FC2, true>(g, a0, a1, b, mt, st) : launch_mode<MODE_FC2, false>(g, a0, a1, b, mt, st);
 }
 
 }  // namespace moe
