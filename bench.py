@@ -827,9 +827,11 @@ def run_fp8(args, cfg, world, rank, local):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     clocks.mark_timed()
+    torch.cuda.nvtx.range_push("timed")
     for i in range(args.steps):
         flush.zero_()
         fused(evs[i])
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -960,9 +962,11 @@ def run_mx(args, cfg, world, rank, local):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     clocks.mark_timed()
+    torch.cuda.nvtx.range_push("timed")
     for i in range(args.steps):
         flush.zero_()
         fused(evs[i])
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()

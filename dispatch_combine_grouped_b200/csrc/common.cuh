@@ -350,12 +350,6 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
       : "memory");
 }
 
-// Rows of a group covered by 256-row pair tiles: whole pairs, plus one more pair when
-// more than 128 rows are left; the remaining 0..128 rows are a 128-row tail block.
-__host__ __device__ __forceinline__ int pair_rows(int rows) {
-  return ((rows >> 8) + ((rows & 255) > 128 ? 1 : 0)) << 8;
-}
-
 // ------------------------------------------------------------------ small math
 __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)); }
 

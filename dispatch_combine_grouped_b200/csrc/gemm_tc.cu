@@ -149,12 +149,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       orow = p.A_routed + s * p.N;
       arow = p.shared_from_map1 ? 0 : orow;
     }
-    if (p.tail_only) {  // the pair kernel covers the first pair_rows(rows) rows
-      const int pr = pair_rows(rows);
-      rows = rows > pr ? rows - pr : 0;
-      arow += pr;
-      orow += pr;
-    }
     s_rows[g] = rows;
     s_arow[g] = arow;
     s_orow[g] = orow;

@@ -64,7 +64,6 @@ struct GemmArgs {
   int n_out;         // valid output columns (E, I or d)
   int I;             // FC1: row offset of W_up inside W13
   int shared_from_map1;
-  int tail_only;        // 1-CTA kernel: only the rows left after the 256-row pair tiles
   const int32_t* n_e;
   const int32_t* expert_off;
   const int32_t* row2tok;
