@@ -1270,6 +1270,15 @@ def bench_layer(args, cfg, world, rank, local, steps, warmup, headline=True):
         eplb_info["owner_max_over_mean_after"] = float(R_after.max() / R_after.mean())
         eplb_info["note"] = ("stages_ms.layout includes the replica assignment; the fused and e2e "
                              "numbers run the layer without copies")
+    graph_ms = None
+    if not R and rank == 0:
+        if S:
+            graph_ms = graph_step_ms(lambda: moe.layer_forward_overlapped(cfg, x, wg, bias, owner, w13, w2, side, y=y,
+                                                                          ws=ws, status=status),
+                                     flush, min(steps, 20), dev)
+        else:
+            graph_ms = graph_step_ms(lambda: moe.layer_forward(cfg, x, wg, bias, owner, w13, w2, y=y, ws=ws,
+                                                               status=status), flush, min(steps, 20), dev)
     if rank != 0:
         return None
     ffn_rec = {"tflops": ffn_seq_tflops, "ms": ffn_seq_ms, "frac_of_peak": ffn_seq_tflops / tpeak, "peak_kind": tkind,
@@ -1320,6 +1329,14 @@ def bench_layer(args, cfg, world, rank, local, steps, warmup, headline=True):
     }
     if chunked is not None:
         line["chunked"] = chunked
+    if graph_ms is not None:
+        ok = isinstance(graph_ms, float)
+        line["graph"] = {"ms_per_step": graph_ms if ok else None,
+                         "tokens_per_s": whole_job_tokens_per_s(cfg.N, 1, graph_ms) if ok else None,
+                         **({} if ok else {"error": graph_ms}),
+                         "how": "moe_layer_forward_overlapped (moe_layer_forward without shared experts) captured once "
+                                "in a CUDA graph and replayed, median of the replays, L2 flushed before each outside "
+                                "the graph: the step without host launch gaps"}
     if headline:
         line["fused_ms_per_step"] = fused_ms
         line["e2e"] = {"value": whole_job_tokens_per_s(cfg.N, world, e2e_ms), "unit": "tokens/s",
@@ -1342,6 +1359,36 @@ def kernel_launches_per_step(cfg, R=0):
     return 2 + 3 + 1 + 2 + (2 if cfg.S else 0) + 1 + (4 if R else 0)
 
 
+def graph_step_ms(call, flush, n, dev):
+    """The product's layer call captured once in a CUDA graph and replayed n times, the
+    256 MiB L2 flush before each replay outside the graph; median replay time in ms, or an
+    error string when the capture fails."""
+    import torch
+    try:
+        cs = torch.cuda.Stream(device=dev)
+        cs.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(cs):
+            call()  # warm-up on the capture stream
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cs):
+            call()
+        ts = []
+        for _ in range(n):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        del g
+        return sorted(ts)[len(ts) // 2]
+    except RuntimeError as e:  # capture refused: report it, keep the eager numbers
+        torch.cuda.synchronize()
+        return f"capture failed: {e}"
+
+
 def summarize(line) -> dict:
     """The per-workload record of the default run's "workloads" field."""
     keep = {"ms_per_step": line["ms_per_step"], "tokens_per_s": line["value"], "config": line["config"]["workload"],
@@ -1354,7 +1401,9 @@ def summarize(line) -> dict:
             "permute": {k: line["permute"][k] for k in ("gbs", "frac_of_hbm", "frac_of_8tbs", "gbs_in_step")},
             "combine": {k: line["combine"][k] for k in ("gbs", "frac_of_hbm", "frac_of_8tbs", "gbs_in_step")},
             "imbalance": line["imbalance"], "clocks": line["clocks"], "steps": line["steps"],
-            "gpu_launches": line["gpu_launches"]}
+            "gpu_launches": line["gpu_launches"],
+            "graph_ms_per_step": line.get("graph", {}).get("ms_per_step"),
+            "graph_tokens_per_s": line.get("graph", {}).get("tokens_per_s")}
     if "cpu_baseline" in line:
         keep["cpu_baseline"] = line["cpu_baseline"]
     if "chunked" in line:

@@ -326,3 +326,30 @@ def test_forward_captures_into_cuda_graph(cfg):
         g.replay()
         torch.cuda.synchronize()
         assert torch.equal(y, y_eager)
+
+
+@pytest.mark.parametrize("cfg", [SMALL[1], SMALL[4]], ids=_ids([SMALL[1], SMALL[4]]))
+def test_overlapped_forward_captures_into_cuda_graph(cfg):
+    """moe_layer_forward_overlapped forks the shared experts onto the side stream with
+    events, so a capture on the calling stream pulls the side stream in; replays give the
+    one-stream forward's bits (the bench times this replay as the graph step)."""
+    inp = gpu_inputs(cfg)
+    ws = moe.alloc_workspace(cfg)
+    args = (cfg, inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], inp["w13"], inp["w2"])
+    y_ref = moe.layer_forward(*args, ws=ws)
+    torch.cuda.synchronize()
+    y = torch.empty_like(y_ref)
+    s, side = torch.cuda.Stream(), torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        moe.layer_forward_overlapped(*args, side, y=y, ws=ws)  # warm-up on the capture stream
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            moe.layer_forward_overlapped(*args, side, y=y, ws=ws)
+    for _ in range(2):
+        y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_ref)
+    del g
