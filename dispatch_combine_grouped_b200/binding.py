@@ -41,7 +41,7 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_checks_en
             "moe_ep_workspace_bytes_fp8", "moe_ep_dispatch_fp8", "moe_ep_expert_ffn_fp8", "moe_ep_layer_forward_fp8",
             "moe_ep_layer_forward_overlapped", "moe_ep_layer_forward_fp8_overlapped",
             "moe_quantize_mx", "moe_permute_mx", "moe_grouped_ffn_mx", "moe_workspace_bytes_mx",
-            "moe_layer_forward_mx"]
+            "moe_layer_forward_mx", "moe_layer_forward_mx_overlapped"]
 
 
 class CConfig(ctypes.Structure):
@@ -123,6 +123,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_grouped_ffn_mx": (i32, [cfgp, layp] + [vp] * 14),
         "moe_workspace_bytes_mx": (sz, [cfgp]),
         "moe_layer_forward_mx": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp]),
+        "moe_layer_forward_mx_overlapped": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp, vp]),
         "moe_layer_forward_fp8": (i32, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, layp, vp, vp, sz, vp]),
         "moe_capacity_drop": (i32, [cfgp, vp, i32, vp, vp, vp, sz, vp]),
         "moe_capacity_rows": (i32, [cfgp, ctypes.c_double, ctypes.POINTER(i32)]),
@@ -607,17 +608,22 @@ def workspace_bytes_mx(cfg) -> int:
 
 
 def layer_forward_mx(cfg, x, w_gate, bias, expert_owner, w13_q, w13_sf, w2_q, w2_sf, y=None, ws=None, layout=None,
-                     status=None):
-    """moe_layer_forward_mx: the layer with the MX expert path on the current stream."""
+                     status=None, side_stream=None):
+    """moe_layer_forward_mx on the current stream, or moe_layer_forward_mx_overlapped when
+    side_stream is given."""
     c = c_config(cfg)
     if y is None:
         y = torch.empty(cfg.N, cfg.d, dtype=torch.bfloat16, device=x.device)
     if ws is None:
         ws = torch.empty(max(workspace_bytes_mx(cfg), 1), dtype=torch.uint8, device=x.device)
-    _check(load().moe_layer_forward_mx(ctypes.byref(c), _p(x), _p(w_gate), _p(bias), _p(expert_owner), _p(w13_q),
-                                       _p(w13_sf), _p(w2_q), _p(w2_sf), _p(y),
-                                       ctypes.byref(layout.c) if layout is not None else None, _p(status), _p(ws),
-                                       ws.numel(), _stream()), "moe_layer_forward_mx")
+    args = [ctypes.byref(c), _p(x), _p(w_gate), _p(bias), _p(expert_owner), _p(w13_q), _p(w13_sf), _p(w2_q),
+            _p(w2_sf), _p(y), ctypes.byref(layout.c) if layout is not None else None, _p(status), _p(ws), ws.numel(),
+            _stream()]
+    if side_stream is None:
+        _check(load().moe_layer_forward_mx(*args), "moe_layer_forward_mx")
+    else:
+        _check(load().moe_layer_forward_mx_overlapped(*args, ctypes.c_void_p(side_stream.cuda_stream)),
+               "moe_layer_forward_mx_overlapped")
     return y
 
 

@@ -1208,10 +1208,10 @@ size_t moe_workspace_bytes_mx(const moe_config* cfg) {
   return carve_forward(*cfg, nullptr, true, true).total;
 }
 
-moe_status moe_layer_forward_mx(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
-                                const int32_t* expert_owner, const void* w13_q, const uint8_t* w13_sf,
-                                const void* w2_q, const uint8_t* w2_sf, void* y, const moe_layout* layout_out,
-                                int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream) {
+static moe_status forward_mx(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
+                             const int32_t* expert_owner, const void* w13_q, const uint8_t* w13_sf, const void* w2_q,
+                             const uint8_t* w2_sf, void* y, const moe_layout* layout_out, int32_t* dev_status,
+                             void* ws, size_t ws_bytes, cudaStream_t st, cudaStream_t side) {
   moe_status s = check_mx(cfg);
   if (s != MOE_OK) return s;
   if ((s = check_router(*cfg)) != MOE_OK) return s;
@@ -1226,20 +1226,56 @@ moe_status moe_layer_forward_mx(const moe_config* cfg, const void* x, const void
   if (c.N == 0) return MOE_OK;
   w = carve_forward(c, static_cast<char*>(ws), true, true);
   const moe_layout& L = layout_out ? *layout_out : w.lay;
-  const cudaStream_t st = (cudaStream_t)stream;
   if ((s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
   if ((s = cuda_status(launch_quantize_mx(x, c.N, c.d, w.x_q, w.x_sf, st), "x quantisation (mx)")) != MOE_OK)
     return s;
-  if ((s = cuda_status(launch_layout(c, expert_owner, w.ids, L, dev_status, w.lay_ws, st), "layout")) != MOE_OK)
-    return s;
-  if ((s = cuda_status(launch_permute_bytes(c, L, w.x_q, w.x_perm, c.d, st), "permute (mx codes)")) != MOE_OK)
-    return s;
-  if ((s = cuda_status(launch_permute_bytes(c, L, w.x_sf, w.x_sf_perm, c.d / 32, st), "permute (mx scales)")) !=
-      MOE_OK)
-    return s;
   MxFfn f{w.x_perm, w.x_sf_perm, w.x_q, w.x_sf, w13_q, w13_sf, w2_q, w2_sf, w.w, w.h, w.h_q, w.h_sf, w.out};
-  if ((s = ffn_mx_impl(c, L, f, st)) != MOE_OK) return s;
+  const bool overlap = side != nullptr && side != st && c.n_shared > 0;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaError_t e = cudaSuccess;
+  if (overlap) {  // the shared experts read only x's codes and scales: they run on the side stream
+    e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
+    if (e != cudaSuccess) {
+      if (fork) cudaEventDestroy(fork);
+      if (join) cudaEventDestroy(join);
+      return cuda_status(e, "fork");
+    }
+    s = ffn_mx_impl(c, L, f, side, c.E, c.n_shared);
+    e = cudaEventRecord(join, side);
+  }
+  if (s == MOE_OK) s = cuda_status(launch_layout(c, expert_owner, w.ids, L, dev_status, w.lay_ws, st), "layout");
+  if (s == MOE_OK) s = cuda_status(launch_permute_bytes(c, L, w.x_q, w.x_perm, c.d, st), "permute (mx codes)");
+  if (s == MOE_OK)
+    s = cuda_status(launch_permute_bytes(c, L, w.x_sf, w.x_sf_perm, c.d / 32, st), "permute (mx scales)");
+  if (s == MOE_OK) s = overlap ? ffn_mx_impl(c, L, f, st, 0, c.E) : ffn_mx_impl(c, L, f, st);
+  if (overlap) {
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, join, 0);  // join even after an error
+    cudaEventDestroy(fork);
+    cudaEventDestroy(join);
+  }
+  if (s != MOE_OK) return s;
+  if (e != cudaSuccess) return cuda_status(e, "join");
   return cuda_status(launch_combine(c, L, w.out, nullptr, y, st), "combine");
+}
+
+moe_status moe_layer_forward_mx(const moe_config* cfg, const void* x, const void* w_gate, const float* bias,
+                                const int32_t* expert_owner, const void* w13_q, const uint8_t* w13_sf,
+                                const void* w2_q, const uint8_t* w2_sf, void* y, const moe_layout* layout_out,
+                                int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return forward_mx(cfg, x, w_gate, bias, expert_owner, w13_q, w13_sf, w2_q, w2_sf, y, layout_out, dev_status, ws,
+                    ws_bytes, (cudaStream_t)stream, nullptr);
+}
+
+moe_status moe_layer_forward_mx_overlapped(const moe_config* cfg, const void* x, const void* w_gate,
+                                           const float* bias, const int32_t* expert_owner, const void* w13_q,
+                                           const uint8_t* w13_sf, const void* w2_q, const uint8_t* w2_sf, void* y,
+                                           const moe_layout* layout_out, int32_t* dev_status, void* ws,
+                                           size_t ws_bytes, moe_stream_t stream, moe_stream_t side_stream) {
+  return forward_mx(cfg, x, w_gate, bias, expert_owner, w13_q, w13_sf, w2_q, w2_sf, y, layout_out, dev_status, ws,
+                    ws_bytes, (cudaStream_t)stream, (cudaStream_t)side_stream);
 }
 
 size_t moe_ep_window_bytes(const moe_config* cfg, int32_t capacity) {

@@ -576,6 +576,18 @@ moe_status moe_layer_forward_mx(const moe_config* cfg, const void* x, const void
                                 const void* w2_q, const uint8_t* w2_sf, void* y, const moe_layout* layout_out,
                                 int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_layer_forward_mx with the shared experts overlapped: after the router and the MX
+ * quantisation of x on `stream`, the shared experts' MX FFN runs on `side_stream` while
+ * the layout, the MX permute and the routed MX FFN run on `stream`; `stream` waits for
+ * `side_stream` before the combine.  Same result as moe_layer_forward_mx, bit for bit; two
+ * events are created and destroyed per call.  With n_shared == 0 or side_stream == stream
+ * this is moe_layer_forward_mx. */
+moe_status moe_layer_forward_mx_overlapped(const moe_config* cfg, const void* x, const void* w_gate,
+                                           const float* bias, const int32_t* expert_owner, const void* w13_q,
+                                           const uint8_t* w13_sf, const void* w2_q, const uint8_t* w2_sf, void* y,
+                                           const moe_layout* layout_out, int32_t* dev_status, void* ws,
+                                           size_t ws_bytes, moe_stream_t stream, moe_stream_t side_stream);
+
 /* ============================================================================
  * Expert parallelism across GPUs ([EP-DeepEP] §2-3: every rank is a source of tokens
  * and the owner of some experts; dispatch sends each assignment to the owner of its
