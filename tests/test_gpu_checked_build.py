@@ -6,8 +6,8 @@ Each case runs in a child process that loads the checked library (MOE_LIB=checke
     it, is caught: the kernel records MOE_ERR_BAD_INDEX in the registered word, skips the
     access, and the guard bands around its output stay untouched:
       tok2row out of range (permute and combine), send2row (staged permute), expert_off
-      and n_e describing rows past the routed block (grouped FFN), row2tok out of range
-      (the FC2 gate).
+      and n_e describing rows past the routed block (grouped FFN, bf16 and block-scaled
+      MX), row2tok out of range (the FC2 gate).
 Nothing traps: every fault is turned into a status before any access.
 """
 import os
@@ -87,6 +87,23 @@ CHILD = textwrap.dedent(r'''
             ob, oo = guarded((A + cfg.N, cfg.d), torch.bfloat16)
             moe.grouped_ffn(cfg, lay, xp, inp["x"], inp["w13"], inp["w2"], topk_w=w, h=hh, out=oo)
             assert fired() == BAD and guards_ok(hb) and guards_ok(ob)
+        elif case == "mx_groups":  # the block-scaled kernel checks its group table the same way
+            c = small_config("chk_mx", cfg_id=130, N=200, d=512, E=8, S=1, k=2, I=256, P=2)
+            inp = make_inputs(c, device="cuda")
+            logits, ids, w = moe.route(c, inp["x"], inp["w_gate"], inp["bias"])
+            lay = moe.dispatch_layout(c, ids)
+            A = c.N * c.k
+            x_q, x_sf = moe.quantize_mx(inp["x"])
+            w13_q, w13_sf = moe.quantize_mx(inp["w13"])
+            w2_q, w2_sf = moe.quantize_mx(inp["w2"])
+            xp, xp_sf = moe.permute_mx(c, lay, x_q, x_sf)
+            moe.grouped_ffn_mx(c, lay, xp, xp_sf, x_q, x_sf, w13_q, w13_sf, w2_q, w2_sf, topk_w=w)
+            assert fired() == 0
+            lay["expert_off"][2] = A - 3
+            hb, hh = guarded((A + c.N, c.I), torch.bfloat16)
+            ob, oo = guarded((A + c.N, c.d), torch.bfloat16)
+            moe.grouped_ffn_mx(c, lay, xp, xp_sf, x_q, x_sf, w13_q, w13_sf, w2_q, w2_sf, topk_w=w, h=hh, out=oo)
+            assert fired() == BAD and guards_ok(hb) and guards_ok(ob)
         elif case == "gate":
             lay["row2tok"][0] = -5
             ob, oo = guarded((A + cfg.N, cfg.d), torch.bfloat16)
@@ -108,7 +125,7 @@ def checked_lib():
     return b.build(checked=True)
 
 
-@pytest.mark.parametrize("case", ["clean", "permute", "staged", "combine", "ffn_groups", "gate"])
+@pytest.mark.parametrize("case", ["clean", "permute", "staged", "combine", "ffn_groups", "mx_groups", "gate"])
 def test_checked_build(checked_lib, case):
     env = dict(os.environ, MOE_LIB="checked")
     r = subprocess.run([sys.executable, "-c", CHILD, ROOT, case], capture_output=True, text=True, env=env,
