@@ -41,7 +41,9 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_last_error", "moe_checks_en
             "moe_ep_workspace_bytes_fp8", "moe_ep_dispatch_fp8", "moe_ep_expert_ffn_fp8", "moe_ep_layer_forward_fp8",
             "moe_ep_layer_forward_overlapped", "moe_ep_layer_forward_fp8_overlapped",
             "moe_quantize_mx", "moe_permute_mx", "moe_grouped_ffn_mx", "moe_workspace_bytes_mx",
-            "moe_layer_forward_mx", "moe_layer_forward_mx_overlapped"]
+            "moe_layer_forward_mx", "moe_layer_forward_mx_overlapped", "moe_ep_workspace_bytes_mx",
+            "moe_ep_dispatch_mx", "moe_ep_expert_ffn_mx", "moe_ep_layer_forward_mx",
+            "moe_ep_layer_forward_mx_overlapped"]
 
 
 class CConfig(ctypes.Structure):
@@ -146,6 +148,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_ep_expert_ffn": (i32, [cfgp, grpp, vp, vp, vp, hdp, vp, vp, sz, vp]),
         "moe_ep_combine": (i32, [cfgp, grpp, hdp, vp, vp, vp]),
         "moe_ep_layer_forward": (i32, [cfgp, grpp, vp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz, vp]),
+        "moe_ep_workspace_bytes_mx": (sz, [cfgp, i32]),
+        "moe_ep_dispatch_mx": (i32, [cfgp, grpp, vp, vp, vp, hdp, vp]),
+        "moe_ep_expert_ffn_mx": (i32, [cfgp, grpp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz, vp]),
+        "moe_ep_layer_forward_mx": (i32, [cfgp, grpp, vp, vp, vp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz, vp]),
+        "moe_ep_layer_forward_mx_overlapped": (i32, [cfgp, grpp, vp, vp, vp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz,
+                                                     vp, vp]),
         "moe_ep_workspace_bytes_fp8": (sz, [cfgp, i32]),
         "moe_ep_dispatch_fp8": (i32, [cfgp, grpp, vp, vp, vp, hdp, vp]),
         "moe_ep_expert_ffn_fp8": (i32, [cfgp, grpp, vp, vp, vp, vp, vp, vp, hdp, vp, vp, sz, vp]),

@@ -239,7 +239,8 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_dispatch_kernel(const __grid
                                                                      const float* __restrict__ topk_w,
                                                                      const float* __restrict__ x_scale, int N,
                                                                      int k, int vpr, int capacity, int P,
-                                                                     int me, int* check) {
+                                                                     int me, int* check,
+                                                                     const uint4* __restrict__ x2, int vpr2) {
   const int lane = threadIdx.x & 31;
   for (int t = blockIdx.x * kEpWarps + (threadIdx.x >> 5); t < N; t += gridDim.x * kEpWarps) {
     int my = lane < k ? dest[(size_t)t * k + lane] : -1;
@@ -250,13 +251,16 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_dispatch_kernel(const __grid
       if (x_scale) at<float>(peers.base[o], off.scale)[my - o * capacity] = x_scale[t];
     }
     uint4* rows[kMaxK];
+    uint4* srows[kMaxK];  // MX scale rows: [capacity, vpr2] vectors after [capacity, vpr] of codes
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
       const int d = __shfl_sync(0xffffffffu, my, j);
       rows[j] = nullptr;
+      srows[j] = nullptr;
       if (j < k && d >= 0) {
         const int o = d / capacity;
         rows[j] = at<uint4>(peers.base[o], off.x_recv) + (size_t)(d - o * capacity) * vpr;
+        if (x2) srows[j] = at<uint4>(peers.base[o], off.x_recv) + (size_t)capacity * vpr + (size_t)(d - o * capacity) * vpr2;
       }
     }
     const uint4* s = x + (size_t)t * vpr;
@@ -276,6 +280,13 @@ __global__ void __launch_bounds__(kEpWarps * 32) ep_dispatch_kernel(const __grid
           if (v < vpr) rows[j][v] = buf[u];
         }
       }
+    }
+    if (x2 && lane < vpr2) {  // MX: the token's scale row (vpr2 <= 32 vectors) to the same
+                              // receive rows of the scale region, which follows the codes
+      const uint4 u = ld_nc(x2 + (size_t)t * vpr2 + lane);
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j)
+        if (srows[j] != nullptr) srows[j][lane] = u;
     }
   }
   // The last CTA to finish publishes this source's epoch to every owner.  Each CTA
@@ -464,10 +475,11 @@ cudaError_t launch_ep_layout(const moe_config& c, const EpPeers& peers, const Ep
 
 cudaError_t launch_ep_dispatch(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me,
                                int capacity, const void* x, const int32_t* dest, const float* topk_w,
-                               const float* x_scale, int row_bytes, cudaStream_t st) {
+                               const float* x_scale, int row_bytes, cudaStream_t st, const void* x2, int row_bytes2) {
+  if (x2 && (row_bytes2 % 16 != 0 || row_bytes2 > 32 * 16)) return cudaErrorInvalidValue;
   ep_dispatch_kernel<<<ep_grid(c.N, kEpWarps), kEpWarps * 32, 0, st>>>(
       peers, off, static_cast<const uint4*>(x), dest, topk_w, x_scale, c.N, c.k, row_bytes / 16, capacity, c.P, me,
-      check_word());
+      check_word(), static_cast<const uint4*>(x2), x2 ? row_bytes2 / 16 : 0);
   return cudaGetLastError();
 }
 

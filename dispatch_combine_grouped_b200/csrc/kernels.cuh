@@ -165,10 +165,13 @@ cudaError_t launch_ep_layout(const moe_config& c, const EpPeers& peers, const Ep
                              int local_experts, const int32_t* owner, const int32_t* ids, const moe_layout& loc,
                              int32_t* dest, int32_t* own_n_e, int32_t* own_off, int* status, cudaStream_t st);
 // rows of row_bytes bytes (d * elem for bf16 / fp32, d for e4m3 codes); x_scale (FP8): each
-// token's scale, stored beside each of its received rows (NULL: none)
+// token's scale, stored beside each of its received rows (NULL: none); x2 (MX): each token's
+// scale row of row_bytes2 bytes (at most 512), stored in the receive region after the
+// capacity rows of codes (NULL: none)
 cudaError_t launch_ep_dispatch(const moe_config& c, const EpPeers& peers, const EpOffsets& off, int me,
                                int capacity, const void* x, const int32_t* dest, const float* topk_w,
-                               const float* x_scale, int row_bytes, cudaStream_t st);
+                               const float* x_scale, int row_bytes, cudaStream_t st, const void* x2 = nullptr,
+                               int row_bytes2 = 0);
 cudaError_t launch_ep_wait(const char* own, const EpOffsets& off, size_t flag_off, int n, int* status,
                            cudaStream_t st);
 cudaError_t launch_ep_signal(const EpPeers& peers, const EpOffsets& off, size_t flag_off, int P, int me,

@@ -380,6 +380,9 @@ struct EpWs {
   float* h_scale;   // [capacity + S*N]
   void* x_q;        // [N, d] e4m3 (moe_ep_layer_forward_fp8)
   float* x_scale;   // [N]
+  // MX only
+  uint8_t* h_sf;    // [capacity + S*N, I/32] E8M0
+  uint8_t* x_sf;    // [N, d/32] (moe_ep_layer_forward_mx)
   size_t total;
 };
 
@@ -389,7 +392,9 @@ moe_config one_owner(const moe_config& c) {
   return c1;
 }
 
-EpWs carve_ep(const moe_config& c, int capacity, char* base, bool fp8 = false) {
+// fp8: the FP8 path's buffers; mx: the MX path's (those plus the scale bytes)
+EpWs carve_ep(const moe_config& c, int capacity, char* base, bool fp8 = false, bool mx = false) {
+  fp8 = fp8 || mx;
   EpWs w;
   memset(&w, 0, sizeof(w));
   const size_t A = (size_t)c.N * c.k, E = c.E, S = c.n_shared, eb = elem_bytes(c);
@@ -426,6 +431,10 @@ EpWs carve_ep(const moe_config& c, int capacity, char* base, bool fp8 = false) {
     w.x_q = take((size_t)c.N * c.d);
     w.x_scale = reinterpret_cast<float*>(take((size_t)c.N * 4));
   }
+  if (mx) {
+    w.h_sf = reinterpret_cast<uint8_t*>(take(((size_t)capacity + S * c.N) * (c.I / 32)));
+    w.x_sf = reinterpret_cast<uint8_t*>(take((size_t)c.N * (c.d / 32)));
+  }
   w.total = off;
   return w;
 }
@@ -449,8 +458,9 @@ moe_status check_ep(const moe_config* cfg, const moe_ep_group* g, EpPeers* peers
   return MOE_OK;
 }
 
-moe_status check_ep_ws(const moe_config& c, const moe_ep_group* g, void* ws, size_t ws_bytes, bool fp8 = false) {
-  if (!ws || ws_bytes < carve_ep(c, g->capacity, nullptr, fp8).total)
+moe_status check_ep_ws(const moe_config& c, const moe_ep_group* g, void* ws, size_t ws_bytes, bool fp8 = false,
+                       bool mx = false) {
+  if (!ws || ws_bytes < carve_ep(c, g->capacity, nullptr, fp8, mx).total)
     return fail(MOE_ERR_WORKSPACE, "EP workspace too small");
   if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return fail(MOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
   return MOE_OK;
@@ -482,17 +492,67 @@ moe_status ep_layout_impl(const moe_config& c, const moe_ep_group& g, const EpPe
 // per-row quantisation of the h rows of the range, FC2 on e4m3 h.
 struct EpFfn {
   bool fp8;
-  const void* x;  // bf16 tokens, or e4m3 codes with x_scale
+  const void* x;  // bf16 tokens, or e4m3 codes with x_scale (FP8) / x_sf (MX)
   const float* x_scale;
   const void* w13;
   const float* w13_scale;
   const void* w2;
   const float* w2_scale;
+  // MX (block-scaled e4m3): E8M0 scale rows beside the codes; the received rows' scales
+  // follow their codes in the window's receive region
+  bool mx = false;
+  const uint8_t* x_sf = nullptr;
+  const uint8_t* w13_sf = nullptr;
+  const uint8_t* w2_sf = nullptr;
 };
+
+// The MX form of ep_gemms: FC1 on the received codes and their scale rows (the shared
+// groups on this rank's own x codes), MX quantisation of the h rows of the range, FC2.
+moe_status ep_gemms_mx(const moe_config& c, const moe_ep_group& g, char* win, const EpOffsets& off, const EpFfn& f,
+                       const moe_ep_handle& hd, const EpWs& w, cudaStream_t st, int g0, int G) {
+  moe_config co = c;
+  co.E = g.local_experts;
+  moe_layout L;
+  memset(&L, 0, sizeof(L));
+  L.n_e = hd.owner_n_e;
+  L.expert_off = hd.owner_off;
+  const int S = c.N > 0 ? c.n_shared : 0;
+  const long long cap = g.capacity;
+  const long long rows = cap + (long long)S * c.N;
+  GemmArgs g1 = fc1_args(co, L, win + off.x_recv, S > 0 ? f.x : nullptr, f.w13, w.h);
+  g1.g0 = g0;
+  g1.G = G;
+  g1.A_routed = g.capacity;
+  g1.max_ctas = shared_cap(co, g0);
+  g1.a0_sf = reinterpret_cast<const uint8_t*>(win + off.x_recv) + cap * c.d;  // after the codes
+  g1.a1_sf = f.x_sf;
+  g1.b_sf = f.w13_sf;
+  g1.a0_rows = cap;
+  g1.a1_rows = c.N > 0 ? c.N : 1;
+  cudaError_t e = launch_tc_gemm_mx(g1, st);
+  if (e != cudaSuccess) return cuda_status(e, "EP FC1 grouped GEMM (mx)");
+  const int Lx = g.local_experts;
+  const long long r0 = g0 < Lx ? 0 : cap + (long long)(g0 - Lx) * c.N;
+  const long long r1 = g0 + G <= Lx ? cap : cap + (long long)(g0 + G - Lx) * c.N;
+  e = launch_quantize_mx(static_cast<const uint16_t*>(w.h) + r0 * c.I, r1 - r0, c.I,
+                         static_cast<uint8_t*>(w.h_q) + r0 * c.I, w.h_sf + r0 * (c.I / 32), st);
+  if (e != cudaSuccess) return cuda_status(e, "h quantisation (mx)");
+  GemmArgs g2 = fc2_args(co, L, w.h_q, f.w2, reinterpret_cast<const float*>(win + off.gate), win + off.out_recv);
+  g2.g0 = g0;
+  g2.G = G;
+  g2.A_routed = g.capacity;
+  g2.max_ctas = shared_cap(co, g0);
+  g2.a0_sf = w.h_sf;
+  g2.b_sf = f.w2_sf;
+  g2.a0_rows = rows;
+  g2.a1_rows = rows;
+  return cuda_status(launch_tc_gemm_mx(g2, st), "EP FC2 grouped GEMM (mx)");
+}
 
 moe_status ep_gemms(const moe_config& c, const moe_ep_group& g, char* win, const EpOffsets& off, const EpFfn& f,
                     const moe_ep_handle& hd, const EpWs& w, cudaStream_t st, int g0, int G) {
   if (G <= 0) return MOE_OK;
+  if (f.mx) return ep_gemms_mx(c, g, win, off, f, hd, w, st, g0, G);
   moe_config co = c;
   co.E = g.local_experts;
   moe_layout L;
@@ -570,7 +630,12 @@ moe_status ep_forward(const moe_config& c, const moe_ep_group& g, const EpPeers&
   moe_status s = MOE_OK;
   if (c.N > 0) {
     if ((s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
-    if (f.fp8) {
+    if (f.mx) {
+      s = cuda_status(launch_quantize_mx(x, c.N, c.d, w.x_q, w.x_sf, st), "x quantisation (mx)");
+      if (s != MOE_OK) return s;
+      f.x = w.x_q;
+      f.x_sf = w.x_sf;
+    } else if (f.fp8) {
       s = cuda_status(launch_quantize_rows(x, c.N, c.d, w.x_q, w.x_scale, st), "x quantisation");
       if (s != MOE_OK) return s;
       f.x = w.x_q;
@@ -597,7 +662,9 @@ moe_status ep_forward(const moe_config& c, const moe_ep_group& g, const EpPeers&
   if (s == MOE_OK) s = ep_layout_impl(c, g, peers, owner, w.ids, hd, status, w, st);
   if (s == MOE_OK)
     s = cuda_status(launch_ep_dispatch(c, peers, off, g.rank, g.capacity, f.x, hd.dest, w.w,
-                                       f.fp8 ? f.x_scale : nullptr, c.d * (f.fp8 ? 1 : elem_bytes(c)), st),
+                                       f.fp8 && !f.mx ? f.x_scale : nullptr,
+                                       c.d * (f.fp8 || f.mx ? 1 : elem_bytes(c)), st, f.mx ? f.x_sf : nullptr,
+                                       c.d / 32),
                     "EP dispatch");
   if (s == MOE_OK) s = ep_ffn_impl(c, g, peers, f, hd, status, w, st, G);
   if (overlap) {
@@ -1403,21 +1470,21 @@ static moe_status ep_layer(const moe_config* cfg, const moe_ep_group* grp, const
                            const float* bias, const int32_t* expert_owner, const EpFfn& f, void* y,
                            const moe_ep_handle* handle_out, int32_t* dev_status, void* ws, size_t ws_bytes,
                            moe_stream_t stream, moe_stream_t side) {
-  moe_status s = f.fp8 ? check_fp8(cfg) : check_config(cfg);
+  moe_status s = f.mx ? check_mx(cfg) : (f.fp8 ? check_fp8(cfg) : check_config(cfg));
   if (s != MOE_OK) return s;
   EpPeers peers;
   if ((s = check_ep(cfg, grp, &peers)) != MOE_OK) return s;
   if ((s = check_router(*cfg)) != MOE_OK) return s;
   if ((s = check_owner(*cfg, expert_owner)) != MOE_OK) return s;
-  if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes, f.fp8)) != MOE_OK) return s;
+  if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes, f.fp8, f.mx)) != MOE_OK) return s;
   if (handle_out && !handle_complete(handle_out)) return fail(MOE_ERR_INVALID_ARG, "incomplete handle_out");
   const moe_config& c = *cfg;
   const bool any = grp->local_experts > 0 || (c.N > 0 && c.n_shared > 0);
   if ((c.N > 0 && (!x || !w_gate || !y)) || (any && (!f.w13 || !f.w2)) ||
-      (any && f.fp8 && (!f.w13_scale || !f.w2_scale)))
+      (any && f.fp8 && (!f.w13_scale || !f.w2_scale)) || (any && f.mx && (!f.w13_sf || !f.w2_sf)))
     return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
   return ep_forward(c, *grp, peers, x, w_gate, bias, expert_owner, f, y, handle_out, dev_status,
-                    carve_ep(c, grp->capacity, static_cast<char*>(ws), f.fp8), (cudaStream_t)stream,
+                    carve_ep(c, grp->capacity, static_cast<char*>(ws), f.fp8, f.mx), (cudaStream_t)stream,
                     (cudaStream_t)side);
 }
 
@@ -1495,6 +1562,75 @@ moe_status moe_ep_layer_forward_fp8_overlapped(const moe_config* cfg, const moe_
   const EpFfn f = {true, nullptr, nullptr, w13_q, w13_scale, w2_q, w2_scale};
   return ep_layer(cfg, grp, x, w_gate, bias, expert_owner, f, y, handle_out, dev_status, ws, ws_bytes, stream,
                   side_stream);
+}
+
+size_t moe_ep_workspace_bytes_mx(const moe_config* cfg, int32_t capacity) {
+  if (check_mx(cfg) != MOE_OK || capacity < 1) return 0;
+  return carve_ep(*cfg, capacity, nullptr, false, true).total;
+}
+
+moe_status moe_ep_dispatch_mx(const moe_config* cfg, const moe_ep_group* grp, const void* x_q, const uint8_t* x_sf,
+                              const float* topk_w, const moe_ep_handle* handle, moe_stream_t stream) {
+  moe_status s = check_mx(cfg);
+  if (s != MOE_OK) return s;
+  EpPeers peers;
+  if ((s = check_ep(cfg, grp, &peers)) != MOE_OK) return s;
+  if (!handle_complete(handle) || (cfg->N > 0 && (!x_q || !x_sf || !topk_w)))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  return cuda_status(launch_ep_dispatch(*cfg, peers, ep_offsets(*cfg, grp->capacity), grp->rank, grp->capacity, x_q,
+                                        handle->dest, topk_w, nullptr, cfg->d, (cudaStream_t)stream, x_sf,
+                                        cfg->d / 32),
+                     "EP dispatch (mx)");
+}
+
+moe_status moe_ep_expert_ffn_mx(const moe_config* cfg, const moe_ep_group* grp, const void* x_q, const uint8_t* x_sf,
+                                const void* w13_q, const uint8_t* w13_sf, const void* w2_q, const uint8_t* w2_sf,
+                                const moe_ep_handle* handle, int32_t* dev_status, void* ws, size_t ws_bytes,
+                                moe_stream_t stream) {
+  moe_status s = check_mx(cfg);
+  if (s != MOE_OK) return s;
+  EpPeers peers;
+  if ((s = check_ep(cfg, grp, &peers)) != MOE_OK) return s;
+  if ((s = check_ep_ws(*cfg, grp, ws, ws_bytes, false, true)) != MOE_OK) return s;
+  const bool any = grp->local_experts > 0 || (cfg->N > 0 && cfg->n_shared > 0);
+  if (!handle_complete(handle) || (any && (!w13_q || !w13_sf || !w2_q || !w2_sf)) ||
+      (cfg->N > 0 && cfg->n_shared > 0 && (!x_q || !x_sf)))
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  EpFfn f = {false, x_q, nullptr, w13_q, nullptr, w2_q, nullptr};
+  f.mx = true;
+  f.x_sf = x_sf;
+  f.w13_sf = w13_sf;
+  f.w2_sf = w2_sf;
+  return ep_ffn_impl(*cfg, *grp, peers, f, *handle, dev_status,
+                     carve_ep(*cfg, grp->capacity, (char*)ws, false, true), (cudaStream_t)stream,
+                     ep_groups(*cfg, *grp));
+}
+
+static EpFfn mx_weights(const void* w13_q, const uint8_t* w13_sf, const void* w2_q, const uint8_t* w2_sf) {
+  EpFfn f = {false, nullptr, nullptr, w13_q, nullptr, w2_q, nullptr};
+  f.mx = true;
+  f.w13_sf = w13_sf;
+  f.w2_sf = w2_sf;
+  return f;
+}
+
+moe_status moe_ep_layer_forward_mx(const moe_config* cfg, const moe_ep_group* grp, const void* x, const void* w_gate,
+                                   const float* bias, const int32_t* expert_owner, const void* w13_q,
+                                   const uint8_t* w13_sf, const void* w2_q, const uint8_t* w2_sf, void* y,
+                                   const moe_ep_handle* handle_out, int32_t* dev_status, void* ws, size_t ws_bytes,
+                                   moe_stream_t stream) {
+  return ep_layer(cfg, grp, x, w_gate, bias, expert_owner, mx_weights(w13_q, w13_sf, w2_q, w2_sf), y, handle_out,
+                  dev_status, ws, ws_bytes, stream, nullptr);
+}
+
+moe_status moe_ep_layer_forward_mx_overlapped(const moe_config* cfg, const moe_ep_group* grp, const void* x,
+                                              const void* w_gate, const float* bias, const int32_t* expert_owner,
+                                              const void* w13_q, const uint8_t* w13_sf, const void* w2_q,
+                                              const uint8_t* w2_sf, void* y, const moe_ep_handle* handle_out,
+                                              int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                              moe_stream_t side_stream) {
+  return ep_layer(cfg, grp, x, w_gate, bias, expert_owner, mx_weights(w13_q, w13_sf, w2_q, w2_sf), y, handle_out,
+                  dev_status, ws, ws_bytes, stream, side_stream);
 }
 
 moe_status moe_capacity_rows(const moe_config* cfg, double factor, int32_t* capacity) {

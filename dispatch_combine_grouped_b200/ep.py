@@ -80,6 +80,8 @@ def window_views(cfg, capacity: int, window: torch.Tensor) -> dict:
                 gate=view(o["gate"], capacity, torch.float32),
                 scale=view(o["scale"], capacity, torch.float32),
                 x_recv_fp8=window[o["x_recv"]:o["x_recv"] + capacity * d].view(capacity, d),
+                x_recv_mx_sf=window[o["x_recv"] + capacity * d:o["x_recv"] + capacity * d + capacity * (d // 32)]
+                .view(capacity, d // 32),
                 x_recv=window[o["x_recv"]:o["x_recv"] + capacity * d * eb].view(dt).view(capacity, d),
                 out_recv=window[o["out_recv"]:o["out_recv"] + (capacity + S * N) * d * eb].view(dt)
                 .view(capacity + S * N, d))
@@ -116,8 +118,14 @@ def workspace_bytes_fp8(cfg, capacity: int) -> int:
     return B.load().moe_ep_workspace_bytes_fp8(ctypes.byref(c), capacity)
 
 
-def alloc_ws(cfg, capacity: int, device="cuda", fp8=False) -> torch.Tensor:
-    n = workspace_bytes_fp8(cfg, capacity) if fp8 else workspace_bytes(cfg, capacity)
+def workspace_bytes_mx(cfg, capacity: int) -> int:
+    c = B.c_config(cfg)
+    return B.load().moe_ep_workspace_bytes_mx(ctypes.byref(c), capacity)
+
+
+def alloc_ws(cfg, capacity: int, device="cuda", fp8=False, mx=False) -> torch.Tensor:
+    n = workspace_bytes_mx(cfg, capacity) if mx else (workspace_bytes_fp8(cfg, capacity) if fp8
+                                                      else workspace_bytes(cfg, capacity))
     return torch.empty(max(n, 1), dtype=torch.uint8, device=device)
 
 
@@ -319,4 +327,38 @@ def layer_forward_fp8(cfg, grp: Group, x, w_gate, bias, w13_q, w13_scale, w2_q, 
     else:
         B._check(B.load().moe_ep_layer_forward_fp8_overlapped(*args, ctypes.c_void_p(side_stream.cuda_stream)),
                  "moe_ep_layer_forward_fp8_overlapped")
+    return y
+
+
+def dispatch_mx(cfg, grp: Group, x_q, x_sf, topk_w, handle: Handle):
+    """MX payload: e4m3 token rows (d bytes) and their E8M0 scale rows (d/32 bytes)."""
+    c = B.c_config(cfg)
+    B._check(B.load().moe_ep_dispatch_mx(ctypes.byref(c), ctypes.byref(grp.c), B._p(x_q), B._p(x_sf),
+                                         B._p(topk_w), ctypes.byref(handle.c), B._stream()), "moe_ep_dispatch_mx")
+
+
+def expert_ffn_mx(cfg, grp: Group, x_q, x_sf, w13_q, w13_sf, w2_q, w2_sf, handle: Handle, ws, status=None):
+    c = B.c_config(cfg)
+    B._check(B.load().moe_ep_expert_ffn_mx(ctypes.byref(c), ctypes.byref(grp.c), B._p(x_q), B._p(x_sf),
+                                           B._p(w13_q), B._p(w13_sf), B._p(w2_q), B._p(w2_sf),
+                                           ctypes.byref(handle.c), B._p(status), B._p(ws), ws.numel(),
+                                           B._stream()), "moe_ep_expert_ffn_mx")
+
+
+def layer_forward_mx(cfg, grp: Group, x, w_gate, bias, w13_q, w13_sf, w2_q, w2_sf, ws, expert_owner=None, y=None,
+                     handle: Handle | None = None, status=None, side_stream=None):
+    """The layer on this rank with MX dispatch and experts, bf16 combine
+    (moe_ep_layer_forward_mx, or ..._overlapped with side_stream); ws from
+    alloc_ws(..., mx=True)."""
+    c = B.c_config(cfg)
+    if y is None:
+        y = torch.empty(cfg.N, cfg.d, dtype=torch.bfloat16, device=x.device)
+    args = [ctypes.byref(c), ctypes.byref(grp.c), B._p(x), B._p(w_gate), B._p(bias), B._p(expert_owner),
+            B._p(w13_q), B._p(w13_sf), B._p(w2_q), B._p(w2_sf), B._p(y),
+            ctypes.byref(handle.c) if handle is not None else None, B._p(status), B._p(ws), ws.numel(), B._stream()]
+    if side_stream is None:
+        B._check(B.load().moe_ep_layer_forward_mx(*args), "moe_ep_layer_forward_mx")
+    else:
+        B._check(B.load().moe_ep_layer_forward_mx_overlapped(*args, ctypes.c_void_p(side_stream.cuda_stream)),
+                 "moe_ep_layer_forward_mx_overlapped")
     return y

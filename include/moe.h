@@ -677,7 +677,8 @@ size_t moe_ep_window_bytes(const moe_config* cfg, int32_t capacity);
  * u64, done flags [32] u64 (each indexed by the signalling rank), step counter u64,
  * dispatch counter u32, failed-step word u64 (the last step in which a wait of this rank
  * gave up), count table [P, E] int32, gates [capacity] fp32, token scales [capacity] fp32
- * (FP8 dispatch), received rows [capacity, d] (of d bytes each for the FP8 dispatch),
+ * (FP8 dispatch), received rows [capacity, d] (of d bytes each for the FP8 dispatch; the
+ * MX dispatch puts its [capacity, d/32] scale rows right after its capacity code rows),
  * output rows [capacity + S*N, d].  (ABI version 101 added the failed-step word.) */
 moe_status moe_ep_window_layout(const moe_config* cfg, int32_t capacity, size_t* offsets);
 /* Bytes of scratch the EP calls of one step need (ws; the same ws for all calls of a step
@@ -761,6 +762,37 @@ moe_status moe_ep_layer_forward_fp8_overlapped(const moe_config* cfg, const moe_
                                                const float* w2_scale, void* y, const moe_ep_handle* handle_out,
                                                int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream,
                                                moe_stream_t side_stream);
+
+/* The EP layer with the MXFP8 expert path (MX dispatch, bf16 combine: the e4m3 code rows
+ * travel with their E8M0 scale rows, which land in the window's receive region after the
+ * capacity rows of codes, [capacity, d/32] bytes; see moe_quantize_mx / moe_grouped_ffn_mx).
+ * dtype = MOE_BF16, d % 512 == 0, I % 128 == 0.
+ *   moe_ep_dispatch_mx: as moe_ep_dispatch, code rows x_q [N, d] and scale rows x_sf
+ *     [N, d/32] of this rank's tokens.
+ *   moe_ep_expert_ffn_mx: as moe_ep_expert_ffn on MX operands: x_q, x_sf are this rank's
+ *     tokens (the shared experts' rows); w13_q [local+S, 2I, d] + w13_sf [local+S, 2I, d/32],
+ *     w2_q [local+S, d, I] + w2_sf [local+S, d, I/32].
+ *   moe_ep_layer_forward_mx(_overlapped): moe_route, moe_quantize_mx(x), then the five EP
+ *     steps with the two above (shared experts on side_stream in the overlapped form).
+ *     ws of moe_ep_workspace_bytes_mx bytes. */
+size_t moe_ep_workspace_bytes_mx(const moe_config* cfg, int32_t capacity);
+moe_status moe_ep_dispatch_mx(const moe_config* cfg, const moe_ep_group* grp, const void* x_q, const uint8_t* x_sf,
+                              const float* topk_w, const moe_ep_handle* handle, moe_stream_t stream);
+moe_status moe_ep_expert_ffn_mx(const moe_config* cfg, const moe_ep_group* grp, const void* x_q, const uint8_t* x_sf,
+                                const void* w13_q, const uint8_t* w13_sf, const void* w2_q, const uint8_t* w2_sf,
+                                const moe_ep_handle* handle, int32_t* dev_status, void* ws, size_t ws_bytes,
+                                moe_stream_t stream);
+moe_status moe_ep_layer_forward_mx(const moe_config* cfg, const moe_ep_group* grp, const void* x, const void* w_gate,
+                                   const float* bias, const int32_t* expert_owner, const void* w13_q,
+                                   const uint8_t* w13_sf, const void* w2_q, const uint8_t* w2_sf, void* y,
+                                   const moe_ep_handle* handle_out, int32_t* dev_status, void* ws, size_t ws_bytes,
+                                   moe_stream_t stream);
+moe_status moe_ep_layer_forward_mx_overlapped(const moe_config* cfg, const moe_ep_group* grp, const void* x,
+                                              const void* w_gate, const float* bias, const int32_t* expert_owner,
+                                              const void* w13_q, const uint8_t* w13_sf, const void* w2_q,
+                                              const uint8_t* w2_sf, void* y, const moe_ep_handle* handle_out,
+                                              int32_t* dev_status, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                              moe_stream_t side_stream);
 
 #ifdef __cplusplus
 }

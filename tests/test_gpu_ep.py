@@ -506,3 +506,80 @@ def test_ep_at_size_limits(cfg):
     y1 = moe.combine(cfg, lay1, out)
     torch.cuda.synchronize()
     assert torch.equal(res["y"], y1)
+
+
+MX_CASES = [
+    (small_config("ep_mx", cfg_id=136, N=512, d=512, E=16, S=1, k=4, I=128, P=4), None),
+    (small_config("ep_mx_owner", cfg_id=137, N=384, d=1024, E=32, S=2, k=4, I=256, P=4, n_groups=4, topk_groups=2,
+                  score="sigmoid"), "random"),
+]
+
+
+@pytest.mark.parametrize("cfg,spec", MX_CASES, ids=[c.name for c, _ in MX_CASES])
+def test_ep_mx_step_matches_one_gpu_mx_layer(cfg, spec):
+    """MX dispatch (e4m3 rows + their E8M0 scale rows over the peer windows), MX expert FFN
+    on the owners, bf16 combine: the received codes and scale rows are the quantised token
+    rows bit for bit, and y equals the one-GPU MX layer bit for bit."""
+    inp = gpu_inputs(cfg)
+    owner = _owner(cfg, spec)
+    em = Emulated(cfg, _shards(cfg, spec), owner)
+    em.ws = [ep.alloc_ws(c, em.capacity, mx=True) for c in em.rcfg]
+    P, n = cfg.P, cfg.N // cfg.P
+    w13_q, w13_sf = moe.quantize_mx(inp["w13"])
+    w2_q, w2_sf = moe.quantize_mx(inp["w2"])
+    xs = [inp["x"][r * n:(r + 1) * n] for r in range(P)]
+    routed = [moe.route(em.rcfg[r], xs[r], inp["w_gate"], inp["bias"]) for r in range(P)]
+    ids, w = [rt[1] for rt in routed], [rt[2] for rt in routed]
+    qs = [moe.quantize_mx(x) for x in xs]
+    E, S = cfg.E, cfg.S
+    ys = []
+    for r in range(P):
+        ep.notify(em.rcfg[r], em.groups[r], ids[r], em.ws[r], em.status)
+    for r in range(P):
+        ep.layout(em.rcfg[r], em.groups[r], ids[r], em.handles[r], em.ws[r], owner, em.status)
+    for r in range(P):
+        ep.dispatch_mx(em.rcfg[r], em.groups[r], qs[r][0], qs[r][1], w[r], em.handles[r])
+    for r in range(P):
+        idx = torch.tensor(list(em.owned[r]) + list(range(E, E + S)), dtype=torch.long, device="cuda")
+        ep.expert_ffn_mx(em.rcfg[r], em.groups[r], qs[r][0], qs[r][1], w13_q.index_select(0, idx),
+                         w13_sf.index_select(0, idx), w2_q.index_select(0, idx), w2_sf.index_select(0, idx),
+                         em.handles[r], em.ws[r], em.status)
+    for r in range(P):
+        ys.append(ep.combine(em.rcfg[r], em.groups[r], em.handles[r], status=em.status))
+    torch.cuda.synchronize()
+    assert int(em.status.item()) == 0
+    own_np = owner.cpu().numpy() if owner is not None else None
+    lay = O.ep_layout([i.cpu().numpy() for i in ids], cfg.E, cfg.P, own_np, em.capacity)
+    check_handles(em, lay)
+    for j in range(P):
+        v = ep.window_views(em.rcfg[j], em.capacity, em.windows[j])
+        rows = lay["recv"][j]
+        R = len(rows)
+        if R == 0:
+            continue
+        assert torch.equal(v["x_recv_fp8"][:R], torch.stack([qs[i][0][a // cfg.k] for i, a in rows]))
+        assert torch.equal(v["x_recv_mx_sf"][:R], torch.stack([qs[i][1][a // cfg.k] for i, a in rows]))
+        assert torch.equal(v["gate"][:R], torch.stack([w[i].reshape(-1)[a] for i, a in rows]))
+    y1 = moe.layer_forward_mx(cfg, inp["x"], inp["w_gate"], inp["bias"], owner, w13_q, w13_sf, w2_q, w2_sf)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(ys), y1)
+
+
+def test_ep_mx_layer_forward_one_rank():
+    """P = 1: moe_ep_layer_forward_mx and its overlapped form equal moe_layer_forward_mx."""
+    cfg = small_config("ep_mx_p1", cfg_id=138, N=300, d=512, E=16, S=1, k=4, I=128, P=1)
+    inp = gpu_inputs(cfg)
+    cap = cfg.N * cfg.k
+    groups, windows = ep.emulated_groups(cfg, cap)
+    ws = ep.alloc_ws(cfg, cap, mx=True)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    w13_q, w13_sf = moe.quantize_mx(inp["w13"])
+    w2_q, w2_sf = moe.quantize_mx(inp["w2"])
+    side = torch.cuda.Stream()
+    for step in range(3):
+        y = ep.layer_forward_mx(cfg, groups[0], inp["x"], inp["w_gate"], inp["bias"], w13_q, w13_sf, w2_q, w2_sf, ws,
+                                status=status, side_stream=side if step == 2 else None)
+        y1 = moe.layer_forward_mx(cfg, inp["x"], inp["w_gate"], inp["bias"], None, w13_q, w13_sf, w2_q, w2_sf)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert torch.equal(y, y1)
