@@ -476,9 +476,10 @@ def run_ep(args, cfg, local):
     inp = make_inputs(gcfg, device=dev)
     n = cfg.N // P
     rc = gcfg.replace(N=n)
-    f8 = bool(args.fp8)
+    mx = bool(args.mx)
+    f8 = bool(args.fp8) and not mx
     E, S, R = cfg.E, cfg.S, args.eplb
-    if R and f8:
+    if R and (f8 or mx):
         raise SystemExit("--ep with --eplb runs the bf16 path")
     # the workload's placement (e.g. the hot-spot table), else contiguous; with EPLB the
     # copies are planned from this batch's counts and the slot weights placed once
@@ -506,23 +507,29 @@ def run_ep(args, cfg, local):
     # buffers from the exchanged counts (+ k*P rows for the per-rank split of copies)
     cap = int(-(-(int(load.max()) + cfg.k * P) // 128) * 128)
     groups, windows = ep.emulated_groups(pc, cap, owner_t)
-    ws = [ep.alloc_ws(pc, cap, fp8=f8) for _ in range(P)]
+    ws = [ep.alloc_ws(pc, cap, fp8=f8, mx=mx) for _ in range(P)]
     handles = [ep.Handle(pc, len(slots_of[r])) for r in range(P)]
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     wts = []
-    if f8:  # weights quantised once (a load-time step), then sliced per owner
-        w13_q, w13_s = moe.quantize_fp8(inp["w13"])
-        w2_q, w2_s = moe.quantize_fp8(inp["w2"])
+    if f8 or mx:  # weights quantised once (a load-time step), then sliced per owner
+        quant = moe.quantize_mx if mx else moe.quantize_fp8
+        w13_q, w13_s = quant(inp["w13"])
+        w2_q, w2_s = quant(inp["w2"])
         del inp["w13"], inp["w2"]
     for r in range(P):
         idx = torch.tensor(slots_of[r] + list(range(E_slots, E_slots + S)), device=dev)
-        if f8:
+        if f8 or mx:
             wts.append(tuple(t.index_select(0, idx) for t in (w13_q, w13_s, w2_q, w2_s)))
         else:
             wts.append((w13_ep.index_select(0, idx), w2_ep.index_select(0, idx)))
     xs = [inp["x"][r * n:(r + 1) * n] for r in range(P)]
-    qs = [(torch.empty(n, cfg.d, dtype=torch.uint8, device=dev), torch.empty(n, dtype=torch.float32, device=dev))
-          for _ in range(P)] if f8 else None
+    qs = None
+    if f8:
+        qs = [(torch.empty(n, cfg.d, dtype=torch.uint8, device=dev), torch.empty(n, dtype=torch.float32, device=dev))
+              for _ in range(P)]
+    elif mx:
+        qs = [(torch.empty(n, cfg.d, dtype=torch.uint8, device=dev),
+               torch.empty(n, cfg.d // 32, dtype=torch.uint8, device=dev)) for _ in range(P)]
     routed = [moe.route(rc, xs[r], inp["w_gate"], inp["bias"]) for r in range(P)]
     ys = [torch.empty(n, cfg.d, dtype=cfg.torch_dtype, device=dev) for _ in range(P)]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -537,6 +544,8 @@ def run_ep(args, cfg, local):
             moe.route(rc, xs[r], inp["w_gate"], inp["bias"], out=routed[r])
             if f8:
                 moe.quantize_fp8(xs[r], out=qs[r][0], scale=qs[r][1])
+            elif mx:
+                moe.quantize_mx(xs[r], out=qs[r][0], sf=qs[r][1])
             if R:
                 moe.eplb_assign(rc, routed[r][1], rep_off, rep_slots, E + R, status=status, out=phys[r], ws=eplb_ws)
         ids_ep = phys if R else [rt[1] for rt in routed]
@@ -550,6 +559,8 @@ def run_ep(args, cfg, local):
         for r in range(P):
             if f8:
                 ep.dispatch_fp8(pc, groups[r], qs[r][0], qs[r][1], routed[r][2], handles[r])
+            elif mx:
+                ep.dispatch_mx(pc, groups[r], qs[r][0], qs[r][1], routed[r][2], handles[r])
             else:
                 ep.dispatch(pc, groups[r], xs[r], routed[r][2], handles[r])
         mark(4)
@@ -558,6 +569,8 @@ def run_ep(args, cfg, local):
                 fev[r][0].record()
             if f8:
                 ep.expert_ffn_fp8(pc, groups[r], qs[r][0], qs[r][1], *wts[r], handles[r], ws[r], status)
+            elif mx:
+                ep.expert_ffn_mx(pc, groups[r], qs[r][0], qs[r][1], *wts[r], handles[r], ws[r], status)
             else:
                 ep.expert_ffn(pc, groups[r], xs[r], wts[r][0], wts[r][1], handles[r], ws[r], status)
             if fev is not None:
@@ -610,6 +623,12 @@ def run_ep(args, cfg, local):
         def one_gpu(y=None):
             return moe.layer_forward_fp8(gcfg, inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], w13_q,
                                          w13_s, w2_q, w2_s, y=y, ws=ws1)
+    elif mx:
+        ws1 = torch.empty(moe.workspace_bytes_mx(gcfg), dtype=torch.uint8, device=dev)
+
+        def one_gpu(y=None):
+            return moe.layer_forward_mx(gcfg, inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], w13_q,
+                                        w13_s, w2_q, w2_s, y=y, ws=ws1)
     else:
         ws1 = moe.alloc_workspace(gcfg, dev)
 
@@ -636,7 +655,8 @@ def run_ep(args, cfg, local):
         cross.append(int((owner != r).sum().item()))
     owner_rows = [int(h.as_dict()["owner_off"][-1].item()) for h in handles]
     row_bytes = cfg.d * eb                      # output rows (combine) and bf16 payload rows
-    pay_bytes = cfg.d * (1 if f8 else eb)       # dispatch payload rows (e4m3: d bytes)
+    pay_bytes = cfg.d + cfg.d // 32 if mx else cfg.d * (1 if f8 else eb)  # dispatch payload rows (e4m3: d
+    #                                                 bytes, plus d/32 scale bytes for MX)
     max_cross = max(cross) * pay_bytes
     med = sorted(step_ms)[len(step_ms) // 2]
     stage_ms = {k: tot[i] / args.steps for i, k in enumerate(stages)}
@@ -644,10 +664,11 @@ def run_ep(args, cfg, local):
     pay_x, pay_rows = cfg.N * pay_bytes, cfg.N * cfg.k * pay_bytes
     print(json.dumps({
         "metric": "MoE-layer tokens/s, expert-parallel path with P ranks emulated on one GPU"
-                  + (" (FP8 dispatch and experts, bf16 combine)" if f8 else ""),
+                  + (" (FP8 dispatch and experts, bf16 combine)" if f8 else "")
+                  + (" (MXFP8 dispatch and experts, bf16 combine)" if mx else ""),
         "value": cfg.N / (med / 1e3), "unit": "tokens/s", "n_gpus": 1, "ep_ranks_emulated": P,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": med,
-        "dtype": "e4m3 (scaled), bf16 out" if f8 else cfg.dtype,
+        "dtype": "e4m3 (scaled), bf16 out" if f8 else ("e4m3 + E8M0 per 32, bf16 out" if mx else cfg.dtype),
         "config": {"workload": describe(gcfg), "tokens_per_rank": n, "capacity_rows_per_owner": cap,
                    "l2": "flushed before every step"},
         "how": "ms_per_step: the emulated step of all P ranks as one CUDA graph replay; stages: eager launches "
