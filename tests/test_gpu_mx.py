@@ -196,3 +196,47 @@ def test_mx_rejects_unsupported_shapes():
     with pytest.raises(moe.MoEError):
         moe.layer_forward_mx(cfg, inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], w13_q, w13_sf, w2_q,
                              w2_sf)
+
+
+@pytest.mark.parametrize("factor", [0.0, 0.7])
+def test_mx_layer_with_capacity_drops(factor):
+    """Assignments dropped by a capacity factor (id -1) take no row: the MX permute skips
+    them and y equals the oracle's MX layer over the kept assignments (factor 0: the shared
+    expert alone)."""
+    cfg = SMALL[0]
+    inp = gpu_inputs(cfg)
+    E, S, N, k, I, d = cfg.E, cfg.S, cfg.N, cfg.k, cfg.I, cfg.d
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    logits, ids, w = moe.route(cfg, inp["x"], inp["w_gate"], inp["bias"])
+    kept = moe.capacity_drop(cfg, ids, moe.capacity_of(factor, cfg), status=status)
+    lay = moe.dispatch_layout(cfg, kept, inp["expert_owner"], status=status)
+    x_q, x_sf = moe.quantize_mx(inp["x"])
+    w13_q, w13_sf = moe.quantize_mx(inp["w13"])
+    w2_q, w2_sf = moe.quantize_mx(inp["w2"])
+    xp, xp_sf = moe.permute_mx(cfg, lay, x_q, x_sf)
+    h, h_q, h_sf, out = moe.grouped_ffn_mx(cfg, lay, xp, xp_sf, x_q, x_sf, w13_q, w13_sf, w2_q, w2_sf, topk_w=w)
+    y = moe.combine(cfg, lay, out)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    kept_np = kept.cpu().numpy().astype(np.int64)
+    assert (kept_np < 0).any()
+    xq_ref, xsf_ref = F.quantize_mx(inp["x"].float().cpu().numpy())
+    w13q, w13sf = F.quantize_mx(inp["w13"].float().cpu().numpy().reshape(-1, d))
+    w2q, w2sf = F.quantize_mx(inp["w2"].float().cpu().numpy().reshape(-1, I))
+    w13q, w13sf = w13q.reshape(E + S, 2 * I, d), w13sf.reshape(E + S, 2 * I, d // 32)
+    w2q, w2sf = w2q.reshape(E + S, d, I), w2sf.reshape(E + S, d, I // 32)
+    gates = O.f64(w)
+
+    def expert(e, toks):  # the MX expert on token rows, h rounded to bf16 and quantised
+        hh = F.fc1_mx(xq_ref[toks], xsf_ref[toks], w13q[e], w13sf[e], I)
+        hq, hs = F.quantize_mx(_to_bf16(hh).astype(np.float32))
+        return F.fc2_mx(hq, hs, w2q[e], w2sf[e])
+
+    y_ref = np.zeros((N, d))
+    for e in range(E):
+        t, j = np.nonzero(kept_np == e)
+        if len(t):
+            y_ref[t] += expert(e, t) * gates[t, j][:, None]
+    for s in range(S):
+        y_ref += expert(E + s, np.arange(N))
+    assert_close_fro(y, y_ref, what=f"MX layer with capacity factor {factor}")
