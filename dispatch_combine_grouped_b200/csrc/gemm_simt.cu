@@ -1,14 +1,15 @@
 // fp32 grouped GEMM on the CUDA cores, for the fp32 configurations (the tensor-core path
 // is bf16).  Same three jobs and the same group / tile scheme as the tcgen05 kernel:
 // router logits (+ bias), FC1 with SwiGLU, FC2 with the gate scale.  64 x 64 output tile
-// per CTA, 16-deep k slices staged in shared memory, 4 x 4 outputs per thread, fp32 FMA
-// in ascending k order.
+// per CTA, 32-deep k slices staged in shared memory (the next slice's loads issued into
+// registers before the current one is multiplied, so that their latency overlaps the
+// FMAs), 4 x 4 outputs per thread, fp32 FMA in ascending k order.
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace moe {
 
-constexpr int SBM = 64, SBN = 64, SBK = 16;
+constexpr int SBM = 64, SBN = 64, SBK = 32;
 constexpr int kSimtThreads = 256;
 constexpr int kSimtGroups = kMaxSlots + kMaxShared;
 
@@ -86,36 +87,43 @@ __global__ void __launch_bounds__(kSimtThreads) simt_gemm_kernel(const GemmArgs 
     const int n0 = n_blk * SBN;
 
     float accg[4][4] = {}, accu[4][4] = {};
-    for (int k0 = 0; k0 < p.K; k0 += SBK) {
-      {  // A slice: 64 rows x 16 k, one float4 per thread
-        const int r = tid / 4, kq = (tid % 4) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (m_blk * SBM + r < rows && k0 + kq < p.K)
-          v = *reinterpret_cast<const float4*>(Abase + (arow0 + r) * p.K + k0 + kq);
-        As[kq + 0][r] = v.x;
-        As[kq + 1][r] = v.y;
-        As[kq + 2][r] = v.z;
-        As[kq + 3][r] = v.w;
-      }
-      {  // B slice(s): 64 output columns x 16 k
-        const int c = tid / 4, kq = (tid % 4) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f), u = v;
-        if (n0 + c < p.n_out && k0 + kq < p.K) {
-          v = *reinterpret_cast<const float4*>(W + (long long)(n0 + c) * p.K + k0 + kq);
-          if (MODE == MODE_FC1) u = *reinterpret_cast<const float4*>(W + (long long)(p.I + n0 + c) * p.K + k0 + kq);
+    // this thread's share of a slice: rows / columns tid / 4, k offsets (tid % 4) * 4 and +16
+    const int lr = tid / 4, kq = (tid % 4) * 4;
+    float4 ra[2], rg[2], ru[2];
+    auto load = [&](int k0) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int kk = k0 + kq + 16 * h;
+        ra[h] = rg[h] = ru[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (m_blk * SBM + lr < rows && kk < p.K) ra[h] = *reinterpret_cast<const float4*>(Abase + (arow0 + lr) * p.K + kk);
+        if (n0 + lr < p.n_out && kk < p.K) {
+          rg[h] = *reinterpret_cast<const float4*>(W + (long long)(n0 + lr) * p.K + kk);
+          if (MODE == MODE_FC1) ru[h] = *reinterpret_cast<const float4*>(W + (long long)(p.I + n0 + lr) * p.K + kk);
         }
-        Bg[kq + 0][c] = v.x;
-        Bg[kq + 1][c] = v.y;
-        Bg[kq + 2][c] = v.z;
-        Bg[kq + 3][c] = v.w;
+      }
+    };
+    load(0);
+    for (int k0 = 0; k0 < p.K; k0 += SBK) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // registers -> shared memory, k-major
+        const int kk = kq + 16 * h;
+        As[kk + 0][lr] = ra[h].x;
+        As[kk + 1][lr] = ra[h].y;
+        As[kk + 2][lr] = ra[h].z;
+        As[kk + 3][lr] = ra[h].w;
+        Bg[kk + 0][lr] = rg[h].x;
+        Bg[kk + 1][lr] = rg[h].y;
+        Bg[kk + 2][lr] = rg[h].z;
+        Bg[kk + 3][lr] = rg[h].w;
         if (MODE == MODE_FC1) {
-          Bu[kq + 0][c] = u.x;
-          Bu[kq + 1][c] = u.y;
-          Bu[kq + 2][c] = u.z;
-          Bu[kq + 3][c] = u.w;
+          Bu[kk + 0][lr] = ru[h].x;
+          Bu[kk + 1][lr] = ru[h].y;
+          Bu[kk + 2][lr] = ru[h].z;
+          Bu[kk + 3][lr] = ru[h].w;
         }
       }
       __syncthreads();
+      if (k0 + SBK < p.K) load(k0 + SBK);  // the next slice, in flight during the FMAs below
 #pragma unroll
       for (int kk = 0; kk < SBK; ++kk) {
         float a[4], bg[4], bu[4];
