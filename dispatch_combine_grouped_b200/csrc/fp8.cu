@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "mx.cuh"
 
 namespace moe {
 
@@ -65,25 +66,9 @@ cudaError_t launch_quantize_rows(const void* src, long long rows, int cols, void
   return cudaGetLastError();
 }
 
-// Block-scaled (MX) e4m3 quantisation: the microscaling format for FP8 elements
-// ("MoE我们喜欢你（四）" names MXFP8 expert compute).  Every 32 consecutive values of a row
-// share one power-of-two scale X = 2^e stored as an E8M0 byte (e + 127), with
-// e = floor(log2 amax) - 8 (8: the exponent of 256, the largest power of two in e4m3),
-// clamped to [-127, 127] (-127 for an all-zero block); code = round-to-nearest-even of
-// v * 2^-e, saturating at +-448.  The scaling by 2^-e is exact (it only moves the exponent)
-// unless the product falls below 2^-126, where every candidate code is 0 anyway.
-//
+// Block-scaled (MX) e4m3 quantisation of rows (the format and its rule: mx.cuh).
 // One warp per row, one 32-value block per lane: four 16-byte loads (64 bytes, adjacent
 // lanes adjacent), two 16-byte stores of codes and one scale byte per lane.
-__device__ __forceinline__ int mx_exponent(float amax) {
-  const uint32_t b = __float_as_uint(amax);
-  if (b == 0u) return -127;
-  const int biased = (int)(b >> 23);
-  const int fl = biased > 0 ? biased - 127 : (31 - __clz((int)(b & 0x7FFFFFu))) - 149;  // floor(log2 amax)
-  const int e = fl - 8;
-  return e < -127 ? -127 : (e > 127 ? 127 : e);
-}
-
 __global__ void __launch_bounds__(kQuantWarps * 32)
     quantize_mx_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, uint8_t* __restrict__ sf,
                        long long rows, int blocks_per_row) {
@@ -107,23 +92,11 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
         f[q * 8 + 2 * h + 1] = t.y;
       }
     }
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(f[i]));
-    const int e = mx_exponent(amax);
-    const float inv = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, a normal float for e <= 119
     uint32_t packed[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
-          make_float2(__fmul_rn(f[4 * i], inv), __fmul_rn(f[4 * i + 1], inv)), __NV_SATFINITE, __NV_E4M3);
-      const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
-          make_float2(__fmul_rn(f[4 * i + 2], inv), __fmul_rn(f[4 * i + 3], inv)), __NV_SATFINITE, __NV_E4M3);
-      packed[i] = (uint32_t)lo | ((uint32_t)hi << 16);
-    }
+    const uint8_t sfb = mx_quantize32(f, packed);
     d[blk * 2] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     d[blk * 2 + 1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-    sf[r * blocks_per_row + blk] = (uint8_t)(e + 127);
+    sf[r * blocks_per_row + blk] = sfb;
   }
 }
 

@@ -22,7 +22,9 @@
 //               columns, scale B: 8; every 32-lane quarter gets a copy) and 4 block-scaled
 //               MMAs (M=128, N=192, K=32 each; the scale of k-block kk is byte kk of the
 //               TMEM words, selected by the instruction descriptor)
-//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes, SwiGLU / gate, bf16 stores
+//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes, SwiGLU / gate, bf16 stores;
+//               FC1 also quantises h to MX as it goes (a 32-column chunk of a row is one
+//               MX block of h, held by one thread), so h needs no pass of its own
 // TMEM: two 192-column fp32 accumulators (columns 0 and 192), the scale columns after
 // them (one copy; the tcgen05 operations of a thread run in issue order, so the next
 // stage's copy follows the MMAs that read the previous one).  N = 192 keeps both
@@ -31,6 +33,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "mx.cuh"
 
 namespace moe {
 namespace {
@@ -437,7 +440,7 @@ __global__ void __launch_bounds__(kThreadsMx, 1)
       const int r = td.m_blk * kBM + r_in_tile;
       const bool row_ok = r < s_rows[td.g];
       const long long orow = (long long)s_orow[td.g] + r;
-      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + orow * p.ldo;
+      __nv_bfloat16* dst = p.out ? static_cast<__nv_bfloat16*>(p.out) + orow * p.ldo : nullptr;
       if (MODE == MODE_FC1) {
         const int col_base = td.n_blk * (kBN / 2);
 #pragma unroll 1
@@ -446,21 +449,35 @@ __global__ void __launch_bounds__(kThreadsMx, 1)
           tmem_ld32(taddr + c0, gv);
           tmem_ld32(taddr + kBN / 2 + c0, uv);
           tmem_wait_ld();
-          if (row_ok) {
+          // n_out % 32 == 0: a 32-column chunk is wholly inside the output or wholly past it
+          if (row_ok && col_base + c0 < p.n_out) {
+            uint32_t w[16];  // the chunk's h rounded to bf16, two per word
 #pragma unroll
-            for (int q = 0; q < 32; q += 8) {
-              const int col = col_base + c0 + q;
-              if (col < p.n_out) {  // n_out % 8 == 0: the whole vector is valid
-                uint32_t w[4];
+            for (int u = 0; u < 16; ++u) {
+              const float h0 = silu_f32(__uint_as_float(gv[2 * u])) * __uint_as_float(uv[2 * u]);
+              const float h1 = silu_f32(__uint_as_float(gv[2 * u + 1])) * __uint_as_float(uv[2 * u + 1]);
+              w[u] = pack_bf16x2(h0, h1);
+            }
+            const int col = col_base + c0;
+            if (p.out) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  const float h0 = silu_f32(__uint_as_float(gv[q + 2 * u])) * __uint_as_float(uv[q + 2 * u]);
-                  const float h1 =
-                      silu_f32(__uint_as_float(gv[q + 2 * u + 1])) * __uint_as_float(uv[q + 2 * u + 1]);
-                  w[u] = pack_bf16x2(h0, h1);
-                }
-                *reinterpret_cast<uint4*>(dst + col) = make_uint4(w[0], w[1], w[2], w[3]);
+              for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4*>(dst + col + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+            }
+            if (p.q_out) {  // the chunk is one MX block of h: quantise the stored (bf16) values
+              float f[32];
+#pragma unroll
+              for (int u = 0; u < 16; ++u) {
+                const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[u]));
+                f[2 * u] = t.x;
+                f[2 * u + 1] = t.y;
               }
+              uint32_t packed[8];
+              const uint8_t sfb = mx_quantize32(f, packed);
+              uint4* qd = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.q_out) + orow * p.n_out + col);
+              qd[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+              qd[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+              p.q_sf[orow * (p.n_out / 32) + col / 32] = sfb;
             }
           }
         }
@@ -524,8 +541,9 @@ cudaError_t launch_mode(const GemmArgs& g, const CUtensorMap& a0, const CUtensor
 }  // namespace
 
 cudaError_t launch_tc_gemm_mx(const GemmArgs& g, cudaStream_t st) {
-  if ((g.mode != MODE_FC1 && g.mode != MODE_FC2) || g.K % kBK != 0 || g.n_out % 8 != 0 || !g.a0_sf || !g.b_sf ||
-      (g.a1 && !g.a1_sf) || g.a0_rows < 1 || g.b_rows < 1)
+  if ((g.mode != MODE_FC1 && g.mode != MODE_FC2) || g.K % kBK != 0 || g.n_out % 32 != 0 || !g.a0_sf || !g.b_sf ||
+      (g.a1 && !g.a1_sf) || g.a0_rows < 1 || g.b_rows < 1 || (g.q_out && !g.q_sf) ||
+      (g.mode == MODE_FC2 && !g.out) || (g.mode == MODE_FC1 && !g.out && !g.q_out))
     return cudaErrorInvalidValue;
   CUtensorMap a0, a1, b;
   if (!make_map_a(&a0, g.a0, g.a0_rows, g.K, kBK, true)) return cudaErrorInvalidValue;

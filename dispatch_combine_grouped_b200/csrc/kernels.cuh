@@ -91,6 +91,11 @@ struct GemmArgs {
   const uint8_t* a1_sf;  // rows of A map 1 (FC1: the tokens, for the shared experts)
   const uint8_t* b_sf;   // [groups, b_rows, K/32]
   long long a0_rows, a1_rows;  // rows of the A tensors (the last row is read for rows past them)
+  // MX FC1: the epilogue also writes h MX-quantised (after its bf16 rounding): codes
+  // [rows, n_out] and E8M0 scale bytes [rows, n_out/32] (NULL: not written); out may then
+  // be NULL (h not stored in bf16)
+  void* q_out;
+  uint8_t* q_sf;
 };
 
 #ifdef __CUDACC__

@@ -123,7 +123,7 @@ FwdWs carve_forward(const moe_config& c, char* base, bool fp8 = false, bool mx =
   w.lay.tile_off = reinterpret_cast<int32_t*>(take((E + S + 1) * 4));
   w.lay_ws = take(layout_scratch(c));
   w.x_perm = take(A * c.d * (fp8 ? 1 : eb));
-  w.h = take((A + S * c.N) * c.I * eb);
+  w.h = take(mx ? 0 : (A + S * c.N) * c.I * eb);  // the MX forward quantises h in FC1's epilogue
   w.out = take((A + S * c.N) * c.d * eb);
   if (fp8) {
     w.x_q = take((size_t)c.N * c.d);
@@ -307,8 +307,9 @@ moe_status ffn_fp8_impl(const moe_config& c, const moe_layout& L, const Fp8Ffn& 
   return cuda_status(tc_grouped(g2, c, (int)(A + (long long)c.n_shared * c.N), 0, st), "FC2 grouped GEMM (fp8)");
 }
 
-// MX expert FFN over groups [g0, g0+G): FC1 on block-scaled e4m3 rows -> h (bf16) -> MX
-// quantisation of h -> FC2 on block-scaled rows, on the block-scaled tile kernel.
+// MX expert FFN over groups [g0, g0+G): FC1 on block-scaled e4m3 rows, whose epilogue
+// rounds h to bf16 (stored when f.h is given) and quantises it to MX, then FC2 on
+// block-scaled rows, on the block-scaled tile kernel.
 struct MxFfn {
   const void* x_q_perm;
   const uint8_t* x_sf_perm;
@@ -339,13 +340,10 @@ moe_status ffn_mx_impl(const moe_config& c, const moe_layout& L, const MxFfn& f,
   g.b_sf = f.w13_sf;
   g.a0_rows = A > 0 ? A : 1;
   g.a1_rows = c.N;
+  g.q_out = f.h_q;  // h quantised by FC1's epilogue (h itself stored only when f.h is given)
+  g.q_sf = f.h_sf;
   cudaError_t e = launch_tc_gemm_mx(g, st);
   if (e != cudaSuccess) return cuda_status(e, "FC1 grouped GEMM (mx)");
-  const long long r0 = g0 < c.E ? 0 : A + (long long)(g0 - c.E) * c.N;
-  const long long r1 = (g0 + G <= c.E) ? A : A + (long long)(g0 + G - c.E) * c.N;
-  e = launch_quantize_mx(static_cast<const uint16_t*>(f.h) + r0 * c.I, r1 - r0, c.I,
-                         static_cast<uint8_t*>(f.h_q) + r0 * c.I, f.h_sf + r0 * (c.I / 32), st);
-  if (e != cudaSuccess) return cuda_status(e, "h quantisation (mx)");
   GemmArgs g2 = fc2_args(c, L, f.h_q, f.w2_q, f.topk_w, f.out);
   g2.g0 = g0;
   g2.G = G;
@@ -417,6 +415,8 @@ EpWs carve_ep(const moe_config& c, int capacity, char* base, bool fp8 = false, b
   w.loc.row2tok = i32(A);
   w.loc.tile_off = i32(E + S + 1);
   w.lay_ws = take(layout_scratch(one_owner(c)));
+  // (the MX path quantises h in FC1's epilogue and leaves this unused; it stays so that an
+  // MX workspace also satisfies the size check of the precision-independent EP calls)
   w.h = take(((size_t)capacity + S * c.N) * c.I * eb);
   w.logits = reinterpret_cast<float*>(take((size_t)c.N * E * 4));
   w.ids = i32(A);
@@ -507,7 +507,7 @@ struct EpFfn {
 };
 
 // The MX form of ep_gemms: FC1 on the received codes and their scale rows (the shared
-// groups on this rank's own x codes), MX quantisation of the h rows of the range, FC2.
+// groups on this rank's own x codes) with h quantised to MX in its epilogue, then FC2.
 moe_status ep_gemms_mx(const moe_config& c, const moe_ep_group& g, char* win, const EpOffsets& off, const EpFfn& f,
                        const moe_ep_handle& hd, const EpWs& w, cudaStream_t st, int g0, int G) {
   moe_config co = c;
@@ -529,14 +529,11 @@ moe_status ep_gemms_mx(const moe_config& c, const moe_ep_group& g, char* win, co
   g1.b_sf = f.w13_sf;
   g1.a0_rows = cap;
   g1.a1_rows = c.N > 0 ? c.N : 1;
+  g1.out = nullptr;  // h quantised by the epilogue, not kept in bf16
+  g1.q_out = w.h_q;
+  g1.q_sf = w.h_sf;
   cudaError_t e = launch_tc_gemm_mx(g1, st);
   if (e != cudaSuccess) return cuda_status(e, "EP FC1 grouped GEMM (mx)");
-  const int Lx = g.local_experts;
-  const long long r0 = g0 < Lx ? 0 : cap + (long long)(g0 - Lx) * c.N;
-  const long long r1 = g0 + G <= Lx ? cap : cap + (long long)(g0 + G - Lx) * c.N;
-  e = launch_quantize_mx(static_cast<const uint16_t*>(w.h) + r0 * c.I, r1 - r0, c.I,
-                         static_cast<uint8_t*>(w.h_q) + r0 * c.I, w.h_sf + r0 * (c.I / 32), st);
-  if (e != cudaSuccess) return cuda_status(e, "h quantisation (mx)");
   GemmArgs g2 = fc2_args(co, L, w.h_q, f.w2, reinterpret_cast<const float*>(win + off.gate), win + off.out_recv);
   g2.g0 = g0;
   g2.G = G;
@@ -1296,7 +1293,8 @@ static moe_status forward_mx(const moe_config* cfg, const void* x, const void* w
   if ((s = route_impl(c, x, w_gate, bias, w.logits, w.ids, w.w, st)) != MOE_OK) return s;
   if ((s = cuda_status(launch_quantize_mx(x, c.N, c.d, w.x_q, w.x_sf, st), "x quantisation (mx)")) != MOE_OK)
     return s;
-  MxFfn f{w.x_perm, w.x_sf_perm, w.x_q, w.x_sf, w13_q, w13_sf, w2_q, w2_sf, w.w, w.h, w.h_q, w.h_sf, w.out};
+  // h is quantised by FC1's epilogue and not kept in bf16
+  MxFfn f{w.x_perm, w.x_sf_perm, w.x_q, w.x_sf, w13_q, w13_sf, w2_q, w2_sf, w.w, nullptr, w.h_q, w.h_sf, w.out};
   const bool overlap = side != nullptr && side != st && c.n_shared > 0;
   cudaEvent_t fork = nullptr, join = nullptr;
   cudaError_t e = cudaSuccess;

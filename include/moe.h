@@ -553,7 +553,8 @@ moe_status moe_permute_mx(const moe_config* cfg, const moe_layout* layout, const
 /*
  * MX grouped SwiGLU FFN, routed and shared experts:
  *   h = SiLU(X W_gate^T) * (X W_up^T) on MX operands         (bf16 [A + S*N, I])
- *   h_q, h_sf = moe_quantize_mx(h)                          (e4m3 [A + S*N, I], E8M0 [A + S*N, I/32])
+ *   h_q, h_sf = the MX quantisation of h (as moe_quantize_mx; done by FC1's epilogue)
+ *                                                           (e4m3 [A + S*N, I], E8M0 [A + S*N, I/32])
  *   out = (h W2^T on MX operands) * gate(row)               (bf16 [A + S*N, d])
  *   x_q_perm [A, d] + x_sf_perm [A, d/32] (moe_permute_mx); x_q [N, d] + x_sf [N, d/32]
  *   (the shared experts' rows; NULL when n_shared == 0); w13_q [E+S, 2I, d] + w13_sf
