@@ -152,11 +152,11 @@ def test_mx_layer_staged(cfg):
     assert torch.equal(y, r["y"]) and torch.equal(y_ov, r["y"])
 
 
-@pytest.mark.parametrize("name", ["fine", "wide"])
+@pytest.mark.parametrize("name", ["fine", "wide", "decode", "hot_cal"])
 def test_mx_full_size_sampled(name):
     """Full-size workloads: x quantisation bit-exact, the sampled experts' weight codes and
     scales bit-exact, sampled rows of h and out against the oracle (covering first and last
-    rows of the sampled groups), fused == staged."""
+    rows of the sampled groups, and of the shared experts), fused == staged."""
     cfg = CONFIGS[name]
     inp = gpu_inputs(cfg)
     r = _staged(cfg, inp)
@@ -181,6 +181,17 @@ def test_mx_full_size_sampled(name):
         g = O.f64(r["w"]).reshape(-1)[row2tok[rows]]
         assert_close_fro(r["out"][torch.tensor(rows)], F.fc2_mx(hq[rows], hsf[rows], w2q_ref, w2sf_ref) * g[:, None],
                          what=f"out expert {e}")
+    A = cfg.N * k
+    for s_ in range(cfg.S):  # the shared experts: sampled token rows, first and last included
+        e = E + s_
+        w13q_ref, w13sf_ref = F.quantize_mx(inp["w13"][e].float().cpu().numpy())
+        w2q_ref, w2sf_ref = F.quantize_mx(inp["w2"][e].float().cpu().numpy())
+        tok = np.unique(np.concatenate([[0, cfg.N - 1], rng.choice(cfg.N, min(6, cfg.N), replace=False)]))
+        rows = A + s_ * cfg.N + tok
+        assert_close_rel(r["h"][torch.tensor(rows)], F.fc1_mx(xq_ref[tok], xsf_ref[tok], w13q_ref, w13sf_ref, I),
+                         what=f"h shared expert {s_}")
+        assert_close_fro(r["out"][torch.tensor(rows)], F.fc2_mx(hq[rows], hsf[rows], w2q_ref, w2sf_ref),
+                         what=f"out shared expert {s_}")
     y = moe.layer_forward_mx(cfg, inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], r["w13_q"],
                              r["w13_sf"], r["w2_q"], r["w2_sf"])
     torch.cuda.synchronize()
@@ -240,3 +251,36 @@ def test_mx_layer_with_capacity_drops(factor):
     for s in range(S):
         y_ref += expert(E + s, np.arange(N))
     assert_close_fro(y, y_ref, what=f"MX layer with capacity factor {factor}")
+
+
+def test_mx_forward_is_deterministic_and_graph_capturable():
+    """Two runs give the same bits; the MX forward, one-stream and overlapped, captured in a
+    CUDA graph and replayed gives them too (workspace and weights set up before capture)."""
+    cfg = SMALL[1]
+    inp = gpu_inputs(cfg)
+    w13_q, w13_sf = moe.quantize_mx(inp["w13"])
+    w2_q, w2_sf = moe.quantize_mx(inp["w2"])
+    ws = torch.empty(moe.workspace_bytes_mx(cfg), dtype=torch.uint8, device="cuda")
+    args = (cfg, inp["x"], inp["w_gate"], inp["bias"], inp["expert_owner"], w13_q, w13_sf, w2_q, w2_sf)
+    y1 = moe.layer_forward_mx(*args, ws=ws)
+    y2 = moe.layer_forward_mx(*args, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    side = torch.cuda.Stream()
+    for overlapped in (False, True):
+        kw = dict(side_stream=side) if overlapped else {}
+        y3 = torch.empty_like(y1)
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            moe.layer_forward_mx(*args, y=y3, ws=ws, **kw)  # warm-up on the capture stream
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            moe.layer_forward_mx(*args, y=y3, ws=ws, **kw)
+        for _ in range(2):
+            y3.zero_()
+            g.replay()
+            torch.cuda.synchronize()
+            assert torch.equal(y3, y1)
+        del g
