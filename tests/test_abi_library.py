@@ -173,3 +173,27 @@ def test_checked_build_loads_and_says_so():
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=dict(os.environ, MOE_LIB="checked"),
                        capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
+
+
+def test_mx_calls_refuse_unsupported_shapes_without_launching():
+    """The MX entry points refuse, before any launch and with a reason: rows whose length
+    is not a multiple of 32 (one E8M0 scale per 32 values), d % 512 != 0 or I % 128 != 0,
+    an fp32 configuration, and NULL operands; the MX workspace covers the codes and scales."""
+    lib = binding.load()
+    assert lib.moe_quantize_mx(ctypes.c_void_p(16), 4, 48, ctypes.c_void_p(16), ctypes.c_void_p(16), None) \
+        == binding.MOE_ERR_INVALID_ARG
+    assert b"32" in lib.moe_last_error()
+    assert lib.moe_quantize_mx(None, 4, 64, None, None, None) == binding.MOE_ERR_INVALID_ARG
+    for kw, want in ((dict(d=256), binding.MOE_ERR_UNSUPPORTED), (dict(I=192), binding.MOE_ERR_UNSUPPORTED),
+                     (dict(dtype="f32"), binding.MOE_ERR_UNSUPPORTED)):
+        c = binding.c_config(small_config(N=8, d=512, E=8, S=1, k=2, I=128, P=2).replace(**kw))
+        assert lib.moe_layer_forward_mx(ctypes.byref(c), None, None, None, None, None, None, None, None, None, None,
+                                        None, None, 0, None) == want, kw
+        assert lib.moe_grouped_ffn_mx(ctypes.byref(c), None, *([None] * 14)) == want, kw
+    c = binding.c_config(small_config(N=8, d=512, E=8, S=1, k=2, I=128, P=2))
+    lay = binding.CLayout()
+    assert lib.moe_grouped_ffn_mx(ctypes.byref(c), ctypes.byref(lay), *([None] * 14)) == binding.MOE_ERR_INVALID_ARG
+    wide = CONFIGS["wide"]
+    A, S = wide.N * wide.k, wide.S
+    need = A * wide.d * (1 + 1 / 32) + (A + S * wide.N) * (wide.I * (1 + 1 / 32) + wide.d * 2)
+    assert moe.workspace_bytes_mx(wide) >= need
