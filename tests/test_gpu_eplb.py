@@ -128,3 +128,57 @@ def test_full_size_skewed_routing_with_replicas(name, R):
                                 inp["w2"])
     torch.cuda.synchronize()
     assert torch.equal(res["y"], y_plain)
+
+
+@pytest.mark.parametrize("R", [8, 16])
+def test_mx_layer_with_replicas_equals_mx_layer_without(R):
+    """Redundant slots on the MXFP8 path: the slots carry copies of the MX codes and scale
+    rows (eplb_place_weights moves any per-expert bytes), and the MX layer over the E + R
+    slots gives the MX layer without copies, bit for bit."""
+    cfg = small_config("e_mx", cfg_id=139, N=700, d=512, E=16, S=1, k=4, I=128, P=8)
+    inp = gpu_inputs(cfg)
+    logits, ids, w = moe.route(cfg, inp["x"], inp["w_gate"], inp["bias"])
+    n_e = torch.bincount(ids.reshape(-1).long(), minlength=cfg.E).cpu().numpy()
+    plan = moe.eplb_plan(n_e, R, cfg.P)
+    ro, rs = _tables(plan)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    phys = moe.eplb_assign(cfg, ids, ro, rs, cfg.E + R, status=status)
+    pcfg = moe.physical_config(cfg, R)
+    w13_q, w13_sf = moe.quantize_mx(inp["w13"])
+    w2_q, w2_sf = moe.quantize_mx(inp["w2"])
+    place = [moe.eplb_place_weights(plan["slot_expert"], cfg.E, cfg.S, t) for t in (w13_q, w13_sf, w2_q, w2_sf)]
+    lay = moe.dispatch_layout(pcfg, phys, None, status=status)
+    x_q, x_sf = moe.quantize_mx(inp["x"])
+    xp, xp_sf = moe.permute_mx(pcfg, lay, x_q, x_sf)
+    _, _, _, out = moe.grouped_ffn_mx(pcfg, lay, xp, xp_sf, x_q, x_sf, *place, topk_w=w)
+    y = moe.combine(pcfg, lay, out)
+    y_plain = moe.layer_forward_mx(cfg, inp["x"], inp["w_gate"], inp["bias"], None, w13_q, w13_sf, w2_q, w2_sf)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(y, y_plain)
+
+
+def test_fp8_layer_with_replicas_equals_fp8_layer_without():
+    """The same on the row-scaled FP8 path: slot copies of the e4m3 codes and row scales."""
+    R = 8
+    cfg = small_config("e_f8", cfg_id=140, N=700, d=256, E=16, S=1, k=4, I=128, P=8)
+    inp = gpu_inputs(cfg)
+    logits, ids, w = moe.route(cfg, inp["x"], inp["w_gate"], inp["bias"])
+    n_e = torch.bincount(ids.reshape(-1).long(), minlength=cfg.E).cpu().numpy()
+    plan = moe.eplb_plan(n_e, R, cfg.P)
+    ro, rs = _tables(plan)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    phys = moe.eplb_assign(cfg, ids, ro, rs, cfg.E + R, status=status)
+    pcfg = moe.physical_config(cfg, R)
+    w13_q, w13_s = moe.quantize_fp8(inp["w13"])
+    w2_q, w2_s = moe.quantize_fp8(inp["w2"])
+    place = [moe.eplb_place_weights(plan["slot_expert"], cfg.E, cfg.S, t) for t in (w13_q, w13_s, w2_q, w2_s)]
+    lay = moe.dispatch_layout(pcfg, phys, None, status=status)
+    x_q, x_s = moe.quantize_fp8(inp["x"])
+    xp = moe.permute_fp8(pcfg, lay, x_q)
+    _, _, _, out = moe.grouped_ffn_fp8(pcfg, lay, xp, x_q, x_s, *place, topk_w=w)
+    y = moe.combine(pcfg, lay, out)
+    y_plain = moe.layer_forward_fp8(cfg, inp["x"], inp["w_gate"], inp["bias"], None, w13_q, w13_s, w2_q, w2_s)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(y, y_plain)
