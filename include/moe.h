@@ -123,8 +123,8 @@ const char* moe_status_string(int32_t status);
 const char* moe_last_error(void);
 
 /*
- * Bounds-checked build (no counterpart in the pages; the survey's substitute for a race /
- * bounds sanitizer, which is closed on this GPU pool).  The same sources compiled with
+ * Bounds-checked build (no counterpart in the pages; it stands in for a race / bounds
+ * sanitizer).  The same sources compiled with
  * -DMOE_CHECKS give libmoe_checked.so, whose kernels check every index they read from a
  * caller-visible map or table before using it: token -> row maps (tok2row, send2row,
  * tok2send) in the permute and combine, row -> assignment (row2tok) in the FC2 gate and
